@@ -1,0 +1,304 @@
+"""Seeded synthetic inputs for the gated delta rule workloads.
+
+This module only draws random numbers and shapes them into the five
+workloads; it holds none of the method's arithmetic (no gate cumsum, no
+decay, no delta update).  Both the fp64 CPU oracle (through the tests) and
+the CUDA library (through the tests and ``bench.py``) are fed from here, so
+the two sides always see bit-identical inputs.
+
+Generator
+---------
+Counter-based SplitMix64: element ``n`` of tensor ``tid`` under ``seed`` is
+``mix64(base(seed, tid) + (n + 1) * 0x9E3779B97F4A7C15)`` (mod 2**64), where
+``mix64`` is the published SplitMix64 output function (Steele, Lea & Flood,
+"Fast splittable pseudorandom number generators", OOPSLA 2014).  The top 53
+bits give a uniform double in [0, 1).  Normals use Box-Muller on the pair of
+counters (2n, 2n+1).  Because every element is a pure function of
+(seed, tid, flat index), any subset of a tensor (a few heads of a large
+workload) can be generated without generating the rest, on CPU or GPU, with
+identical results.
+
+Value recipes follow the workload descriptions: q, k ~ N(0,1) L2-normalised
+per token, v ~ N(0,1), beta = sigmoid(N(0,1)), per-channel or scalar
+log-decay g, S0 zero or N(0, 0.02) (0.02 is the standard deviation).
+Low-precision tensors are produced by rounding fp64 -> fp32 -> bf16, both
+round-to-nearest-even.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Dict, Optional, Sequence
+
+import torch
+
+_M64 = (1 << 64) - 1
+_GOLDEN = 0x9E3779B97F4A7C15
+_MIX1 = 0xBF58476D1CE4E5B9
+_MIX2 = 0x94D049BB133111EB
+_STREAM = 0xD1B54A32D192ED03
+
+# tensor ids: one independent stream per input tensor
+TID_Q, TID_K, TID_V, TID_G, TID_BETA, TID_S0, TID_CHAN = 1, 2, 3, 4, 5, 6, 7
+
+
+def _s64(c: int) -> int:
+    """Unsigned 64-bit constant -> the int64 with the same bits."""
+    c &= _M64
+    return c - (1 << 64) if c >= (1 << 63) else c
+
+
+def mix64_int(z: int) -> int:
+    """SplitMix64 output function on a Python int (exact, for reference)."""
+    z &= _M64
+    z = ((z ^ (z >> 30)) * _MIX1) & _M64
+    z = ((z ^ (z >> 27)) * _MIX2) & _M64
+    return z ^ (z >> 31)
+
+
+def stream_base(seed: int, tid: int) -> int:
+    return mix64_int(mix64_int(seed) ^ ((tid * _STREAM) & _M64))
+
+
+def _srl(z: torch.Tensor, s: int) -> torch.Tensor:
+    """Logical right shift of int64 bit patterns."""
+    return torch.bitwise_and(torch.bitwise_right_shift(z, s), (1 << (64 - s)) - 1)
+
+
+def _mix64_t(z: torch.Tensor) -> torch.Tensor:
+    z = torch.bitwise_xor(z, _srl(z, 30)) * _s64(_MIX1)
+    z = torch.bitwise_xor(z, _srl(z, 27)) * _s64(_MIX2)
+    return torch.bitwise_xor(z, _srl(z, 31))
+
+
+def raw_u64(seed: int, tid: int, counters: torch.Tensor) -> torch.Tensor:
+    """int64 tensor holding the 64-bit outputs for the given counters."""
+    base = _s64(stream_base(seed, tid))
+    z = base + (counters.to(torch.int64) + 1) * _s64(_GOLDEN)
+    return _mix64_t(z)
+
+
+def uniform(seed: int, tid: int, counters: torch.Tensor) -> torch.Tensor:
+    """fp64 uniforms in [0, 1) for the given counters."""
+    u = _srl(raw_u64(seed, tid, counters), 11)
+    return u.to(torch.float64) * (2.0 ** -53)
+
+
+def normal(seed: int, tid: int, index: torch.Tensor) -> torch.Tensor:
+    """fp64 standard normals for element indices (Box-Muller on 2n, 2n+1)."""
+    index = index.to(torch.int64)
+    u1 = uniform(seed, tid, 2 * index)
+    u2 = uniform(seed, tid, 2 * index + 1)
+    return torch.sqrt(-2.0 * torch.log1p(-u1)) * torch.cos((2.0 * math.pi) * u2)
+
+
+def _softplus64(x: torch.Tensor) -> torch.Tensor:
+    return torch.where(x > 30.0, x, torch.log1p(torch.exp(torch.clamp(x, max=30.0))))
+
+
+def _sigmoid64(x: torch.Tensor) -> torch.Tensor:
+    return 1.0 / (1.0 + torch.exp(-x))
+
+
+def to_dtype(x64: torch.Tensor, dtype: torch.dtype) -> torch.Tensor:
+    """fp64 -> fp32 (RNE) -> dtype (RNE)."""
+    x32 = x64.to(torch.float32)
+    return x32 if dtype == torch.float32 else x32.to(dtype)
+
+
+# --------------------------------------------------------------------------
+# workloads
+# --------------------------------------------------------------------------
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    kind: str            # "chunk" or "decode"
+    B: int
+    H: int
+    T: int               # tokens per sequence (chunk) or steps (decode)
+    dk: int
+    dv: int
+    C: int
+    gate: str            # "per_channel" or "scalar"
+    dtype: torch.dtype   # dtype of q, k, v, O
+    g_recipe: str
+    s0: str              # "zero" or "normal002"
+    seed: int
+    description: str
+
+    @property
+    def tokens(self) -> int:
+        """Tokens one pass processes: B*T for the forward, B per decode step."""
+        return self.B * self.T
+
+
+WORKLOADS: Dict[str, Workload] = {
+    "kda_tiny_fp32": Workload(
+        "kda_tiny_fp32", "chunk", 1, 2, 256, 64, 64, 64, "per_channel", torch.float32,
+        "softplus_n01_plus1_clamp5", "zero", 0,
+        "KDA forward, tiny, fp32: B1 H2 T256 d64 C64"),
+    "gdn_scalar_t4096": Workload(
+        "gdn_scalar_t4096", "chunk", 4, 16, 4096, 128, 128, 64, "scalar", torch.bfloat16,
+        "scalar_softplus_n01_plus2", "zero", 1,
+        "Gated DeltaNet (scalar gate) forward: B4 H16 T4096 d128 C64 bf16"),
+    "kda_d128_t8192": Workload(
+        "kda_d128_t8192", "chunk", 2, 32, 8192, 128, 128, 64, "per_channel", torch.bfloat16,
+        "softplus_n02_clamp5", "normal002", 2,
+        "KDA forward at head dim 128: B2 H32 T8192 d128 C64 bf16"),
+    "kda_long_t65536": Workload(
+        "kda_long_t65536", "chunk", 1, 32, 65536, 128, 128, 64, "per_channel", torch.bfloat16,
+        "long_context_mix", "normal002", 3,
+        "KDA long-context forward: B1 H32 T65536 d128 C64 bf16"),
+    "kda_decode_b256": Workload(
+        "kda_decode_b256", "decode", 256, 32, 1000, 128, 128, 1, "per_channel", torch.bfloat16,
+        "softplus_n01_plus1_clamp5", "normal002", 4,
+        "KDA recurrent decode: B256 H32 d128, 1000 steps, fp32 state"),
+}
+
+# the five workloads in the order the method's configurations list them
+ORDER = ["kda_tiny_fp32", "gdn_scalar_t4096", "kda_d128_t8192", "kda_long_t65536", "kda_decode_b256"]
+
+LONG_FAST_CHANNELS = 13  # round(0.1 * 128) channels per head pinned at g = -5
+
+
+def _g_from_recipe(w: Workload, seed: int, idx: torch.Tensor, b: torch.Tensor, h: torch.Tensor,
+                   c: Optional[torch.Tensor], fast: Optional[Dict]) -> torch.Tensor:
+    r = w.g_recipe
+    if r == "softplus_n01_plus1_clamp5":
+        return torch.clamp(-_softplus64(normal(seed, TID_G, idx) + 1.0), min=-5.0)
+    if r == "scalar_softplus_n01_plus2":
+        return -_softplus64(normal(seed, TID_G, idx) + 2.0)
+    if r == "softplus_n02_clamp5":
+        return torch.clamp(-_softplus64(2.0 * normal(seed, TID_G, idx)), min=-5.0)
+    if r == "long_context_mix":
+        u = uniform(seed, TID_G, idx)
+        slow = -(0.001 + 0.049 * u)
+        is_fast = fast["mask"][b * w.H + h, c]
+        return torch.where(is_fast, torch.full_like(slow, -5.0), slow)
+    raise ValueError(r)
+
+
+def fast_channel_mask(w: Workload, device="cpu") -> torch.Tensor:
+    """[B*H, dk] bool: the channels pinned at g=-5 in the long-context workload.
+
+    Per head, the LONG_FAST_CHANNELS channels with the smallest draw from
+    stream TID_CHAN are chosen.
+    """
+    n = w.B * w.H * w.dk
+    u = uniform(w.seed, TID_CHAN, torch.arange(n, device=device)).view(w.B * w.H, w.dk)
+    order = torch.argsort(u, dim=1)
+    mask = torch.zeros(w.B * w.H, w.dk, dtype=torch.bool, device=device)
+    mask.scatter_(1, order[:, :LONG_FAST_CHANNELS], True)
+    return mask
+
+
+def _chunked(n: int, block: int):
+    s = 0
+    while s < n:
+        e = min(n, s + block)
+        yield s, e
+        s = e
+
+
+def generate(w: Workload, device="cpu", heads: Optional[Sequence[int]] = None,
+             steps: Optional[int] = None, block: int = 1 << 24) -> Dict[str, torch.Tensor]:
+    """Inputs of workload ``w``.
+
+    ``heads``: optional list of flat head ids (b*H + h); when given, tensors
+    keep their full (B, H) extent only along the selected heads, returned as
+    shape [len(heads), 1, ...] with the same values the full tensor holds
+    there.  ``steps`` (decode only) limits the number of steps generated.
+
+    Chunk workloads return q, k [B,H,T,dk], v [B,H,T,dv], g [B,H,T,dk] or
+    [B,H,T], beta [B,H,T], S0 [B,H,dv,dk] (fp32).  Decode returns the same
+    keys with a leading steps axis: q [S,B,H,dk] ... and S0 [B,H,dv,dk].
+    """
+    B, H, dk, dv = w.B, w.H, w.dk, w.dv
+    if heads is None:
+        head_ids = torch.arange(B * H, dtype=torch.int64, device=device)
+        outB, outH = B, H
+    else:
+        head_ids = torch.as_tensor(list(heads), dtype=torch.int64, device=device)
+        outB, outH = len(heads), 1
+    nh = head_ids.numel()
+    fast = {"mask": fast_channel_mask(w, device)} if w.g_recipe == "long_context_mix" else None
+    seed = w.seed
+    decode = w.kind == "decode"
+    T = (steps if steps is not None else w.T)
+
+    def field(tid, width, make, out_dtype):
+        # flat index of element (t, head, j) in the full tensor
+        if decode:
+            shape = (T, nh, width) if width else (T, nh)
+        else:
+            shape = (nh, T, width) if width else (nh, T)
+        out = torch.empty(shape, dtype=out_dtype, device=device)
+        flat = out.view(-1)
+        n = flat.numel()
+        per_row = width if width else 1
+        for s, e in _chunked(n, block):
+            lin = torch.arange(s, e, dtype=torch.int64, device=device)
+            j = lin % per_row
+            rest = lin // per_row
+            if decode:
+                hsel = rest % nh
+                t = rest // nh
+                hid = head_ids[hsel]
+                full = (t * (B * H) + hid) * per_row + j
+            else:
+                t = rest % T
+                hsel = rest // T
+                hid = head_ids[hsel]
+                full = (hid * w.T + t) * per_row + j
+            flat[s:e] = make(tid, full, hid // H, hid % H, j if width else None, t)
+        return out
+
+    def qk_field(tid):
+        raw = field(tid, dk, lambda tid_, full, b, h, c, t: normal(seed, tid_, full), torch.float64)
+        nrm = torch.sqrt((raw * raw).sum(-1, keepdim=True))
+        return to_dtype(raw / nrm, w.dtype)
+
+    q = qk_field(TID_Q)
+    k = qk_field(TID_K)
+    v = to_dtype(field(TID_V, dv, lambda tid_, full, b, h, c, t: normal(seed, tid_, full), torch.float64), w.dtype)
+    if w.gate == "per_channel":
+        g = field(TID_G, dk, lambda tid_, full, b, h, c, t: _g_from_recipe(w, seed, full, b, h, c, fast),
+                  torch.float64).to(torch.float32)
+    else:
+        g = field(TID_G, 0, lambda tid_, full, b, h, c, t: _g_from_recipe(w, seed, full, b, h, c, fast),
+                  torch.float64).to(torch.float32)
+    beta = field(TID_BETA, 0, lambda tid_, full, b, h, c, t: _sigmoid64(normal(seed, tid_, full)),
+                 torch.float64).to(torch.float32)
+
+    # initial state: [head, dv, dk], flat index over the full [B,H,dv,dk]
+    if w.s0 == "zero":
+        S0 = torch.zeros(nh, dv, dk, dtype=torch.float32, device=device)
+    else:
+        per = dv * dk
+        S0 = torch.empty(nh, dv, dk, dtype=torch.float32, device=device)
+        flat = S0.view(-1)
+        for s, e in _chunked(flat.numel(), block):
+            lin = torch.arange(s, e, dtype=torch.int64, device=device)
+            full = head_ids[lin // per] * per + lin % per
+            flat[s:e] = (0.02 * normal(seed, TID_S0, full)).to(torch.float32)
+
+    if decode:
+        shp = lambda x, *tail: x.view(T, outB, outH, *tail)
+        out = dict(q=shp(q, dk), k=shp(k, dk), v=shp(v, dv),
+                   g=shp(g, dk) if w.gate == "per_channel" else shp(g),
+                   beta=shp(beta), S0=S0.view(outB, outH, dv, dk))
+    else:
+        shp = lambda x, *tail: x.view(outB, outH, T, *tail)
+        out = dict(q=shp(q, dk), k=shp(k, dk), v=shp(v, dv),
+                   g=shp(g, dk) if w.gate == "per_channel" else shp(g),
+                   beta=shp(beta), S0=S0.view(outB, outH, dv, dk))
+    return out
+
+
+def small_chunk_case(B: int, H: int, T: int, dk: int, dv: int, gate: str, dtype: torch.dtype,
+                     g_recipe: str = "softplus_n01_plus1_clamp5", s0: str = "normal002",
+                     seed: int = 11, C: int = 64) -> Workload:
+    """An ad-hoc chunk workload with the same value recipes (parity tests)."""
+    return Workload(f"case_B{B}H{H}T{T}d{dk}x{dv}_{gate}", "chunk", B, H, T, dk, dv, C, gate, dtype,
+                    g_recipe, s0, seed, "parity case")

@@ -1,0 +1,123 @@
+"""fp64 CPU oracle of the gated delta rule -- TEST INFRASTRUCTURE.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline / reference
+leg of ``bench.py`` may import this package.  The CUDA library never imports,
+links or calls it, and it never imports the CUDA library.  It shares with the
+GPU side only the seeded input generator (``gdr_workloads``), which holds none
+of the method's arithmetic.
+
+Contents
+  * ``forward``   -- the token-by-token fp64 recurrence (``gdr_oracle.c``),
+    the parity reference for the chunked forward and the decode step.
+  * ``decode``    -- the same recurrence driven one decode step per token.
+  * ``chunk_form`` (module) -- an fp64 restatement of the chunkwise WY/UT
+    equations, used only to pin ``forward`` (it is not a parity reference).
+
+Every function reads exactly the values the GPU receives: bf16 and fp32
+tensors are widened to fp64 exactly before the recurrence runs.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+from typing import Optional, Tuple
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gdr_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle into ``oracle/liboracle.so`` (gcc, no FMA contraction)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared", "-pthread",
+               "-o", _LIB, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB)
+            P = ctypes.c_void_p
+            I = ctypes.c_int
+            lib.gdr_oracle_forward.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I]
+            lib.gdr_oracle_forward.restype = I
+            lib.gdr_oracle_online_cores.restype = I
+            _lib = lib
+    return _lib
+
+
+def online_cores() -> int:
+    return int(_load().gdr_oracle_online_cores())
+
+
+def _f64(x) -> Optional[np.ndarray]:
+    if x is None:
+        return None
+    if isinstance(x, torch.Tensor):
+        x = x.detach().to("cpu").to(torch.float64).contiguous().numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def forward(q, k, v, g, beta, S0=None, gate: str = "per_channel", erase=None, write=None,
+            clamp: bool = True, threads: int = 0) -> Tuple[np.ndarray, np.ndarray]:
+    """fp64 recurrence over T tokens.
+
+    Shapes: q, k [B,H,T,dk]; v [B,H,T,dv]; g [B,H,T,dk] (per_channel) or
+    [B,H,T] (scalar); beta [B,H,T]; S0 [B,H,dv,dk] or None.
+    ``erase`` / ``write`` ([B,H,T]) replace beta on the erase and write sides
+    (pins only).  Returns (O [B,H,T,dv], S_T [B,H,dv,dk]) as fp64 numpy arrays.
+    """
+    qa, ka, va, ga = _f64(q), _f64(k), _f64(v), _f64(g)
+    ba = _f64(beta)
+    ea, wa = _f64(erase), _f64(write)
+    B, H, T, dk = qa.shape
+    dv = va.shape[-1]
+    assert ka.shape == (B, H, T, dk) and va.shape == (B, H, T, dv)
+    if gate == "per_channel":
+        assert ga.shape == (B, H, T, dk)
+    elif gate == "scalar":
+        assert ga.shape == (B, H, T)
+    else:
+        raise ValueError(gate)
+    for x in (ba, ea, wa):
+        assert x is None or x.shape == (B, H, T)
+    s0 = _f64(S0)
+    if s0 is not None:
+        assert s0.shape == (B, H, dv, dk)
+    O = np.empty((B, H, T, dv), dtype=np.float64)
+    ST = np.empty((B, H, dv, dk), dtype=np.float64)
+    rc = _load().gdr_oracle_forward(_ptr(qa), _ptr(ka), _ptr(va), _ptr(ga), _ptr(ba), _ptr(ea), _ptr(wa),
+                                    _ptr(s0), _ptr(O), _ptr(ST), B, H, T, dk, dv,
+                                    1 if gate == "scalar" else 0, 1 if clamp else 0, int(threads))
+    if rc != 0:
+        raise RuntimeError("oracle forward failed")
+    return O, ST
+
+
+def decode(q, k, v, g, beta, S, gate: str = "per_channel", threads: int = 0) -> Tuple[np.ndarray, np.ndarray]:
+    """``steps`` consecutive single-token updates.
+
+    q, k [steps,B,H,dk]; v [steps,B,H,dv]; g [steps,B,H,dk] or [steps,B,H];
+    beta [steps,B,H]; S [B,H,dv,dk].  A decode step is one token of the
+    recurrence, so this runs ``forward`` with the steps as the token axis.
+    Returns (o [steps,B,H,dv], S_final [B,H,dv,dk]).
+    """
+    mv = lambda x: _f64(x).transpose(1, 2, 0, *range(3, _f64(x).ndim)).copy()
+    O, ST = forward(mv(q), mv(k), mv(v), mv(g), mv(beta), S0=S, gate=gate, threads=threads)
+    return O.transpose(2, 0, 1, 3).copy(), ST

@@ -1,0 +1,185 @@
+/*
+ * gdr_oracle.c -- fp64 CPU oracle of the gated delta rule.
+ *
+ * TEST INFRASTRUCTURE.  Only the tests, the smoke check and the CPU-baseline
+ * leg of the benchmark load this file's library.  It shares no code, header,
+ * table or constant with the CUDA library and never touches a GPU.
+ *
+ * What it computes: the plain token-by-token recurrence, in the d_v x d_k
+ * orientation,
+ *
+ *     S_t = S_{t-1} Diag(alpha_t) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,
+ *     o_t = S_t q_t,
+ *
+ * as the first line of the induction in "Reading notes: Kimi Delta
+ * Attention" (mzeromiko), section 4 "Forward pass", writes it:
+ * S_t = S_{t-1}Diag(alpha_t) + beta_t (v_t - S_{t-1}Diag(alpha_t) k_t) k_t^T.
+ * Each token is done in the order the pseudo-code of "KDA vs Gated DeltaNet"
+ * (brenchcc), section 4 "How the source maps to the formulas", gives:
+ * decay the state, predict the value from the decayed state, form the
+ * delta, write it along the key, read the output with the query.
+ *
+ *   - per-channel gate (KDA): alpha_t = exp(max(g_t, -5)) per key channel;
+ *     the -5 lower bound is the g_min of the KDA gate in "Lightweight LLM
+ *     reproduction: Linear Attention" (aitujian), section 3.1 [7a].
+ *   - scalar gate (Gated DeltaNet): alpha_t = exp(g_t) for the whole head,
+ *     "Token Mixer I", section "Gated Delta Networks" (no bound applied).
+ *
+ * Oracle-only extension used by the pins: the erase and write strengths may
+ * be given apart from beta (the tied-scalar case of Gated DeltaNet-2's erase
+ * and write gates, "Token Mixer I", section "Gated DeltaNet-2 / Decoupling
+ * erase and write"): delta = w_t v_t - e_t (S~ k_t).  With e = w = beta it is
+ * the method itself; e = 0, w = 1 gives (gated) linear attention.
+ *
+ * Layouts (row-major, contiguous, fp64):
+ *   q, k   [B,H,T,dk]      v, O [B,H,T,dv]
+ *   g      [B,H,T,dk] (per-channel) or [B,H,T] (scalar)
+ *   beta, erase, write  [B,H,T]      (erase / write may be NULL -> beta)
+ *   S0, S_T [B,H,dv,dk]              (S0 NULL -> zeros, S_T NULL -> not written)
+ * Heads are independent; they are spread over nthreads POSIX threads
+ * (nthreads <= 0 -> all online cores).  Returns 0, or -1 on a bad argument
+ * or allocation failure.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdlib.h>
+#include <string.h>
+#include <unistd.h>
+
+typedef struct {
+    const double *q, *k, *v, *g, *beta, *erase, *write, *S0;
+    double *O, *S_T;
+    int B, H, T, dk, dv, per_channel, clamp;
+    int head_begin, head_end;
+    int status;
+} oracle_job;
+
+static void run_head(const oracle_job *J, int head, double *S, double *a, double *delta)
+{
+    const int T = J->T, dk = J->dk, dv = J->dv;
+    const size_t hk = (size_t)head * T * dk, hv = (size_t)head * T * dv, hs = (size_t)head * T;
+    const size_t hS = (size_t)head * dv * dk;
+
+    if (J->S0) memcpy(S, J->S0 + hS, sizeof(double) * dv * dk);
+    else memset(S, 0, sizeof(double) * dv * dk);
+
+    for (int t = 0; t < T; ++t) {
+        const double *qt = J->q + hk + (size_t)t * dk;
+        const double *kt = J->k + hk + (size_t)t * dk;
+        const double *vt = J->v + hv + (size_t)t * dv;
+        double *ot = J->O + hv + (size_t)t * dv;
+
+        /* gate: alpha_t */
+        if (J->per_channel) {
+            const double *gt = J->g + hk + (size_t)t * dk;
+            for (int c = 0; c < dk; ++c) {
+                double gc = gt[c];
+                if (J->clamp && gc < -5.0) gc = -5.0;
+                a[c] = exp(gc);
+            }
+        } else {
+            const double as = exp(J->g[hs + t]);
+            for (int c = 0; c < dk; ++c) a[c] = as;
+        }
+        const double e = J->erase ? J->erase[hs + t] : J->beta[hs + t];
+        const double w = J->write ? J->write[hs + t] : J->beta[hs + t];
+
+        /* decay, then predict from the decayed state: p = S~ k */
+        for (int i = 0; i < dv; ++i) {
+            double *row = S + (size_t)i * dk;
+            double p = 0.0;
+            for (int c = 0; c < dk; ++c) {
+                row[c] *= a[c];
+                p += row[c] * kt[c];
+            }
+            delta[i] = w * vt[i] - e * p;
+        }
+        /* write the delta along k, then read with q: o = S_t q */
+        for (int i = 0; i < dv; ++i) {
+            double *row = S + (size_t)i * dk;
+            double o = 0.0;
+            for (int c = 0; c < dk; ++c) {
+                row[c] += delta[i] * kt[c];
+                o += row[c] * qt[c];
+            }
+            ot[i] = o;
+        }
+    }
+    if (J->S_T) memcpy(J->S_T + hS, S, sizeof(double) * dv * dk);
+}
+
+static void *worker(void *arg)
+{
+    oracle_job *J = (oracle_job *)arg;
+    double *S = (double *)malloc(sizeof(double) * (size_t)J->dv * J->dk);
+    double *a = (double *)malloc(sizeof(double) * (size_t)J->dk);
+    double *delta = (double *)malloc(sizeof(double) * (size_t)J->dv);
+    if (!S || !a || !delta) {
+        J->status = -1;
+    } else {
+        for (int h = J->head_begin; h < J->head_end; ++h) run_head(J, h, S, a, delta);
+    }
+    free(S);
+    free(a);
+    free(delta);
+    return NULL;
+}
+
+int gdr_oracle_forward(const double *q, const double *k, const double *v, const double *g,
+                       const double *beta, const double *erase, const double *write,
+                       const double *S0, double *O, double *S_T,
+                       int B, int H, int T, int dk, int dv,
+                       int gate_scalar, int clamp, int nthreads)
+{
+    if (!q || !k || !v || !g || !O || B < 0 || H < 0 || T < 0 || dk <= 0 || dv <= 0) return -1;
+    if (!beta && (!erase || !write)) return -1;
+    const int heads = B * H;
+    if (heads == 0) return 0;
+    if (nthreads <= 0) nthreads = (int)sysconf(_SC_NPROCESSORS_ONLN);
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > heads) nthreads = heads;
+
+    oracle_job *jobs = (oracle_job *)calloc((size_t)nthreads, sizeof(oracle_job));
+    pthread_t *tid = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
+    if (!jobs || !tid) {
+        free(jobs);
+        free(tid);
+        return -1;
+    }
+    int status = 0;
+    for (int j = 0; j < nthreads; ++j) {
+        oracle_job *J = &jobs[j];
+        J->q = q; J->k = k; J->v = v; J->g = g; J->beta = beta;
+        J->erase = erase; J->write = write; J->S0 = S0; J->O = O; J->S_T = S_T;
+        J->B = B; J->H = H; J->T = T; J->dk = dk; J->dv = dv;
+        J->per_channel = !gate_scalar;
+        J->clamp = clamp;
+        J->head_begin = (int)((long long)heads * j / nthreads);
+        J->head_end = (int)((long long)heads * (j + 1) / nthreads);
+        J->status = 0;
+    }
+    int started = 0;
+    for (int j = 1; j < nthreads; ++j) {
+        if (pthread_create(&tid[j], NULL, worker, &jobs[j]) != 0) {
+            /* fall back to running this share on the calling thread */
+            worker(&jobs[j]);
+            tid[j] = 0;
+        } else {
+            ++started;
+        }
+    }
+    worker(&jobs[0]);
+    for (int j = 1; j < nthreads; ++j)
+        if (tid[j]) pthread_join(tid[j], NULL);
+    for (int j = 0; j < nthreads; ++j)
+        if (jobs[j].status) status = -1;
+    (void)started;
+    free(jobs);
+    free(tid);
+    return status;
+}
+
+int gdr_oracle_online_cores(void)
+{
+    return (int)sysconf(_SC_NPROCESSORS_ONLN);
+}

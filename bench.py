@@ -1,0 +1,428 @@
+#!/usr/bin/env python
+"""Throughput of the gated delta rule on B200: one JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole hot path over one batch: one chunked forward
+(``gdr_chunk_fwd``) of the workload, or for the decode workload its 1000
+consecutive single-token steps.  Default workload: the KDA forward at head
+dim 128 (B=2, H=32, T=8192, d_k=d_v=128, C=64, bf16) -- the size the method's
+throughput target is quoted at.
+
+Multi-GPU (launched with torch.distributed.run, one process per GPU): every
+(b, h) sequence is an independent recurrence, so each rank runs its own batch
+of the same shape (different seed) with no collective on the data path
+(weak scaling).  Timing: W untimed warm-up steps, then K steps bracketed by a
+barrier and a device synchronize on both sides, timed with CUDA events on the
+launching stream; the job time is the max over ranks; ``value`` is the
+tokens all ranks processed divided by that time.
+
+``--impl reference`` times the fp64 CPU oracle (the only reference this
+method has) on the host cores, rank 0 only, each step a bounded sample of
+the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import gdr_workloads as W  # noqa: E402
+
+METRIC = "tokens/s (device-timed) of gated-delta-rule chunk fwd; % of roofline"
+METRIC_DECODE = "tokens/s (device-timed) of gated-delta-rule recurrent decode step; % of HBM roofline"
+DEFAULT_WORKLOAD = "kda_d128_t8192"
+
+# DRAM traffic per launch of the dominant kernel, from one ncu capture, keyed
+# by the kernel's source file and that file's hash when captured; the entry
+# is ignored (traffic = null) as soon as the source changes.
+TRAFFIC = {}
+
+
+# ----------------------------------------------------------------- helpers
+
+def algorithmic_bytes(w: W.Workload) -> int:
+    """Bytes one step must move at least: every input read once, every output
+    written once (no intermediates)."""
+    e = 2 if w.dtype == torch.bfloat16 else 4
+    gate = w.dk * 4 if w.gate == "per_channel" else 4
+    per_token = 2 * w.dk * e + w.dv * e + gate + 4 + w.dv * e       # q, k, v, g, beta, O
+    heads = w.B * w.H
+    state = 2 * w.dv * w.dk * 4                                     # S0 read + S_T write
+    if w.kind == "decode":
+        return w.T * heads * (per_token + state)                    # the state moves every step
+    return heads * w.T * per_token + heads * state
+
+
+def dense_flops(w: W.Workload) -> int:
+    """Tensor-core flops of one step of the chunk form (C x C tiles counted full)."""
+    if w.kind == "decode":
+        return w.T * w.B * w.H * 8 * w.dk * w.dv
+    C, dk, dv = w.C, w.dk, w.dv
+    per_chunk = 2 * C * C * (3 * dk + 2 * dv) + 6 * C * dk * dv
+    return w.B * w.H * (w.T // C) * per_chunk
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def roofline(w: W.Workload, seconds_per_launch: float, peaks, kernel_src: str = None):
+    byts = algorithmic_bytes(w)
+    flops = dense_flops(w)
+    t_hbm = byts / (peaks["hbm_gbs"] * 1e9)
+    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+    traffic = None
+    ent = TRAFFIC.get(w.name)
+    if ent and kernel_src and ent.get("src_sha") == file_sha(kernel_src):
+        traffic = ent["bytes_per_launch"]
+    if t_hbm >= t_tc:
+        ach = byts / seconds_per_launch / 1e9
+        return {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(ach / peaks["hbm_gbs"], 4), "traffic": traffic,
+                "peak_source": peaks["source"] + " (copy bandwidth)", "algorithmic_bytes": byts}
+    ach = flops / seconds_per_launch / 1e12
+    return {"bound": "tensor", "achieved": round(ach, 2), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": round(ach / peaks["bf16_tflops"], 4), "traffic": traffic,
+            "peak_source": peaks["source"], "algorithmic_flops": flops}
+
+
+def file_sha(path: str) -> str:
+    try:
+        return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+    except OSError:
+        return ""
+
+
+def rank_workload(w: W.Workload, rank: int) -> W.Workload:
+    """Weak scaling: rank r runs the same shapes with its own seed."""
+    import dataclasses
+    return dataclasses.replace(w, seed=w.seed + 1000 * rank)
+
+
+def reduce_max(x: float, world: int, device) -> float:
+    if world <= 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------ clock sampler
+
+_REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+
+class ClockSampler:
+    """nvidia-smi samples (SM clock, max clock, throttle reasons) in the background."""
+
+    def __init__(self, gpu_id: str, period_ms: int = 50):
+        self.samples = []
+        self.proc = None
+        fields = "timestamp,clocks.sm,clocks.max.sm,power.draw," + ",".join(
+            "clocks_event_reasons." + r for r in _REASONS)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", gpu_id, f"--query-gpu={fields}", "--format=csv,noheader,nounits",
+                 f"-lms={period_ms}"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 4 + len(_REASONS):
+                continue
+            try:
+                self.samples.append((time.time(), float(parts[1]), float(parts[2]),
+                                     [r for r, v in zip(_REASONS, parts[4:]) if v.lower() == "active"]))
+            except ValueError:
+                pass
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0: float, t1: float):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "note": "nvidia-smi unavailable"}
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        note = "samples inside the timed region"
+        if not inside:
+            inside = sorted(self.samples, key=lambda s: min(abs(s[0] - t0), abs(s[0] - t1)))[:3]
+            note = "timed region shorter than the sampling period; nearest samples"
+        reasons = sorted({r for s in inside for r in s[3]})
+        return {"sm_mhz": statistics.median(s[1] for s in inside), "sm_max_mhz": max(s[2] for s in inside),
+                "reasons": reasons, "samples": len(inside), "note": note}
+
+
+def gpu_id_for(device) -> str:
+    try:
+        u = torch.cuda.get_device_properties(device).uuid
+        s = str(u)
+        return s if s.startswith("GPU-") else "GPU-" + s
+    except Exception:
+        return str(device.index if device.index is not None else 0)
+
+
+# ------------------------------------------------------------ CPU oracle leg
+
+def oracle_sample(w: W.Workload, budget_s: float, seed_rank: int = 0):
+    """Time the fp64 oracle on a bounded sample of workload ``w``.
+
+    The sample is ``heads`` whole heads (as many as host threads, at most all
+    of them) over the first ``tokens`` tokens (or decode steps), sized from a
+    short calibration run to take about ``budget_s`` seconds.  Returns
+    (tokens/s in the workload's unit, description dict).
+    """
+    import oracle
+    cores = oracle.online_cores()
+    heads_total = w.B * w.H
+    heads = min(heads_total, cores)
+    hl = list(range(0, heads_total, max(1, heads_total // heads)))[:heads]
+
+    def run(ntok):
+        if w.kind == "decode":
+            x = W.generate(w, heads=hl, steps=ntok)
+            t = time.perf_counter()
+            oracle.decode(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], gate=w.gate, threads=cores)
+            return time.perf_counter() - t
+        x = W.generate(w, heads=hl)
+        sl = lambda a: a[:, :, :ntok]
+        t = time.perf_counter()
+        oracle.forward(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["g"]), sl(x["beta"]), x["S0"],
+                       gate=w.gate, threads=cores)
+        return time.perf_counter() - t
+
+    cal_tok = min(w.T, 64)
+    t_cal = run(cal_tok)
+    per_tok = t_cal / cal_tok
+    ntok = int(max(cal_tok, min(w.T, budget_s / max(per_tok, 1e-9))))
+    if ntok != cal_tok:
+        dt = run(ntok)
+    else:
+        dt = t_cal
+    head_tokens_per_s = len(hl) * ntok / dt
+    # a workload token (one position of one sequence) spans all H heads
+    tokens_per_s = head_tokens_per_s / w.H
+    unit_note = "decode steps" if w.kind == "decode" else "tokens"
+    return tokens_per_s, {"kind": "oracle", "cores": min(cores, len(hl)),
+                          "sample": f"fp64 oracle on {len(hl)} of {heads_total} heads x {ntok} {unit_note} "
+                                    f"of {w.name} ({dt:.1f} s)", "seconds": round(dt, 2)}
+
+
+# ------------------------------------------------------------------ main
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(W.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def base_line(w: W.Workload, args, world: int):
+    return {
+        "metric": METRIC_DECODE if w.kind == "decode" else METRIC,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32",
+        "data": "synthetic (seeded counter-based generator, shapes and value recipes of the workload)",
+        "config": {
+            "workload": w.name, "description": w.description, "B": w.B, "H": w.H, "T": w.T,
+            "dk": w.dk, "dv": w.dv, "C": w.C, "gate": w.gate,
+            "global_batch": w.B * world, "seq_len": w.T,
+            "parallelism": f"dp{world} (independent sequences per GPU, no collective)",
+            "l2": "inputs larger than L2 (%.0f MB per step vs 126 MB)" % (algorithmic_bytes(w) / 1e6),
+        },
+    }
+
+
+def run_reference(args, w: W.Workload, rank: int, world: int):
+    if rank != 0:
+        return 0
+    budget = max(1.0, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
+    vals = []
+    desc = None
+    for i in range(args.warmup + args.steps):
+        v, desc = oracle_sample(w, budget)
+        if i >= args.warmup:
+            vals.append(v)
+    value = statistics.median(vals)
+    line = base_line(w, args, world)
+    line.update({"impl": "reference", "value": value,
+                 "ms_per_step": (w.tokens / value) * 1e3,
+                 "cpu_baseline": dict(desc, value=value, unit="tokens/s"),
+                 "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+                 "gpu_launches": 0})
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", str(args.gpus)))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w0 = W.WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        return run_reference(args, w0, rank, world if "WORLD_SIZE" in os.environ else args.gpus)
+
+    import gated_delta_rule_89_b200 as gdr
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    w = rank_workload(w0, rank)
+    stream = torch.cuda.current_stream(device)
+
+    # ---- inputs resident in HBM before timing
+    if w.kind == "decode":
+        steps_needed = w.T
+        x = W.generate(w, device=device, steps=steps_needed)
+        S = x["S0"].clone()
+        o = torch.empty(w.B, w.H, w.dv, dtype=w.dtype, device=device)
+
+        def step():
+            for s in range(w.T):
+                gdr.recurrent_step(x["q"][s], x["k"][s], x["v"][s], x["g"][s], x["beta"][s], S, o=o)
+    else:
+        x = W.generate(w, device=device)
+        O = torch.empty(w.B, w.H, w.T, w.dv, dtype=w.dtype, device=device)
+        S_T = torch.empty(w.B, w.H, w.dv, w.dk, dtype=torch.float32, device=device)
+
+        def step():
+            gdr.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], C=w.C, gate=w.gate,
+                          O=O, S_T=S_T)
+    torch.cuda.synchronize(device)
+
+    sampler = ClockSampler(gpu_id_for(device)) if rank == 0 else None
+    for _ in range(args.warmup):
+        step()
+    launches_per_step = gdr.last_launch_count() * (w.T if w.kind == "decode" else 1)
+    torch.cuda.synchronize(device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t_wall0 = time.time()
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize(device)
+    t_wall1 = time.time()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = sum(step_ms)
+    total_ms = reduce_max(total_ms, world, device)
+    ms_per_step = total_ms / args.steps
+    # chunk: B*T tokens per step; decode: B sequences x T consecutive steps
+    tokens_job = w.B * w.T * world
+    value = tokens_job / (ms_per_step / 1e3)
+
+    # ---- end to end through the public API with host buffers (pinned)
+    e2e = None
+    if w.kind != "decode" and args.e2e_steps > 0:
+        hx = {k: v.to("cpu").pin_memory() for k, v in x.items()}
+        h2d = sum(v.numel() * v.element_size() for v in hx.values())
+        d2h = O.numel() * O.element_size() + S_T.numel() * S_T.element_size()
+        gdr.chunk_fwd(hx["q"], hx["k"], hx["v"], hx["g"], hx["beta"], hx["S0"], C=w.C, gate=w.gate)  # warm
+        torch.cuda.synchronize(device)
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            Oh, Sh = gdr.chunk_fwd(hx["q"], hx["k"], hx["v"], hx["g"], hx["beta"], hx["S0"], C=w.C, gate=w.gate)
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        e2e_ms = reduce_max(e0.elapsed_time(e1), world, device) / args.e2e_steps
+        e2e = {"value": w.tokens * world / (e2e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3)}
+        del hx
+    elif w.kind == "decode":
+        e2e = {"value": None, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0,
+               "note": "not measured for the decode workload"}
+
+    clocks = None
+    if sampler is not None:
+        sampler.stop()
+        clocks = sampler.summary(t_wall0, t_wall1)
+
+    if rank == 0:
+        peaks = load_peaks()
+        per_launch_s = statistics.mean(step_ms) / 1e3 / (w.T if w.kind == "decode" else 1)
+        wk = w0
+        if w.kind == "decode":
+            import dataclasses
+            wk = dataclasses.replace(w0, T=1)   # one launch = one decode step
+        src = os.path.join(ROOT, "gated_delta_rule_89_b200", "csrc",
+                           "recurrent_step.cu" if w.kind == "decode" else "chunk_tc.cu")
+        line = base_line(w0, args, world)
+        line.update({
+            "value": value,
+            "ms_per_step": round(ms_per_step, 4),
+            "roofline": roofline(wk, per_launch_s, peaks, src),
+            "gpu_launches": launches_per_step * args.steps,
+            "e2e": e2e,
+            "clocks": clocks,
+        })
+        if world == 1 and not args.no_cpu_baseline:
+            v, desc = oracle_sample(w0, args.cpu_budget)
+            line["cpu_baseline"] = dict(desc, value=v, unit="tokens/s")
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,200 @@
+"""B200-native gated delta rule (KDA / Gated DeltaNet): Python binding.
+
+A thin ctypes layer over ``libgdr.so`` (the C ABI declared in
+``include/gdr.h``).  It only marshals arguments: it checks dtypes, devices
+and contiguity, allocates outputs with PyTorch, passes raw device pointers
+and the current CUDA stream, and raises on a non-OK status.  Every step of
+the computation runs in the library's CUDA kernels; there is no fallback.
+If the library has not been built, importing the functions raises.
+
+Host tensors are accepted too: they are copied to the current CUDA device,
+processed, and the outputs are copied back to host memory (this is what the
+end-to-end measurement times).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+__all__ = ["chunk_fwd", "recurrent_step", "chunk_fwd_workspace_size", "GDRError", "library_path",
+           "last_launch_count", "GATE_PER_CHANNEL", "GATE_SCALAR"]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libgdr.so")
+_lib = None
+
+GDR_OK = 0
+GATE_PER_CHANNEL = 0
+GATE_SCALAR = 1
+_DTYPES = {torch.float32: 0, torch.bfloat16: 1}
+
+
+class GDRError(RuntimeError):
+    pass
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def lib() -> ctypes.CDLL:
+    """Load libgdr.so (raises ImportError when it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise ImportError(f"libgdr.so is not built ({_LIB_PATH}); run "
+                              "`python -m gated_delta_rule_89_b200.build`")
+        L = ctypes.CDLL(_LIB_PATH)
+        P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        L.gdr_chunk_fwd.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P, Z, P]
+        L.gdr_chunk_fwd.restype = I
+        L.gdr_recurrent_step.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, P]
+        L.gdr_recurrent_step.restype = I
+        L.gdr_chunk_fwd_workspace_size.argtypes = [I, I, I, I, I, I, I, I]
+        L.gdr_chunk_fwd_workspace_size.restype = Z
+        L.gdr_status_string.argtypes = [I]
+        L.gdr_status_string.restype = ctypes.c_char_p
+        L.gdr_last_cuda_error.restype = I
+        L.gdr_last_launch_count.restype = I
+        _lib = L
+    return _lib
+
+
+def _check(status: int, what: str) -> None:
+    if status != GDR_OK:
+        L = lib()
+        name = L.gdr_status_string(status).decode()
+        extra = f" (cudaError {L.gdr_last_cuda_error()})" if name == "GDR_ERR_CUDA" else ""
+        raise GDRError(f"{what}: {name}{extra}")
+
+
+def last_launch_count() -> int:
+    """Kernels launched by this thread's last successful library call."""
+    return int(lib().gdr_last_launch_count())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(device: torch.device, stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    h = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    return ctypes.c_void_p(h)
+
+
+def _need(t: torch.Tensor, name: str, dtype=None, device=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def chunk_fwd_workspace_size(B, H, T, dk, dv, C=64, gate="per_channel", dtype=torch.bfloat16) -> int:
+    g = GATE_PER_CHANNEL if gate == "per_channel" else GATE_SCALAR
+    return int(lib().gdr_chunk_fwd_workspace_size(B, H, T, dk, dv, C, g, _DTYPES[dtype]))
+
+
+def _to_device(x, device):
+    return None if x is None else x.to(device, non_blocking=True)
+
+
+def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor, beta: torch.Tensor,
+              S0: Optional[torch.Tensor] = None, C: int = 64, gate: Optional[str] = None,
+              O: Optional[torch.Tensor] = None, S_T: Optional[torch.Tensor] = None,
+              final_state: bool = True, workspace: Optional[torch.Tensor] = None,
+              stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Chunkwise forward of the gated delta rule (``gdr_chunk_fwd``).
+
+    q, k [B,H,T,dk] and v [B,H,T,dv] (fp32 or bf16, same dtype); g fp32
+    [B,H,T,dk] (per-channel, KDA) or [B,H,T] (scalar, Gated DeltaNet);
+    beta fp32 [B,H,T]; S0 fp32 [B,H,dv,dk] or None (zeros).  Returns
+    (O [B,H,T,dv] in v's dtype, S_T [B,H,dv,dk] fp32 or None).
+    """
+    host = not q.is_cuda
+    if host:
+        dev = torch.device("cuda", torch.cuda.current_device())
+        q, k, v, g, beta, S0 = (_to_device(x, dev) for x in (q, k, v, g, beta, S0))
+    dev = q.device
+    if gate is None:
+        gate = "per_channel" if g.dim() == 4 else "scalar"
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    if dt not in _DTYPES:
+        raise TypeError("q, k, v must be float32 or bfloat16")
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, dt, dev)
+    _need(g, "g", torch.float32, dev)
+    _need(beta, "beta", torch.float32, dev)
+    if tuple(k.shape) != (B, H, T, dk) or tuple(v.shape[:3]) != (B, H, T) or tuple(beta.shape) != (B, H, T):
+        raise ValueError("inconsistent shapes")
+    if gate == "per_channel" and tuple(g.shape) != (B, H, T, dk):
+        raise ValueError("per-channel g must be [B,H,T,dk]")
+    if gate == "scalar" and tuple(g.shape) != (B, H, T):
+        raise ValueError("scalar g must be [B,H,T]")
+    if S0 is not None:
+        _need(S0, "S0", torch.float32, dev)
+        if tuple(S0.shape) != (B, H, dv, dk):
+            raise ValueError("S0 must be [B,H,dv,dk]")
+    if O is None:
+        O = torch.empty(B, H, T, dv, dtype=dt, device=dev)
+    _need(O, "O", dt, dev)
+    if S_T is None and final_state:
+        S_T = torch.empty(B, H, dv, dk, dtype=torch.float32, device=dev)
+    if S_T is not None:
+        _need(S_T, "S_T", torch.float32, dev)
+    gm = GATE_PER_CHANNEL if gate == "per_channel" else GATE_SCALAR
+    L = lib()
+    ws_bytes = int(L.gdr_chunk_fwd_workspace_size(B, H, T, dk, dv, C, gm, _DTYPES[dt]))
+    if ws_bytes and (workspace is None or workspace.numel() * workspace.element_size() < ws_bytes):
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    st = L.gdr_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(O), _ptr(S_T),
+                         B, H, T, dk, dv, C, gm, _DTYPES[dt],
+                         _ptr(workspace) if ws_bytes else None, ws_bytes, _stream_handle(dev, stream))
+    _check(st, "gdr_chunk_fwd")
+    if host:
+        O = O.to("cpu")
+        S_T = None if S_T is None else S_T.to("cpu")
+    return O, S_T
+
+
+def recurrent_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor, beta: torch.Tensor,
+                   S: torch.Tensor, o: Optional[torch.Tensor] = None, gate: Optional[str] = None,
+                   stream=None) -> torch.Tensor:
+    """One decode step (``gdr_recurrent_step``); S [B,H,dv,dk] fp32 is updated in place.
+
+    q, k [B,H,dk], v [B,H,dv] (fp32 or bf16); g fp32 [B,H,dk] (per-channel)
+    or [B,H] (scalar); beta fp32 [B,H].  Returns o [B,H,dv] in v's dtype.
+    """
+    dev = S.device
+    if gate is None:
+        gate = "per_channel" if g.dim() == 3 else "scalar"
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    if dt not in _DTYPES:
+        raise TypeError("q, k, v must be float32 or bfloat16")
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, dt, dev)
+    _need(g, "g", torch.float32, dev)
+    _need(beta, "beta", torch.float32, dev)
+    _need(S, "S", torch.float32, dev)
+    if tuple(S.shape) != (B, H, dv, dk) or tuple(beta.shape) != (B, H):
+        raise ValueError("inconsistent shapes")
+    if o is None:
+        o = torch.empty(B, H, dv, dtype=dt, device=dev)
+    _need(o, "o", dt, dev)
+    gm = GATE_PER_CHANNEL if gate == "per_channel" else GATE_SCALAR
+    st = lib().gdr_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(o),
+                                  B, H, dk, dv, gm, _DTYPES[dt], _stream_handle(dev, stream))
+    _check(st, "gdr_recurrent_step")
+    return o

@@ -1,0 +1,126 @@
+// C entry points of libgdr.so: argument validation, dispatch, status codes.
+// The declarations and the contract of every call are in include/gdr.h.
+#include <stdint.h>
+
+#include "gdr.h"
+#include "gdr_internal.cuh"
+
+#define GDR_API extern "C" __attribute__((visibility("default")))
+
+namespace {
+
+thread_local int tl_last_cuda_error = 0;
+thread_local int tl_last_launches = 0;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int finish(cudaError_t e, int launches)
+{
+    if (e != cudaSuccess) {
+        tl_last_cuda_error = (int)e;
+        return GDR_ERR_CUDA;
+    }
+    tl_last_launches = launches;
+    return GDR_OK;
+}
+
+bool size_ok(int d) { return d == 64 || d == 128; }
+
+}  // namespace
+
+GDR_API const char *gdr_status_string(int status)
+{
+    switch (status) {
+        case GDR_OK: return "GDR_OK";
+        case GDR_ERR_INVALID_ARG: return "GDR_ERR_INVALID_ARG";
+        case GDR_ERR_UNSUPPORTED: return "GDR_ERR_UNSUPPORTED";
+        case GDR_ERR_ALIGNMENT: return "GDR_ERR_ALIGNMENT";
+        case GDR_ERR_CUDA: return "GDR_ERR_CUDA";
+        case GDR_ERR_GATE_RANGE: return "GDR_ERR_GATE_RANGE";
+        case GDR_ERR_TIMEOUT: return "GDR_ERR_TIMEOUT";
+        default: return "GDR_ERR_UNKNOWN";
+    }
+}
+
+GDR_API int gdr_last_cuda_error(void) { return tl_last_cuda_error; }
+
+GDR_API int gdr_last_launch_count(void) { return tl_last_launches; }
+
+GDR_API size_t gdr_chunk_fwd_workspace_size(int B, int H, int T, int dk, int dv, int C, int gate_mode, int dtype)
+{
+    (void)B; (void)H; (void)T; (void)dk; (void)dv; (void)C; (void)gate_mode; (void)dtype;
+    return 0;
+}
+
+GDR_API int gdr_chunk_fwd(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                          const float *S0, void *O, float *S_T,
+                          int B, int H, int T, int dk, int dv, int C, int gate_mode, int dtype,
+                          void *workspace, size_t ws_bytes, void *stream)
+{
+    if (B < 0 || H < 0 || T < 0) return GDR_ERR_INVALID_ARG;
+    if (gate_mode != GDR_GATE_PER_CHANNEL && gate_mode != GDR_GATE_SCALAR) return GDR_ERR_INVALID_ARG;
+    if (dtype != GDR_F32 && dtype != GDR_BF16) return GDR_ERR_INVALID_ARG;
+    if (dk <= 0 || dv <= 0 || C <= 0) return GDR_ERR_INVALID_ARG;
+    if (!size_ok(dk) || !size_ok(dv) || !(C == 16 || C == 32 || C == 64)) return GDR_ERR_UNSUPPORTED;
+    if (ws_bytes < gdr_chunk_fwd_workspace_size(B, H, T, dk, dv, C, gate_mode, dtype)) return GDR_ERR_INVALID_ARG;
+    if ((long long)B * H * T * (dk > dv ? dk : dv) >= (1LL << 40)) return GDR_ERR_UNSUPPORTED;
+    (void)workspace;
+    const long long heads = (long long)B * H;
+    if (heads == 0) {
+        tl_last_launches = 0;
+        return GDR_OK;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (T == 0) {
+        // nothing to read or write per token; the final state is the initial one
+        if (S_T && !aligned16(S_T)) return GDR_ERR_ALIGNMENT;
+        if (S0 && !aligned16(S0)) return GDR_ERR_ALIGNMENT;
+        cudaError_t e = cudaSuccess;
+        const size_t bytes = sizeof(float) * (size_t)heads * dv * dk;
+        if (S_T && S0 && S_T != S0) e = cudaMemcpyAsync(S_T, S0, bytes, cudaMemcpyDeviceToDevice, st);
+        else if (S_T && !S0) e = cudaMemsetAsync(S_T, 0, bytes, st);
+        return finish(e, 0);
+    }
+    if (!q || !k || !v || !g || !beta || !O) return GDR_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, g, beta, S0, O, S_T};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return GDR_ERR_ALIGNMENT;
+
+    gdr::ChunkArgs a;
+    a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.S0 = S0; a.O = O; a.S_T = S_T;
+    a.B = B; a.H = H; a.T = T; a.dk = dk; a.dv = dv; a.C = C;
+    a.scalar_gate = (gate_mode == GDR_GATE_SCALAR);
+    a.bf16 = (dtype == GDR_BF16);
+    int launches = 0;
+    cudaError_t e = gdr::chunk_tc_supports(a) ? gdr::launch_chunk_tc(a, st, &launches)
+                                              : gdr::launch_chunk_simt(a, st, &launches);
+    return finish(e, launches);
+}
+
+GDR_API int gdr_recurrent_step(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                               float *S, void *o, int B, int H, int dk, int dv, int gate_mode, int dtype,
+                               void *stream)
+{
+    if (B < 0 || H < 0) return GDR_ERR_INVALID_ARG;
+    if (gate_mode != GDR_GATE_PER_CHANNEL && gate_mode != GDR_GATE_SCALAR) return GDR_ERR_INVALID_ARG;
+    if (dtype != GDR_F32 && dtype != GDR_BF16) return GDR_ERR_INVALID_ARG;
+    if (dk <= 0 || dv <= 0) return GDR_ERR_INVALID_ARG;
+    if (!size_ok(dk) || !size_ok(dv)) return GDR_ERR_UNSUPPORTED;
+    if ((long long)B * H * dv * dk >= (1LL << 40)) return GDR_ERR_UNSUPPORTED;
+    if ((long long)B * H == 0) {
+        tl_last_launches = 0;
+        return GDR_OK;
+    }
+    if (!q || !k || !v || !g || !beta || !S || !o) return GDR_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, g, beta, S, o};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return GDR_ERR_ALIGNMENT;
+    gdr::StepArgs a;
+    a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.S = S; a.o = o;
+    a.B = B; a.H = H; a.dk = dk; a.dv = dv;
+    a.scalar_gate = (gate_mode == GDR_GATE_SCALAR);
+    a.bf16 = (dtype == GDR_BF16);
+    int launches = 0;
+    cudaError_t e = gdr::launch_recurrent_step(a, static_cast<cudaStream_t>(stream), &launches);
+    return finish(e, launches);
+}

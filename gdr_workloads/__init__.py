@@ -171,6 +171,8 @@ def _g_from_recipe(w: Workload, seed: int, idx: torch.Tensor, b: torch.Tensor, h
         return -_softplus64(normal(seed, TID_G, idx) + 2.0)
     if r == "softplus_n02_clamp5":
         return torch.clamp(-_softplus64(2.0 * normal(seed, TID_G, idx)), min=-5.0)
+    if r == "softplus_n02_unbounded":   # parity cases only: some values below -5
+        return -_softplus64(2.0 * normal(seed, TID_G, idx) + 2.0)
     if r == "long_context_mix":
         u = uniform(seed, TID_G, idx)
         slow = -(0.001 + 0.049 * u)
@@ -202,7 +204,7 @@ def _chunked(n: int, block: int):
 
 
 def generate(w: Workload, device="cpu", heads: Optional[Sequence[int]] = None,
-             steps: Optional[int] = None, block: int = 1 << 24) -> Dict[str, torch.Tensor]:
+             steps: Optional[int] = None, step0: int = 0, block: int = 1 << 24) -> Dict[str, torch.Tensor]:
     """Inputs of workload ``w``.
 
     ``heads``: optional list of flat head ids (b*H + h); when given, tensors
@@ -243,7 +245,7 @@ def generate(w: Workload, device="cpu", heads: Optional[Sequence[int]] = None,
             rest = lin // per_row
             if decode:
                 hsel = rest % nh
-                t = rest // nh
+                t = rest // nh + step0
                 hid = head_ids[hsel]
                 full = (t * (B * H) + hid) * per_row + j
             else:

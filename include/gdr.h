@@ -1,0 +1,139 @@
+/*
+ * gdr.h -- C ABI of the B200 (sm_100a) gated delta rule library (libgdr.so).
+ *
+ * The method (d_v x d_k orientation, o_t = S_t q_t):
+ *
+ *     S_t = S_{t-1} Diag(alpha_t) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+ *
+ * as written in "Reading notes: Kimi Delta Attention" (mzeromiko), section 4
+ * "Forward pass" (KDA: alpha_t in (0,1)^{d_k}, one decay per key channel) and
+ * in "Token Mixer I", section "Gated Delta Networks" (Gated DeltaNet: one
+ * scalar alpha_t per head).  The gate is passed as its logarithm g = log alpha
+ * ("KDA vs Gated DeltaNet" (brenchcc), section 4: the state is multiplied by
+ * exp(decay)).  In per-channel mode the library applies the KDA lower bound
+ * g >= -5 ("Lightweight LLM reproduction: Linear Attention" (aitujian),
+ * section 3.1 [7a], g_min = -5) by computing with max(g, -5); scalar gates
+ * are used as given.
+ *
+ * Conventions shared by every call
+ *   - Every tensor pointer is a DEVICE pointer owned by the caller; the
+ *     library never allocates, frees or keeps a pointer after the call.
+ *   - Tensors are dense, row-major (last index fastest), with the shapes
+ *     given per argument below, and must be 16-byte aligned.
+ *   - dtype GDR_F32 means q, k, v and the output are float; GDR_BF16 means
+ *     they are bfloat16.  g, beta and every state tensor are always float.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream).  Argument errors are detected on the host and
+ *     returned before anything is launched; a launch failure returns
+ *     GDR_ERR_CUDA and the CUDA error code is kept for gdr_last_cuda_error().
+ *   - Outputs must not overlap inputs, except where an argument says so.
+ *   - Supported sizes: d_k, d_v in {64, 128}; chunk C in {16, 32, 64};
+ *     any T >= 0, B >= 0, H >= 0.  Other sizes return GDR_ERR_UNSUPPORTED.
+ *   - Functions return a gdr_status value as int.
+ */
+#ifndef GDR_H_
+#define GDR_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum gdr_status {
+    GDR_OK = 0,
+    GDR_ERR_INVALID_ARG = 1,  /* null pointer, negative size, bad enum, short workspace */
+    GDR_ERR_UNSUPPORTED = 2,  /* valid but unsupported size (d_k, d_v, C) */
+    GDR_ERR_ALIGNMENT = 3,    /* a tensor pointer is not 16-byte aligned */
+    GDR_ERR_CUDA = 4,         /* a CUDA call failed; see gdr_last_cuda_error() */
+    GDR_ERR_GATE_RANGE = 5,   /* reserved: gate outside its domain */
+    GDR_ERR_TIMEOUT = 6       /* reserved: a bounded device wait ran out */
+} gdr_status;
+
+typedef enum gdr_dtype { GDR_F32 = 0, GDR_BF16 = 1 } gdr_dtype;
+
+typedef enum gdr_gate_mode {
+    GDR_GATE_PER_CHANNEL = 0, /* KDA: g has one value per key channel */
+    GDR_GATE_SCALAR = 1       /* Gated DeltaNet: g has one value per head and token */
+} gdr_gate_mode;
+
+/*
+ * Bytes of device workspace gdr_chunk_fwd needs for these sizes (0 when the
+ * chosen kernels need none).  Returns 0 for unsupported arguments too; the
+ * forward call itself reports those.
+ */
+size_t gdr_chunk_fwd_workspace_size(int B, int H, int T, int dk, int dv, int C,
+                                    int gate_mode, int dtype);
+
+/*
+ * Chunkwise-parallel forward over a whole sequence.
+ *
+ * Computes, for every (b, h), O[t] = S_t q_t for t = 0..T-1 and the final
+ * state S_T, starting from S0.  The work follows the chunk form of "Reading
+ * notes: Kimi Delta Attention", section 4 (also "Token Mixer I", section
+ * "Kimi Delta Attention: Improving Delta Rule with Fine-grained Gating", the
+ * UT transform, chunk state update and chunk output equations): chunks of C
+ * tokens, a per-chunk log-gate cumulative sum, the UT transform
+ * A~ = (I + StrictTril(Diag(beta) (Gamma*K)(K/Gamma)^T))^{-1}, W = A~ Diag(beta)(Gamma*K),
+ * U = A~ Diag(beta) V, then sequentially over chunks
+ * V_new = U - W S^T,  O = (Gamma*Q) S^T + Tril((Gamma*Q)(K/Gamma)^T) V_new,
+ * S <- S Diag(gamma_C) + V_new^T (K * gamma_C/Gamma).
+ * The result equals the token recurrence above up to rounding; a last
+ * partial chunk (T not a multiple of C) is handled exactly.
+ *
+ *   q, k   [B,H,T,dk]  dtype           queries / keys (not normalised here)
+ *   v      [B,H,T,dv]  dtype           values
+ *   g      [B,H,T,dk] (per-channel) or [B,H,T] (scalar), float: log-decay
+ *   beta   [B,H,T]     float           write strength
+ *   S0     [B,H,dv,dk] float           initial state; NULL = zeros
+ *   O      [B,H,T,dv]  dtype           output (written)
+ *   S_T    [B,H,dv,dk] float           final state (written); NULL = not
+ *                                      written; may be the same pointer as
+ *                                      S0 (in-place update of the state)
+ *   C                                   chunk size (64 is the tuned size)
+ *   workspace / ws_bytes                device scratch of at least
+ *                                      gdr_chunk_fwd_workspace_size() bytes
+ *                                      (may be NULL when that is 0)
+ *   stream                              cudaStream_t
+ */
+int gdr_chunk_fwd(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                  const float *S0, void *O, float *S_T,
+                  int B, int H, int T, int dk, int dv, int C, int gate_mode, int dtype,
+                  void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * One single-token recurrent update per (b, h): the decode step.
+ *
+ * Follows the order of the pseudo-code in "KDA vs Gated DeltaNet", section 4
+ * (decay the state, predict from the decayed state, delta, write, read), in a
+ * single pass over S: S~ = S Diag(alpha); p = S~ k; delta = beta (v - p);
+ * S <- S~ + delta k^T; o = S q.
+ *
+ *   q, k   [B,H,dk]    dtype
+ *   v      [B,H,dv]    dtype
+ *   g      [B,H,dk] (per-channel) or [B,H] (scalar), float
+ *   beta   [B,H]       float
+ *   S      [B,H,dv,dk] float           state, updated IN PLACE
+ *   o      [B,H,dv]    dtype           output (written)
+ */
+int gdr_recurrent_step(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                       float *S, void *o, int B, int H, int dk, int dv, int gate_mode, int dtype,
+                       void *stream);
+
+/* Human-readable name of a status value (static string, never NULL). */
+const char *gdr_status_string(int status);
+
+/* The last cudaError_t value a call of this thread met (0 if none). */
+int gdr_last_cuda_error(void);
+
+/*
+ * Number of kernel launches the last successful call of this thread issued
+ * (lets a caller count device launches without a profiler).
+ */
+int gdr_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDR_H_ */

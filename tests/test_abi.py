@@ -1,0 +1,92 @@
+"""The C ABI library loads, exports every symbol include/gdr.h declares, and
+rejects bad arguments on the host before any device work (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gated_delta_rule_89_b200 as gdr
+from gated_delta_rule_89_b200 import build as gbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+OK, INVALID, UNSUPPORTED, ALIGN = 0, 1, 2, 3
+
+
+@pytest.fixture(scope="module")
+def L():
+    gbuild.build()
+    return gdr.lib()
+
+
+def declared_functions():
+    names = []
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if h.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", h)).read()
+            txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+            names += re.findall(r"\b(gdr_[a-z0-9_]+)\s*\(", txt)
+    return sorted(set(names))
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert "gdr_chunk_fwd" in names and "gdr_recurrent_step" in names
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings(L):
+    assert L.gdr_status_string(0) == b"GDR_OK"
+    assert L.gdr_status_string(3) == b"GDR_ERR_ALIGNMENT"
+    assert L.gdr_status_string(99) == b"GDR_ERR_UNKNOWN"
+
+
+P = ctypes.c_void_p
+GOOD = P(0x100000)      # never dereferenced: every case below fails validation first
+ODD = P(0x100008)
+
+
+def chunk(L, B=1, H=1, T=64, dk=128, dv=128, C=64, gate=0, dtype=1, ptr=GOOD, S0=None, ST=None, ws=0):
+    return L.gdr_chunk_fwd(ptr, ptr, ptr, ptr, ptr, S0, ptr, ST, B, H, T, dk, dv, C, gate, dtype, None, ws, None)
+
+
+def test_chunk_argument_validation(L):
+    assert chunk(L, B=-1) == INVALID
+    assert chunk(L, T=-3) == INVALID
+    assert chunk(L, gate=2) == INVALID
+    assert chunk(L, dtype=5) == INVALID
+    assert chunk(L, dk=0) == INVALID
+    assert chunk(L, dk=96) == UNSUPPORTED
+    assert chunk(L, dv=256) == UNSUPPORTED
+    assert chunk(L, C=48) == UNSUPPORTED
+    assert chunk(L, ptr=ODD) == ALIGN
+    assert chunk(L, ptr=None) == INVALID
+    assert chunk(L, ST=ODD) == ALIGN
+    # empty problems succeed without touching the device
+    assert chunk(L, B=0) == OK and L.gdr_last_launch_count() == 0
+    assert chunk(L, H=0) == OK
+    assert chunk(L, T=0) == OK          # no S_T requested: nothing to do
+
+
+def test_step_argument_validation(L):
+    def step(B=2, H=2, dk=128, dv=128, gate=0, dtype=1, ptr=GOOD):
+        return L.gdr_recurrent_step(ptr, ptr, ptr, ptr, ptr, ptr, ptr, B, H, dk, dv, gate, dtype, None)
+    assert step(B=-1) == INVALID
+    assert step(gate=7) == INVALID
+    assert step(dk=32) == UNSUPPORTED
+    assert step(ptr=ODD) == ALIGN
+    assert step(ptr=None) == INVALID
+    assert step(B=0) == OK
+
+
+def test_workspace_query(L):
+    assert L.gdr_chunk_fwd_workspace_size(2, 32, 8192, 128, 128, 64, 0, 1) >= 0
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(gdr, "_lib", None)
+    monkeypatch.setattr(gdr, "_LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(ImportError):
+        gdr.lib()

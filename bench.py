@@ -199,45 +199,62 @@ def gpu_id_for(device) -> str:
 def oracle_sample(w: W.Workload, budget_s: float, seed_rank: int = 0):
     """Time the fp64 oracle on a bounded sample of workload ``w``.
 
-    The sample is ``heads`` whole heads (as many as host threads, at most all
-    of them) over the first ``tokens`` tokens (or decode steps), sized from a
-    short calibration run to take about ``budget_s`` seconds.  Returns
-    (tokens/s in the workload's unit, description dict).
+    The sample is whole heads (spread over the batch) over the first
+    ``tokens`` tokens (or decode steps), sized from a short calibration run to
+    take about ``budget_s`` seconds; when the whole workload takes less than
+    that, the whole workload is run, repeatedly, until the budget is used.
+    Returns (tokens/s in the workload's unit, description dict).
     """
     import oracle
     cores = oracle.online_cores()
     heads_total = w.B * w.H
-    heads = min(heads_total, cores)
-    hl = list(range(0, heads_total, max(1, heads_total // heads)))[:heads]
 
-    def run(ntok):
+    def pick(nh):
+        step = max(1, heads_total // nh)
+        return list(range(0, heads_total, step))[:nh]
+
+    def run(hl, ntok):
         if w.kind == "decode":
             x = W.generate(w, heads=hl, steps=ntok)
             t = time.perf_counter()
             oracle.decode(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], gate=w.gate, threads=cores)
             return time.perf_counter() - t
         x = W.generate(w, heads=hl)
-        sl = lambda a: a[:, :, :ntok]
+        sl = lambda a: a[:, :, :ntok].contiguous()
+        args = [sl(x[k]) for k in ("q", "k", "v", "g", "beta")]
         t = time.perf_counter()
-        oracle.forward(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["g"]), sl(x["beta"]), x["S0"],
-                       gate=w.gate, threads=cores)
+        oracle.forward(*args, x["S0"], gate=w.gate, threads=cores)
         return time.perf_counter() - t
 
-    cal_tok = min(w.T, 64)
-    t_cal = run(cal_tok)
-    per_tok = t_cal / cal_tok
-    ntok = int(max(cal_tok, min(w.T, budget_s / max(per_tok, 1e-9))))
-    if ntok != cal_tok:
-        dt = run(ntok)
+    # calibrate on one head per core
+    hl = pick(min(heads_total, cores))
+    cal_tok = min(w.T, 256)
+    per_head_tok = run(hl, cal_tok) / (len(hl) * cal_tok) * min(len(hl), cores)
+    full_est = per_head_tok * heads_total * w.T / min(heads_total, cores)
+    if full_est <= budget_s:
+        hl, ntok = pick(heads_total), w.T
     else:
-        dt = t_cal
+        ntok = w.T
+        nh = int(budget_s / (per_head_tok * ntok) * min(heads_total, cores))
+        if nh < min(heads_total, cores):
+            nh = min(heads_total, cores)
+            ntok = max(cal_tok, int(budget_s / (per_head_tok * ntok) * ntok))
+        hl = pick(max(1, min(heads_total, nh)))
+    times = []
+    t_all = time.perf_counter()
+    while True:
+        times.append(run(hl, ntok))
+        if time.perf_counter() - t_all >= budget_s or len(times) >= 50:
+            break
+    dt = statistics.median(times)
     head_tokens_per_s = len(hl) * ntok / dt
     # a workload token (one position of one sequence) spans all H heads
     tokens_per_s = head_tokens_per_s / w.H
     unit_note = "decode steps" if w.kind == "decode" else "tokens"
     return tokens_per_s, {"kind": "oracle", "cores": min(cores, len(hl)),
                           "sample": f"fp64 oracle on {len(hl)} of {heads_total} heads x {ntok} {unit_note} "
-                                    f"of {w.name} ({dt:.1f} s)", "seconds": round(dt, 2)}
+                                    f"of {w.name}, median of {len(times)} runs ({sum(times):.1f} s total)",
+                          "seconds": round(sum(times), 2)}
 
 
 # ------------------------------------------------------------------ main

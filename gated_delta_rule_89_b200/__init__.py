@@ -20,7 +20,7 @@ from typing import Optional, Tuple
 import torch
 
 __all__ = ["chunk_fwd", "recurrent_step", "chunk_fwd_workspace_size", "GDRError", "library_path",
-           "last_launch_count", "GATE_PER_CHANNEL", "GATE_SCALAR"]
+           "last_launch_count", "device_status", "GATE_PER_CHANNEL", "GATE_SCALAR"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libgdr.so")
@@ -59,6 +59,8 @@ def lib() -> ctypes.CDLL:
         L.gdr_status_string.restype = ctypes.c_char_p
         L.gdr_last_cuda_error.restype = I
         L.gdr_last_launch_count.restype = I
+        L.gdr_device_status.argtypes = [P]
+        L.gdr_device_status.restype = I
         _lib = L
     return _lib
 
@@ -74,6 +76,13 @@ def _check(status: int, what: str) -> None:
 def last_launch_count() -> int:
     """Kernels launched by this thread's last successful library call."""
     return int(lib().gdr_last_launch_count())
+
+
+def device_status(device=None, stream=None) -> int:
+    """Synchronize the stream and return (and clear) the library's device
+    status word: 0 unless a kernel ran out of a bounded wait (GDR_ERR_TIMEOUT)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    return int(lib().gdr_device_status(_stream_handle(dev, stream)))
 
 
 def _ptr(t: Optional[torch.Tensor]):

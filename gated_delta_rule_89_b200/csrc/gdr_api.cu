@@ -48,8 +48,24 @@ GDR_API int gdr_last_launch_count(void) { return tl_last_launches; }
 
 GDR_API size_t gdr_chunk_fwd_workspace_size(int B, int H, int T, int dk, int dv, int C, int gate_mode, int dtype)
 {
-    (void)B; (void)H; (void)T; (void)dk; (void)dv; (void)C; (void)gate_mode; (void)dtype;
-    return 0;
+    if (B <= 0 || H <= 0 || T <= 0) return 0;
+    if (gate_mode != GDR_GATE_PER_CHANNEL && gate_mode != GDR_GATE_SCALAR) return 0;
+    gdr::ChunkArgs a = {};
+    a.B = B; a.H = H; a.T = T; a.dk = dk; a.dv = dv; a.C = C;
+    a.scalar_gate = (gate_mode == GDR_GATE_SCALAR);
+    a.bf16 = (dtype == GDR_BF16);
+    return gdr::chunk_tc_supports(a) ? gdr::chunk_tc_workspace_bytes(B, H, T) : 0;
+}
+
+GDR_API int gdr_device_status(void *stream)
+{
+    int v = 0;
+    cudaError_t e = gdr::read_device_status(static_cast<cudaStream_t>(stream), &v);
+    if (e != cudaSuccess) {
+        tl_last_cuda_error = (int)e;
+        return GDR_ERR_CUDA;
+    }
+    return v;
 }
 
 GDR_API int gdr_chunk_fwd(const void *q, const void *k, const void *v, const float *g, const float *beta,
@@ -62,9 +78,9 @@ GDR_API int gdr_chunk_fwd(const void *q, const void *k, const void *v, const flo
     if (dtype != GDR_F32 && dtype != GDR_BF16) return GDR_ERR_INVALID_ARG;
     if (dk <= 0 || dv <= 0 || C <= 0) return GDR_ERR_INVALID_ARG;
     if (!size_ok(dk) || !size_ok(dv) || !(C == 16 || C == 32 || C == 64)) return GDR_ERR_UNSUPPORTED;
-    if (ws_bytes < gdr_chunk_fwd_workspace_size(B, H, T, dk, dv, C, gate_mode, dtype)) return GDR_ERR_INVALID_ARG;
     if ((long long)B * H * T * (dk > dv ? dk : dv) >= (1LL << 40)) return GDR_ERR_UNSUPPORTED;
-    (void)workspace;
+    const size_t ws_need = gdr_chunk_fwd_workspace_size(B, H, T, dk, dv, C, gate_mode, dtype);
+    if (ws_bytes < ws_need || (ws_need && !workspace)) return GDR_ERR_INVALID_ARG;
     const long long heads = (long long)B * H;
     if (heads == 0) {
         tl_last_launches = 0;
@@ -82,7 +98,7 @@ GDR_API int gdr_chunk_fwd(const void *q, const void *k, const void *v, const flo
         return finish(e, 0);
     }
     if (!q || !k || !v || !g || !beta || !O) return GDR_ERR_INVALID_ARG;
-    const void *ptrs[] = {q, k, v, g, beta, S0, O, S_T};
+    const void *ptrs[] = {q, k, v, g, beta, S0, O, S_T, workspace};
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return GDR_ERR_ALIGNMENT;
 
@@ -91,6 +107,7 @@ GDR_API int gdr_chunk_fwd(const void *q, const void *k, const void *v, const flo
     a.B = B; a.H = H; a.T = T; a.dk = dk; a.dv = dv; a.C = C;
     a.scalar_gate = (gate_mode == GDR_GATE_SCALAR);
     a.bf16 = (dtype == GDR_BF16);
+    a.workspace = workspace;
     int launches = 0;
     cudaError_t e = gdr::chunk_tc_supports(a) ? gdr::launch_chunk_tc(a, st, &launches)
                                               : gdr::launch_chunk_simt(a, st, &launches);

@@ -16,6 +16,7 @@ struct ChunkArgs {
     int B, H, T, dk, dv, C;
     bool scalar_gate;
     bool bf16;
+    void *workspace;   // device scratch of chunk_tc_workspace_bytes() bytes (tensor-core path)
 };
 
 // Arguments of one decode step, already validated.
@@ -35,6 +36,9 @@ cudaError_t launch_recurrent_step(const StepArgs &a, cudaStream_t stream, int *l
 cudaError_t launch_chunk_simt(const ChunkArgs &a, cudaStream_t stream, int *launches);
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream, int *launches);
 bool chunk_tc_supports(const ChunkArgs &a);
+size_t chunk_tc_workspace_bytes(int B, int H, int T);
+// Synchronizes `stream`, then reads and clears the device status word.
+cudaError_t read_device_status(cudaStream_t stream, int *status);
 
 // The KDA lower bound on the per-channel log-decay.
 constexpr float kGateMin = -5.0f;

@@ -120,6 +120,16 @@ int gdr_recurrent_step(const void *q, const void *k, const void *v, const float 
                        float *S, void *o, int B, int H, int dk, int dv, int gate_mode, int dtype,
                        void *stream);
 
+/*
+ * Device-side status.  Kernels that wait on other warps of their own block
+ * bound every wait (about a second); when one runs out the kernel records
+ * GDR_ERR_TIMEOUT in a device status word, stops, and leaves its outputs
+ * undefined.  This call synchronizes `stream`, returns that word (GDR_OK if
+ * no kernel recorded anything since the last call) and clears it.  It may
+ * return GDR_ERR_CUDA if the synchronization itself fails.
+ */
+int gdr_device_status(void *stream);
+
 /* Human-readable name of a status value (static string, never NULL). */
 const char *gdr_status_string(int status);
 

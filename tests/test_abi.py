@@ -48,8 +48,9 @@ GOOD = P(0x100000)      # never dereferenced: every case below fails validation 
 ODD = P(0x100008)
 
 
-def chunk(L, B=1, H=1, T=64, dk=128, dv=128, C=64, gate=0, dtype=1, ptr=GOOD, S0=None, ST=None, ws=0):
-    return L.gdr_chunk_fwd(ptr, ptr, ptr, ptr, ptr, S0, ptr, ST, B, H, T, dk, dv, C, gate, dtype, None, ws, None)
+def chunk(L, B=1, H=1, T=64, dk=128, dv=128, C=64, gate=0, dtype=1, ptr=GOOD, S0=None, ST=None,
+          ws=1 << 40, wsp=GOOD):
+    return L.gdr_chunk_fwd(ptr, ptr, ptr, ptr, ptr, S0, ptr, ST, B, H, T, dk, dv, C, gate, dtype, wsp, ws, None)
 
 
 def test_chunk_argument_validation(L):
@@ -64,6 +65,12 @@ def test_chunk_argument_validation(L):
     assert chunk(L, ptr=ODD) == ALIGN
     assert chunk(L, ptr=None) == INVALID
     assert chunk(L, ST=ODD) == ALIGN
+    assert chunk(L, wsp=ODD) == ALIGN
+    # the tensor-core path needs its workspace; a short or missing one is refused
+    need = L.gdr_chunk_fwd_workspace_size(1, 1, 64, 128, 128, 64, 0, 1)
+    assert need > 0
+    assert chunk(L, ws=need - 1) == INVALID
+    assert chunk(L, wsp=None) == INVALID
     # empty problems succeed without touching the device
     assert chunk(L, B=0) == OK and L.gdr_last_launch_count() == 0
     assert chunk(L, H=0) == OK
@@ -82,7 +89,12 @@ def test_step_argument_validation(L):
 
 
 def test_workspace_query(L):
-    assert L.gdr_chunk_fwd_workspace_size(2, 32, 8192, 128, 128, 64, 0, 1) >= 0
+    # bf16, d = 128, C = 64: T' and Aqk, 2 x 64 x 64 bf16 per chunk
+    assert L.gdr_chunk_fwd_workspace_size(2, 32, 8192, 128, 128, 64, 0, 1) == 2 * 2 * 32 * 128 * 64 * 64 * 2
+    assert L.gdr_chunk_fwd_workspace_size(1, 1, 65, 128, 128, 64, 1, 1) == 2 * 2 * 64 * 64 * 2
+    # fp32 inputs or other sizes run on the CUDA-core path, which needs none
+    assert L.gdr_chunk_fwd_workspace_size(1, 2, 256, 64, 64, 64, 0, 0) == 0
+    assert L.gdr_chunk_fwd_workspace_size(1, 2, 256, 128, 128, 32, 0, 1) == 0
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):

@@ -47,6 +47,7 @@ def check_chunk(w, C=None, S0_none=False):
                          C=C or w.C, gate=w.gate)
     torch.cuda.synchronize()
     assert gdr.last_launch_count() >= 1
+    assert gdr.device_status() == 0
     eo, es = relerr(O, O_ref), relerr(S, S_ref)
     tol = TOL[w.dtype]
     assert eo <= tol and es <= tol, (w.name, eo, es)
@@ -150,6 +151,7 @@ def test_full_size_sampled(name, heads):
     d = W.generate(w, device="cuda")
     O, S = gdr.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], C=w.C, gate=w.gate)
     torch.cuda.synchronize()
+    assert gdr.device_status() == 0
     assert bool(torch.isfinite(O).all()) and bool(torch.isfinite(S).all())
     H = w.H
     sel = lambda t: torch.stack([t[h // H, h % H] for h in heads])[:, None].cpu()

@@ -137,7 +137,7 @@ _REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_pow
 class ClockSampler:
     """nvidia-smi samples (SM clock, max clock, throttle reasons) in the background."""
 
-    def __init__(self, gpu_id: str, period_ms: int = 50):
+    def __init__(self, gpu_id: str, period_ms: int = 20):
         self.samples = []
         self.proc = None
         fields = "timestamp,clocks.sm,clocks.max.sm,power.draw," + ",".join(
@@ -162,6 +162,12 @@ class ClockSampler:
                                      [r for r, v in zip(_REASONS, parts[4:]) if v.lower() == "active"]))
             except ValueError:
                 pass
+
+    def wait_first(self, timeout_s: float = 5.0):
+        """Block until the sampler has produced a sample (so the timed region is covered)."""
+        t0 = time.time()
+        while self.proc is not None and not self.samples and time.time() - t0 < timeout_s:
+            time.sleep(0.01)
 
     def stop(self):
         if self.proc is not None:
@@ -357,6 +363,8 @@ def main():
     torch.cuda.synchronize(device)
 
     sampler = ClockSampler(gpu_id_for(device)) if rank == 0 else None
+    if sampler is not None:
+        sampler.wait_first()
     for _ in range(args.warmup):
         step()
     launches_per_step = gdr.last_launch_count() * (w.T if w.kind == "decode" else 1)

@@ -66,16 +66,17 @@ constexpr uint32_t OFF_KT = OFF_AQ + 2 * 8192;     // K_tail (2 panels)         
 constexpr uint32_t OFF_W = OFF_KT + 16384;         // W (2 panels x 8 KB)               16 KB
 constexpr uint32_t OFF_S = OFF_W + 16384;          // bf16 S (2 panels x 16 KB)         32 KB
 constexpr uint32_t OFF_VN = OFF_S + 32768;         // V_new^T (1 panel, 128 rows)       16 KB
-constexpr uint32_t OFF_GAM = OFF_VN + 16384;       // gamma_C [2][128] fp32             1 KB
-constexpr uint32_t OFF_BAR = OFF_GAM + 1024;       // mbarriers, TMEM slot, abort flag
+constexpr uint32_t OFF_GAM = OFF_VN + 16384;       // gamma_C ring [4][128] fp32        2 KB
+constexpr uint32_t OFF_BAR = OFF_GAM + 2048;       // mbarriers, TMEM slot, abort flag
 constexpr uint32_t SMEM_USED = OFF_BAR + 512;
 constexpr uint32_t SMEM_ALLOC = SMEM_USED + 1024;  // alignment slack
 
 // TMEM columns (fp32)
-constexpr uint32_t TM_S = 0;      // state, 128 columns
-constexpr uint32_t TM_W = 128;    // W^T, 64 columns
-constexpr uint32_t TM_V = 192;    // V_new^T accumulators, 2 x 64 columns
-constexpr uint32_t TM_O = 320;    // O^T accumulators, 2 x 64 columns
+constexpr uint32_t TM_S = 0;      // state S_n, 128 columns (written only by the conversion warps)
+constexpr uint32_t TM_D = 128;    // state increment V_new^T K_tail of the last chunk, 128 columns
+constexpr uint32_t TM_W = 256;    // W^T, 64 columns
+constexpr uint32_t TM_V = 320;    // V_new^T accumulator, 64 columns
+constexpr uint32_t TM_O = 384;    // O^T accumulators, 2 x 64 columns
 constexpr uint32_t TM_COLS = 512;
 
 enum Bar {
@@ -87,7 +88,7 @@ enum Bar {
     B_KQ_READY, B_KQ_READY1, B_KT_READY, B_KT_FREE,
     B_WT_FULL, B_WT_EMPTY, B_W_READY, B_W_FREE,
     B_S_READY, B_S_FULL, B_X_FULL, B_VN_READY,
-    B_VACC_EMPTY, B_VACC_EMPTY1, B_O_FULL, B_O_FULL1, B_OACC_EMPTY, B_OACC_EMPTY1,
+    B_VACC_EMPTY, B_O_FULL, B_O_FULL1, B_OACC_EMPTY, B_OACC_EMPTY1,
     B_FINAL,
     B_COUNT
 };
@@ -98,6 +99,19 @@ struct Maps {
 };
 
 __device__ __forceinline__ void record_error(int code) { atomicCAS(&g_device_status, 0, code); }
+
+// Optional phase timestamps of block 0 (SM clock), compiled only with -DGDR_TRACE.
+#ifdef GDR_TRACE
+__device__ long long g_trace[16][1024];
+#define GDR_TRACE_AT(ev, n)                                                   \
+    do {                                                                      \
+        if (blockIdx.x == 0 && (n) < 1024) g_trace[(ev)][(n)] = clock64();    \
+    } while (0)
+#else
+#define GDR_TRACE_AT(ev, n) \
+    do {                    \
+    } while (0)
+#endif
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
 {
@@ -134,7 +148,7 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
             128, 128, 128, 1,   // kq ready (E) x2, kt ready (E), kt free (MMA)
             1, 128, 128, 1,     // wt full (MMA), wt empty (M), w ready (M), w free (MMA)
             128, 1, 1, 128,     // s ready (M), s full (MMA), x full (MMA), vn ready (M)
-            128, 128, 1, 1, 128, 128,   // vacc empty (M) x2, o full (MMA) x2, oacc empty (E) x2
+            128, 1, 1, 128, 128,        // vacc empty (M), o full (MMA) x2, oacc empty (E) x2
             1};
         for (int i = 0; i < B_COUNT; ++i) mbar_init(&bar[i], counts[i]);
         *abort_flag = 0;
@@ -150,12 +164,23 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
     const uint32_t tmem = *tmem_slot;
     const uint32_t sbase = smem_u32(sm);
 
+    // Single-thread roles (TMA producer, MMA issuer) wait with `wait`.
     auto wait = [&](int b, uint32_t parity) -> bool {
         if (*abort_flag) return false;
         if (mbar_wait(&bar[b], parity, kWaitBudget)) return true;
         record_error(6 /* GDR_ERR_TIMEOUT */);
         *abort_flag = 1;
         return false;
+    };
+    // Warp-wide roles wait with `waitw`: every lane acquires the barrier
+    // phase, the result is made warp-uniform, and the warp reconverges -- the
+    // tcgen05.ld/st that follow are .sync.aligned and need all 32 lanes
+    // converged (lanes leave a spin loop at different times).
+    auto waitw = [&](int b, uint32_t parity) -> bool {
+        bool ok = wait(b, parity);
+        ok = __all_sync(0xffffffffu, ok);
+        __syncwarp();
+        return ok;
     };
 
     if (warp == 0) {
@@ -191,6 +216,7 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
                 if (!wait(B_EMPTY_AQ + b, upar ^ 1)) break;
                 mbar_arrive_expect_tx(&bar[B_FULL_AQ + b], 8192);
                 tma_load_2d(sm + OFF_AQ + b * 8192, &maps.aq, &bar[B_FULL_AQ + b], 0, crow);
+                GDR_TRACE_AT(0, n);
                 issued = n + 1;
             }
             if (*abort_flag && issued > 0) {
@@ -218,9 +244,10 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
                 const uint32_t par = (uint32_t)(n & 1), upar = (uint32_t)((n >> 1) & 1);
                 // ---- W^T = K<-^T T'^T ; U^T = V^T T'^T
                 if (!wait(B_KQ_READY + b, upar) || !wait(B_FULL_T, par) || !wait(B_FULL_V, par) ||
-                    !wait(B_WT_EMPTY, par ^ 1) || !wait(B_VACC_EMPTY + b, upar ^ 1))
+                    !wait(B_WT_EMPTY, par ^ 1) || !wait(B_VACC_EMPTY, par ^ 1))
                     break;
                 tc_fence_after();
+                GDR_TRACE_AT(1, n);
                 const uint32_t kb = sbase + OFF_K + b * 16384;
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
@@ -228,7 +255,7 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
                              sdesc_sw128(sbase + OFF_T + s * 32, 16, 1024), ID_WU, s > 0);
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
-                    mma_bf16(tmem + TM_V + 64 * b, sdesc_sw128(sbase + OFF_V + s * 2048, 8192, 1024),
+                    mma_bf16(tmem + TM_V, sdesc_sw128(sbase + OFF_V + s * 2048, 8192, 1024),
                              sdesc_sw128(sbase + OFF_T + s * 32, 16, 1024), ID_WU, s > 0);
                 mma_commit(&bar[B_WT_FULL]);
                 mma_commit(&bar[B_EMPTY_K + b]);
@@ -237,10 +264,11 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
                 // ---- V_new^T += -S W^T ; O^T = S Q<-^T
                 if (!wait(B_S_READY, par) || !wait(B_W_READY, par) || !wait(B_OACC_EMPTY + b, upar ^ 1)) break;
                 tc_fence_after();
+                GDR_TRACE_AT(2, n);
                 const uint32_t qb = sbase + OFF_Q + b * 16384;
 #pragma unroll
                 for (int s = 0; s < 8; ++s)
-                    mma_bf16(tmem + TM_V + 64 * b, sdesc_sw128(sbase + OFF_S + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024),
+                    mma_bf16(tmem + TM_V, sdesc_sw128(sbase + OFF_S + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024),
                              sdesc_sw128(sbase + OFF_W + (s >> 2) * 8192 + (s & 3) * 32, 16, 1024), ID_X, 1);
 #pragma unroll
                 for (int s = 0; s < 8; ++s)
@@ -252,14 +280,15 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
                 // ---- O^T += V_new^T Aqk^T ; S += V_new^T K_tail
                 if (!wait(B_VN_READY, par) || !wait(B_FULL_AQ + b, upar) || !wait(B_KT_READY, par)) break;
                 tc_fence_after();
+                GDR_TRACE_AT(3, n);
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
                     mma_bf16(tmem + TM_O + 64 * b, sdesc_sw128(sbase + OFF_VN + s * 32, 16, 1024),
                              sdesc_sw128(sbase + OFF_AQ + b * 8192 + s * 32, 16, 1024), ID_O, 1);
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
-                    mma_bf16(tmem + TM_S, sdesc_sw128(sbase + OFF_VN + s * 32, 16, 1024),
-                             sdesc_sw128(sbase + OFF_KT + s * 2048, 8192, 1024), ID_S, 1);
+                    mma_bf16(tmem + TM_D, sdesc_sw128(sbase + OFF_VN + s * 32, 16, 1024),
+                             sdesc_sw128(sbase + OFF_KT + s * 2048, 8192, 1024), ID_S, s > 0);
                 mma_commit(&bar[B_O_FULL + b]);
                 mma_commit(&bar[B_S_FULL]);
                 mma_commit(&bar[B_EMPTY_AQ + b]);
@@ -276,13 +305,14 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
         const int orow = (int)lq + lane;             // d_v index for the epilogue
         auto epilogue = [&](int m) -> bool {
             const int bb = m & 1;
-            if (!wait(B_O_FULL + bb, (uint32_t)((m >> 1) & 1))) return false;
+            if (!waitw(B_O_FULL + bb, (uint32_t)((m >> 1) & 1))) return false;
             tc_fence_after();
             const int nvalid = min(kC, T_len - m * kC);
             __nv_bfloat16 *orow_ptr = O + (tok0 + (size_t)m * kC) * kD + orow;
 #pragma unroll
             for (int cb = 0; cb < 4; ++cb) {
                 uint32_t r[16];
+                __syncwarp();   // the bounded stores below diverge the warp; tcgen05.ld needs it converged
                 tmem_ld16(tmem + (lq << 16) + TM_O + 64 * bb + 16 * cb, r);
                 tmem_ld_wait(r);
 #pragma unroll
@@ -300,13 +330,18 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
             const int b = n & 1;
             const uint32_t par = (uint32_t)(n & 1), upar = (uint32_t)((n >> 1) & 1);
             const int t0 = n * kC;
-            if (!SCALAR && !wait(B_FULL_G, par)) break;
-            if (!wait(B_FULL_K + b, upar) || !wait(B_FULL_Q + b, upar)) break;
+            if (!SCALAR && !waitw(B_FULL_G, par)) break;
+            if (!waitw(B_FULL_K + b, upar) || !waitw(B_FULL_Q + b, upar)) break;
+            if (tid == 64) GDR_TRACE_AT(4, n);
             float al[kC];
             if (!SCALAR) {
                 const float *gt = reinterpret_cast<const float *>(sm + OFF_G);
 #pragma unroll
                 for (int r = 0; r < kC; ++r) al[r] = __expf(fmaxf(gt[r * kD + c], kGateMin));
+                // The next TMA load overwrites this tile as soon as the barrier
+                // completes; an arrive does not wait for this thread's shared
+                // loads, so order them before the async-proxy write first.
+                fence_async_smem();
                 mbar_arrive(&bar[B_EMPTY_G]);
             } else {
 #pragma unroll
@@ -330,11 +365,13 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
                 *kk = __float2bfloat16_rn(kv * p);
                 *qq = __float2bfloat16_rn(qv * p);
             }
-            gam[b * kD + c] = p;
+            gam[(n & 3) * kD + c] = p;
             fence_async_smem();
             mbar_arrive(&bar[B_KQ_READY + b]);
+            if (tid == 64) GDR_TRACE_AT(5, n);
             // K_tail = k * exp(G_C - G): reverse running product
-            if (!wait(B_KT_FREE, par ^ 1)) break;
+            if (!waitw(B_KT_FREE, par ^ 1)) break;
+            if (tid == 64) GDR_TRACE_AT(6, n);
             unsigned char *ktp = sm + OFF_KT + (c >> 6) * 8192;
             p = 1.f;
 #pragma unroll
@@ -346,11 +383,17 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
             }
             fence_async_smem();
             mbar_arrive(&bar[B_KT_READY]);
+            if (tid == 64) GDR_TRACE_AT(7, n);
             if (n > 0) ok = epilogue(n - 1);
+            if (tid == 64 && n > 0) GDR_TRACE_AT(8, n - 1);
         }
         if (ok && !*abort_flag && nchunks > 0) epilogue(nchunks - 1);
     } else {
         // ================================================================ M: sequential-path conversions
+        // The state S_n lives at TM_S and is written only here.  At chunk n
+        // (n > 0) this group forms S_n = S_{n-1} * gamma_{n-1} + dS_{n-1}, with
+        // dS_{n-1} = V_new^T K_tail of chunk n-1 taken from TM_D, stores it
+        // back, and writes its bf16 copy for the MMAs of chunk n.
         const uint32_t lq = 32u * (warp & 3);
         const int i = (int)lq + lane;                // TMEM lane: row of S / V_new^T, key channel of W^T
         const uint32_t trow = tmem + (lq << 16);
@@ -364,13 +407,47 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
             tmem_st16(trow + TM_S + 16 * cb, r);
         }
         tmem_st_wait();
+        // S_{n} = S_{n-1} * gamma_{n-1} + dS_{n-1}, in TMEM and (optionally) as bf16 in smem
+        auto advance_state = [&](int n, bool to_smem) {
+            const float *gm = gam + ((n - 1) & 3) * kD;
+#pragma unroll 2
+            for (int cb = 0; cb < 8; ++cb) {
+                uint32_t r[16], dr[16];
+                tmem_ld16(trow + TM_S + 16 * cb, r);
+                tmem_ld16(trow + TM_D + 16 * cb, dr);
+                tmem_ld_wait(r);
+                reg_touch(dr);
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                    r[j] = __float_as_uint(fmaf(__uint_as_float(r[j]), gm[16 * cb + j], __uint_as_float(dr[j])));
+                tmem_st16(trow + TM_S + 16 * cb, r);
+                if (to_smem) {
+                    unsigned char *sp = sm + OFF_S + (cb >> 2) * 16384;
+                    uint4 lo, hi;
+                    lo.x = pack_bf16(__uint_as_float(r[0]), __uint_as_float(r[1]));
+                    lo.y = pack_bf16(__uint_as_float(r[2]), __uint_as_float(r[3]));
+                    lo.z = pack_bf16(__uint_as_float(r[4]), __uint_as_float(r[5]));
+                    lo.w = pack_bf16(__uint_as_float(r[6]), __uint_as_float(r[7]));
+                    hi.x = pack_bf16(__uint_as_float(r[8]), __uint_as_float(r[9]));
+                    hi.y = pack_bf16(__uint_as_float(r[10]), __uint_as_float(r[11]));
+                    hi.z = pack_bf16(__uint_as_float(r[12]), __uint_as_float(r[13]));
+                    hi.w = pack_bf16(__uint_as_float(r[14]), __uint_as_float(r[15]));
+                    *reinterpret_cast<uint4 *>(sp + sw128_off(i, (16 * cb) & 63)) = lo;
+                    *reinterpret_cast<uint4 *>(sp + sw128_off(i, ((16 * cb) & 63) + 8)) = hi;
+                }
+            }
+            tmem_st_wait();
+        };
         bool ok = true;
         for (int n = 0; n < nchunks; ++n) {
-            const int b = n & 1;
             const uint32_t par = (uint32_t)(n & 1);
             // ---- W^T -> W (bf16, K-major [64 tokens x 128 channels])
-            if (!wait(B_WT_FULL, par) || !wait(B_W_FREE, par ^ 1)) { ok = false; break; }
+            // KQ_READY(n) has completed (W^T(n) needed it); waiting on it here only
+            // acquires gamma_C(n), which the next chunk boundary reads.
+            if (!waitw(B_WT_FULL, par) || !waitw(B_W_FREE, par ^ 1) ||
+                !waitw(B_KQ_READY + (n & 1), (uint32_t)((n >> 1) & 1))) { ok = false; break; }
             tc_fence_after();
+            if (tid == 192) GDR_TRACE_AT(9, n);
             {
                 unsigned char *wp = sm + OFF_W + (i >> 6) * 8192;
                 const uint32_t cc = (uint32_t)(i & 63);
@@ -389,12 +466,15 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
             tc_fence_before();
             mbar_arrive(&bar[B_W_READY]);
             mbar_arrive(&bar[B_WT_EMPTY]);
-            // ---- S -> bf16 smem, S * gamma_C -> TMEM
-            if (n > 0 && !wait(B_S_FULL, par ^ 1)) { ok = false; break; }
-            if (!wait(B_KQ_READY + b, (uint32_t)((n >> 1) & 1))) { ok = false; break; }
-            tc_fence_after();
-            {
-                const float *gm = gam + b * kD;
+            if (tid == 192) GDR_TRACE_AT(10, n);
+            // ---- state of this chunk -> bf16 smem
+            if (n > 0) {
+                if (!waitw(B_S_FULL, par ^ 1)) { ok = false; break; }
+                tc_fence_after();
+                if (tid == 192) GDR_TRACE_AT(11, n);
+                advance_state(n, true);
+            } else {
+                if (tid == 192) GDR_TRACE_AT(11, n);
 #pragma unroll
                 for (int cb = 0; cb < 8; ++cb) {
                     uint32_t r[16];
@@ -412,22 +492,20 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
                     hi.w = pack_bf16(__uint_as_float(r[14]), __uint_as_float(r[15]));
                     *reinterpret_cast<uint4 *>(sp + sw128_off(i, (16 * cb) & 63)) = lo;
                     *reinterpret_cast<uint4 *>(sp + sw128_off(i, ((16 * cb) & 63) + 8)) = hi;
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * gm[16 * cb + j]);
-                    tmem_st16(trow + TM_S + 16 * cb, r);
                 }
-                tmem_st_wait();
             }
             fence_async_smem();
             tc_fence_before();
             mbar_arrive(&bar[B_S_READY]);
+            if (tid == 192) GDR_TRACE_AT(12, n);
             // ---- V_new^T (TMEM) -> bf16 smem
-            if (!wait(B_X_FULL, par)) { ok = false; break; }
+            if (!waitw(B_X_FULL, par)) { ok = false; break; }
             tc_fence_after();
+            if (tid == 192) GDR_TRACE_AT(13, n);
 #pragma unroll
             for (int cb = 0; cb < 4; ++cb) {
                 uint32_t r[16];
-                tmem_ld16(trow + TM_V + 64 * b + 16 * cb, r);
+                tmem_ld16(trow + TM_V + 16 * cb, r);
                 tmem_ld_wait(r);
                 uint4 lo, hi;
                 lo.x = pack_bf16(__uint_as_float(r[0]), __uint_as_float(r[1]));
@@ -444,11 +522,13 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
             fence_async_smem();
             tc_fence_before();
             mbar_arrive(&bar[B_VN_READY]);
-            mbar_arrive(&bar[B_VACC_EMPTY + b]);
+            mbar_arrive(&bar[B_VACC_EMPTY]);
+            if (tid == 192) GDR_TRACE_AT(14, n);
         }
-        // ---- final state
-        if (ok && nchunks > 0 && wait(B_S_FULL, (uint32_t)((nchunks - 1) & 1))) {
+        // ---- final state S_N = S_{N-1} gamma_{N-1} + dS_{N-1}
+        if (ok && nchunks > 0 && waitw(B_S_FULL, (uint32_t)((nchunks - 1) & 1))) {
             tc_fence_after();
+            advance_state(nchunks, false);
             if (ST) {
 #pragma unroll
                 for (int cb = 0; cb < 8; ++cb) {
@@ -562,6 +642,13 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream, int *launch
     if (e == cudaSuccess) *launches += 1;
     return e;
 }
+
+#ifdef GDR_TRACE
+extern "C" __attribute__((visibility("default"))) int gdr_trace_dump(long long *host)
+{
+    return (int)cudaMemcpyFromSymbol(host, g_trace, sizeof(g_trace));
+}
+#endif
 
 cudaError_t read_device_status(cudaStream_t stream, int *status)
 {

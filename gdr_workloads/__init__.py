@@ -171,6 +171,8 @@ def _g_from_recipe(w: Workload, seed: int, idx: torch.Tensor, b: torch.Tensor, h
         return -_softplus64(normal(seed, TID_G, idx) + 2.0)
     if r == "softplus_n02_clamp5":
         return torch.clamp(-_softplus64(2.0 * normal(seed, TID_G, idx)), min=-5.0)
+    if r == "slow_decay":               # parity cases only: the state carries across chunks
+        return -(0.001 + 0.049 * uniform(seed, TID_G, idx))
     if r == "softplus_n02_unbounded":   # parity cases only: some values below -5
         return -_softplus64(2.0 * normal(seed, TID_G, idx) + 2.0)
     if r == "long_context_mix":

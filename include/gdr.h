@@ -121,6 +121,39 @@ int gdr_recurrent_step(const void *q, const void *k, const void *v, const float 
                        void *stream);
 
 /*
+ * Chunked forward that allocates nothing, for callers that cannot allocate
+ * device memory or pass a workspace at the point of the call: serving or
+ * real-time loops that forbid allocator calls on their hot path, code that
+ * keeps allocator calls out of a region it records as a CUDA graph, hosts
+ * whose device memory belongs to another runtime or a pool the caller cannot
+ * reach.  The pages have no counterpart to this call; it is an interface
+ * convenience of this library.
+ *
+ * Same arguments, layouts and results as gdr_chunk_fwd, without the
+ * workspace: the scratch the tensor-core path needs comes from one fixed
+ * array the library holds in device memory, GDR_NOALLOC_SCRATCH_BYTES on
+ * every GPU where the library is loaded, until the process exits.
+ *   - Problems whose gdr_chunk_fwd_workspace_size() exceeds
+ *     GDR_NOALLOC_SCRATCH_BYTES are rejected with GDR_ERR_UNSUPPORTED before
+ *     any launch (for example B*H*ceil(T/64) > 2048 chunks of bf16 d=128).
+ *   - Every call shares that array.  Calls that may overlap on the GPU
+ *     (unordered streams, several host threads) race on it and give
+ *     undefined results; order them.  Nothing has to be cleared between
+ *     calls.
+ *   - The first call made with a given device current looks up the array's
+ *     device address (cudaGetSymbolAddress) and caches it; make that first
+ *     call before any stream capture begins.  A failed look-up returns
+ *     GDR_ERR_CUDA without launching anything.
+ *   - It calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+#define GDR_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+int gdr_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                          const float *S0, void *O, float *S_T,
+                          int B, int H, int T, int dk, int dv, int C, int gate_mode, int dtype,
+                          void *stream);
+
+/*
  * Device-side status.  Kernels that wait on other warps of their own block
  * bound every wait (about a second); when one runs out the kernel records
  * GDR_ERR_TIMEOUT in a device status word, stops, and leaves its outputs

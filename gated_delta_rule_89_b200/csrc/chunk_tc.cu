@@ -63,13 +63,14 @@ constexpr uint32_t OFF_V = OFF_Q + 2 * 16384;      // v (2 panels)              
 constexpr uint32_t OFF_T = OFF_V + 16384;          // T' (1 panel)                      8 KB
 constexpr uint32_t OFF_AQ = OFF_T + 8192;          // 2 x Aqk                           2 x 8 KB
 constexpr uint32_t OFF_KT = OFF_AQ + 2 * 8192;     // K_tail (2 panels)                 16 KB
-constexpr uint32_t OFF_W = OFF_KT + 16384;         // W (2 panels x 8 KB)               16 KB
+constexpr uint32_t OFF_W = OFF_KT + 16384;         // W, MN-major [128 ch x 64 tok]     16 KB
 constexpr uint32_t OFF_S = OFF_W + 16384;          // bf16 S (2 panels x 16 KB)         32 KB
 constexpr uint32_t OFF_VN = OFF_S + 32768;         // V_new^T (1 panel, 128 rows)       16 KB
 constexpr uint32_t OFF_GAM = OFF_VN + 16384;       // gamma_C ring [4][128] fp32        2 KB
 constexpr uint32_t OFF_BAR = OFF_GAM + 2048;       // mbarriers, TMEM slot, abort flag
 constexpr uint32_t SMEM_USED = OFF_BAR + 512;
 constexpr uint32_t SMEM_ALLOC = SMEM_USED + 1024;  // alignment slack
+static_assert(SMEM_ALLOC <= 232448, "dynamic shared memory above the 227 KB per-block limit");
 
 // TMEM columns (fp32)
 constexpr uint32_t TM_S = 0;      // state S_n, 128 columns (written only by the conversion warps)
@@ -89,6 +90,7 @@ enum Bar {
     B_WT_FULL, B_WT_EMPTY, B_W_READY, B_W_FREE,
     B_S_READY, B_S_FULL, B_X_FULL, B_VN_READY,
     B_VACC_EMPTY, B_O_FULL, B_O_FULL1, B_OACC_EMPTY, B_OACC_EMPTY1,
+    B_XCH, B_XCH1,
     B_FINAL,
     B_COUNT
 };
@@ -117,6 +119,30 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
 {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// Eight bf16 (one 16-byte chunk) times eight fp32 factors, rounded back to bf16.
+__device__ __forceinline__ uint4 scale8(uint4 v, const float (&f)[8])
+{
+    uint4 o;
+    o.x = pack_bf16(__uint_as_float(v.x << 16) * f[0], __uint_as_float(v.x & 0xffff0000u) * f[1]);
+    o.y = pack_bf16(__uint_as_float(v.y << 16) * f[2], __uint_as_float(v.y & 0xffff0000u) * f[3]);
+    o.z = pack_bf16(__uint_as_float(v.z << 16) * f[4], __uint_as_float(v.z & 0xffff0000u) * f[5]);
+    o.w = pack_bf16(__uint_as_float(v.w << 16) * f[6], __uint_as_float(v.w & 0xffff0000u) * f[7]);
+    return o;
+}
+
+// Sixteen fp32 TMEM words -> two 16-byte bf16 chunks.
+__device__ __forceinline__ void pack16(const uint32_t (&r)[16], uint4 &lo, uint4 &hi)
+{
+    lo.x = pack_bf16(__uint_as_float(r[0]), __uint_as_float(r[1]));
+    lo.y = pack_bf16(__uint_as_float(r[2]), __uint_as_float(r[3]));
+    lo.z = pack_bf16(__uint_as_float(r[4]), __uint_as_float(r[5]));
+    lo.w = pack_bf16(__uint_as_float(r[6]), __uint_as_float(r[7]));
+    hi.x = pack_bf16(__uint_as_float(r[8]), __uint_as_float(r[9]));
+    hi.y = pack_bf16(__uint_as_float(r[10]), __uint_as_float(r[11]));
+    hi.z = pack_bf16(__uint_as_float(r[12]), __uint_as_float(r[13]));
+    hi.w = pack_bf16(__uint_as_float(r[14]), __uint_as_float(r[15]));
 }
 
 template <bool SCALAR>
@@ -149,6 +175,7 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
             1, 128, 128, 1,     // wt full (MMA), wt empty (M), w ready (M), w free (MMA)
             128, 1, 1, 128,     // s ready (M), s full (MMA), x full (MMA), vn ready (M)
             128, 1, 1, 128, 128,        // vacc empty (M), o full (MMA) x2, oacc empty (E) x2
+            128, 128,                   // row-group exchange (E) x2
             1};
         for (int i = 0; i < B_COUNT; ++i) mbar_init(&bar[i], counts[i]);
         *abort_flag = 0;
@@ -236,7 +263,7 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
         // ================================================================ MMA issuer
         if (lane == 0) {
             constexpr uint32_t ID_WU = idesc_bf16(128, 64, true, false);         // A MN-major, B K-major
-            constexpr uint32_t ID_X = idesc_bf16(128, 64, false, false, true);   // -A
+            constexpr uint32_t ID_X = idesc_bf16(128, 64, false, true, true);    // -A, B (W) MN-major
             constexpr uint32_t ID_O = idesc_bf16(128, 64, false, false);
             constexpr uint32_t ID_S = idesc_bf16(128, 128, false, true);         // B MN-major
             for (int n = 0; n < nchunks; ++n) {
@@ -266,33 +293,35 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
                 tc_fence_after();
                 GDR_TRACE_AT(2, n);
                 const uint32_t qb = sbase + OFF_Q + b * 16384;
+                // V_new^T first: it is on the sequential path
 #pragma unroll
                 for (int s = 0; s < 8; ++s)
                     mma_bf16(tmem + TM_V, sdesc_sw128(sbase + OFF_S + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024),
-                             sdesc_sw128(sbase + OFF_W + (s >> 2) * 8192 + (s & 3) * 32, 16, 1024), ID_X, 1);
+                             sdesc_sw128(sbase + OFF_W + s * 2048, 8192, 1024), ID_X, 1);
+                mma_commit(&bar[B_X_FULL]);
+                mma_commit(&bar[B_W_FREE]);
 #pragma unroll
                 for (int s = 0; s < 8; ++s)
                     mma_bf16(tmem + TM_O + 64 * b, sdesc_sw128(sbase + OFF_S + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024),
                              sdesc_sw128(qb + (s >> 2) * 8192 + (s & 3) * 32, 16, 1024), ID_O, s > 0);
-                mma_commit(&bar[B_X_FULL]);
-                mma_commit(&bar[B_W_FREE]);
                 mma_commit(&bar[B_EMPTY_Q + b]);
                 // ---- O^T += V_new^T Aqk^T ; S += V_new^T K_tail
                 if (!wait(B_VN_READY, par) || !wait(B_FULL_AQ + b, upar) || !wait(B_KT_READY, par)) break;
                 tc_fence_after();
                 GDR_TRACE_AT(3, n);
-#pragma unroll
-                for (int s = 0; s < 4; ++s)
-                    mma_bf16(tmem + TM_O + 64 * b, sdesc_sw128(sbase + OFF_VN + s * 32, 16, 1024),
-                             sdesc_sw128(sbase + OFF_AQ + b * 8192 + s * 32, 16, 1024), ID_O, 1);
+                // the state increment first: it is on the sequential path
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
                     mma_bf16(tmem + TM_D, sdesc_sw128(sbase + OFF_VN + s * 32, 16, 1024),
                              sdesc_sw128(sbase + OFF_KT + s * 2048, 8192, 1024), ID_S, s > 0);
-                mma_commit(&bar[B_O_FULL + b]);
                 mma_commit(&bar[B_S_FULL]);
-                mma_commit(&bar[B_EMPTY_AQ + b]);
                 mma_commit(&bar[B_KT_FREE]);
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_bf16(tmem + TM_O + 64 * b, sdesc_sw128(sbase + OFF_VN + s * 32, 16, 1024),
+                             sdesc_sw128(sbase + OFF_AQ + b * 8192 + s * 32, 16, 1024), ID_O, 1);
+                mma_commit(&bar[B_O_FULL + b]);
+                mma_commit(&bar[B_EMPTY_AQ + b]);
             }
             // every MMA issued above has completed before TMEM is released
             mma_commit(&bar[B_FINAL]);
@@ -300,7 +329,6 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
         }
     } else if (warp < 6) {
         // ================================================================ E: gate products, operands, epilogue
-        const int c = tid - 64;                      // key channel 0..127
         const uint32_t lq = 32u * (warp & 3);        // TMEM lane quarter of this warp
         const int orow = (int)lq + lane;             // d_v index for the epilogue
         auto epilogue = [&](int m) -> bool {
@@ -325,6 +353,14 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
             mbar_arrive(&bar[B_OACC_EMPTY + bb]);
             return true;
         };
+        // Vectorised gate pass: thread (rg, cg) owns rows 8rg..8rg+7 and key
+        // channels 8cg..8cg+7, so every shared access is one 16-byte chunk of
+        // a 128B-swizzled row.  The running products exp(G_r) and exp(G_C - G_r)
+        // per channel combine the thread's own 8 rows with the products of the
+        // other row groups, exchanged through shared memory once per chunk.
+        const int et = tid - 64;
+        const int cg = et & 15, rg = et >> 4;
+        const uint32_t pan = (uint32_t)(cg >> 3) * 8192u;   // panel holding this channel group
         bool ok = true;
         for (int n = 0; n < nchunks && ok; ++n) {
             const int b = n & 1;
@@ -333,53 +369,108 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
             if (!SCALAR && !waitw(B_FULL_G, par)) break;
             if (!waitw(B_FULL_K + b, upar) || !waitw(B_FULL_Q + b, upar)) break;
             if (tid == 64) GDR_TRACE_AT(4, n);
-            float al[kC];
+            float a[8][8];
             if (!SCALAR) {
-                const float *gt = reinterpret_cast<const float *>(sm + OFF_G);
+                const float *gt = reinterpret_cast<const float *>(sm + OFF_G) + (8 * rg) * kD + 8 * cg;
 #pragma unroll
-                for (int r = 0; r < kC; ++r) al[r] = __expf(fmaxf(gt[r * kD + c], kGateMin));
-                // The next TMA load overwrites this tile as soon as the barrier
-                // completes; an arrive does not wait for this thread's shared
-                // loads, so order them before the async-proxy write first.
-                fence_async_smem();
-                mbar_arrive(&bar[B_EMPTY_G]);
+                for (int rr = 0; rr < 8; ++rr) {
+                    const float4 x0 = *reinterpret_cast<const float4 *>(gt + rr * kD);
+                    const float4 x1 = *reinterpret_cast<const float4 *>(gt + rr * kD + 4);
+                    a[rr][0] = __expf(fmaxf(x0.x, kGateMin)); a[rr][1] = __expf(fmaxf(x0.y, kGateMin));
+                    a[rr][2] = __expf(fmaxf(x0.z, kGateMin)); a[rr][3] = __expf(fmaxf(x0.w, kGateMin));
+                    a[rr][4] = __expf(fmaxf(x1.x, kGateMin)); a[rr][5] = __expf(fmaxf(x1.y, kGateMin));
+                    a[rr][6] = __expf(fmaxf(x1.z, kGateMin)); a[rr][7] = __expf(fmaxf(x1.w, kGateMin));
+                }
             } else {
 #pragma unroll
-                for (int r = 0; r < kC; ++r) al[r] = (t0 + r < T_len) ? __expf(__ldg(g_scalar + tok0 + t0 + r)) : 1.f;
-            }
-            unsigned char *kp = sm + OFF_K + b * 16384 + (c >> 6) * 8192;
-            unsigned char *qp = sm + OFF_Q + b * 16384 + (c >> 6) * 8192;
-            const uint32_t cc = (uint32_t)(c & 63);
-            uint32_t kraw[kC / 2];
-            float p = 1.f;
+                for (int rr = 0; rr < 8; ++rr) {
+                    const int t = t0 + 8 * rg + rr;
+                    const float e = (t < T_len) ? __expf(__ldg(g_scalar + tok0 + t)) : 1.f;
 #pragma unroll
-            for (int r = 0; r < kC; ++r) {
-                const uint32_t off = sw128_off(r, cc);
-                __nv_bfloat16 *kk = reinterpret_cast<__nv_bfloat16 *>(kp + off);
-                __nv_bfloat16 *qq = reinterpret_cast<__nv_bfloat16 *>(qp + off);
-                const float kv = __bfloat162float(*kk);
-                const float qv = __bfloat162float(*qq);
-                if (r & 1) kraw[r >> 1] |= (uint32_t)__bfloat16_as_ushort(*kk) << 16;
-                else kraw[r >> 1] = (uint32_t)__bfloat16_as_ushort(*kk);
-                p *= al[r];
-                *kk = __float2bfloat16_rn(kv * p);
-                *qq = __float2bfloat16_rn(qv * p);
+                    for (int c = 0; c < 8; ++c) a[rr][c] = e;
+                }
             }
-            gam[(n & 3) * kD + c] = p;
+            // product of this row group, exchanged with the other seven
+            float L[8], F[8], Bk[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                L[c] = a[0][c];
+#pragma unroll
+                for (int rr = 1; rr < 8; ++rr) L[c] *= a[rr][c];
+                F[c] = 1.f;
+                Bk[c] = 1.f;
+            }
+            // Exchange area: with per-channel gates, row 8j of the g tile, which
+            // only the threads of row group j read, and which they overwrite
+            // after reading it; the tile is released after the exchange.  With
+            // a scalar gate the g region holds no tile, so two [8][128] buffers
+            // live there.
+            float *xb = reinterpret_cast<float *>(sm + OFF_G) + (SCALAR ? b * 8 * kD : 0);
+            constexpr int xrow = SCALAR ? kD : 8 * kD;
+            *reinterpret_cast<float4 *>(xb + rg * xrow + 8 * cg) = make_float4(L[0], L[1], L[2], L[3]);
+            *reinterpret_cast<float4 *>(xb + rg * xrow + 8 * cg + 4) = make_float4(L[4], L[5], L[6], L[7]);
+            mbar_arrive(&bar[B_XCH + b]);
+            if (!waitw(B_XCH + b, upar)) break;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                if (j == rg) continue;
+                const float4 y0 = *reinterpret_cast<const float4 *>(xb + j * xrow + 8 * cg);
+                const float4 y1 = *reinterpret_cast<const float4 *>(xb + j * xrow + 8 * cg + 4);
+                const float y[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    if (j < rg) F[c] *= y[c];
+                    else Bk[c] *= y[c];
+                }
+            }
+            if (!SCALAR) {
+                // The next TMA load overwrites the g tile as soon as this
+                // barrier completes; an arrive does not wait for this thread's
+                // shared loads, so order them before the async-proxy write.
+                fence_async_smem();
+                mbar_arrive(&bar[B_EMPTY_G]);
+            }
+            // K<- = k exp(G_r), Q<- = q exp(G_r) in place; raw k kept for K_tail
+            unsigned char *kp = sm + OFF_K + b * 16384 + pan;
+            unsigned char *qp = sm + OFF_Q + b * 16384 + pan;
+            uint4 kraw[8];
+            float pf[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) pf[c] = F[c];
+#pragma unroll
+            for (int rr = 0; rr < 8; ++rr) {
+                const uint32_t r = (uint32_t)(8 * rg + rr);
+                const uint32_t off = r * 128u + ((((uint32_t)(cg & 7)) ^ (r & 7u)) << 4);
+                const uint4 kv = *reinterpret_cast<const uint4 *>(kp + off);
+                const uint4 qv = *reinterpret_cast<const uint4 *>(qp + off);
+                kraw[rr] = kv;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) pf[c] *= a[rr][c];
+                *reinterpret_cast<uint4 *>(kp + off) = scale8(kv, pf);
+                *reinterpret_cast<uint4 *>(qp + off) = scale8(qv, pf);
+            }
+            if (rg == 0) {   // gamma_C = product over all 64 rows
+                float *gw = gam + (n & 3) * kD + 8 * cg;
+                *reinterpret_cast<float4 *>(gw) = make_float4(L[0] * Bk[0], L[1] * Bk[1], L[2] * Bk[2], L[3] * Bk[3]);
+                *reinterpret_cast<float4 *>(gw + 4) = make_float4(L[4] * Bk[4], L[5] * Bk[5], L[6] * Bk[6], L[7] * Bk[7]);
+            }
             fence_async_smem();
             mbar_arrive(&bar[B_KQ_READY + b]);
             if (tid == 64) GDR_TRACE_AT(5, n);
-            // K_tail = k * exp(G_C - G): reverse running product
+            // K_tail = k exp(G_C - G_r): exclusive running product from the end
             if (!waitw(B_KT_FREE, par ^ 1)) break;
             if (tid == 64) GDR_TRACE_AT(6, n);
-            unsigned char *ktp = sm + OFF_KT + (c >> 6) * 8192;
-            p = 1.f;
+            unsigned char *ktp = sm + OFF_KT + pan;
+            float sf[8];
 #pragma unroll
-            for (int r = kC - 1; r >= 0; --r) {
-                const uint32_t bits = (r & 1) ? (kraw[r >> 1] >> 16) : (kraw[r >> 1] & 0xffffu);
-                const float kv = __bfloat162float(__ushort_as_bfloat16((unsigned short)bits));
-                *reinterpret_cast<__nv_bfloat16 *>(ktp + sw128_off(r, cc)) = __float2bfloat16_rn(kv * p);
-                p *= al[r];
+            for (int c = 0; c < 8; ++c) sf[c] = Bk[c];
+#pragma unroll
+            for (int rr = 7; rr >= 0; --rr) {
+                const uint32_t r = (uint32_t)(8 * rg + rr);
+                const uint32_t off = r * 128u + ((((uint32_t)(cg & 7)) ^ (r & 7u)) << 4);
+                *reinterpret_cast<uint4 *>(ktp + off) = scale8(kraw[rr], sf);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) sf[c] *= a[rr][c];
             }
             fence_async_smem();
             mbar_arrive(&bar[B_KT_READY]);
@@ -410,30 +501,34 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
         // S_{n} = S_{n-1} * gamma_{n-1} + dS_{n-1}, in TMEM and (optionally) as bf16 in smem
         auto advance_state = [&](int n, bool to_smem) {
             const float *gm = gam + ((n - 1) & 3) * kD;
-#pragma unroll 2
-            for (int cb = 0; cb < 8; ++cb) {
-                uint32_t r[16], dr[16];
-                tmem_ld16(trow + TM_S + 16 * cb, r);
-                tmem_ld16(trow + TM_D + 16 * cb, dr);
-                tmem_ld_wait(r);
-                reg_touch(dr);
 #pragma unroll
-                for (int j = 0; j < 16; ++j)
-                    r[j] = __float_as_uint(fmaf(__uint_as_float(r[j]), gm[16 * cb + j], __uint_as_float(dr[j])));
-                tmem_st16(trow + TM_S + 16 * cb, r);
+            for (int cb = 0; cb < 8; cb += 2) {
+                uint32_t r0[16], r1[16], d0[16], d1[16];
+                tmem_ld16(trow + TM_S + 16 * cb, r0);
+                tmem_ld16(trow + TM_S + 16 * cb + 16, r1);
+                tmem_ld16(trow + TM_D + 16 * cb, d0);
+                tmem_ld16(trow + TM_D + 16 * cb + 16, d1);
+                tmem_ld_wait(r0);
+                reg_touch(r1);
+                reg_touch(d0);
+                reg_touch(d1);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    r0[j] = __float_as_uint(fmaf(__uint_as_float(r0[j]), gm[16 * cb + j], __uint_as_float(d0[j])));
+                    r1[j] = __float_as_uint(fmaf(__uint_as_float(r1[j]), gm[16 * cb + 16 + j], __uint_as_float(d1[j])));
+                }
+                tmem_st16(trow + TM_S + 16 * cb, r0);
+                tmem_st16(trow + TM_S + 16 * cb + 16, r1);
                 if (to_smem) {
                     unsigned char *sp = sm + OFF_S + (cb >> 2) * 16384;
+                    const uint32_t col = (uint32_t)((16 * cb) & 63);
                     uint4 lo, hi;
-                    lo.x = pack_bf16(__uint_as_float(r[0]), __uint_as_float(r[1]));
-                    lo.y = pack_bf16(__uint_as_float(r[2]), __uint_as_float(r[3]));
-                    lo.z = pack_bf16(__uint_as_float(r[4]), __uint_as_float(r[5]));
-                    lo.w = pack_bf16(__uint_as_float(r[6]), __uint_as_float(r[7]));
-                    hi.x = pack_bf16(__uint_as_float(r[8]), __uint_as_float(r[9]));
-                    hi.y = pack_bf16(__uint_as_float(r[10]), __uint_as_float(r[11]));
-                    hi.z = pack_bf16(__uint_as_float(r[12]), __uint_as_float(r[13]));
-                    hi.w = pack_bf16(__uint_as_float(r[14]), __uint_as_float(r[15]));
-                    *reinterpret_cast<uint4 *>(sp + sw128_off(i, (16 * cb) & 63)) = lo;
-                    *reinterpret_cast<uint4 *>(sp + sw128_off(i, ((16 * cb) & 63) + 8)) = hi;
+                    pack16(r0, lo, hi);
+                    *reinterpret_cast<uint4 *>(sp + sw128_off(i, col)) = lo;
+                    *reinterpret_cast<uint4 *>(sp + sw128_off(i, col + 8)) = hi;
+                    pack16(r1, lo, hi);
+                    *reinterpret_cast<uint4 *>(sp + sw128_off(i, col + 16)) = lo;
+                    *reinterpret_cast<uint4 *>(sp + sw128_off(i, col + 24)) = hi;
                 }
             }
             tmem_st_wait();
@@ -449,18 +544,30 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
             tc_fence_after();
             if (tid == 192) GDR_TRACE_AT(9, n);
             {
-                unsigned char *wp = sm + OFF_W + (i >> 6) * 8192;
-                const uint32_t cc = (uint32_t)(i & 63);
-#pragma unroll
-                for (int cb = 0; cb < 4; ++cb) {
-                    uint32_t r[16];
-                    tmem_ld16(trow + TM_W + 16 * cb, r);
-                    tmem_ld_wait(r);
-#pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        *reinterpret_cast<__nv_bfloat16 *>(wp + sw128_off(16 * cb + j, cc)) =
-                            __float2bfloat16_rn(__uint_as_float(r[j]));
-                }
+                // W^T row of key channel i = 64 tokens = one 128-byte row of the
+                // MN-major W operand
+                uint32_t r0[16], r1[16];
+                tmem_ld16(trow + TM_W, r0);
+                tmem_ld16(trow + TM_W + 16, r1);
+                tmem_ld_wait(r0);
+                reg_touch(r1);
+                uint4 lo, hi;
+                pack16(r0, lo, hi);
+                *reinterpret_cast<uint4 *>(sm + OFF_W + sw128_off(i, 0)) = lo;
+                *reinterpret_cast<uint4 *>(sm + OFF_W + sw128_off(i, 8)) = hi;
+                pack16(r1, lo, hi);
+                *reinterpret_cast<uint4 *>(sm + OFF_W + sw128_off(i, 16)) = lo;
+                *reinterpret_cast<uint4 *>(sm + OFF_W + sw128_off(i, 24)) = hi;
+                tmem_ld16(trow + TM_W + 32, r0);
+                tmem_ld16(trow + TM_W + 48, r1);
+                tmem_ld_wait(r0);
+                reg_touch(r1);
+                pack16(r0, lo, hi);
+                *reinterpret_cast<uint4 *>(sm + OFF_W + sw128_off(i, 32)) = lo;
+                *reinterpret_cast<uint4 *>(sm + OFF_W + sw128_off(i, 40)) = hi;
+                pack16(r1, lo, hi);
+                *reinterpret_cast<uint4 *>(sm + OFF_W + sw128_off(i, 48)) = lo;
+                *reinterpret_cast<uint4 *>(sm + OFF_W + sw128_off(i, 56)) = hi;
             }
             fence_async_smem();
             tc_fence_before();

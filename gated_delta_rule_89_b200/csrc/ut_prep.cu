@@ -1,4 +1,4 @@
-// UT-transform preparation of the chunked forward, one CTA per chunk.
+// UT-transform preparation of the chunked forward.
 //
 // For every chunk of C = 64 tokens (rows r, i) this kernel forms
 //   A[r][i]   = beta_r sum_c k_rc k_ic exp(G_rc - G_ic)     (i <  r)
@@ -12,6 +12,13 @@
 // output equation.  Neither depends on the state, so all chunks of all heads
 // run in parallel here and the sequential kernel only consumes them.
 //
+// Execution.  Persistent CTAs of 8 warps, two per SM, walk the chunks
+// blockIdx.x, blockIdx.x + gridDim.x, ...  The gate pass reads k, q and g of
+// a chunk straight from global memory (each warp a contiguous row segment)
+// and writes the scaled operands into shared memory in the 128B-swizzled
+// layout, which makes the ldmatrix reads of the block products conflict
+// free; the other CTA on the SM runs its own phases while one waits.
+
 // Decay ratios (per-channel gate).  G is the cumulative log-decay inside the
 // chunk; exp(G_r - G_i) is formed without overflow by splitting the chunk
 // into four 16-token blocks.  With base_R the cumulative sum just before
@@ -31,36 +38,55 @@
 // A scalar gate needs no splitting: the products use k and q as they are and
 // the decay exp(G_r - G_i) multiplies each entry afterwards.
 //
-// Inverse.  (I + A) is unit lower triangular.  Its two 32 x 32 diagonal
-// blocks are inverted by forward substitution, one thread per column, and
-// the off-diagonal block is Y = -Z A_10 X (X, Z the diagonal inverses).
+// Inverse of N = I + A (unit lower triangular), in 16 x 16 blocks N_im.
+// D_i = N_ii^{-1} by forward substitution (one thread per column).  With
+// Nt_im = D_i N_im (i > m) the blocks U_ij of N^{-1} below the diagonal
+// follow column block by column block:
+//   U_{i,i-1} = -Nt_{i,i-1} D_{i-1},
+//   U_20 = -Nt_20 D_0 - Nt_21 U_10,   U_31 = -Nt_31 D_1 - Nt_32 U_21,
+//   U_30 = -Nt_30 D_0 - Nt_31 U_10 - Nt_32 U_20,
+// (from N N^{-1} = I, left-multiplied by D_i).  These 16 products of 16 x 16
+// fp32 blocks run on mma.sync (m16n8k8, tf32) with each operand split into a
+// high and a low tf32 part (x = hi + lo) and the product taken as
+// hi*hi + hi*lo + lo*hi, the three-pass tf32 error compensation of
+// Ootomo and Yokota (2022), which keeps fp32-level accuracy.
+
+#include <mutex>
+
 #include "gdr_internal.cuh"
+#include "sm100_ptx.cuh"
 
 namespace gdr {
 namespace {
 
-constexpr int kC = 64;        // chunk
-constexpr int kDK = 128;      // key dim
-constexpr int kLdB = kDK + 8; // padded bf16 row stride (272 B: ldmatrix conflict free)
-constexpr int kLdA = kC + 1;  // padded fp32 row stride
+using namespace sm100;
 
-struct PrepSmem {
-    __nv_bfloat16 kh[kC][kLdB];   // Khat (left operand of A)
-    __nv_bfloat16 qh[kC][kLdB];   // Qhat (left operand of Aqk)
-    __nv_bfloat16 kc[kC][kLdB];   // Kchk (right operand)
-    float fac[7][kDK];            // block-pair channel factors (see pair_factor)
-    float A[kC][kLdA];            // A, then its inverse
-    float Aq[kC][kLdA];           // Aqk
-    float P[32][33];              // A_10 X
-    float beta[kC];
-    float G[kC];                  // scalar-gate cumulative sum
-};
+constexpr int kC = 64;         // chunk
+constexpr int kDK = 128;       // key dim
+constexpr int kThreads = 256;  // 8 warps
+constexpr int kLdA = 68;       // fp32 row stride: 16-byte rows, conflict-free fragment stores
 
-__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void *p)
+// shared memory (offsets from a 1024-byte aligned base)
+constexpr uint32_t OFF_K = 0;                      // Khat (or k), two swizzled panels   16 KB
+constexpr uint32_t OFF_Q = 16384;                  // Qhat (or q)                         16 KB
+constexpr uint32_t OFF_KC = 32768;                 // Kchk                                16 KB
+constexpr uint32_t OFF_BD = 49152;                 // bd[4][128], 1/bd[4][128] fp32         4 KB
+constexpr int kLdD = 24;       // row stride of the 16 x 16 blocks (conflict-free mma B fragments)
+constexpr uint32_t OFF_D = OFF_BD + 4096;          // D_i = N_ii^{-1}, [4][16][24]           6 KB
+constexpr uint32_t OFF_A = OFF_D + 4 * 16 * kLdD * 4;   // A
+constexpr uint32_t OFF_AQ = OFF_A + kC * kLdA * 4; // Aqk, then Nt / X'
+constexpr uint32_t OFF_U = OFF_AQ + kC * kLdA * 4; // U_10, U_21, U_20 [3][16][24]
+constexpr uint32_t OFF_BETA = OFF_U + 3 * 16 * kLdD * 4;   // beta, two buffers by chunk parity
+constexpr uint32_t OFF_GC = OFF_BETA + 512;        // scalar gate: inclusive cumulative sum
+constexpr uint32_t SMEM_USED = OFF_GC + 256;
+constexpr uint32_t SMEM_ALLOC = SMEM_USED + 1024;  // alignment slack
+static_assert(2 * (SMEM_ALLOC + 1024) <= 233472, "two CTAs per SM must fit in shared memory");
+
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr)
 {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"((uint32_t)__cvta_generic_to_shared(p)));
+                 : "r"(addr));
 }
 
 __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
@@ -72,245 +98,415 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ uint32_t scale_bf16x2(uint32_t v, float s0, float s1)
+// two bf16 (packed) times two fp32 factors, rounded back to bf16
+__device__ __forceinline__ uint32_t scale2(uint32_t v, float s0, float s1)
 {
-    __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162 *>(&v);
-    float2 f = __bfloat1622float2(h);
-    __nv_bfloat162 o = __floats2bfloat162_rn(f.x * s0, f.y * s1);
+    __nv_bfloat162 o = __floats2bfloat162_rn(__uint_as_float(v << 16) * s0, __uint_as_float(v & 0xffff0000u) * s1);
     return *reinterpret_cast<uint32_t *>(&o);
 }
 
-// factor row for block pair (R, I): -1 = none (adjacent blocks), else index into fac
-__device__ __forceinline__ int pair_factor(int R, int I)
+__device__ __forceinline__ uint32_t pack2(float lo, float hi)
 {
-    if (R == I) return 3 + R;          // 1 / bd_R
-    if (R == I + 1) return -1;         // exp(base_R - base_{I+1}) = 1
-    if (R == 2 && I == 0) return 0;    // bd_1
-    if (R == 3 && I == 1) return 1;    // bd_2
-    return 2;                          // (3, 0): bd_1 bd_2
+    __nv_bfloat162 o = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&o);
+}
+
+// packed fp32 pair multiply (sm_100 f32x2)
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b)
+{
+    unsigned long long x = *reinterpret_cast<unsigned long long *>(&a), y = *reinterpret_cast<unsigned long long *>(&b), z;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(z) : "l"(x), "l"(y));
+    return *reinterpret_cast<float2 *>(&z);
+}
+
+// bf16 pair (packed) times an fp32 pair, rounded back to a bf16 pair
+__device__ __forceinline__ uint32_t scale2p(uint32_t v, float2 f)
+{
+    const float2 r = fmul2(make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u)), f);
+    return pack2(r.x, r.y);
+}
+
+__device__ __forceinline__ void split_tf32(float x, uint32_t &hi, uint32_t &lo)
+{
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(hi) : "f"(x));
+    const float r = x - __uint_as_float(hi);
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(lo) : "f"(r));
+}
+
+__device__ __forceinline__ void mma1688(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// One warp: c[16x16] -= A[16x16] B[16x16] in fp32 accuracy (three tf32
+// passes).  A, B row-major in shared memory with row strides lda, ldb.
+// Fragment of c: c[nt][e] is row g + 8 (e >> 1), column 8 nt + 2 t + (e & 1),
+// with g = lane / 4, t = lane % 4.
+__device__ __forceinline__ void mm16_sub(float (&c)[2][4], const float *A, int lda, const float *B, int ldb, int g,
+                                         int t)
+{
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+        uint32_t ah[4], al[4];
+        split_tf32(-A[g * lda + 8 * ks + t], ah[0], al[0]);
+        split_tf32(-A[(g + 8) * lda + 8 * ks + t], ah[1], al[1]);
+        split_tf32(-A[g * lda + 8 * ks + t + 4], ah[2], al[2]);
+        split_tf32(-A[(g + 8) * lda + 8 * ks + t + 4], ah[3], al[3]);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            uint32_t bh0, bl0, bh1, bl1;
+            split_tf32(B[(8 * ks + t) * ldb + 8 * nt + g], bh0, bl0);
+            split_tf32(B[(8 * ks + t + 4) * ldb + 8 * nt + g], bh1, bl1);
+            mma1688(c[nt], al, bh0, bh1);
+            mma1688(c[nt], ah, bl0, bl1);
+            mma1688(c[nt], ah, bh0, bh1);
+        }
+    }
+}
+
+// byte offset of (row, col) in a [64 rows x 128 cols] bf16 tile held as two
+// 128B-swizzled panels of 64 columns
+__device__ __forceinline__ uint32_t tile_off(uint32_t row, uint32_t col)
+{
+    return (col >> 6) * 8192u + sw128_off(row, col & 63u);
+}
+
+// channel factors of block pair (R, I) (I <= R, I != R - 1) at channels c, c + 1
+// (bd holds bd[4][128] followed by 1/bd[4][128])
+__device__ __forceinline__ float2 pair_factor(const float *bd, int R, int I, int c)
+{
+    if (I == R) return *reinterpret_cast<const float2 *>(bd + (4 + R) * kDK + c);
+    if (I == R - 2) return *reinterpret_cast<const float2 *>(bd + (R - 1) * kDK + c);
+    const float2 a = *reinterpret_cast<const float2 *>(bd + 1 * kDK + c);   // (3, 0): bd_1 bd_2
+    const float2 b = *reinterpret_cast<const float2 *>(bd + 2 * kDK + c);
+    return make_float2(a.x * b.x, a.y * b.y);
 }
 
 template <bool SCALAR>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(kThreads, 2)
 ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__restrict__ qg,
-               const float *__restrict__ gg, const float *__restrict__ betag,
-               __nv_bfloat16 *__restrict__ Tout, __nv_bfloat16 *__restrict__ Aqout, int T_len, int nchunks)
+               const float *__restrict__ gg, const float *__restrict__ betag, __nv_bfloat16 *__restrict__ Tout,
+               __nv_bfloat16 *__restrict__ Aqout, int T_len, int nchunks, int total)
 {
-    extern __shared__ __align__(16) unsigned char prep_raw[];
-    PrepSmem &sm = *reinterpret_cast<PrepSmem *>(prep_raw);
+    extern __shared__ unsigned char prep_raw[];
+    unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(prep_raw) + 1023) &
+                                                          ~static_cast<uintptr_t>(1023));
+    float(*sA)[kLdA] = reinterpret_cast<float(*)[kLdA]>(sm + OFF_A);
+    float(*sQ)[kLdA] = reinterpret_cast<float(*)[kLdA]>(sm + OFF_AQ);   // Aqk, later Nt
+    float(*sU)[16][kLdD] = reinterpret_cast<float(*)[16][kLdD]>(sm + OFF_U);
+    float *sBd = reinterpret_cast<float *>(sm + OFF_BD);              // [4][128] bd, then [4][128] 1/bd
+    float(*sD)[16][kLdD] = reinterpret_cast<float(*)[16][kLdD]>(sm + OFF_D);
+    float *sGc = reinterpret_cast<float *>(sm + OFF_GC);
+
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
-    const size_t head = blockIdx.x / nchunks;
-    const int chunk = blockIdx.x - (int)(head * nchunks);
-    const int t0 = chunk * kC;
-    const int n = min(kC, T_len - t0);
-    const size_t row0 = head * (size_t)T_len + t0;   // first token row of this chunk
+    const int g = lane >> 2, t = lane & 3;   // mma fragment coordinates
 
-    if (tid < kC) sm.beta[tid] = tid < n ? betag[row0 + tid] : 0.f;
+    int parity = 0;
+    for (int ci = blockIdx.x; ci < total; ci += gridDim.x, parity ^= 1) {
+        const int head = ci / nchunks;
+        const int t0 = (ci - head * nchunks) * kC;
+        const int nrows = min(kC, T_len - t0);
+        const size_t row0 = (size_t)head * T_len + t0;   // first token row of this chunk
+        const size_t cbase = (size_t)ci * kC * kC;       // this chunk's T' and Aqk
+        // beta alternates between two buffers: the last T' stores of the
+        // previous chunk may still read theirs while this chunk starts
+        float *sBeta = reinterpret_cast<float *>(sm + OFF_BETA) + kC * parity;
 
-    // ---- operands (thread = key channel)
-    {
-        const int c = tid;
-        if (!SCALAR) {
-            float bd[4];
+        // ---- operands.  Warp (R, panel) covers rows 16R..16R+15 and the 64
+        // channels of one panel; lane = (half, quad): rows 16R + 8 half + 0..7,
+        // channels 64 panel + 4 quad + 0..3.
+        {
+            const int R = warp >> 1, half = lane >> 4;
+            const uint32_t c = 64u * (warp & 1) + 4u * (lane & 15);
+            const int rbase = 16 * R + 8 * half;
+            uint2 kr[8], qr[8];
+            float4 gv[8];
 #pragma unroll
-            for (int R = 0; R < 4; ++R) {
-                float al[16], kv[16], qv[16];
+            for (int rr = 0; rr < 8; ++rr) {
+                const int r = rbase + rr;
+                const bool ok = r < nrows;
+                const size_t e = (row0 + r) * kDK + c;
+                kr[rr] = ok ? __ldg(reinterpret_cast<const uint2 *>(kg + e)) : make_uint2(0u, 0u);
+                qr[rr] = ok ? __ldg(reinterpret_cast<const uint2 *>(qg + e)) : make_uint2(0u, 0u);
+                if (!SCALAR)
+                    gv[rr] = ok ? __ldg(reinterpret_cast<const float4 *>(gg + e)) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+            if (tid < kC) sBeta[tid] = tid < nrows ? __ldg(betag + row0 + tid) : 0.f;
+            if (SCALAR && warp == 0) {
+                // inclusive scan of the scalar log-decay over the chunk (2 values per lane)
+                const float a0 = (2 * lane < nrows) ? __ldg(gg + row0 + 2 * lane) : 0.f;
+                const float a1 = (2 * lane + 1 < nrows) ? __ldg(gg + row0 + 2 * lane + 1) : 0.f;
+                float sum = a0 + a1;
 #pragma unroll
-                for (int r = 0; r < 16; ++r) {
-                    const int rr = R * 16 + r;
-                    const bool ok = rr < n;
-                    const size_t gi = (row0 + rr) * kDK + c;
-                    al[r] = ok ? __expf(fmaxf(gg[gi], kGateMin)) : 1.f;
-                    kv[r] = ok ? __bfloat162float(kg[gi]) : 0.f;
-                    qv[r] = ok ? __bfloat162float(qg[gi]) : 0.f;
+                for (int off = 1; off < 32; off <<= 1) {
+                    const float o = __shfl_up_sync(0xffffffffu, sum, off);
+                    if (lane >= off) sum += o;
                 }
-                float p = 1.f;
+                sGc[2 * lane + 1] = sum;
+                sGc[2 * lane] = sum - a1;
+            }
+            if (SCALAR) {
 #pragma unroll
-                for (int r = 0; r < 16; ++r) {
-                    p *= al[r];
-                    sm.kh[R * 16 + r][c] = __float2bfloat16_rn(kv[r] * p);
-                    sm.qh[R * 16 + r][c] = __float2bfloat16_rn(qv[r] * p);
+                for (int rr = 0; rr < 8; ++rr) {
+                    const uint32_t off = tile_off(rbase + rr, c);
+                    *reinterpret_cast<uint2 *>(sm + OFF_K + off) = kr[rr];
+                    *reinterpret_cast<uint2 *>(sm + OFF_Q + off) = qr[rr];
                 }
-                bd[R] = p;
-                p = 1.f;
+            } else {
+                // alpha = exp(max(g, -5)) and the product over this thread's 8 rows
+                const float2 log2e = make_float2(1.4426950408889634f, 1.4426950408889634f);
+                float2 la = make_float2(1.f, 1.f), lb = make_float2(1.f, 1.f);   // channels (0,1), (2,3)
 #pragma unroll
-                for (int r = 15; r >= 0; --r) {
-                    sm.kc[R * 16 + r][c] = __float2bfloat16_rn(kv[r] * p);
-                    p *= al[r];
+                for (int rr = 0; rr < 8; ++rr) {
+                    float2 x = fmul2(make_float2(fmaxf(gv[rr].x, kGateMin), fmaxf(gv[rr].y, kGateMin)), log2e);
+                    float2 y = fmul2(make_float2(fmaxf(gv[rr].z, kGateMin), fmaxf(gv[rr].w, kGateMin)), log2e);
+                    gv[rr] = make_float4(exp2f(x.x), exp2f(x.y), exp2f(y.x), exp2f(y.y));
+                    la = fmul2(la, make_float2(gv[rr].x, gv[rr].y));
+                    lb = fmul2(lb, make_float2(gv[rr].z, gv[rr].w));
+                }
+                // the other half of the 16-row block (lane ^ 16)
+                const float2 oa = make_float2(__shfl_xor_sync(0xffffffffu, la.x, 16), __shfl_xor_sync(0xffffffffu, la.y, 16));
+                const float2 ob = make_float2(__shfl_xor_sync(0xffffffffu, lb.x, 16), __shfl_xor_sync(0xffffffffu, lb.y, 16));
+                // Khat, Qhat: inclusive running product from the block start
+                float2 pa = half ? oa : make_float2(1.f, 1.f), pb = half ? ob : make_float2(1.f, 1.f);
+#pragma unroll
+                for (int rr = 0; rr < 8; ++rr) {
+                    const uint32_t off = tile_off(rbase + rr, c);
+                    pa = fmul2(pa, make_float2(gv[rr].x, gv[rr].y));
+                    pb = fmul2(pb, make_float2(gv[rr].z, gv[rr].w));
+                    *reinterpret_cast<uint2 *>(sm + OFF_K + off) = make_uint2(scale2p(kr[rr].x, pa), scale2p(kr[rr].y, pb));
+                    *reinterpret_cast<uint2 *>(sm + OFF_Q + off) = make_uint2(scale2p(qr[rr].x, pa), scale2p(qr[rr].y, pb));
+                }
+                if (half) {   // pa, pb now hold bd_R
+                    *reinterpret_cast<float4 *>(sBd + R * kDK + c) = make_float4(pa.x, pa.y, pb.x, pb.y);
+                    *reinterpret_cast<float4 *>(sBd + (4 + R) * kDK + c) =
+                        make_float4(1.f / pa.x, 1.f / pa.y, 1.f / pb.x, 1.f / pb.y);
+                }
+                // Kchk: exclusive running product to the block end
+                pa = half ? make_float2(1.f, 1.f) : oa;
+                pb = half ? make_float2(1.f, 1.f) : ob;
+#pragma unroll
+                for (int rr = 7; rr >= 0; --rr) {
+                    const uint32_t off = tile_off(rbase + rr, c);
+                    *reinterpret_cast<uint2 *>(sm + OFF_KC + off) = make_uint2(scale2p(kr[rr].x, pa), scale2p(kr[rr].y, pb));
+                    pa = fmul2(pa, make_float2(gv[rr].x, gv[rr].y));
+                    pb = fmul2(pb, make_float2(gv[rr].z, gv[rr].w));
                 }
             }
-            sm.fac[0][c] = bd[1];
-            sm.fac[1][c] = bd[2];
-            sm.fac[2][c] = bd[1] * bd[2];
+        }
+        __syncthreads();
+
+        // ---- block products on tensor cores: 10 block pairs over 8 warps, each
+        // pair gives both A and Aqk (the right operand and its scaling are shared)
+        {
+            const uint32_t left_k = smem_u32(sm + OFF_K), left_q = smem_u32(sm + OFF_Q);
+            const uint32_t right = SCALAR ? left_k : smem_u32(sm + OFF_KC);
+            for (int p = warp; p < 10; p += 8) {
+                // pairs (R, I), I <= R, in row-major order of the lower block triangle
+                const int R = p < 1 ? 0 : p < 3 ? 1 : p < 6 ? 2 : 3;
+                const int I = p - R * (R + 1) / 2;
+                const bool scaled = !SCALAR && I != R - 1;
+                float acc[2][2][4] = {};
 #pragma unroll
-            for (int R = 0; R < 4; ++R) sm.fac[3 + R][c] = 1.f / bd[R];
+                for (int ks = 0; ks < kDK / 16; ++ks) {
+                    uint32_t ak[4], aq[4], b[4];
+                    const uint32_t aoff = tile_off(R * 16 + (lane & 15), ks * 16 + (lane >> 4) * 8);
+                    ldsm_x4(ak, left_k + aoff);
+                    ldsm_x4(aq, left_q + aoff);
+                    ldsm_x4(b, right + tile_off(I * 16 + (lane & 7) + ((lane >> 4) << 3),
+                                                ks * 16 + ((lane >> 3) & 1) * 8));
+                    if (scaled) {
+                        const int c = ks * 16 + 2 * t;
+                        const float2 f0 = pair_factor(sBd, R, I, c), f8 = pair_factor(sBd, R, I, c + 8);
+                        b[0] = scale2p(b[0], f0);
+                        b[1] = scale2p(b[1], f8);
+                        b[2] = scale2p(b[2], f0);
+                        b[3] = scale2p(b[3], f8);
+                    }
+                    mma16816(acc[0][0], ak, b[0], b[1]);
+                    mma16816(acc[0][1], ak, b[2], b[3]);
+                    mma16816(acc[1][0], aq, b[0], b[1]);
+                    mma16816(acc[1][1], aq, b[2], b[3]);
+                }
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int r = R * 16 + g + h * 8;
+                        const int i = I * 16 + nt * 8 + 2 * t;
+                        float va[2], vq[2];
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            va[e] = acc[0][nt][2 * h + e];
+                            vq[e] = acc[1][nt][2 * h + e];
+                            if (SCALAR) {
+                                const float dec = __expf(sGc[r] - sGc[i + e]);   // masked below when i > r
+                                va[e] *= dec;
+                                vq[e] *= dec;
+                            }
+                            va[e] = (i + e < r) ? sBeta[r] * va[e] : 0.f;
+                            vq[e] = (i + e <= r) ? vq[e] : 0.f;
+                        }
+                        *reinterpret_cast<float2 *>(&sA[r][i]) = make_float2(va[0], va[1]);
+                        *reinterpret_cast<float2 *>(&sQ[r][i]) = make_float2(vq[0], vq[1]);
+                    }
+            }
+        }
+        __syncthreads();
+
+        if (tid < 64) {
+            // D_b = N_bb^{-1}: thread = (block b, column jc), forward substitution
+            const int base = (tid >> 4) * 16, jc = tid & 15;
+            float x[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) x[r] = (r == jc) ? 1.f : 0.f;
+            // right-looking: once x[m] is final, remove it from every later row
+#pragma unroll
+            for (int m = 0; m < 15; ++m)
+#pragma unroll
+                for (int r = m + 1; r < 16; ++r) x[r] = fmaf(-sA[base + r][base + m], x[m], x[r]);
+#pragma unroll
+            for (int r = 0; r < 16; ++r) sD[tid >> 4][r][jc] = x[r];
         } else {
-            for (int r = 0; r < kC; ++r) {
-                const bool ok = r < n;
-                const size_t gi = (row0 + r) * kDK + c;
-                const __nv_bfloat16 z = __float2bfloat16_rn(0.f);
-                const __nv_bfloat16 kk = ok ? kg[gi] : z;
-                sm.kh[r][c] = kk;
-                sm.kc[r][c] = kk;
-                sm.qh[r][c] = ok ? qg[gi] : z;
-            }
-        }
-    }
-    if (SCALAR && warp == 0) {
-        // inclusive scan of the scalar log-decay over the chunk (2 values per lane)
-        float a0 = (2 * lane < n) ? gg[row0 + 2 * lane] : 0.f;
-        float a1 = (2 * lane + 1 < n) ? gg[row0 + 2 * lane + 1] : 0.f;
-        float s = a0 + a1;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            float o = __shfl_up_sync(0xffffffffu, s, off);
-            if (lane >= off) s += o;
-        }
-        sm.G[2 * lane + 1] = s;
-        sm.G[2 * lane] = s - a1;
-    }
-    for (int idx = tid; idx < kC * kLdA; idx += 128) {
-        (&sm.A[0][0])[idx] = 0.f;
-        (&sm.Aq[0][0])[idx] = 0.f;
-    }
-    __syncthreads();
-
-    // ---- block products on tensor cores: warp (which, half)
-    {
-        const int which = warp >> 1;        // 0: A from Khat, 1: Aqk from Qhat
-        const int half = warp & 1;
-        const __nv_bfloat16(*L)[kLdB] = which ? sm.qh : sm.kh;
-        float(*D)[kLdA] = which ? sm.Aq : sm.A;
-        const int g = lane >> 2, t = lane & 3;
-        static const int kPairs[2][5][2] = {{{0, 0}, {1, 0}, {1, 1}, {2, 0}, {2, 1}},
-                                            {{2, 2}, {3, 0}, {3, 1}, {3, 2}, {3, 3}}};
-#pragma unroll 1
-        for (int p = 0; p < 5; ++p) {
-            const int R = kPairs[half][p][0], I = kPairs[half][p][1];
-            const int fi = SCALAR ? -1 : pair_factor(R, I);
-            float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-            for (int s = 0; s < kDK / 16; ++s) {
-                uint32_t a[4], b[4];
-                ldsm_x4(a, &L[R * 16 + (lane & 15)][s * 16 + (lane >> 4) * 8]);
-                ldsm_x4(b, &sm.kc[I * 16 + (lane & 7) + ((lane >> 4) << 3)][s * 16 + ((lane >> 3) & 1) * 8]);
-                if (fi >= 0) {
-                    const float *f = sm.fac[fi] + s * 16 + 2 * t;
-                    b[0] = scale_bf16x2(b[0], f[0], f[1]);
-                    b[1] = scale_bf16x2(b[1], f[8], f[9]);
-                    b[2] = scale_bf16x2(b[2], f[0], f[1]);
-                    b[3] = scale_bf16x2(b[3], f[8], f[9]);
+            // Aqk out (bf16 row-major): blocks above the diagonal are zero
+            for (int task = tid - 64; task < kC * 8; task += kThreads - 64) {
+                const int r = task >> 3, g8 = task & 7;
+                uint4 o = make_uint4(0u, 0u, 0u, 0u);
+                if ((g8 >> 1) <= (r >> 4)) {
+                    const float4 a0 = *reinterpret_cast<const float4 *>(&sQ[r][8 * g8]);
+                    const float4 a1 = *reinterpret_cast<const float4 *>(&sQ[r][8 * g8 + 4]);
+                    o.x = pack2(a0.x, a0.y);
+                    o.y = pack2(a0.z, a0.w);
+                    o.z = pack2(a1.x, a1.y);
+                    o.w = pack2(a1.z, a1.w);
                 }
-                mma16816(acc[0], a, b[0], b[1]);
-                mma16816(acc[1], a, b[2], b[3]);
+                *reinterpret_cast<uint4 *>(Aqout + cbase + r * kC + 8 * g8) = o;
             }
+        }
+        __syncthreads();
+
+        // T' block (i, j) = U_ij Diag(beta_j) from a 16 x 16 accumulator fragment
+        auto store_t = [&](const float (&c)[2][4], int i, int j) {
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                const int col = 16 * j + 8 * nt + 2 * t;
+                const float b0 = sBeta[col], b1 = sBeta[col + 1];
+                __nv_bfloat16 *dst = Tout + cbase + (size_t)(16 * i + g) * kC + col;
+                *reinterpret_cast<uint32_t *>(dst) = pack2(c[nt][0] * b0, c[nt][1] * b1);
+                *reinterpret_cast<uint32_t *>(dst + 8 * kC) = pack2(c[nt][2] * b0, c[nt][3] * b1);
+            }
+        };
+        auto store_s = [&](const float (&c)[2][4], float (*dst)[kLdD]) {
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                *reinterpret_cast<float2 *>(&dst[g][8 * nt + 2 * t]) = make_float2(c[nt][0], c[nt][1]);
+                *reinterpret_cast<float2 *>(&dst[g + 8][8 * nt + 2 * t]) = make_float2(c[nt][2], c[nt][3]);
+            }
+        };
+        float acc[2][4] = {};
+        if (warp < 6) {
+            // Nt_im = D_i A_im for the six blocks below the diagonal (into sQ)
+            const int i = warp < 1 ? 1 : warp < 3 ? 2 : 3;
+            const int m = warp - i * (i - 1) / 2;
+            float nt_[2][4] = {};
+            mm16_sub(nt_, &sD[i][0][0], kLdD, &sA[16 * i][16 * m], kLdA, g, t);   // = -D_i A_im
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int r = R * 16 + g + (e >> 1) * 8;
-                    const int i = I * 16 + nt * 8 + 2 * t + (e & 1);
-                    float v = acc[nt][e];
-                    if (SCALAR) v *= __expf(sm.G[r] - sm.G[i]);
-                    if (which == 0) v = (i < r) ? sm.beta[r] * v : 0.f;
-                    else v = (i <= r) ? v : 0.f;
-                    D[r][i] = v;
-                }
-        }
-    }
-    __syncthreads();
-
-    // ---- inverse of (I + A): diagonal 32 x 32 blocks, one thread per column
-    if (tid < 64) {
-        const int base = (tid >> 5) * 32;   // 0: X (top-left), 32: Z (bottom-right)
-        const int j = tid & 31;
-        float x[32];
+                for (int e = 0; e < 4; ++e) nt_[nt][e] = -nt_[nt][e];
+            float(*dst)[kLdA] = reinterpret_cast<float(*)[kLdA]>(&sQ[16 * i][16 * m]);
 #pragma unroll
-        for (int r = 0; r < 32; ++r) {
-            float s = (r == j) ? 1.f : 0.f;
-#pragma unroll
-            for (int m = 0; m < r; ++m) s = fmaf(-sm.A[base + r][base + m], x[m], s);
-            x[r] = s;
-        }
-        // every lane of this warp has finished reading its diagonal block of A
-        // before any lane overwrites it (the other warp owns the other block)
-        __syncwarp();
-#pragma unroll
-        for (int r = 0; r < 32; ++r) sm.A[base + r][base + j] = x[r];
-    }
-    __syncthreads();
-    // P = A_10 X   (32 x 32): thread -> 8 entries
-    {
-        const int r = tid >> 2, c0 = (tid & 3) * 8;
-        float acc[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-        for (int m = 0; m < 32; ++m) {
-            const float a = sm.A[32 + r][m];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) acc[e] = fmaf(a, sm.A[m][c0 + e], acc[e]);
-        }
-        __syncthreads();
-#pragma unroll
-        for (int e = 0; e < 8; ++e) sm.P[r][c0 + e] = acc[e];
-        __syncthreads();
-        // Y = -Z P
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-        for (int m = 0; m < 32; ++m) {
-            const float z = sm.A[32 + r][32 + m];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) acc[e] = fmaf(z, sm.P[m][c0 + e], acc[e]);
-        }
-#pragma unroll
-        for (int e = 0; e < 8; ++e) sm.A[32 + r][c0 + e] = -acc[e];
-        // upper-right block of the inverse is zero
-#pragma unroll
-        for (int e = 0; e < 8; ++e) sm.A[r][32 + c0 + e] = 0.f;
-    }
-    __syncthreads();
-
-    // ---- write T' = A~ Diag(beta) and Aqk (bf16, row-major 64 x 64)
-    {
-        const size_t cbase = ((size_t)blockIdx.x) * kC * kC;
-        for (int idx = tid; idx < kC * kC / 8; idx += 128) {
-            const int r = idx >> 3, c0 = (idx & 7) * 8;
-            __align__(16) __nv_bfloat16 tv[8], qv[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                tv[e] = __float2bfloat16_rn(sm.A[r][c0 + e] * sm.beta[c0 + e]);
-                qv[e] = __float2bfloat16_rn(sm.Aq[r][c0 + e]);
+            for (int nt = 0; nt < 2; ++nt) {
+                *reinterpret_cast<float2 *>(&dst[g][8 * nt + 2 * t]) = make_float2(nt_[nt][0], nt_[nt][1]);
+                *reinterpret_cast<float2 *>(&dst[g + 8][8 * nt + 2 * t]) = make_float2(nt_[nt][2], nt_[nt][3]);
             }
-            *reinterpret_cast<uint4 *>(Tout + cbase + r * kC + c0) = *reinterpret_cast<uint4 *>(tv);
-            *reinterpret_cast<uint4 *>(Aqout + cbase + r * kC + c0) = *reinterpret_cast<uint4 *>(qv);
+        } else {
+            // diagonal blocks D_i Diag(beta) and the zero blocks above them
+            for (int task = tid - 192; task < kC * 8; task += 64) {
+                const int r = task >> 3, g8 = task & 7, i = r >> 4, jb = g8 >> 1;
+                if (jb < i) continue;
+                uint4 o = make_uint4(0u, 0u, 0u, 0u);
+                if (jb == i) {
+                    const int ch = 8 * (g8 & 1), cl = 16 * jb + ch;
+                    const float4 d0 = *reinterpret_cast<const float4 *>(&sD[i][r & 15][ch]);
+                    const float4 d1 = *reinterpret_cast<const float4 *>(&sD[i][r & 15][ch + 4]);
+                    o.x = pack2(d0.x * sBeta[cl + 0], d0.y * sBeta[cl + 1]);
+                    o.y = pack2(d0.z * sBeta[cl + 2], d0.w * sBeta[cl + 3]);
+                    o.z = pack2(d1.x * sBeta[cl + 4], d1.y * sBeta[cl + 5]);
+                    o.w = pack2(d1.z * sBeta[cl + 6], d1.w * sBeta[cl + 7]);
+                }
+                *reinterpret_cast<uint4 *>(Tout + cbase + r * kC + 8 * g8) = o;
+            }
         }
+        __syncthreads();
+        // first products of every block below the diagonal
+        if (warp < 6) {
+            // warp -> (i, j): (1,0) (2,1) (3,2) (2,0) (3,1) (3,0)
+            const int i = warp < 3 ? warp + 1 : (warp == 3 ? 2 : 3);
+            const int j = warp < 3 ? warp : (warp == 4 ? 1 : 0);
+            mm16_sub(acc, &sQ[16 * i][16 * j], kLdA, &sD[j][0][0], kLdD, g, t);   // -Nt_ij D_j
+            if (warp < 3) {
+                store_t(acc, i, j);
+                if (warp < 2) store_s(acc, sU[warp]);   // U_10, U_21
+            }
+        }
+        __syncthreads();
+        if (warp == 3) {          // U_20 = -Nt_20 D_0 - Nt_21 U_10
+            mm16_sub(acc, &sQ[32][16], kLdA, &sU[0][0][0], kLdD, g, t);
+            store_t(acc, 2, 0);
+            store_s(acc, sU[2]);
+        } else if (warp == 4) {   // U_31 = -Nt_31 D_1 - Nt_32 U_21
+            mm16_sub(acc, &sQ[48][32], kLdA, &sU[1][0][0], kLdD, g, t);
+            store_t(acc, 3, 1);
+        } else if (warp == 5) {   // U_30 so far: -Nt_30 D_0 - Nt_31 U_10
+            mm16_sub(acc, &sQ[48][16], kLdA, &sU[0][0][0], kLdD, g, t);
+        }
+        __syncthreads();
+        if (warp == 5) {          // U_30 -= Nt_32 U_20
+            mm16_sub(acc, &sQ[48][32], kLdA, &sU[2][0][0], kLdD, g, t);
+            store_t(acc, 3, 0);
+        }
+        // no barrier here: the next chunk's first writes (operand tiles, the
+        // other beta buffer) touch nothing warp 5 still reads, and its next
+        // barrier waits for warp 5
     }
+}
+
+int sm_count()
+{
+    static int counts[64];
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    std::lock_guard<std::mutex> lock(mu);
+    if (counts[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        counts[dev] = n;
+    }
+    return counts[dev];
 }
 
 }  // namespace
 
-size_t ut_prep_smem_bytes() { return sizeof(PrepSmem); }
-
 cudaError_t launch_ut_prep(const ChunkArgs &a, __nv_bfloat16 *Tout, __nv_bfloat16 *Aqout, cudaStream_t stream)
 {
     const int nchunks = (a.T + kC - 1) / kC;
-    const long long blocks = (long long)a.B * a.H * nchunks;
-    if (blocks == 0) return cudaSuccess;
-    const size_t smem = sizeof(PrepSmem);
-    if (a.scalar_gate) {
-        cudaError_t e = cudaFuncSetAttribute(ut_prep_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
-        if (e != cudaSuccess) return e;
-        ut_prep_kernel<true><<<(unsigned)blocks, 128, smem, stream>>>(
-            (const __nv_bfloat16 *)a.k, (const __nv_bfloat16 *)a.q, a.g, a.beta, Tout, Aqout, a.T, nchunks);
-    } else {
-        cudaError_t e = cudaFuncSetAttribute(ut_prep_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
-        if (e != cudaSuccess) return e;
-        ut_prep_kernel<false><<<(unsigned)blocks, 128, smem, stream>>>(
-            (const __nv_bfloat16 *)a.k, (const __nv_bfloat16 *)a.q, a.g, a.beta, Tout, Aqout, a.T, nchunks);
-    }
+    const long long total = (long long)a.B * a.H * nchunks;
+    if (total == 0) return cudaSuccess;
+    if (total > 0x7fffffffLL) return cudaErrorInvalidValue;
+    const long long slots = 2LL * sm_count();   // two resident CTAs per SM
+    const int grid = (int)(total < slots ? total : slots);
+    auto kern = a.scalar_gate ? ut_prep_kernel<true> : ut_prep_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_ALLOC);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kThreads, SMEM_ALLOC, stream>>>((const __nv_bfloat16 *)a.k, (const __nv_bfloat16 *)a.q, a.g,
+                                                 a.beta, Tout, Aqout, a.T, nchunks, (int)total);
     return cudaGetLastError();
 }
 

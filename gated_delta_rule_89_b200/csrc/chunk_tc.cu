@@ -3,34 +3,40 @@
 //
 // Two kernels per call:
 //   1. ut_prep (ut_prep.cu): every chunk of every head in parallel -> the
-//      UT-transform matrix T' = (I + A)^{-1} Diag(beta) and the masked
-//      intra-chunk matrix Aqk, bf16, into the workspace.
+//      UT-transform matrix T' = (I + A)^{-1} Diag(beta), the masked
+//      intra-chunk matrix Aqk and, with G the cumulative log-decay inside the
+//      chunk, K<- = K*exp(G), Q<- = Q*exp(G), K_tail = K*exp(G_C - G) and
+//      gamma_C = exp(G_C), all into the workspace.
 //   2. chunk_scan (this file): one CTA per (b, h) walks the chunks in order.
 //      The fp32 state S [d_v x d_k] lives in tensor memory for the whole
-//      sequence.  Per chunk, with G the cumulative log-decay, K<- = K*exp(G),
-//      Q<- = Q*exp(G), K_tail = K*exp(G_C - G) and gamma_C = exp(G_C):
+//      sequence.  Per chunk:
 //        W^T     = K<-^T T'^T                (= (T' K<-)^T)
 //        V_new^T = V^T T'^T - S W^T          (U^T, then -S W^T accumulated)
 //        O^T     = S Q<-^T + V_new^T Aqk^T
-//        S       = S Diag(gamma_C) + V_new^T K_tail
+//        S       = S Diag(gamma_C) + V_new^T K_tail   (the scaling in place in
+//                  TMEM, the increment accumulated onto it by the MMA)
 //      which is the chunk state update and chunk output of "Reading notes:
 //      Kimi Delta Attention" (mzeromiko), section 4, and of "Token Mixer I",
 //      section "Kimi Delta Attention: Improving Delta Rule with Fine-grained
 //      Gating", in the d_v x d_k orientation.  Every product is one
 //      tcgen05.mma chain with M = 128 (rows of S, or key channels), fp32
-//      accumulators in TMEM; inputs arrive by TMA with 128-byte swizzle and
-//      the same tiles serve as K-major or MN-major operands.
+//      accumulators in TMEM; all inputs arrive by TMA with 128-byte swizzle
+//      into double-buffered tiles, and the same tiles serve as K-major or
+//      MN-major operands.
 //
 // Warp roles (320 threads):
-//   warp 0      TMA producer (one lane)
-//   warp 1      TMEM allocation and the MMA issuer (one lane)
-//   warps 2-5   "E": the gate products exp(G) and exp(G_C - G) (running
-//               products of alpha = exp(g)), the scaled operands K<-, Q<-
-//               (in place over the TMA tiles) and K_tail, and the output
-//               epilogue (TMEM -> bf16 -> global)
-//   warps 6-9   "M": the conversions on the sequential path: W^T (TMEM) ->
-//               W (bf16 smem), S -> bf16 S plus S*gamma_C back into TMEM,
-//               V_new^T (TMEM) -> bf16 smem
+//   warp 0      TMA producer (one lane): all tiles of a chunk land in one of
+//               two stages and complete one barrier; gamma_C in two slots
+//   warp 1      TMEM allocation and the MMA issuer (one lane), in the order
+//               X^T(n), O^T(n), W^T(n+1), dS(n), O(n), U^T(n+1), so the
+//               products that do not depend on the state run while the state
+//               is updated
+//   warps 2-9   every conversion, split by columns between warps 2-5 and
+//               6-9: on the sequential path S (TMEM) -> bf16 smem and
+//               V_new^T (TMEM) -> bf16 smem; off it, in the gaps while the
+//               tensor core runs, S *= gamma_C in TMEM, W^T (TMEM) -> W
+//               (bf16 smem) and the output epilogue O^T (TMEM) -> bf16 -> global.
+// The sequential chain per chunk is dS -> S to bf16 -> X^T -> V_new -> dS.
 // Every wait is bounded (about a second); on timeout the kernel records
 // GDR_ERR_TIMEOUT in a device status word, lets the copies and MMAs it
 // issued finish, frees its tensor memory and returns.
@@ -44,7 +50,7 @@ namespace gdr {
 
 __device__ int g_device_status;   // 0 = OK, else the first gdr_status a kernel recorded
 
-cudaError_t launch_ut_prep(const ChunkArgs &a, __nv_bfloat16 *Tout, __nv_bfloat16 *Aqout, cudaStream_t stream);
+cudaError_t launch_ut_prep(const ChunkArgs &a, const TcWorkspace &w, cudaStream_t stream);
 
 namespace {
 
@@ -52,52 +58,55 @@ using namespace sm100;
 
 constexpr int kC = 64;
 constexpr int kD = 128;
-constexpr int kThreads = 320;
+constexpr int kThreads = 320;   // 10 warps: TMA, MMA, 4 x E, 4 x M
 constexpr long long kWaitBudget = 2000000000LL;   // clock cycles per wait (~1 s)
 
-// shared memory map (bytes from a 1024-aligned base)
-constexpr uint32_t OFF_G = 0;                      // [64][128] fp32 gate tile          32 KB
-constexpr uint32_t OFF_K = OFF_G + 32768;          // 2 x k -> K<-  (2 panels x 8 KB)   2 x 16 KB
-constexpr uint32_t OFF_Q = OFF_K + 2 * 16384;      // 2 x q -> Q<-                      2 x 16 KB
-constexpr uint32_t OFF_V = OFF_Q + 2 * 16384;      // v (2 panels)                      16 KB
-constexpr uint32_t OFF_T = OFF_V + 16384;          // T' (1 panel)                      8 KB
-constexpr uint32_t OFF_AQ = OFF_T + 8192;          // 2 x Aqk                           2 x 8 KB
-constexpr uint32_t OFF_KT = OFF_AQ + 2 * 8192;     // K_tail (2 panels)                 16 KB
-constexpr uint32_t OFF_W = OFF_KT + 16384;         // W, MN-major [128 ch x 64 tok]     16 KB
-constexpr uint32_t OFF_S = OFF_W + 16384;          // bf16 S (2 panels x 16 KB)         32 KB
-constexpr uint32_t OFF_VN = OFF_S + 32768;         // V_new^T (1 panel, 128 rows)       16 KB
-constexpr uint32_t OFF_GAM = OFF_VN + 16384;       // gamma_C ring [4][128] fp32        2 KB
-constexpr uint32_t OFF_BAR = OFF_GAM + 2048;       // mbarriers, TMEM slot, abort flag
-constexpr uint32_t SMEM_USED = OFF_BAR + 512;
+// shared memory map (bytes from a 1024-aligned base).  The input tiles of a
+// chunk form one stage (gamma_C in a slot of its own); two stages alternate
+// by chunk parity.
+constexpr uint32_t ST_K = 0;                       // K<-  (2 panels x 8 KB)              16 KB
+constexpr uint32_t ST_Q = 16384;                   // Q<-                                  16 KB
+constexpr uint32_t ST_KT = 32768;                  // K_tail                               16 KB
+constexpr uint32_t ST_V = 49152;                   // v                                    16 KB
+constexpr uint32_t ST_T = 65536;                   // T' (1 panel)                          8 KB
+constexpr uint32_t ST_AQ = 73728;                  // Aqk                                   8 KB
+constexpr uint32_t STAGE = 81920;                  // stage stride (1024-aligned)
+constexpr uint32_t STAGE_TX = 4 * 16384 + 2 * 8192;   // bytes one stage receives
+constexpr uint32_t OFF_W = 2 * STAGE;              // W, MN-major [128 ch x 64 tok]         16 KB
+constexpr uint32_t OFF_S = OFF_W + 16384;          // bf16 S (2 panels x 16 KB)             32 KB
+constexpr uint32_t OFF_VN = OFF_S + 32768;         // V_new^T (1 panel, 128 rows)           16 KB
+constexpr uint32_t OFF_GAM = OFF_VN + 16384;       // gamma_C of each stage, [2][128] fp32   1 KB
+constexpr uint32_t OFF_BAR = OFF_GAM + 1024;       // mbarriers, TMEM slot, abort flag
+constexpr uint32_t SMEM_USED = OFF_BAR + 256;
 constexpr uint32_t SMEM_ALLOC = SMEM_USED + 1024;  // alignment slack
 static_assert(SMEM_ALLOC <= 232448, "dynamic shared memory above the 227 KB per-block limit");
 
 // TMEM columns (fp32)
-constexpr uint32_t TM_S = 0;      // state S_n, 128 columns (written only by the conversion warps)
-constexpr uint32_t TM_D = 128;    // state increment V_new^T K_tail of the last chunk, 128 columns
-constexpr uint32_t TM_W = 256;    // W^T, 64 columns
-constexpr uint32_t TM_V = 320;    // V_new^T accumulator, 64 columns
-constexpr uint32_t TM_O = 384;    // O^T accumulators, 2 x 64 columns
-constexpr uint32_t TM_COLS = 512;
+constexpr uint32_t TM_S = 0;      // state S_n, 128 columns: scaled by gamma_C in place, dS accumulated onto it
+constexpr uint32_t TM_W = 128;    // W^T, 64 columns
+constexpr uint32_t TM_V = 192;    // V_new^T accumulator, 64 columns
+constexpr uint32_t TM_O = 256;    // O^T accumulators, 2 x 64 columns
+constexpr uint32_t TM_COLS = 512; // allocation granularity (power of two); 384 used
 
 enum Bar {
-    B_FULL_G, B_EMPTY_G,
-    B_FULL_K, B_FULL_K1, B_EMPTY_K, B_EMPTY_K1,
-    B_FULL_Q, B_FULL_Q1, B_EMPTY_Q, B_EMPTY_Q1,
-    B_FULL_V, B_EMPTY_V, B_FULL_T, B_EMPTY_T,
-    B_FULL_AQ, B_FULL_AQ1, B_EMPTY_AQ, B_EMPTY_AQ1,
-    B_KQ_READY, B_KQ_READY1, B_KT_READY, B_KT_FREE,
-    B_WT_FULL, B_WT_EMPTY, B_W_READY, B_W_FREE,
-    B_S_READY, B_S_FULL, B_X_FULL, B_VN_READY,
-    B_VACC_EMPTY, B_O_FULL, B_O_FULL1, B_OACC_EMPTY, B_OACC_EMPTY1,
-    B_XCH, B_XCH1,
+    B_FULL, B_FULL1,          // stage landed (TMA transaction bytes)
+    B_EMPTY, B_EMPTY1,        // stage released (MMA commit)
+    B_GFULL, B_GFULL1,        // gamma_C slot landed
+    B_GEMPTY, B_GEMPTY1,      // gamma_C slot read by the state-update threads
+    B_WT_FULL,                // W^T(n), U^T(n) in TMEM
+    B_SW_READY,               // W(n) and S_n (bf16) in smem, TMEM W read
+    B_X_FULL,                 // V_new^T(n) in TMEM
+    B_VN_READY,               // V_new^T(n) bf16 in smem, TM_V read, S_n scaled by gamma_C(n)
+    B_S_FULL,                 // S_{n+1} complete in TMEM
+    B_O_FULL, B_O_FULL1,      // O^T(n) complete
+    B_OACC_EMPTY, B_OACC_EMPTY1,   // O^T accumulator drained by the epilogue
     B_FINAL,
     B_COUNT
 };
-static_assert(8 * B_COUNT + 8 <= 512, "barrier area");
+static_assert(8 * B_COUNT + 8 <= 256, "barrier area");
 
 struct Maps {
-    CUtensorMap k, q, v, g, t, aq;
+    CUtensorMap k, q, kt, v, t, aq;   // K<-, Q<-, K_tail, v: [BH][T][128]; T', Aqk: [chunks*64][64]
 };
 
 __device__ __forceinline__ void record_error(int code) { atomicCAS(&g_device_status, 0, code); }
@@ -121,17 +130,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
-// Eight bf16 (one 16-byte chunk) times eight fp32 factors, rounded back to bf16.
-__device__ __forceinline__ uint4 scale8(uint4 v, const float (&f)[8])
-{
-    uint4 o;
-    o.x = pack_bf16(__uint_as_float(v.x << 16) * f[0], __uint_as_float(v.x & 0xffff0000u) * f[1]);
-    o.y = pack_bf16(__uint_as_float(v.y << 16) * f[2], __uint_as_float(v.y & 0xffff0000u) * f[3]);
-    o.z = pack_bf16(__uint_as_float(v.z << 16) * f[4], __uint_as_float(v.z & 0xffff0000u) * f[5]);
-    o.w = pack_bf16(__uint_as_float(v.w << 16) * f[6], __uint_as_float(v.w & 0xffff0000u) * f[7]);
-    return o;
-}
-
 // Sixteen fp32 TMEM words -> two 16-byte bf16 chunks.
 __device__ __forceinline__ void pack16(const uint32_t (&r)[16], uint4 &lo, uint4 &hi)
 {
@@ -147,7 +145,7 @@ __device__ __forceinline__ void pack16(const uint32_t (&r)[16], uint4 &lo, uint4
 
 template <bool SCALAR>
 __global__ void __launch_bounds__(kThreads, 1)
-chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g_scalar,
+chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ gamma_c,
                   const float *__restrict__ S0, __nv_bfloat16 *__restrict__ O, float *__restrict__ ST,
                   int T_len, int nchunks)
 {
@@ -157,7 +155,6 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_BAR + 8 * B_COUNT);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + OFF_BAR + 8 * B_COUNT + 4);
-    float *gam = reinterpret_cast<float *>(sm + OFF_GAM);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -166,16 +163,11 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
 
     if (tid == 0) {
         const uint32_t counts[B_COUNT] = {
-            1, 128,             // g full / empty (E threads release)
-            1, 1, 1, 1,         // k full x2, empty x2
-            1, 1, 1, 1,         // q
-            1, 1, 1, 1,         // v full/empty, T' full/empty
-            1, 1, 1, 1,         // Aqk
-            128, 128, 128, 1,   // kq ready (E) x2, kt ready (E), kt free (MMA)
-            1, 128, 128, 1,     // wt full (MMA), wt empty (M), w ready (M), w free (MMA)
-            128, 1, 1, 128,     // s ready (M), s full (MMA), x full (MMA), vn ready (M)
-            128, 1, 1, 128, 128,        // vacc empty (M), o full (MMA) x2, oacc empty (E) x2
-            128, 128,                   // row-group exchange (E) x2
+            1, 1, 1, 1,       // stage full (TMA), stage empty (MMA commit)
+            1, 1, 256, 256,   // gamma full (TMA), gamma empty (warps 2-9)
+            1, 256, 1, 256,   // wt full (MMA), sw ready (warps 2-9), x full (MMA), vn ready (warps 2-9)
+            1,                // s full (MMA)
+            1, 1, 256, 256,   // o full (MMA) x2, oacc empty (warps 2-9) x2
             1};
         for (int i = 0; i < B_COUNT; ++i) mbar_init(&bar[i], counts[i]);
         *abort_flag = 0;
@@ -191,8 +183,10 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
     const uint32_t tmem = *tmem_slot;
     const uint32_t sbase = smem_u32(sm);
 
-    // Single-thread roles (TMA producer, MMA issuer) wait with `wait`.
+    // Single-thread roles (TMA producer, MMA issuer) wait with `wait`: one
+    // try first, and only a thread that has to wait looks at the abort flag.
     auto wait = [&](int b, uint32_t parity) -> bool {
+        if (mbar_try_wait(&bar[b], parity)) return true;
         if (*abort_flag) return false;
         if (mbar_wait(&bar[b], parity, kWaitBudget)) return true;
         record_error(6 /* GDR_ERR_TIMEOUT */);
@@ -218,45 +212,35 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
             for (int n = 0; n < nchunks; ++n) {
                 const int t0 = n * kC;
                 const int b = n & 1;
-                const uint32_t par = (uint32_t)(n & 1), upar = (uint32_t)((n >> 1) & 1);
-                const int crow = (head * nchunks + n) * kC;   // row of this chunk in the workspace
-                if (!SCALAR) {
-                    if (!wait(B_EMPTY_G, par ^ 1)) break;
-                    mbar_arrive_expect_tx(&bar[B_FULL_G], 32768);
-                    tma_load_3d(sm + OFF_G, &maps.g, &bar[B_FULL_G], 0, t0, head);
-                }
-                if (!wait(B_EMPTY_K + b, upar ^ 1)) break;
-                mbar_arrive_expect_tx(&bar[B_FULL_K + b], 16384);
-                tma_load_3d(sm + OFF_K + b * 16384, &maps.k, &bar[B_FULL_K + b], 0, t0, head);
-                tma_load_3d(sm + OFF_K + b * 16384 + 8192, &maps.k, &bar[B_FULL_K + b], 64, t0, head);
-                if (!wait(B_EMPTY_Q + b, upar ^ 1)) break;
-                mbar_arrive_expect_tx(&bar[B_FULL_Q + b], 16384);
-                tma_load_3d(sm + OFF_Q + b * 16384, &maps.q, &bar[B_FULL_Q + b], 0, t0, head);
-                tma_load_3d(sm + OFF_Q + b * 16384 + 8192, &maps.q, &bar[B_FULL_Q + b], 64, t0, head);
-                if (!wait(B_EMPTY_T, par ^ 1)) break;
-                mbar_arrive_expect_tx(&bar[B_FULL_T], 8192);
-                tma_load_2d(sm + OFF_T, &maps.t, &bar[B_FULL_T], 0, crow);
-                if (!wait(B_EMPTY_V, par ^ 1)) break;
-                mbar_arrive_expect_tx(&bar[B_FULL_V], 16384);
-                tma_load_3d(sm + OFF_V, &maps.v, &bar[B_FULL_V], 0, t0, head);
-                tma_load_3d(sm + OFF_V + 8192, &maps.v, &bar[B_FULL_V], 64, t0, head);
-                if (!wait(B_EMPTY_AQ + b, upar ^ 1)) break;
-                mbar_arrive_expect_tx(&bar[B_FULL_AQ + b], 8192);
-                tma_load_2d(sm + OFF_AQ + b * 8192, &maps.aq, &bar[B_FULL_AQ + b], 0, crow);
+                const uint32_t upar = (uint32_t)((n >> 1) & 1);
+                const int crow = (head * nchunks + n) * kC;   // row of this chunk in T' / Aqk
+                unsigned char *st = sm + b * STAGE;
+                uint64_t *full = &bar[B_FULL + b];
+                if (!wait(B_EMPTY + b, upar ^ 1)) break;
+                mbar_arrive_expect_tx(full, STAGE_TX);
+                tma_load_3d(st + ST_K, &maps.k, full, 0, t0, head);
+                tma_load_3d(st + ST_K + 8192, &maps.k, full, 64, t0, head);
+                tma_load_2d(st + ST_T, &maps.t, full, 0, crow);
+                tma_load_3d(st + ST_V, &maps.v, full, 0, t0, head);
+                tma_load_3d(st + ST_V + 8192, &maps.v, full, 64, t0, head);
+                tma_load_3d(st + ST_Q, &maps.q, full, 0, t0, head);
+                tma_load_3d(st + ST_Q + 8192, &maps.q, full, 64, t0, head);
+                tma_load_3d(st + ST_KT, &maps.kt, full, 0, t0, head);
+                tma_load_3d(st + ST_KT + 8192, &maps.kt, full, 64, t0, head);
+                tma_load_2d(st + ST_AQ, &maps.aq, full, 0, crow);
+                // gamma_C has its own slots, released by the state update, so the
+                // stage itself only waits for the MMAs that read it
+                if (!wait(B_GEMPTY + b, upar ^ 1)) break;
+                mbar_arrive_expect_tx(&bar[B_GFULL + b], 512);
+                bulk_load(sm + OFF_GAM + b * 512, gamma_c + (size_t)(head * nchunks + n) * kD, 512, &bar[B_GFULL + b]);
                 GDR_TRACE_AT(0, n);
                 issued = n + 1;
             }
             if (*abort_flag && issued > 0) {
                 // let the copies of the last issued chunk land before the CTA exits
-                const int n = issued - 1, b = n & 1;
-                const uint32_t par = (uint32_t)(n & 1), upar = (uint32_t)((n >> 1) & 1);
-                const long long small = kWaitBudget / 4;
-                if (!SCALAR) mbar_wait(&bar[B_FULL_G], par, small);
-                mbar_wait(&bar[B_FULL_K + b], upar, small);
-                mbar_wait(&bar[B_FULL_Q + b], upar, small);
-                mbar_wait(&bar[B_FULL_T], par, small);
-                mbar_wait(&bar[B_FULL_V], par, small);
-                mbar_wait(&bar[B_FULL_AQ + b], upar, small);
+                const int n = issued - 1;
+                mbar_wait(&bar[B_FULL + (n & 1)], (uint32_t)((n >> 1) & 1), kWaitBudget / 4);
+                mbar_wait(&bar[B_GFULL + (n & 1)], (uint32_t)((n >> 1) & 1), kWaitBudget / 4);
             }
         }
     } else if (warp == 1) {
@@ -266,86 +250,196 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
             constexpr uint32_t ID_X = idesc_bf16(128, 64, false, true, true);    // -A, B (W) MN-major
             constexpr uint32_t ID_O = idesc_bf16(128, 64, false, false);
             constexpr uint32_t ID_S = idesc_bf16(128, 128, false, true);         // B MN-major
-            for (int n = 0; n < nchunks; ++n) {
+            // W^T = K<-^T T'^T and U^T = V^T T'^T of chunk n (stage n & 1), as
+            // separate groups: W^T feeds the W conversion early, U^T has to
+            // wait until V_new^T of the previous chunk has left TM_V
+            auto mma_w = [&](int n) {
+                const uint32_t st = sbase + (n & 1) * STAGE;
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_bf16(tmem + TM_W, sdesc_sw128(st + ST_K + s * 2048, 8192, 1024),
+                             sdesc_sw128(st + ST_T + s * 32, 16, 1024), ID_WU, s > 0);
+                mma_commit(&bar[B_WT_FULL]);
+            };
+            auto mma_u = [&](int n) {
+                const uint32_t st = sbase + (n & 1) * STAGE;
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_bf16(tmem + TM_V, sdesc_sw128(st + ST_V + s * 2048, 8192, 1024),
+                             sdesc_sw128(st + ST_T + s * 32, 16, 1024), ID_WU, s > 0);
+            };
+            bool ok = nchunks > 0 && wait(B_FULL, 0);
+            if (ok) {
+                tc_fence_after();
+                GDR_TRACE_AT(1, 0);
+                mma_w(0);
+                mma_u(0);
+            }
+            for (int n = 0; n < nchunks && ok; ++n) {
                 const int b = n & 1;
                 const uint32_t par = (uint32_t)(n & 1), upar = (uint32_t)((n >> 1) & 1);
-                // ---- W^T = K<-^T T'^T ; U^T = V^T T'^T
-                if (!wait(B_KQ_READY + b, upar) || !wait(B_FULL_T, par) || !wait(B_FULL_V, par) ||
-                    !wait(B_WT_EMPTY, par ^ 1) || !wait(B_VACC_EMPTY, par ^ 1))
-                    break;
-                tc_fence_after();
-                GDR_TRACE_AT(1, n);
-                const uint32_t kb = sbase + OFF_K + b * 16384;
-#pragma unroll
-                for (int s = 0; s < 4; ++s)
-                    mma_bf16(tmem + TM_W, sdesc_sw128(kb + s * 2048, 8192, 1024),
-                             sdesc_sw128(sbase + OFF_T + s * 32, 16, 1024), ID_WU, s > 0);
-#pragma unroll
-                for (int s = 0; s < 4; ++s)
-                    mma_bf16(tmem + TM_V, sdesc_sw128(sbase + OFF_V + s * 2048, 8192, 1024),
-                             sdesc_sw128(sbase + OFF_T + s * 32, 16, 1024), ID_WU, s > 0);
-                mma_commit(&bar[B_WT_FULL]);
-                mma_commit(&bar[B_EMPTY_K + b]);
-                mma_commit(&bar[B_EMPTY_V]);
-                mma_commit(&bar[B_EMPTY_T]);
+                const uint32_t st = sbase + b * STAGE;
+                const bool more = n + 1 < nchunks;
+                const uint32_t npar = (uint32_t)(((n + 1) >> 1) & 1);   // next stage's phase
                 // ---- V_new^T += -S W^T ; O^T = S Q<-^T
-                if (!wait(B_S_READY, par) || !wait(B_W_READY, par) || !wait(B_OACC_EMPTY + b, upar ^ 1)) break;
+                if (!wait(B_SW_READY, par) || !wait(B_OACC_EMPTY + b, upar ^ 1)) break;
                 tc_fence_after();
                 GDR_TRACE_AT(2, n);
-                const uint32_t qb = sbase + OFF_Q + b * 16384;
-                // V_new^T first: it is on the sequential path
 #pragma unroll
                 for (int s = 0; s < 8; ++s)
                     mma_bf16(tmem + TM_V, sdesc_sw128(sbase + OFF_S + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024),
                              sdesc_sw128(sbase + OFF_W + s * 2048, 8192, 1024), ID_X, 1);
                 mma_commit(&bar[B_X_FULL]);
-                mma_commit(&bar[B_W_FREE]);
 #pragma unroll
                 for (int s = 0; s < 8; ++s)
-                    mma_bf16(tmem + TM_O + 64 * b, sdesc_sw128(sbase + OFF_S + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024),
-                             sdesc_sw128(qb + (s >> 2) * 8192 + (s & 3) * 32, 16, 1024), ID_O, s > 0);
-                mma_commit(&bar[B_EMPTY_Q + b]);
-                // ---- O^T += V_new^T Aqk^T ; S += V_new^T K_tail
-                if (!wait(B_VN_READY, par) || !wait(B_FULL_AQ + b, upar) || !wait(B_KT_READY, par)) break;
+                    mma_bf16(tmem + TM_O + 64 * b,
+                             sdesc_sw128(sbase + OFF_S + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024),
+                             sdesc_sw128(st + ST_Q + (s >> 2) * 8192 + (s & 3) * 32, 16, 1024), ID_O, s > 0);
+                // ---- W^T of the next chunk now if its stage has landed (never
+                // block here: this stage is only released below)
+                bool w_done = false;
+                if (more && mbar_try_wait(&bar[B_FULL + (b ^ 1)], npar)) {
+                    tc_fence_after();
+                    GDR_TRACE_AT(1, n + 1);
+                    mma_w(n + 1);
+                    w_done = true;
+                }
+                // ---- S += V_new^T K_tail (the sequential path; S already scaled by
+                // gamma_C); O^T += V_new^T Aqk^T
+                if (!wait(B_VN_READY, par)) break;
                 tc_fence_after();
                 GDR_TRACE_AT(3, n);
-                // the state increment first: it is on the sequential path
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
-                    mma_bf16(tmem + TM_D, sdesc_sw128(sbase + OFF_VN + s * 32, 16, 1024),
-                             sdesc_sw128(sbase + OFF_KT + s * 2048, 8192, 1024), ID_S, s > 0);
+                    mma_bf16(tmem + TM_S, sdesc_sw128(sbase + OFF_VN + s * 32, 16, 1024),
+                             sdesc_sw128(st + ST_KT + s * 2048, 8192, 1024), ID_S, 1);
                 mma_commit(&bar[B_S_FULL]);
-                mma_commit(&bar[B_KT_FREE]);
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
                     mma_bf16(tmem + TM_O + 64 * b, sdesc_sw128(sbase + OFF_VN + s * 32, 16, 1024),
-                             sdesc_sw128(sbase + OFF_AQ + b * 8192 + s * 32, 16, 1024), ID_O, 1);
+                             sdesc_sw128(st + ST_AQ + s * 32, 16, 1024), ID_O, 1);
                 mma_commit(&bar[B_O_FULL + b]);
-                mma_commit(&bar[B_EMPTY_AQ + b]);
+                mma_commit(&bar[B_EMPTY + b]);   // every read of this stage is issued
+                // ---- U^T of the next chunk (and W^T if its stage came late)
+                if (more) {
+                    if (!w_done) {
+                        if (!wait(B_FULL + (b ^ 1), npar)) break;
+                        tc_fence_after();
+                        GDR_TRACE_AT(1, n + 1);
+                        mma_w(n + 1);
+                    }
+                    mma_u(n + 1);
+                }
             }
             // every MMA issued above has completed before TMEM is released
             mma_commit(&bar[B_FINAL]);
             mbar_wait(&bar[B_FINAL], 0, kWaitBudget);
         }
-    } else if (warp < 6) {
-        // ================================================================ E: gate products, operands, epilogue
-        const uint32_t lq = 32u * (warp & 3);        // TMEM lane quarter of this warp
-        const int orow = (int)lq + lane;             // d_v index for the epilogue
+    } else {
+        // ================================================================ state update, conversions, epilogue
+        // The state S_n lives at TM_S.  At chunk n these warps copy it to bf16
+        // smem for the MMAs of chunk n (on the sequential path), then scale it
+        // in place by gamma_C(n) (off the path, while X^T(n) runs); the MMA of
+        // S += V_new^T K_tail then leaves S_{n+1} in TM_S.  Warps 2-5 take key
+        // channels 64..127 of S and tokens 32..63 of V_new^T, warps 6-9 the
+        // other halves; the same split applies to W^T and O^T.
+        const bool ga = warp < 6;                     // warps 2-5
+        const uint32_t lq = 32u * (warp & 3);         // TMEM lane quarter of this warp
+        const int i = (int)lq + lane;                 // TMEM lane: row of S / V_new^T / O^T, key channel of W^T
+        const uint32_t trow = tmem + (lq << 16);
+        const int sc0 = ga ? 64 : 0;                  // first state column of this warp
+        const int vc0 = ga ? 32 : 0;                  // first V_new^T / W^T / O^T column (token)
+        // initial state into TMEM
+#pragma unroll
+        for (int cb = 0; cb < 4; ++cb) {
+            uint32_t r[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                r[j] = __float_as_uint(S0 ? S0[((size_t)head * kD + i) * kD + sc0 + 16 * cb + j] : 0.f);
+            tmem_st16(trow + TM_S + sc0 + 16 * cb, r);
+        }
+        tmem_st_wait();
+        // One pass over this warp's 64 columns of S_n (TMEM): the bf16 copy goes
+        // to smem and is released to the MMAs at once (the sequential path);
+        // then S_n *= gamma_C(n) is stored back in place for the accumulation
+        // of chunk n's increment.
+        auto state_pass = [&](int n) -> bool {
+            unsigned char *sp = sm + OFF_S + (sc0 >> 6) * 16384;
+            uint32_t r[4][16];
+#pragma unroll
+            for (int cb = 0; cb < 4; ++cb) tmem_ld16(trow + TM_S + sc0 + 16 * cb, r[cb]);
+            tmem_ld_wait(r[0]);
+            reg_touch(r[1]);
+            reg_touch(r[2]);
+            reg_touch(r[3]);
+#pragma unroll
+            for (int cb = 0; cb < 4; ++cb) {
+                uint4 lo, hi;
+                pack16(r[cb], lo, hi);
+                *reinterpret_cast<uint4 *>(sp + sw128_off(i, 16 * cb)) = lo;
+                *reinterpret_cast<uint4 *>(sp + sw128_off(i, 16 * cb + 8)) = hi;
+            }
+            fence_async_smem();
+            tc_fence_before();
+            mbar_arrive(&bar[B_SW_READY]);   // W(n) was converted before
+            if (tid == 192) GDR_TRACE_AT(12, n);
+            if (!waitw(B_GFULL + (n & 1), (uint32_t)((n >> 1) & 1))) return false;
+            const float4 *gm = reinterpret_cast<const float4 *>(sm + OFF_GAM + (n & 1) * 512) + (sc0 >> 2);
+#pragma unroll
+            for (int cb = 0; cb < 4; ++cb) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float4 gv = gm[4 * cb + q];
+                    r[cb][4 * q + 0] = __float_as_uint(__uint_as_float(r[cb][4 * q + 0]) * gv.x);
+                    r[cb][4 * q + 1] = __float_as_uint(__uint_as_float(r[cb][4 * q + 1]) * gv.y);
+                    r[cb][4 * q + 2] = __float_as_uint(__uint_as_float(r[cb][4 * q + 2]) * gv.z);
+                    r[cb][4 * q + 3] = __float_as_uint(__uint_as_float(r[cb][4 * q + 3]) * gv.w);
+                }
+                tmem_st16(trow + TM_S + sc0 + 16 * cb, r[cb]);
+            }
+            tmem_st_wait();
+            mbar_arrive(&bar[B_GEMPTY + (n & 1)]);
+            return true;
+        };
+        // W^T(n) -> W: the row of key channel i = 64 tokens = one 128-byte row of
+        // the MN-major operand.  WT_FULL(n) was committed after every MMA of
+        // chunk n - 1 that reads W, so the buffer is free.
+        auto convert_w = [&](int n) -> bool {
+            if (!waitw(B_WT_FULL, (uint32_t)(n & 1))) return false;
+            tc_fence_after();
+            if (tid == 192) GDR_TRACE_AT(4, n);
+            {
+                uint32_t r0[16], r1[16];
+                tmem_ld16(trow + TM_W + vc0, r0);
+                tmem_ld16(trow + TM_W + vc0 + 16, r1);
+                tmem_ld_wait(r0);
+                reg_touch(r1);
+                uint4 lo, hi;
+                pack16(r0, lo, hi);
+                *reinterpret_cast<uint4 *>(sm + OFF_W + sw128_off(i, vc0)) = lo;
+                *reinterpret_cast<uint4 *>(sm + OFF_W + sw128_off(i, vc0 + 8)) = hi;
+                pack16(r1, lo, hi);
+                *reinterpret_cast<uint4 *>(sm + OFF_W + sw128_off(i, vc0 + 16)) = lo;
+                *reinterpret_cast<uint4 *>(sm + OFF_W + sw128_off(i, vc0 + 24)) = hi;
+            }
+            if (tid == 192) GDR_TRACE_AT(5, n);
+            return true;
+        };
         auto epilogue = [&](int m) -> bool {
             const int bb = m & 1;
             if (!waitw(B_O_FULL + bb, (uint32_t)((m >> 1) & 1))) return false;
             tc_fence_after();
             const int nvalid = min(kC, T_len - m * kC);
-            __nv_bfloat16 *orow_ptr = O + (tok0 + (size_t)m * kC) * kD + orow;
+            __nv_bfloat16 *orow_ptr = O + (tok0 + (size_t)m * kC) * kD + i;
 #pragma unroll
-            for (int cb = 0; cb < 4; ++cb) {
+            for (int cb = 0; cb < 2; ++cb) {
                 uint32_t r[16];
                 __syncwarp();   // the bounded stores below diverge the warp; tcgen05.ld needs it converged
-                tmem_ld16(tmem + (lq << 16) + TM_O + 64 * bb + 16 * cb, r);
+                tmem_ld16(trow + TM_O + 64 * bb + vc0 + 16 * cb, r);
                 tmem_ld_wait(r);
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
-                    const int t = 16 * cb + j;
+                    const int t = vc0 + 16 * cb + j;
                     if (t < nvalid) orow_ptr[(size_t)t * kD] = __float2bfloat16_rn(__uint_as_float(r[j]));
                 }
             }
@@ -353,296 +447,54 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
             mbar_arrive(&bar[B_OACC_EMPTY + bb]);
             return true;
         };
-        // Vectorised gate pass: thread (rg, cg) owns rows 8rg..8rg+7 and key
-        // channels 8cg..8cg+7, so every shared access is one 16-byte chunk of
-        // a 128B-swizzled row.  The running products exp(G_r) and exp(G_C - G_r)
-        // per channel combine the thread's own 8 rows with the products of the
-        // other row groups, exchanged through shared memory once per chunk.
-        const int et = tid - 64;
-        const int cg = et & 15, rg = et >> 4;
-        const uint32_t pan = (uint32_t)(cg >> 3) * 8192u;   // panel holding this channel group
-        bool ok = true;
+        bool ok = nchunks == 0 || convert_w(0);
         for (int n = 0; n < nchunks && ok; ++n) {
-            const int b = n & 1;
-            const uint32_t par = (uint32_t)(n & 1), upar = (uint32_t)((n >> 1) & 1);
-            const int t0 = n * kC;
-            if (!SCALAR && !waitw(B_FULL_G, par)) break;
-            if (!waitw(B_FULL_K + b, upar) || !waitw(B_FULL_Q + b, upar)) break;
-            if (tid == 64) GDR_TRACE_AT(4, n);
-            float a[8][8];
-            if (!SCALAR) {
-                const float *gt = reinterpret_cast<const float *>(sm + OFF_G) + (8 * rg) * kD + 8 * cg;
-#pragma unroll
-                for (int rr = 0; rr < 8; ++rr) {
-                    const float4 x0 = *reinterpret_cast<const float4 *>(gt + rr * kD);
-                    const float4 x1 = *reinterpret_cast<const float4 *>(gt + rr * kD + 4);
-                    a[rr][0] = __expf(fmaxf(x0.x, kGateMin)); a[rr][1] = __expf(fmaxf(x0.y, kGateMin));
-                    a[rr][2] = __expf(fmaxf(x0.z, kGateMin)); a[rr][3] = __expf(fmaxf(x0.w, kGateMin));
-                    a[rr][4] = __expf(fmaxf(x1.x, kGateMin)); a[rr][5] = __expf(fmaxf(x1.y, kGateMin));
-                    a[rr][6] = __expf(fmaxf(x1.z, kGateMin)); a[rr][7] = __expf(fmaxf(x1.w, kGateMin));
-                }
-            } else {
-#pragma unroll
-                for (int rr = 0; rr < 8; ++rr) {
-                    const int t = t0 + 8 * rg + rr;
-                    const float e = (t < T_len) ? __expf(__ldg(g_scalar + tok0 + t)) : 1.f;
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) a[rr][c] = e;
-                }
-            }
-            // product of this row group, exchanged with the other seven
-            float L[8], F[8], Bk[8];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                L[c] = a[0][c];
-#pragma unroll
-                for (int rr = 1; rr < 8; ++rr) L[c] *= a[rr][c];
-                F[c] = 1.f;
-                Bk[c] = 1.f;
-            }
-            // Exchange area: with per-channel gates, row 8j of the g tile, which
-            // only the threads of row group j read, and which they overwrite
-            // after reading it; the tile is released after the exchange.  With
-            // a scalar gate the g region holds no tile, so two [8][128] buffers
-            // live there.
-            float *xb = reinterpret_cast<float *>(sm + OFF_G) + (SCALAR ? b * 8 * kD : 0);
-            constexpr int xrow = SCALAR ? kD : 8 * kD;
-            *reinterpret_cast<float4 *>(xb + rg * xrow + 8 * cg) = make_float4(L[0], L[1], L[2], L[3]);
-            *reinterpret_cast<float4 *>(xb + rg * xrow + 8 * cg + 4) = make_float4(L[4], L[5], L[6], L[7]);
-            mbar_arrive(&bar[B_XCH + b]);
-            if (!waitw(B_XCH + b, upar)) break;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                if (j == rg) continue;
-                const float4 y0 = *reinterpret_cast<const float4 *>(xb + j * xrow + 8 * cg);
-                const float4 y1 = *reinterpret_cast<const float4 *>(xb + j * xrow + 8 * cg + 4);
-                const float y[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    if (j < rg) F[c] *= y[c];
-                    else Bk[c] *= y[c];
-                }
-            }
-            if (!SCALAR) {
-                // The next TMA load overwrites the g tile as soon as this
-                // barrier completes; an arrive does not wait for this thread's
-                // shared loads, so order them before the async-proxy write.
-                fence_async_smem();
-                mbar_arrive(&bar[B_EMPTY_G]);
-            }
-            // K<- = k exp(G_r), Q<- = q exp(G_r) in place; raw k kept for K_tail
-            unsigned char *kp = sm + OFF_K + b * 16384 + pan;
-            unsigned char *qp = sm + OFF_Q + b * 16384 + pan;
-            uint4 kraw[8];
-            float pf[8];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) pf[c] = F[c];
-#pragma unroll
-            for (int rr = 0; rr < 8; ++rr) {
-                const uint32_t r = (uint32_t)(8 * rg + rr);
-                const uint32_t off = r * 128u + ((((uint32_t)(cg & 7)) ^ (r & 7u)) << 4);
-                const uint4 kv = *reinterpret_cast<const uint4 *>(kp + off);
-                const uint4 qv = *reinterpret_cast<const uint4 *>(qp + off);
-                kraw[rr] = kv;
-#pragma unroll
-                for (int c = 0; c < 8; ++c) pf[c] *= a[rr][c];
-                *reinterpret_cast<uint4 *>(kp + off) = scale8(kv, pf);
-                *reinterpret_cast<uint4 *>(qp + off) = scale8(qv, pf);
-            }
-            if (rg == 0) {   // gamma_C = product over all 64 rows
-                float *gw = gam + (n & 3) * kD + 8 * cg;
-                *reinterpret_cast<float4 *>(gw) = make_float4(L[0] * Bk[0], L[1] * Bk[1], L[2] * Bk[2], L[3] * Bk[3]);
-                *reinterpret_cast<float4 *>(gw + 4) = make_float4(L[4] * Bk[4], L[5] * Bk[5], L[6] * Bk[6], L[7] * Bk[7]);
-            }
-            fence_async_smem();
-            mbar_arrive(&bar[B_KQ_READY + b]);
-            if (tid == 64) GDR_TRACE_AT(5, n);
-            // K_tail = k exp(G_C - G_r): exclusive running product from the end
-            if (!waitw(B_KT_FREE, par ^ 1)) break;
-            if (tid == 64) GDR_TRACE_AT(6, n);
-            unsigned char *ktp = sm + OFF_KT + pan;
-            float sf[8];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) sf[c] = Bk[c];
-#pragma unroll
-            for (int rr = 7; rr >= 0; --rr) {
-                const uint32_t r = (uint32_t)(8 * rg + rr);
-                const uint32_t off = r * 128u + ((((uint32_t)(cg & 7)) ^ (r & 7u)) << 4);
-                *reinterpret_cast<uint4 *>(ktp + off) = scale8(kraw[rr], sf);
-#pragma unroll
-                for (int c = 0; c < 8; ++c) sf[c] *= a[rr][c];
-            }
-            fence_async_smem();
-            mbar_arrive(&bar[B_KT_READY]);
-            if (tid == 64) GDR_TRACE_AT(7, n);
-            if (n > 0) ok = epilogue(n - 1);
-            if (tid == 64 && n > 0) GDR_TRACE_AT(8, n - 1);
-        }
-        if (ok && !*abort_flag && nchunks > 0) epilogue(nchunks - 1);
-    } else {
-        // ================================================================ M: sequential-path conversions
-        // The state S_n lives at TM_S and is written only here.  At chunk n
-        // (n > 0) this group forms S_n = S_{n-1} * gamma_{n-1} + dS_{n-1}, with
-        // dS_{n-1} = V_new^T K_tail of chunk n-1 taken from TM_D, stores it
-        // back, and writes its bf16 copy for the MMAs of chunk n.
-        const uint32_t lq = 32u * (warp & 3);
-        const int i = (int)lq + lane;                // TMEM lane: row of S / V_new^T, key channel of W^T
-        const uint32_t trow = tmem + (lq << 16);
-        // initial state into TMEM
-#pragma unroll
-        for (int cb = 0; cb < 8; ++cb) {
-            uint32_t r[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j)
-                r[j] = __float_as_uint(S0 ? S0[((size_t)head * kD + i) * kD + 16 * cb + j] : 0.f);
-            tmem_st16(trow + TM_S + 16 * cb, r);
-        }
-        tmem_st_wait();
-        // S_{n} = S_{n-1} * gamma_{n-1} + dS_{n-1}, in TMEM and (optionally) as bf16 in smem
-        auto advance_state = [&](int n, bool to_smem) {
-            const float *gm = gam + ((n - 1) & 3) * kD;
-#pragma unroll
-            for (int cb = 0; cb < 8; cb += 2) {
-                uint32_t r0[16], r1[16], d0[16], d1[16];
-                tmem_ld16(trow + TM_S + 16 * cb, r0);
-                tmem_ld16(trow + TM_S + 16 * cb + 16, r1);
-                tmem_ld16(trow + TM_D + 16 * cb, d0);
-                tmem_ld16(trow + TM_D + 16 * cb + 16, d1);
-                tmem_ld_wait(r0);
-                reg_touch(r1);
-                reg_touch(d0);
-                reg_touch(d1);
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    r0[j] = __float_as_uint(fmaf(__uint_as_float(r0[j]), gm[16 * cb + j], __uint_as_float(d0[j])));
-                    r1[j] = __float_as_uint(fmaf(__uint_as_float(r1[j]), gm[16 * cb + 16 + j], __uint_as_float(d1[j])));
-                }
-                tmem_st16(trow + TM_S + 16 * cb, r0);
-                tmem_st16(trow + TM_S + 16 * cb + 16, r1);
-                if (to_smem) {
-                    unsigned char *sp = sm + OFF_S + (cb >> 2) * 16384;
-                    const uint32_t col = (uint32_t)((16 * cb) & 63);
-                    uint4 lo, hi;
-                    pack16(r0, lo, hi);
-                    *reinterpret_cast<uint4 *>(sp + sw128_off(i, col)) = lo;
-                    *reinterpret_cast<uint4 *>(sp + sw128_off(i, col + 8)) = hi;
-                    pack16(r1, lo, hi);
-                    *reinterpret_cast<uint4 *>(sp + sw128_off(i, col + 16)) = lo;
-                    *reinterpret_cast<uint4 *>(sp + sw128_off(i, col + 24)) = hi;
-                }
-            }
-            tmem_st_wait();
-        };
-        bool ok = true;
-        for (int n = 0; n < nchunks; ++n) {
             const uint32_t par = (uint32_t)(n & 1);
-            // ---- W^T -> W (bf16, K-major [64 tokens x 128 channels])
-            // KQ_READY(n) has completed (W^T(n) needed it); waiting on it here only
-            // acquires gamma_C(n), which the next chunk boundary reads.
-            if (!waitw(B_WT_FULL, par) || !waitw(B_W_FREE, par ^ 1) ||
-                !waitw(B_KQ_READY + (n & 1), (uint32_t)((n >> 1) & 1))) { ok = false; break; }
-            tc_fence_after();
-            if (tid == 192) GDR_TRACE_AT(9, n);
-            {
-                // W^T row of key channel i = 64 tokens = one 128-byte row of the
-                // MN-major W operand
-                uint32_t r0[16], r1[16];
-                tmem_ld16(trow + TM_W, r0);
-                tmem_ld16(trow + TM_W + 16, r1);
-                tmem_ld_wait(r0);
-                reg_touch(r1);
-                uint4 lo, hi;
-                pack16(r0, lo, hi);
-                *reinterpret_cast<uint4 *>(sm + OFF_W + sw128_off(i, 0)) = lo;
-                *reinterpret_cast<uint4 *>(sm + OFF_W + sw128_off(i, 8)) = hi;
-                pack16(r1, lo, hi);
-                *reinterpret_cast<uint4 *>(sm + OFF_W + sw128_off(i, 16)) = lo;
-                *reinterpret_cast<uint4 *>(sm + OFF_W + sw128_off(i, 24)) = hi;
-                tmem_ld16(trow + TM_W + 32, r0);
-                tmem_ld16(trow + TM_W + 48, r1);
-                tmem_ld_wait(r0);
-                reg_touch(r1);
-                pack16(r0, lo, hi);
-                *reinterpret_cast<uint4 *>(sm + OFF_W + sw128_off(i, 32)) = lo;
-                *reinterpret_cast<uint4 *>(sm + OFF_W + sw128_off(i, 40)) = hi;
-                pack16(r1, lo, hi);
-                *reinterpret_cast<uint4 *>(sm + OFF_W + sw128_off(i, 48)) = lo;
-                *reinterpret_cast<uint4 *>(sm + OFF_W + sw128_off(i, 56)) = hi;
-            }
-            fence_async_smem();
-            tc_fence_before();
-            mbar_arrive(&bar[B_W_READY]);
-            mbar_arrive(&bar[B_WT_EMPTY]);
-            if (tid == 192) GDR_TRACE_AT(10, n);
-            // ---- state of this chunk -> bf16 smem
+            // ---- S_n -> bf16 smem (the MMAs of chunk n - 1 that read the old
+            // copy completed before S_FULL(n - 1), which also completed S_n)
             if (n > 0) {
                 if (!waitw(B_S_FULL, par ^ 1)) { ok = false; break; }
                 tc_fence_after();
-                if (tid == 192) GDR_TRACE_AT(11, n);
-                advance_state(n, true);
-            } else {
-                if (tid == 192) GDR_TRACE_AT(11, n);
-#pragma unroll
-                for (int cb = 0; cb < 8; ++cb) {
-                    uint32_t r[16];
-                    tmem_ld16(trow + TM_S + 16 * cb, r);
-                    tmem_ld_wait(r);
-                    unsigned char *sp = sm + OFF_S + (cb >> 2) * 16384;
-                    uint4 lo, hi;
-                    lo.x = pack_bf16(__uint_as_float(r[0]), __uint_as_float(r[1]));
-                    lo.y = pack_bf16(__uint_as_float(r[2]), __uint_as_float(r[3]));
-                    lo.z = pack_bf16(__uint_as_float(r[4]), __uint_as_float(r[5]));
-                    lo.w = pack_bf16(__uint_as_float(r[6]), __uint_as_float(r[7]));
-                    hi.x = pack_bf16(__uint_as_float(r[8]), __uint_as_float(r[9]));
-                    hi.y = pack_bf16(__uint_as_float(r[10]), __uint_as_float(r[11]));
-                    hi.z = pack_bf16(__uint_as_float(r[12]), __uint_as_float(r[13]));
-                    hi.w = pack_bf16(__uint_as_float(r[14]), __uint_as_float(r[15]));
-                    *reinterpret_cast<uint4 *>(sp + sw128_off(i, (16 * cb) & 63)) = lo;
-                    *reinterpret_cast<uint4 *>(sp + sw128_off(i, ((16 * cb) & 63) + 8)) = hi;
-                }
             }
-            fence_async_smem();
-            tc_fence_before();
-            mbar_arrive(&bar[B_S_READY]);
-            if (tid == 192) GDR_TRACE_AT(12, n);
-            // ---- V_new^T (TMEM) -> bf16 smem
+            if (tid == 192) GDR_TRACE_AT(11, n);
+            if (!state_pass(n)) { ok = false; break; }
+            // ---- V_new^T (TMEM) -> bf16 smem (the MMAs of chunk n - 1 that read
+            // the old copy completed before X_FULL(n))
             if (!waitw(B_X_FULL, par)) { ok = false; break; }
             tc_fence_after();
             if (tid == 192) GDR_TRACE_AT(13, n);
 #pragma unroll
-            for (int cb = 0; cb < 4; ++cb) {
+            for (int cb = 0; cb < 2; ++cb) {
                 uint32_t r[16];
-                tmem_ld16(trow + TM_V + 16 * cb, r);
+                tmem_ld16(trow + TM_V + vc0 + 16 * cb, r);
                 tmem_ld_wait(r);
                 uint4 lo, hi;
-                lo.x = pack_bf16(__uint_as_float(r[0]), __uint_as_float(r[1]));
-                lo.y = pack_bf16(__uint_as_float(r[2]), __uint_as_float(r[3]));
-                lo.z = pack_bf16(__uint_as_float(r[4]), __uint_as_float(r[5]));
-                lo.w = pack_bf16(__uint_as_float(r[6]), __uint_as_float(r[7]));
-                hi.x = pack_bf16(__uint_as_float(r[8]), __uint_as_float(r[9]));
-                hi.y = pack_bf16(__uint_as_float(r[10]), __uint_as_float(r[11]));
-                hi.z = pack_bf16(__uint_as_float(r[12]), __uint_as_float(r[13]));
-                hi.w = pack_bf16(__uint_as_float(r[14]), __uint_as_float(r[15]));
-                *reinterpret_cast<uint4 *>(sm + OFF_VN + sw128_off(i, 16 * cb)) = lo;
-                *reinterpret_cast<uint4 *>(sm + OFF_VN + sw128_off(i, 16 * cb + 8)) = hi;
+                pack16(r, lo, hi);
+                *reinterpret_cast<uint4 *>(sm + OFF_VN + sw128_off(i, vc0 + 16 * cb)) = lo;
+                *reinterpret_cast<uint4 *>(sm + OFF_VN + sw128_off(i, vc0 + 16 * cb + 8)) = hi;
             }
             fence_async_smem();
             tc_fence_before();
-            mbar_arrive(&bar[B_VN_READY]);
-            mbar_arrive(&bar[B_VACC_EMPTY]);
+            mbar_arrive(&bar[B_VN_READY]);   // also: S_n scaled
             if (tid == 192) GDR_TRACE_AT(14, n);
+            // ---- off the sequential path while S += dS runs: next chunk's W,
+            // last chunk's output
+            if (n + 1 < nchunks && !convert_w(n + 1)) { ok = false; break; }
+            if (tid == 192) GDR_TRACE_AT(6, n);
+            if (n > 0 && !epilogue(n - 1)) { ok = false; break; }
+            if (tid == 192) GDR_TRACE_AT(7, n);
         }
-        // ---- final state S_N = S_{N-1} gamma_{N-1} + dS_{N-1}
+        if (ok && nchunks > 0) ok = epilogue(nchunks - 1);
+        // ---- final state S_N: the last accumulation has completed
         if (ok && nchunks > 0 && waitw(B_S_FULL, (uint32_t)((nchunks - 1) & 1))) {
             tc_fence_after();
-            advance_state(nchunks, false);
             if (ST) {
 #pragma unroll
-                for (int cb = 0; cb < 8; ++cb) {
+                for (int cb = 0; cb < 4; ++cb) {
                     uint32_t r[16];
-                    tmem_ld16(trow + TM_S + 16 * cb, r);
+                    tmem_ld16(trow + TM_S + sc0 + 16 * cb, r);
                     tmem_ld_wait(r);
-                    float4 *dst = reinterpret_cast<float4 *>(ST + ((size_t)head * kD + i) * kD + 16 * cb);
+                    float4 *dst = reinterpret_cast<float4 *>(ST + ((size_t)head * kD + i) * kD + sc0 + 16 * cb);
 #pragma unroll
                     for (int j = 0; j < 4; ++j)
                         dst[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
@@ -694,56 +546,41 @@ bool chunk_tc_supports(const ChunkArgs &a)
     return a.bf16 && a.dk == kD && a.dv == kD && a.C == kC;
 }
 
-size_t chunk_tc_workspace_bytes(int B, int H, int T)
-{
-    const size_t nchunks = (size_t)(T + kC - 1) / kC;
-    return 2 * (size_t)B * H * nchunks * kC * kC * sizeof(__nv_bfloat16);
-}
+size_t chunk_tc_workspace_bytes(int B, int H, int T) { return tc_workspace_bytes(B, H, T); }
 
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream, int *launches)
 {
     const int BH = a.B * a.H;
     const int nchunks = (a.T + kC - 1) / kC;
-    __nv_bfloat16 *Tw = static_cast<__nv_bfloat16 *>(a.workspace);
-    __nv_bfloat16 *Aw = Tw + (size_t)BH * nchunks * kC * kC;
+    const TcWorkspace w = carve_tc_workspace(a.workspace, a.B, a.H, a.T);
 
     Maps maps;
     {
         const cuuint64_t dims3[3] = {(cuuint64_t)kD, (cuuint64_t)a.T, (cuuint64_t)BH};
         const cuuint64_t str_bf[2] = {(cuuint64_t)kD * 2, (cuuint64_t)a.T * kD * 2};
         const cuuint32_t box_bf[3] = {64, 64, 1};
-        if (!make_map(&maps.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(a.k), dims3, str_bf, box_bf,
-                      CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_map(&maps.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(a.q), dims3, str_bf, box_bf,
-                      CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_map(&maps.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(a.v), dims3, str_bf, box_bf,
-                      CU_TENSOR_MAP_SWIZZLE_128B))
-            return cudaErrorInvalidValue;
-        if (!a.scalar_gate) {
-            const cuuint64_t str_f[2] = {(cuuint64_t)kD * 4, (cuuint64_t)a.T * kD * 4};
-            const cuuint32_t box_f[3] = {128, 64, 1};
-            if (!make_map(&maps.g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float *>(a.g), dims3, str_f, box_f,
-                          CU_TENSOR_MAP_SWIZZLE_NONE))
+        void *tiles[4] = {w.Kl, w.Ql, w.Kt, const_cast<void *>(a.v)};
+        CUtensorMap *dst[4] = {&maps.k, &maps.q, &maps.kt, &maps.v};
+        for (int i = 0; i < 4; ++i)
+            if (!make_map(dst[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, tiles[i], dims3, str_bf, box_bf,
+                          CU_TENSOR_MAP_SWIZZLE_128B))
                 return cudaErrorInvalidValue;
-        } else {
-            maps.g = maps.k;   // unused in scalar mode
-        }
         const cuuint64_t dims2[2] = {(cuuint64_t)kC, (cuuint64_t)BH * nchunks * kC};
         const cuuint64_t str2[1] = {(cuuint64_t)kC * 2};
         const cuuint32_t box2[2] = {64, 64};
-        if (!make_map(&maps.t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Tw, dims2, str2, box2, CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_map(&maps.aq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Aw, dims2, str2, box2, CU_TENSOR_MAP_SWIZZLE_128B))
+        if (!make_map(&maps.t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w.T, dims2, str2, box2, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_map(&maps.aq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w.Aqk, dims2, str2, box2, CU_TENSOR_MAP_SWIZZLE_128B))
             return cudaErrorInvalidValue;
     }
 
-    cudaError_t e = launch_ut_prep(a, Tw, Aw, stream);
+    cudaError_t e = launch_ut_prep(a, w, stream);
     if (e != cudaSuccess) return e;
     *launches += 1;
 
     auto kern = a.scalar_gate ? chunk_scan_kernel<true> : chunk_scan_kernel<false>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_ALLOC);
     if (e != cudaSuccess) return e;
-    kern<<<BH, kThreads, SMEM_ALLOC, stream>>>(maps, a.g, a.S0, static_cast<__nv_bfloat16 *>(a.O), a.S_T, a.T,
+    kern<<<BH, kThreads, SMEM_ALLOC, stream>>>(maps, w.gam, a.S0, static_cast<__nv_bfloat16 *>(a.O), a.S_T, a.T,
                                               nchunks);
     e = cudaGetLastError();
     if (e == cudaSuccess) *launches += 1;

@@ -30,6 +30,39 @@ struct StepArgs {
     bool bf16;
 };
 
+// The tensor-core path's scratch, carved out of ChunkArgs::workspace (every
+// part starts on a 256-byte boundary):
+//   T, Aqk      [B*H*chunks][64][64] bf16   T' = (I + A)^{-1} Diag(beta) and Aqk
+//   Kl, Ql, Kt  [B, H, T, 128] bf16         K<-, Q<-, K_tail (chunk-relative decays)
+//   gam         [B*H*chunks][128] fp32      gamma_C per key channel
+struct TcWorkspace {
+    __nv_bfloat16 *T, *Aqk, *Kl, *Ql, *Kt;
+    float *gam;
+};
+inline size_t tc_workspace_bytes(int B, int H, int T)
+{
+    const size_t bh = (size_t)B * H, nch = (size_t)(T + 63) / 64;
+    return 2 * bh * nch * 64 * 64 * 2 + 3 * bh * (size_t)T * 128 * 2 + bh * nch * 128 * 4;
+}
+inline TcWorkspace carve_tc_workspace(void *ws, int B, int H, int T)
+{
+    const size_t bh = (size_t)B * H, nch = (size_t)(T + 63) / 64;
+    unsigned char *p = static_cast<unsigned char *>(ws);
+    TcWorkspace w;
+    w.T = reinterpret_cast<__nv_bfloat16 *>(p);
+    p += bh * nch * 64 * 64 * 2;
+    w.Aqk = reinterpret_cast<__nv_bfloat16 *>(p);
+    p += bh * nch * 64 * 64 * 2;
+    w.Kl = reinterpret_cast<__nv_bfloat16 *>(p);
+    p += bh * (size_t)T * 128 * 2;
+    w.Ql = reinterpret_cast<__nv_bfloat16 *>(p);
+    p += bh * (size_t)T * 128 * 2;
+    w.Kt = reinterpret_cast<__nv_bfloat16 *>(p);
+    p += bh * (size_t)T * 128 * 2;
+    w.gam = reinterpret_cast<float *>(p);
+    return w;
+}
+
 // Each launcher enqueues its kernels on `stream`, adds the number of kernels
 // it launched to *launches and returns the first launch error.
 cudaError_t launch_recurrent_step(const StepArgs &a, cudaStream_t stream, int *launches);

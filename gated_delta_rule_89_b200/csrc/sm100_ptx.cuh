@@ -68,16 +68,42 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
     return ok != 0;
 }
 
+// try_wait that lets the hardware suspend the thread for up to `ns`
+// nanoseconds (it resumes as soon as the phase completes), so a waiting warp
+// does not spin on the issue slots its SM sub-partition shares.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t ns)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete, giving up after
 // `budget` clock cycles.  Returns false on timeout (the caller reports it).
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, long long budget)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity)) {
+    while (!mbar_try_wait_sleep(bar, parity, 20000u)) {
         if (clock64() - t0 > budget) return false;
     }
     return true;
+}
+
+// ------------------------------------------------------------- f32x2 math
+
+// Packed fp32 pair multiply (one sm_100 f32x2 instruction, round to nearest).
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b)
+{
+    unsigned long long x = *reinterpret_cast<unsigned long long *>(&a), y = *reinterpret_cast<unsigned long long *>(&b), z;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(z) : "l"(x), "l"(y));
+    return *reinterpret_cast<float2 *>(&z);
 }
 
 // ------------------------------------------------------------------- TMA

@@ -4,7 +4,9 @@
 //   A[r][i]   = beta_r sum_c k_rc k_ic exp(G_rc - G_ic)     (i <  r)
 //   Aqk[r][i] =        sum_c q_rc k_ic exp(G_rc - G_ic)     (i <= r)
 //   T' = (I + A)^{-1} Diag(beta)
-// and writes T' and Aqk (bf16, row-major 64 x 64) to the workspace.  T' is
+// and writes T' and Aqk (bf16, row-major 64 x 64) to the workspace, together
+// with the chunk-relative operands of the state scan (K<-, Q<-, K_tail and
+// gamma_C, defined where they are written).  T' is
 // the matrix the UT transform of "Token Mixer I", section "Kimi Delta
 // Attention: Improving Delta Rule with Fine-grained Gating" calls
 // M = (I + StrictTril(Diag(beta)(Gamma*K)(K/Gamma)^T))^{-1} Diag(beta), so
@@ -98,25 +100,10 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// two bf16 (packed) times two fp32 factors, rounded back to bf16
-__device__ __forceinline__ uint32_t scale2(uint32_t v, float s0, float s1)
-{
-    __nv_bfloat162 o = __floats2bfloat162_rn(__uint_as_float(v << 16) * s0, __uint_as_float(v & 0xffff0000u) * s1);
-    return *reinterpret_cast<uint32_t *>(&o);
-}
-
 __device__ __forceinline__ uint32_t pack2(float lo, float hi)
 {
     __nv_bfloat162 o = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&o);
-}
-
-// packed fp32 pair multiply (sm_100 f32x2)
-__device__ __forceinline__ float2 fmul2(float2 a, float2 b)
-{
-    unsigned long long x = *reinterpret_cast<unsigned long long *>(&a), y = *reinterpret_cast<unsigned long long *>(&b), z;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(z) : "l"(x), "l"(y));
-    return *reinterpret_cast<float2 *>(&z);
 }
 
 // bf16 pair (packed) times an fp32 pair, rounded back to a bf16 pair
@@ -190,7 +177,8 @@ template <bool SCALAR>
 __global__ void __launch_bounds__(kThreads, 2)
 ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__restrict__ qg,
                const float *__restrict__ gg, const float *__restrict__ betag, __nv_bfloat16 *__restrict__ Tout,
-               __nv_bfloat16 *__restrict__ Aqout, int T_len, int nchunks, int total)
+               __nv_bfloat16 *__restrict__ Aqout, __nv_bfloat16 *__restrict__ Klo, __nv_bfloat16 *__restrict__ Qlo,
+               __nv_bfloat16 *__restrict__ Kto, float *__restrict__ gamo, int T_len, int nchunks, int total)
 {
     extern __shared__ unsigned char prep_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(prep_raw) + 1023) &
@@ -220,21 +208,30 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
         // ---- operands.  Warp (R, panel) covers rows 16R..16R+15 and the 64
         // channels of one panel; lane = (half, quad): rows 16R + 8 half + 0..7,
         // channels 64 panel + 4 quad + 0..3.
+        const int R = warp >> 1, half = lane >> 4;
+        const uint32_t c = 64u * (warp & 1) + 4u * (lane & 15);
+        const int rbase = 16 * R + 8 * half;
+        uint2 kr[8], qr[8];
+        float4 gv[8];                       // g, then alpha = exp(max(g, -5))
+        float2 oa = make_float2(1.f, 1.f), ob = oa;   // alpha product of the other half block
         {
-            const int R = warp >> 1, half = lane >> 4;
-            const uint32_t c = 64u * (warp & 1) + 4u * (lane & 15);
-            const int rbase = 16 * R + 8 * half;
-            uint2 kr[8], qr[8];
-            float4 gv[8];
+            // Unconditional loads from rows clamped into the chunk (a
+            // conditional load makes the compiler wait for each one before the
+            // next); rows past T are zeroed (k, q) or given g = 0 afterwards.
 #pragma unroll
             for (int rr = 0; rr < 8; ++rr) {
-                const int r = rbase + rr;
-                const bool ok = r < nrows;
-                const size_t e = (row0 + r) * kDK + c;
-                kr[rr] = ok ? __ldg(reinterpret_cast<const uint2 *>(kg + e)) : make_uint2(0u, 0u);
-                qr[rr] = ok ? __ldg(reinterpret_cast<const uint2 *>(qg + e)) : make_uint2(0u, 0u);
-                if (!SCALAR)
-                    gv[rr] = ok ? __ldg(reinterpret_cast<const float4 *>(gg + e)) : make_float4(0.f, 0.f, 0.f, 0.f);
+                const size_t e = (row0 + min(rbase + rr, nrows - 1)) * kDK + c;
+                kr[rr] = __ldg(reinterpret_cast<const uint2 *>(kg + e));
+                qr[rr] = __ldg(reinterpret_cast<const uint2 *>(qg + e));
+                if (!SCALAR) gv[rr] = __ldg(reinterpret_cast<const float4 *>(gg + e));
+            }
+#pragma unroll
+            for (int rr = 0; rr < 8; ++rr) {
+                if (rbase + rr >= nrows) {
+                    kr[rr] = make_uint2(0u, 0u);
+                    qr[rr] = make_uint2(0u, 0u);
+                    if (!SCALAR) gv[rr] = make_float4(0.f, 0.f, 0.f, 0.f);
+                }
             }
             if (tid < kC) sBeta[tid] = tid < nrows ? __ldg(betag + row0 + tid) : 0.f;
             if (SCALAR && warp == 0) {
@@ -270,8 +267,8 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
                     lb = fmul2(lb, make_float2(gv[rr].z, gv[rr].w));
                 }
                 // the other half of the 16-row block (lane ^ 16)
-                const float2 oa = make_float2(__shfl_xor_sync(0xffffffffu, la.x, 16), __shfl_xor_sync(0xffffffffu, la.y, 16));
-                const float2 ob = make_float2(__shfl_xor_sync(0xffffffffu, lb.x, 16), __shfl_xor_sync(0xffffffffu, lb.y, 16));
+                oa = make_float2(__shfl_xor_sync(0xffffffffu, la.x, 16), __shfl_xor_sync(0xffffffffu, la.y, 16));
+                ob = make_float2(__shfl_xor_sync(0xffffffffu, lb.x, 16), __shfl_xor_sync(0xffffffffu, lb.y, 16));
                 // Khat, Qhat: inclusive running product from the block start
                 float2 pa = half ? oa : make_float2(1.f, 1.f), pb = half ? ob : make_float2(1.f, 1.f);
 #pragma unroll
@@ -300,6 +297,74 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
             }
         }
         __syncthreads();
+
+        // ---- chunk-relative operands of the state scan, to global memory in
+        // the layout of k ([B, H, T, 128] bf16), G counted from the chunk start:
+        //   K<-_r = k_r exp(G_r),  Q<-_r = q_r exp(G_r),  K_tail_r = k_r exp(G_C - G_r)
+        // and gamma_C = exp(G_C) per key channel (fp32, [B H chunks][128]).
+        // Formed in fp32 from the registers above, with the block decays bd_J.
+        {
+            const size_t e0 = row0 * kDK + c;
+            if (!SCALAR) {
+                float2 Fa = make_float2(1.f, 1.f), Fb = Fa, Ba = Fa, Bb = Fa;
+#pragma unroll
+                for (int J = 0; J < 4; ++J) {
+                    const float4 bdj = *reinterpret_cast<const float4 *>(sBd + J * kDK + c);
+                    if (J < R) {
+                        Fa = fmul2(Fa, make_float2(bdj.x, bdj.y));
+                        Fb = fmul2(Fb, make_float2(bdj.z, bdj.w));
+                    } else if (J > R) {
+                        Ba = fmul2(Ba, make_float2(bdj.x, bdj.y));
+                        Bb = fmul2(Bb, make_float2(bdj.z, bdj.w));
+                    }
+                }
+                float2 pa = half ? fmul2(Fa, oa) : Fa, pb = half ? fmul2(Fb, ob) : Fb;
+#pragma unroll
+                for (int rr = 0; rr < 8; ++rr) {
+                    pa = fmul2(pa, make_float2(gv[rr].x, gv[rr].y));
+                    pb = fmul2(pb, make_float2(gv[rr].z, gv[rr].w));
+                    if (rbase + rr < nrows) {
+                        const size_t e = e0 + (size_t)(rbase + rr) * kDK;
+                        *reinterpret_cast<uint2 *>(Klo + e) = make_uint2(scale2p(kr[rr].x, pa), scale2p(kr[rr].y, pb));
+                        *reinterpret_cast<uint2 *>(Qlo + e) = make_uint2(scale2p(qr[rr].x, pa), scale2p(qr[rr].y, pb));
+                    }
+                }
+                if (R == 0 && half == 0) {   // gamma_C = product of the four block decays
+                    const float4 b0 = *reinterpret_cast<const float4 *>(sBd + c);
+                    const float2 ga = fmul2(Ba, make_float2(b0.x, b0.y)), gb = fmul2(Bb, make_float2(b0.z, b0.w));
+                    *reinterpret_cast<float4 *>(gamo + (size_t)ci * kDK + c) = make_float4(ga.x, ga.y, gb.x, gb.y);
+                }
+                pa = half ? Ba : fmul2(Ba, oa);
+                pb = half ? Bb : fmul2(Bb, ob);
+#pragma unroll
+                for (int rr = 7; rr >= 0; --rr) {
+                    if (rbase + rr < nrows) {
+                        const size_t e = e0 + (size_t)(rbase + rr) * kDK;
+                        *reinterpret_cast<uint2 *>(Kto + e) = make_uint2(scale2p(kr[rr].x, pa), scale2p(kr[rr].y, pb));
+                    }
+                    pa = fmul2(pa, make_float2(gv[rr].x, gv[rr].y));
+                    pb = fmul2(pb, make_float2(gv[rr].z, gv[rr].w));
+                }
+            } else {
+                const float Gl = sGc[kC - 1];   // rows past T carry g = 0
+#pragma unroll
+                for (int rr = 0; rr < 8; ++rr) {
+                    const int r = rbase + rr;
+                    if (r < nrows) {
+                        const float ef = __expf(sGc[r]), et = __expf(Gl - sGc[r]);
+                        const float2 fe = make_float2(ef, ef), ft = make_float2(et, et);
+                        const size_t e = e0 + (size_t)r * kDK;
+                        *reinterpret_cast<uint2 *>(Klo + e) = make_uint2(scale2p(kr[rr].x, fe), scale2p(kr[rr].y, fe));
+                        *reinterpret_cast<uint2 *>(Qlo + e) = make_uint2(scale2p(qr[rr].x, fe), scale2p(qr[rr].y, fe));
+                        *reinterpret_cast<uint2 *>(Kto + e) = make_uint2(scale2p(kr[rr].x, ft), scale2p(kr[rr].y, ft));
+                    }
+                }
+                if (R == 0 && half == 0) {
+                    const float gl = __expf(Gl);
+                    *reinterpret_cast<float4 *>(gamo + (size_t)ci * kDK + c) = make_float4(gl, gl, gl, gl);
+                }
+            }
+        }
 
         // ---- block products on tensor cores: 10 block pairs over 8 warps, each
         // pair gives both A and Aqk (the right operand and its scaling are shared)
@@ -494,7 +559,7 @@ int sm_count()
 
 }  // namespace
 
-cudaError_t launch_ut_prep(const ChunkArgs &a, __nv_bfloat16 *Tout, __nv_bfloat16 *Aqout, cudaStream_t stream)
+cudaError_t launch_ut_prep(const ChunkArgs &a, const TcWorkspace &w, cudaStream_t stream)
 {
     const int nchunks = (a.T + kC - 1) / kC;
     const long long total = (long long)a.B * a.H * nchunks;
@@ -506,7 +571,8 @@ cudaError_t launch_ut_prep(const ChunkArgs &a, __nv_bfloat16 *Tout, __nv_bfloat1
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_ALLOC);
     if (e != cudaSuccess) return e;
     kern<<<grid, kThreads, SMEM_ALLOC, stream>>>((const __nv_bfloat16 *)a.k, (const __nv_bfloat16 *)a.q, a.g,
-                                                 a.beta, Tout, Aqout, a.T, nchunks, (int)total);
+                                                 a.beta, w.T, w.Aqk, w.Kl, w.Ql, w.Kt, w.gam, a.T, nchunks,
+                                                 (int)total);
     return cudaGetLastError();
 }
 

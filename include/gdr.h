@@ -135,7 +135,8 @@ int gdr_recurrent_step(const void *q, const void *k, const void *v, const float 
  * every GPU where the library is loaded, until the process exits.
  *   - Problems whose gdr_chunk_fwd_workspace_size() exceeds
  *     GDR_NOALLOC_SCRATCH_BYTES are rejected with GDR_ERR_UNSUPPORTED before
- *     any launch (for example B*H*ceil(T/64) > 2048 chunks of bf16 d=128).
+ *     any launch (bf16 d=128 needs 66,048 bytes per 64-token chunk, so at
+ *     most 508 full chunks, B*H*ceil(T/64) <= 508, fit).
  *   - Every call shares that array.  Calls that may overlap on the GPU
  *     (unordered streams, several host threads) race on it and give
  *     undefined results; order them.  Nothing has to be cleared between

@@ -88,10 +88,16 @@ def test_step_argument_validation(L):
     assert step(B=0) == OK
 
 
+def _tc_workspace(B, H, T):
+    # per chunk: T' and Aqk (2 x 64 x 64 bf16) and gamma_C (128 fp32);
+    # per token: K<-, Q<-, K_tail (3 x 128 bf16)
+    nch = (T + 63) // 64
+    return B * H * (nch * (2 * 64 * 64 * 2 + 128 * 4) + T * 3 * 128 * 2)
+
+
 def test_workspace_query(L):
-    # bf16, d = 128, C = 64: T' and Aqk, 2 x 64 x 64 bf16 per chunk
-    assert L.gdr_chunk_fwd_workspace_size(2, 32, 8192, 128, 128, 64, 0, 1) == 2 * 2 * 32 * 128 * 64 * 64 * 2
-    assert L.gdr_chunk_fwd_workspace_size(1, 1, 65, 128, 128, 64, 1, 1) == 2 * 2 * 64 * 64 * 2
+    assert L.gdr_chunk_fwd_workspace_size(2, 32, 8192, 128, 128, 64, 0, 1) == _tc_workspace(2, 32, 8192)
+    assert L.gdr_chunk_fwd_workspace_size(1, 1, 65, 128, 128, 64, 1, 1) == _tc_workspace(1, 1, 65)
     # fp32 inputs or other sizes run on the CUDA-core path, which needs none
     assert L.gdr_chunk_fwd_workspace_size(1, 2, 256, 64, 64, 64, 0, 0) == 0
     assert L.gdr_chunk_fwd_workspace_size(1, 2, 256, 128, 128, 32, 0, 1) == 0

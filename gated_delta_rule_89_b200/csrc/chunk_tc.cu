@@ -5,12 +5,11 @@
 //   1. ut_prep (ut_prep.cu): every chunk of every head in parallel -> the
 //      UT-transform matrix T' = (I + A)^{-1} Diag(beta), the masked
 //      intra-chunk matrix Aqk and, with G the cumulative log-decay inside the
-//      chunk, K<- = K*exp(G), Q<- = Q*exp(G), K_tail = K*exp(G_C - G) and
-//      gamma_C = exp(G_C), all into the workspace.
+//      chunk, W = T' (K*exp(G)) (stored transposed), Q<- = Q*exp(G),
+//      K_tail = K*exp(G_C - G) and gamma_C = exp(G_C), all into the workspace.
 //   2. chunk_scan (this file): one CTA per (b, h) walks the chunks in order.
 //      The fp32 state S [d_v x d_k] lives in tensor memory for the whole
 //      sequence.  Per chunk:
-//        W^T     = K<-^T T'^T                (= (T' K<-)^T)
 //        V_new^T = V^T T'^T - S W^T          (U^T, then -S W^T accumulated)
 //        O^T     = S Q<-^T + V_new^T Aqk^T
 //        S       = S Diag(gamma_C) + V_new^T K_tail   (the scaling in place in
@@ -25,17 +24,17 @@
 //      MN-major operands.
 //
 // Warp roles (320 threads):
-//   warp 0      TMA producer (one lane): all tiles of a chunk land in one of
-//               two stages and complete one barrier; gamma_C in two slots
+//   warp 0      TMA producer (lane 0): all tiles of a chunk land in one of
+//               two stages and complete one barrier; gamma_C in two slots.
+//               Lane 1 issues the TMA stores of the output tiles.
 //   warp 1      TMEM allocation and the MMA issuer (one lane), in the order
-//               X^T(n), O^T(n), W^T(n+1), dS(n), O(n), U^T(n+1), so the
-//               products that do not depend on the state run while the state
-//               is updated
+//               X^T(n), O^T(n), dS(n), O(n), U^T(n+1), so the products that do
+//               not depend on the state run while the state is updated
 //   warps 2-9   every conversion, split by columns between warps 2-5 and
 //               6-9: on the sequential path S (TMEM) -> bf16 smem and
 //               V_new^T (TMEM) -> bf16 smem; off it, in the gaps while the
-//               tensor core runs, S *= gamma_C in TMEM, W^T (TMEM) -> W
-//               (bf16 smem) and the output epilogue O^T (TMEM) -> bf16 -> global.
+//               tensor core runs, S *= gamma_C in TMEM and the output
+//               epilogue O^T (TMEM) -> bf16 smem tile -> TMA store.
 // The sequential chain per chunk is dS -> S to bf16 -> X^T -> V_new -> dS.
 // Every wait is bounded (about a second); on timeout the kernel records
 // GDR_ERR_TIMEOUT in a device status word, lets the copies and MMAs it
@@ -64,7 +63,7 @@ constexpr long long kWaitBudget = 2000000000LL;   // clock cycles per wait (~1 s
 // shared memory map (bytes from a 1024-aligned base).  The input tiles of a
 // chunk form one stage (gamma_C in a slot of its own); two stages alternate
 // by chunk parity.
-constexpr uint32_t ST_K = 0;                       // K<-  (2 panels x 8 KB)              16 KB
+constexpr uint32_t ST_W = 0;                       // W^T, MN-major [128 ch x 64 tok]      16 KB
 constexpr uint32_t ST_Q = 16384;                   // Q<-                                  16 KB
 constexpr uint32_t ST_KT = 32768;                  // K_tail                               16 KB
 constexpr uint32_t ST_V = 49152;                   // v                                    16 KB
@@ -72,8 +71,8 @@ constexpr uint32_t ST_T = 65536;                   // T' (1 panel)              
 constexpr uint32_t ST_AQ = 73728;                  // Aqk                                   8 KB
 constexpr uint32_t STAGE = 81920;                  // stage stride (1024-aligned)
 constexpr uint32_t STAGE_TX = 4 * 16384 + 2 * 8192;   // bytes one stage receives
-constexpr uint32_t OFF_W = 2 * STAGE;              // W, MN-major [128 ch x 64 tok]         16 KB
-constexpr uint32_t OFF_S = OFF_W + 16384;          // bf16 S (2 panels x 16 KB)             32 KB
+constexpr uint32_t OFF_OST = 2 * STAGE;            // O^T staging for the TMA store (2 panels) 16 KB
+constexpr uint32_t OFF_S = OFF_OST + 16384;        // bf16 S (2 panels x 16 KB)             32 KB
 constexpr uint32_t OFF_VN = OFF_S + 32768;         // V_new^T (1 panel, 128 rows)           16 KB
 constexpr uint32_t OFF_GAM = OFF_VN + 16384;       // gamma_C of each stage, [2][128] fp32   1 KB
 constexpr uint32_t OFF_BAR = OFF_GAM + 1024;       // mbarriers, TMEM slot, abort flag
@@ -83,30 +82,31 @@ static_assert(SMEM_ALLOC <= 232448, "dynamic shared memory above the 227 KB per-
 
 // TMEM columns (fp32)
 constexpr uint32_t TM_S = 0;      // state S_n, 128 columns: scaled by gamma_C in place, dS accumulated onto it
-constexpr uint32_t TM_W = 128;    // W^T, 64 columns
-constexpr uint32_t TM_V = 192;    // V_new^T accumulator, 64 columns
-constexpr uint32_t TM_O = 256;    // O^T accumulators, 2 x 64 columns
-constexpr uint32_t TM_COLS = 512; // allocation granularity (power of two); 384 used
+constexpr uint32_t TM_V = 128;    // V_new^T accumulator, 64 columns
+constexpr uint32_t TM_O = 192;    // O^T accumulators, 2 x 64 columns
+constexpr uint32_t TM_COLS = 512; // allocation granularity (power of two); 320 used
 
 enum Bar {
     B_FULL, B_FULL1,          // stage landed (TMA transaction bytes)
     B_EMPTY, B_EMPTY1,        // stage released (MMA commit)
     B_GFULL, B_GFULL1,        // gamma_C slot landed
     B_GEMPTY, B_GEMPTY1,      // gamma_C slot read by the state-update threads
-    B_WT_FULL,                // W^T(n), U^T(n) in TMEM
-    B_SW_READY,               // W(n) and S_n (bf16) in smem, TMEM W read
+    B_SW_READY,               // S_n (bf16) in smem
     B_X_FULL,                 // V_new^T(n) in TMEM
     B_VN_READY,               // V_new^T(n) bf16 in smem, TM_V read, S_n scaled by gamma_C(n)
     B_S_FULL,                 // S_{n+1} complete in TMEM
     B_O_FULL, B_O_FULL1,      // O^T(n) complete
     B_OACC_EMPTY, B_OACC_EMPTY1,   // O^T accumulator drained by the epilogue
+    B_EPI_FULL,               // O^T staging tile written (warps 2-9)
+    B_EPI_FREE,               // O^T staging tile free again (the previous store has read it)
     B_FINAL,
     B_COUNT
 };
 static_assert(8 * B_COUNT + 8 <= 256, "barrier area");
 
 struct Maps {
-    CUtensorMap k, q, kt, v, t, aq;   // K<-, Q<-, K_tail, v: [BH][T][128]; T', Aqk: [chunks*64][64]
+    CUtensorMap w, q, kt, v, t, aq, o;   // Q<-, K_tail, v, O: [BH][T][128]; T', Aqk: [chunks*64][64];
+                                         // W^T: [chunks*128][64]
 };
 
 __device__ __forceinline__ void record_error(int code) { atomicCAS(&g_device_status, 0, code); }
@@ -165,9 +165,10 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
         const uint32_t counts[B_COUNT] = {
             1, 1, 1, 1,       // stage full (TMA), stage empty (MMA commit)
             1, 1, 256, 256,   // gamma full (TMA), gamma empty (warps 2-9)
-            1, 256, 1, 256,   // wt full (MMA), sw ready (warps 2-9), x full (MMA), vn ready (warps 2-9)
+            256, 1, 256,      // sw ready (warps 2-9), x full (MMA), vn ready (warps 2-9)
             1,                // s full (MMA)
             1, 1, 256, 256,   // o full (MMA) x2, oacc empty (warps 2-9) x2
+            256, 1,           // epilogue tile written (warps 2-9), free (warp 0 lane 1)
             1};
         for (int i = 0; i < B_COUNT; ++i) mbar_init(&bar[i], counts[i]);
         *abort_flag = 0;
@@ -205,9 +206,23 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
     };
 
     if (warp == 0) {
-        // ================================================================ TMA producer
+        // ================================================================ TMA producer, output stores
+        if (lane == 1) {
+            // Output tile m: stored once the conversion warps have written it;
+            // the tile is handed back once the store has read it.
+            mbar_arrive(&bar[B_EPI_FREE]);
+            for (int m = 0; m < nchunks; ++m) {
+                if (!wait(B_EPI_FULL, (uint32_t)(m & 1))) break;
+                tma_store_3d(&maps.o, sm + OFF_OST, 0, m * kC, head);
+                tma_store_3d(&maps.o, sm + OFF_OST + 8192, 64, m * kC, head);
+                bulk_commit_group();
+                bulk_wait_read_all();
+                mbar_arrive(&bar[B_EPI_FREE]);
+            }
+            bulk_wait_all();   // the last store has completed before the CTA exits
+        }
         if (lane == 0) {
-            for (int i = 0; i < 6; ++i) tma_prefetch_desc(&maps.k + i);
+            for (int i = 0; i < 6; ++i) tma_prefetch_desc(&maps.w + i);
             int issued = 0;
             for (int n = 0; n < nchunks; ++n) {
                 const int t0 = n * kC;
@@ -218,8 +233,7 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
                 uint64_t *full = &bar[B_FULL + b];
                 if (!wait(B_EMPTY + b, upar ^ 1)) break;
                 mbar_arrive_expect_tx(full, STAGE_TX);
-                tma_load_3d(st + ST_K, &maps.k, full, 0, t0, head);
-                tma_load_3d(st + ST_K + 8192, &maps.k, full, 64, t0, head);
+                tma_load_2d(st + ST_W, &maps.w, full, 0, (head * nchunks + n) * kD);
                 tma_load_2d(st + ST_T, &maps.t, full, 0, crow);
                 tma_load_3d(st + ST_V, &maps.v, full, 0, t0, head);
                 tma_load_3d(st + ST_V + 8192, &maps.v, full, 64, t0, head);
@@ -246,21 +260,12 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
     } else if (warp == 1) {
         // ================================================================ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t ID_WU = idesc_bf16(128, 64, true, false);         // A MN-major, B K-major
+            constexpr uint32_t ID_WU = idesc_bf16(128, 64, true, false);         // A (v) MN-major, B K-major
             constexpr uint32_t ID_X = idesc_bf16(128, 64, false, true, true);    // -A, B (W) MN-major
             constexpr uint32_t ID_O = idesc_bf16(128, 64, false, false);
             constexpr uint32_t ID_S = idesc_bf16(128, 128, false, true);         // B MN-major
-            // W^T = K<-^T T'^T and U^T = V^T T'^T of chunk n (stage n & 1), as
-            // separate groups: W^T feeds the W conversion early, U^T has to
-            // wait until V_new^T of the previous chunk has left TM_V
-            auto mma_w = [&](int n) {
-                const uint32_t st = sbase + (n & 1) * STAGE;
-#pragma unroll
-                for (int s = 0; s < 4; ++s)
-                    mma_bf16(tmem + TM_W, sdesc_sw128(st + ST_K + s * 2048, 8192, 1024),
-                             sdesc_sw128(st + ST_T + s * 32, 16, 1024), ID_WU, s > 0);
-                mma_commit(&bar[B_WT_FULL]);
-            };
+            // U^T = V^T T'^T of chunk n (stage n & 1); it has to wait until
+            // V_new^T of the previous chunk has left TM_V
             auto mma_u = [&](int n) {
                 const uint32_t st = sbase + (n & 1) * STAGE;
 #pragma unroll
@@ -272,15 +277,12 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
             if (ok) {
                 tc_fence_after();
                 GDR_TRACE_AT(1, 0);
-                mma_w(0);
                 mma_u(0);
             }
             for (int n = 0; n < nchunks && ok; ++n) {
                 const int b = n & 1;
                 const uint32_t par = (uint32_t)(n & 1), upar = (uint32_t)((n >> 1) & 1);
                 const uint32_t st = sbase + b * STAGE;
-                const bool more = n + 1 < nchunks;
-                const uint32_t npar = (uint32_t)(((n + 1) >> 1) & 1);   // next stage's phase
                 // ---- V_new^T += -S W^T ; O^T = S Q<-^T
                 if (!wait(B_SW_READY, par) || !wait(B_OACC_EMPTY + b, upar ^ 1)) break;
                 tc_fence_after();
@@ -288,22 +290,13 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
 #pragma unroll
                 for (int s = 0; s < 8; ++s)
                     mma_bf16(tmem + TM_V, sdesc_sw128(sbase + OFF_S + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024),
-                             sdesc_sw128(sbase + OFF_W + s * 2048, 8192, 1024), ID_X, 1);
+                             sdesc_sw128(st + ST_W + s * 2048, 8192, 1024), ID_X, 1);
                 mma_commit(&bar[B_X_FULL]);
 #pragma unroll
                 for (int s = 0; s < 8; ++s)
                     mma_bf16(tmem + TM_O + 64 * b,
                              sdesc_sw128(sbase + OFF_S + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024),
                              sdesc_sw128(st + ST_Q + (s >> 2) * 8192 + (s & 3) * 32, 16, 1024), ID_O, s > 0);
-                // ---- W^T of the next chunk now if its stage has landed (never
-                // block here: this stage is only released below)
-                bool w_done = false;
-                if (more && mbar_try_wait(&bar[B_FULL + (b ^ 1)], npar)) {
-                    tc_fence_after();
-                    GDR_TRACE_AT(1, n + 1);
-                    mma_w(n + 1);
-                    w_done = true;
-                }
                 // ---- S += V_new^T K_tail (the sequential path; S already scaled by
                 // gamma_C); O^T += V_new^T Aqk^T
                 if (!wait(B_VN_READY, par)) break;
@@ -320,14 +313,11 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
                              sdesc_sw128(st + ST_AQ + s * 32, 16, 1024), ID_O, 1);
                 mma_commit(&bar[B_O_FULL + b]);
                 mma_commit(&bar[B_EMPTY + b]);   // every read of this stage is issued
-                // ---- U^T of the next chunk (and W^T if its stage came late)
-                if (more) {
-                    if (!w_done) {
-                        if (!wait(B_FULL + (b ^ 1), npar)) break;
-                        tc_fence_after();
-                        GDR_TRACE_AT(1, n + 1);
-                        mma_w(n + 1);
-                    }
+                // ---- U^T of the next chunk
+                if (n + 1 < nchunks) {
+                    if (!wait(B_FULL + (b ^ 1), (uint32_t)(((n + 1) >> 1) & 1))) break;
+                    tc_fence_after();
+                    GDR_TRACE_AT(1, n + 1);
                     mma_u(n + 1);
                 }
             }
@@ -381,7 +371,7 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
             }
             fence_async_smem();
             tc_fence_before();
-            mbar_arrive(&bar[B_SW_READY]);   // W(n) was converted before
+            mbar_arrive(&bar[B_SW_READY]);
             if (tid == 192) GDR_TRACE_AT(12, n);
             if (!waitw(B_GFULL + (n & 1), (uint32_t)((n >> 1) & 1))) return false;
             const float4 *gm = reinterpret_cast<const float4 *>(sm + OFF_GAM + (n & 1) * 512) + (sc0 >> 2);
@@ -401,53 +391,35 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
             mbar_arrive(&bar[B_GEMPTY + (n & 1)]);
             return true;
         };
-        // W^T(n) -> W: the row of key channel i = 64 tokens = one 128-byte row of
-        // the MN-major operand.  WT_FULL(n) was committed after every MMA of
-        // chunk n - 1 that reads W, so the buffer is free.
-        auto convert_w = [&](int n) -> bool {
-            if (!waitw(B_WT_FULL, (uint32_t)(n & 1))) return false;
-            tc_fence_after();
-            if (tid == 192) GDR_TRACE_AT(4, n);
-            {
-                uint32_t r0[16], r1[16];
-                tmem_ld16(trow + TM_W + vc0, r0);
-                tmem_ld16(trow + TM_W + vc0 + 16, r1);
-                tmem_ld_wait(r0);
-                reg_touch(r1);
-                uint4 lo, hi;
-                pack16(r0, lo, hi);
-                *reinterpret_cast<uint4 *>(sm + OFF_W + sw128_off(i, vc0)) = lo;
-                *reinterpret_cast<uint4 *>(sm + OFF_W + sw128_off(i, vc0 + 8)) = hi;
-                pack16(r1, lo, hi);
-                *reinterpret_cast<uint4 *>(sm + OFF_W + sw128_off(i, vc0 + 16)) = lo;
-                *reinterpret_cast<uint4 *>(sm + OFF_W + sw128_off(i, vc0 + 24)) = hi;
-            }
-            if (tid == 192) GDR_TRACE_AT(5, n);
-            return true;
-        };
+        // Output of chunk m: O^T (TMEM, rows d_v) -> bf16 into the staging tile
+        // laid out as the TMA store wants it ([64 tokens x 64 d_v] panels,
+        // 128-byte swizzle), then one thread stores it.  The staging tile is
+        // reused only after the previous store has finished reading it.
         auto epilogue = [&](int m) -> bool {
             const int bb = m & 1;
-            if (!waitw(B_O_FULL + bb, (uint32_t)((m >> 1) & 1))) return false;
+            if (!waitw(B_EPI_FREE, (uint32_t)(m & 1)) || !waitw(B_O_FULL + bb, (uint32_t)((m >> 1) & 1))) return false;
             tc_fence_after();
-            const int nvalid = min(kC, T_len - m * kC);
-            __nv_bfloat16 *orow_ptr = O + (tok0 + (size_t)m * kC) * kD + i;
+            // row t of a panel, column i & 63: t * 128 + (((i & 63) / 8) ^ (t % 8)) * 16 + (i % 8) * 2
+            unsigned char *ost = sm + OFF_OST + (i >> 6) * 8192 + (i & 7) * 2 + vc0 * 128;
+            const uint32_t c8 = (uint32_t)((i & 63) >> 3);
+#pragma unroll 2
+            for (int cb = 0; cb < 4; ++cb) {   // 8 tokens per step: rows vc0 + 8 cb + j, j = t % 8
+                uint32_t r[8];
+                tmem_ld8(trow + TM_O + 64 * bb + vc0 + 8 * cb, r);
+                tmem_ld_wait8(r);
+                unsigned char *rowp = ost + cb * 1024;
 #pragma unroll
-            for (int cb = 0; cb < 2; ++cb) {
-                uint32_t r[16];
-                __syncwarp();   // the bounded stores below diverge the warp; tcgen05.ld needs it converged
-                tmem_ld16(trow + TM_O + 64 * bb + vc0 + 16 * cb, r);
-                tmem_ld_wait(r);
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int t = vc0 + 16 * cb + j;
-                    if (t < nvalid) orow_ptr[(size_t)t * kD] = __float2bfloat16_rn(__uint_as_float(r[j]));
-                }
+                for (int j = 0; j < 8; ++j)
+                    *reinterpret_cast<__nv_bfloat16 *>(rowp + j * 128 + ((c8 ^ (uint32_t)j) << 4)) =
+                        __float2bfloat16_rn(__uint_as_float(r[j]));
             }
             tc_fence_before();
             mbar_arrive(&bar[B_OACC_EMPTY + bb]);
+            fence_async_smem();
+            mbar_arrive(&bar[B_EPI_FULL]);
             return true;
         };
-        bool ok = nchunks == 0 || convert_w(0);
+        bool ok = true;
         for (int n = 0; n < nchunks && ok; ++n) {
             const uint32_t par = (uint32_t)(n & 1);
             // ---- S_n -> bf16 smem (the MMAs of chunk n - 1 that read the old
@@ -477,10 +449,7 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
             tc_fence_before();
             mbar_arrive(&bar[B_VN_READY]);   // also: S_n scaled
             if (tid == 192) GDR_TRACE_AT(14, n);
-            // ---- off the sequential path while S += dS runs: next chunk's W,
-            // last chunk's output
-            if (n + 1 < nchunks && !convert_w(n + 1)) { ok = false; break; }
-            if (tid == 192) GDR_TRACE_AT(6, n);
+            // ---- off the sequential path while S += dS runs: last chunk's output
             if (n > 0 && !epilogue(n - 1)) { ok = false; break; }
             if (tid == 192) GDR_TRACE_AT(7, n);
         }
@@ -559,8 +528,8 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream, int *launch
         const cuuint64_t dims3[3] = {(cuuint64_t)kD, (cuuint64_t)a.T, (cuuint64_t)BH};
         const cuuint64_t str_bf[2] = {(cuuint64_t)kD * 2, (cuuint64_t)a.T * kD * 2};
         const cuuint32_t box_bf[3] = {64, 64, 1};
-        void *tiles[4] = {w.Kl, w.Ql, w.Kt, const_cast<void *>(a.v)};
-        CUtensorMap *dst[4] = {&maps.k, &maps.q, &maps.kt, &maps.v};
+        void *tiles[4] = {w.Ql, w.Kt, const_cast<void *>(a.v), a.O};
+        CUtensorMap *dst[4] = {&maps.q, &maps.kt, &maps.v, &maps.o};
         for (int i = 0; i < 4; ++i)
             if (!make_map(dst[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, tiles[i], dims3, str_bf, box_bf,
                           CU_TENSOR_MAP_SWIZZLE_128B))
@@ -568,7 +537,10 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream, int *launch
         const cuuint64_t dims2[2] = {(cuuint64_t)kC, (cuuint64_t)BH * nchunks * kC};
         const cuuint64_t str2[1] = {(cuuint64_t)kC * 2};
         const cuuint32_t box2[2] = {64, 64};
-        if (!make_map(&maps.t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w.T, dims2, str2, box2, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        const cuuint64_t dimsw[2] = {(cuuint64_t)kC, (cuuint64_t)BH * nchunks * kD};
+        const cuuint32_t boxw[2] = {64, 128};
+        if (!make_map(&maps.w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w.W, dimsw, str2, boxw, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_map(&maps.t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w.T, dims2, str2, box2, CU_TENSOR_MAP_SWIZZLE_128B) ||
             !make_map(&maps.aq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w.Aqk, dims2, str2, box2, CU_TENSOR_MAP_SWIZZLE_128B))
             return cudaErrorInvalidValue;
     }

@@ -32,17 +32,18 @@ struct StepArgs {
 
 // The tensor-core path's scratch, carved out of ChunkArgs::workspace (every
 // part starts on a 256-byte boundary):
-//   T, Aqk      [B*H*chunks][64][64] bf16   T' = (I + A)^{-1} Diag(beta) and Aqk
-//   Kl, Ql, Kt  [B, H, T, 128] bf16         K<-, Q<-, K_tail (chunk-relative decays)
-//   gam         [B*H*chunks][128] fp32      gamma_C per key channel
+//   T, Aqk   [B*H*chunks][64][64] bf16    T' = (I + A)^{-1} Diag(beta) and Aqk
+//   W        [B*H*chunks][128][64] bf16   W^T, W = T' K<- (key channel rows)
+//   Ql, Kt   [B, H, T, 128] bf16          Q<-, K_tail (chunk-relative decays)
+//   gam      [B*H*chunks][128] fp32       gamma_C per key channel
 struct TcWorkspace {
-    __nv_bfloat16 *T, *Aqk, *Kl, *Ql, *Kt;
+    __nv_bfloat16 *T, *Aqk, *W, *Ql, *Kt;
     float *gam;
 };
 inline size_t tc_workspace_bytes(int B, int H, int T)
 {
     const size_t bh = (size_t)B * H, nch = (size_t)(T + 63) / 64;
-    return 2 * bh * nch * 64 * 64 * 2 + 3 * bh * (size_t)T * 128 * 2 + bh * nch * 128 * 4;
+    return 2 * bh * nch * 64 * 64 * 2 + bh * nch * 128 * 64 * 2 + 2 * bh * (size_t)T * 128 * 2 + bh * nch * 128 * 4;
 }
 inline TcWorkspace carve_tc_workspace(void *ws, int B, int H, int T)
 {
@@ -53,8 +54,8 @@ inline TcWorkspace carve_tc_workspace(void *ws, int B, int H, int T)
     p += bh * nch * 64 * 64 * 2;
     w.Aqk = reinterpret_cast<__nv_bfloat16 *>(p);
     p += bh * nch * 64 * 64 * 2;
-    w.Kl = reinterpret_cast<__nv_bfloat16 *>(p);
-    p += bh * (size_t)T * 128 * 2;
+    w.W = reinterpret_cast<__nv_bfloat16 *>(p);
+    p += bh * nch * 128 * 64 * 2;
     w.Ql = reinterpret_cast<__nv_bfloat16 *>(p);
     p += bh * (size_t)T * 128 * 2;
     w.Kt = reinterpret_cast<__nv_bfloat16 *>(p);

@@ -5,8 +5,9 @@
 //   Aqk[r][i] =        sum_c q_rc k_ic exp(G_rc - G_ic)     (i <= r)
 //   T' = (I + A)^{-1} Diag(beta)
 // and writes T' and Aqk (bf16, row-major 64 x 64) to the workspace, together
-// with the chunk-relative operands of the state scan (K<-, Q<-, K_tail and
-// gamma_C, defined where they are written).  T' is
+// with the operands of the state scan that do not depend on the state:
+// W = T' K<- (stored transposed), Q<-, K_tail and gamma_C (defined where they
+// are written).  T' is
 // the matrix the UT transform of "Token Mixer I", section "Kimi Delta
 // Attention: Improving Delta Rule with Fine-grained Gating" calls
 // M = (I + StrictTril(Diag(beta)(Gamma*K)(K/Gamma)^T))^{-1} Diag(beta), so
@@ -70,8 +71,9 @@ constexpr int kLdA = 68;       // fp32 row stride: 16-byte rows, conflict-free f
 
 // shared memory (offsets from a 1024-byte aligned base)
 constexpr uint32_t OFF_K = 0;                      // Khat (or k), two swizzled panels   16 KB
-constexpr uint32_t OFF_Q = 16384;                  // Qhat (or q)                         16 KB
-constexpr uint32_t OFF_KC = 32768;                 // Kchk                                16 KB
+constexpr uint32_t OFF_Q = 16384;                  // Qhat (or q); then T' bf16 [64][72]   16 KB
+constexpr uint32_t OFF_KC = 32768;                 // Kchk; then W^T staging, 2 KB/warp   16 KB
+constexpr int kLdT = 72;                           // bf16 row stride of T' (ldmatrix conflict free)
 constexpr uint32_t OFF_BD = 49152;                 // bd[4][128], 1/bd[4][128] fp32         4 KB
 constexpr int kLdD = 24;       // row stride of the 16 x 16 blocks (conflict-free mma B fragments)
 constexpr uint32_t OFF_D = OFF_BD + 4096;          // D_i = N_ii^{-1}, [4][16][24]           6 KB
@@ -89,6 +91,21 @@ __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr)
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                  : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], uint32_t addr)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+// two 8x8 bf16 matrices from mma fragments, stored transposed (lanes 0..15
+// give the row addresses of the transposed matrices)
+__device__ __forceinline__ void stsm_x2_trans(uint32_t addr, uint32_t r0, uint32_t r1)
+{
+    asm volatile("stmatrix.sync.aligned.m8n8.x2.trans.shared.b16 [%0], {%1, %2};" ::"r"(addr), "r"(r0), "r"(r1)
+                 : "memory");
 }
 
 __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
@@ -177,7 +194,7 @@ template <bool SCALAR>
 __global__ void __launch_bounds__(kThreads, 2)
 ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__restrict__ qg,
                const float *__restrict__ gg, const float *__restrict__ betag, __nv_bfloat16 *__restrict__ Tout,
-               __nv_bfloat16 *__restrict__ Aqout, __nv_bfloat16 *__restrict__ Klo, __nv_bfloat16 *__restrict__ Qlo,
+               __nv_bfloat16 *__restrict__ Aqout, __nv_bfloat16 *__restrict__ Wout, __nv_bfloat16 *__restrict__ Qlo,
                __nv_bfloat16 *__restrict__ Kto, float *__restrict__ gamo, int T_len, int nchunks, int total)
 {
     extern __shared__ unsigned char prep_raw[];
@@ -300,9 +317,10 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
 
         // ---- chunk-relative operands of the state scan, to global memory in
         // the layout of k ([B, H, T, 128] bf16), G counted from the chunk start:
-        //   K<-_r = k_r exp(G_r),  Q<-_r = q_r exp(G_r),  K_tail_r = k_r exp(G_C - G_r)
+        //   Q<-_r = q_r exp(G_r),  K_tail_r = k_r exp(G_C - G_r)
         // and gamma_C = exp(G_C) per key channel (fp32, [B H chunks][128]).
         // Formed in fp32 from the registers above, with the block decays bd_J.
+        // (K<-_r = k_r exp(G_r) is only needed inside W = T' K<-, formed below.)
         {
             const size_t e0 = row0 * kDK + c;
             if (!SCALAR) {
@@ -325,7 +343,6 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
                     pb = fmul2(pb, make_float2(gv[rr].z, gv[rr].w));
                     if (rbase + rr < nrows) {
                         const size_t e = e0 + (size_t)(rbase + rr) * kDK;
-                        *reinterpret_cast<uint2 *>(Klo + e) = make_uint2(scale2p(kr[rr].x, pa), scale2p(kr[rr].y, pb));
                         *reinterpret_cast<uint2 *>(Qlo + e) = make_uint2(scale2p(qr[rr].x, pa), scale2p(qr[rr].y, pb));
                     }
                 }
@@ -354,7 +371,6 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
                         const float ef = __expf(sGc[r]), et = __expf(Gl - sGc[r]);
                         const float2 fe = make_float2(ef, ef), ft = make_float2(et, et);
                         const size_t e = e0 + (size_t)r * kDK;
-                        *reinterpret_cast<uint2 *>(Klo + e) = make_uint2(scale2p(kr[rr].x, fe), scale2p(kr[rr].y, fe));
                         *reinterpret_cast<uint2 *>(Qlo + e) = make_uint2(scale2p(qr[rr].x, fe), scale2p(qr[rr].y, fe));
                         *reinterpret_cast<uint2 *>(Kto + e) = make_uint2(scale2p(kr[rr].x, ft), scale2p(kr[rr].y, ft));
                     }
@@ -455,6 +471,11 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
         }
         __syncthreads();
 
+        // T' (bf16) is also kept in shared memory as the left operand of
+        // W = T' K<-; with a scalar gate its columns carry exp(G_r) there, so
+        // that W = (T' Diag(exp(G))) K.
+        __nv_bfloat16(*sT)[kLdT] = reinterpret_cast<__nv_bfloat16(*)[kLdT]>(sm + OFF_Q);
+        auto tcol = [&](int col) { return SCALAR ? sBeta[col] * __expf(sGc[col]) : sBeta[col]; };
         // T' block (i, j) = U_ij Diag(beta_j) from a 16 x 16 accumulator fragment
         auto store_t = [&](const float (&c)[2][4], int i, int j) {
 #pragma unroll
@@ -464,6 +485,9 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
                 __nv_bfloat16 *dst = Tout + cbase + (size_t)(16 * i + g) * kC + col;
                 *reinterpret_cast<uint32_t *>(dst) = pack2(c[nt][0] * b0, c[nt][1] * b1);
                 *reinterpret_cast<uint32_t *>(dst + 8 * kC) = pack2(c[nt][2] * b0, c[nt][3] * b1);
+                const float s0 = SCALAR ? tcol(col) : b0, s1 = SCALAR ? tcol(col + 1) : b1;
+                *reinterpret_cast<uint32_t *>(&sT[16 * i + g][col]) = pack2(c[nt][0] * s0, c[nt][1] * s1);
+                *reinterpret_cast<uint32_t *>(&sT[16 * i + g + 8][col]) = pack2(c[nt][2] * s0, c[nt][3] * s1);
             }
         };
         auto store_s = [&](const float (&c)[2][4], float (*dst)[kLdD]) {
@@ -495,7 +519,7 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
             for (int task = tid - 192; task < kC * 8; task += 64) {
                 const int r = task >> 3, g8 = task & 7, i = r >> 4, jb = g8 >> 1;
                 if (jb < i) continue;
-                uint4 o = make_uint4(0u, 0u, 0u, 0u);
+                uint4 o = make_uint4(0u, 0u, 0u, 0u), os = o;
                 if (jb == i) {
                     const int ch = 8 * (g8 & 1), cl = 16 * jb + ch;
                     const float4 d0 = *reinterpret_cast<const float4 *>(&sD[i][r & 15][ch]);
@@ -504,8 +528,17 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
                     o.y = pack2(d0.z * sBeta[cl + 2], d0.w * sBeta[cl + 3]);
                     o.z = pack2(d1.x * sBeta[cl + 4], d1.y * sBeta[cl + 5]);
                     o.w = pack2(d1.z * sBeta[cl + 6], d1.w * sBeta[cl + 7]);
+                    if (SCALAR) {
+                        os.x = pack2(d0.x * tcol(cl + 0), d0.y * tcol(cl + 1));
+                        os.y = pack2(d0.z * tcol(cl + 2), d0.w * tcol(cl + 3));
+                        os.z = pack2(d1.x * tcol(cl + 4), d1.y * tcol(cl + 5));
+                        os.w = pack2(d1.z * tcol(cl + 6), d1.w * tcol(cl + 7));
+                    } else {
+                        os = o;
+                    }
                 }
                 *reinterpret_cast<uint4 *>(Tout + cbase + r * kC + 8 * g8) = o;
+                *reinterpret_cast<uint4 *>(&sT[r][8 * g8]) = os;
             }
         }
         __syncthreads();
@@ -536,9 +569,76 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
             mm16_sub(acc, &sQ[48][32], kLdA, &sU[2][0][0], kLdD, g, t);
             store_t(acc, 3, 0);
         }
-        // no barrier here: the next chunk's first writes (operand tiles, the
-        // other beta buffer) touch nothing warp 5 still reads, and its next
-        // barrier waits for warp 5
+        __syncthreads();
+
+        // ---- W = T' K<- for the state scan, stored as W^T [128 channels][64 tokens].
+        // Per-channel gate: K<-_r = Khat_r * F_R with F_R = prod_{J<R} bd_J (row r
+        // in block R), so W = sum_R (T'[:, block R] Khat_R) Diag(F_R): one fp32
+        // accumulator per block, combined after the products.  Scalar gate: the
+        // decay sits in T' (above) and Khat is k.  Warp w owns channels
+        // 16w..16w+15 (two 8-channel tiles), all 64 tokens, in 4 token blocks.
+        {
+            const int c0 = 16 * warp;
+            unsigned char *stg = sm + OFF_KC + warp * 2048;   // 16 rows x 128 B, 16-byte chunks XOR-swizzled
+            const uint32_t khat = smem_u32(sm + OFF_K);
+#pragma unroll
+            for (int ct = 0; ct < 2; ++ct) {
+                const int cs = c0 + 8 * ct;                  // first channel of this tile
+                float2 fr[4];                                // F_R at channels cs + 2t, + 1
+                fr[0] = make_float2(1.f, 1.f);
+#pragma unroll
+                for (int R = 1; R < 4; ++R) {
+                    const float2 bdp = SCALAR ? make_float2(1.f, 1.f)
+                                              : *reinterpret_cast<const float2 *>(sBd + (R - 1) * kDK + cs + 2 * t);
+                    fr[R] = make_float2(fr[R - 1].x * bdp.x, fr[R - 1].y * bdp.y);
+                }
+                // B fragments (Khat rows of block R, channels cs..cs+7), shared by all token blocks
+                uint32_t bf[4][2];
+#pragma unroll
+                for (int R = 0; R < 4; ++R) {
+                    uint32_t r4[4];
+                    ldsm_x4_trans(r4, khat + tile_off(16 * R + (lane & 15), cs));
+                    bf[R][0] = r4[0];
+                    bf[R][1] = r4[1];
+                }
+#pragma unroll
+                for (int I = 0; I < 4; ++I) {
+                    float w4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int R = 0; R <= I; ++R) {
+                        uint32_t a[4];
+                        ldsm_x4(a, smem_u32(&sT[16 * I + (lane & 15)][16 * R + (lane >> 4) * 8]));
+                        float accR[4] = {0.f, 0.f, 0.f, 0.f};
+                        mma16816(accR, a, bf[R][0], bf[R][1]);
+                        w4[0] = fmaf(accR[0], fr[R].x, w4[0]);
+                        w4[1] = fmaf(accR[1], fr[R].y, w4[1]);
+                        w4[2] = fmaf(accR[2], fr[R].x, w4[2]);
+                        w4[3] = fmaf(accR[3], fr[R].y, w4[3]);
+                    }
+                    // W^T[channel][token]: the fragment (tokens 16I + g (+8), channels
+                    // 2t, 2t + 1) is two 8x8 matrices; stored transposed, matrix h
+                    // lands in channel rows 8 ct .. 8 ct + 7, token chunk 2I + h.
+                    {
+                        const int row = 8 * ct + (lane & 7), chunk = (2 * I + ((lane >> 3) & 1)) ^ (row & 7);
+                        stsm_x2_trans(smem_u32(stg + row * 128 + chunk * 16), pack2(w4[0], w4[1]), pack2(w4[2], w4[3]));
+                    }
+                }
+            }
+            __syncwarp();
+            // this warp's 16 rows (2 KB) of W^T to global: lane -> row lane/2, half a row
+            {
+                const int row = lane >> 1, h = lane & 1;
+                __nv_bfloat16 *dst = Wout + ((size_t)ci * kDK + c0 + row) * kC + 32 * h;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int chunk = 4 * h + q;
+                    *reinterpret_cast<uint4 *>(dst + 8 * q) =
+                        *reinterpret_cast<const uint4 *>(stg + row * 128 + ((chunk ^ (row & 7)) << 4));
+                }
+            }
+        }
+        // the next chunk overwrites Khat, T' and the staging area
+        __syncthreads();
     }
 }
 
@@ -571,7 +671,7 @@ cudaError_t launch_ut_prep(const ChunkArgs &a, const TcWorkspace &w, cudaStream_
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_ALLOC);
     if (e != cudaSuccess) return e;
     kern<<<grid, kThreads, SMEM_ALLOC, stream>>>((const __nv_bfloat16 *)a.k, (const __nv_bfloat16 *)a.q, a.g,
-                                                 a.beta, w.T, w.Aqk, w.Kl, w.Ql, w.Kt, w.gam, a.T, nchunks,
+                                                 a.beta, w.T, w.Aqk, w.W, w.Ql, w.Kt, w.gam, a.T, nchunks,
                                                  (int)total);
     return cudaGetLastError();
 }

@@ -46,10 +46,19 @@ METRIC = "tokens/s (device-timed) of gated-delta-rule chunk fwd; % of roofline"
 METRIC_DECODE = "tokens/s (device-timed) of gated-delta-rule recurrent decode step; % of HBM roofline"
 DEFAULT_WORKLOAD = "kda_d128_t8192"
 
-# DRAM traffic per launch of the dominant kernel, from one ncu capture, keyed
-# by the kernel's source file and that file's hash when captured; the entry
-# is ignored (traffic = null) as soon as the source changes.
-TRAFFIC = {}
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per call of the
+# path, from one ncu capture of every kernel the call launches, keyed by
+# workload with the hash of the sources those kernels are built from; an
+# entry is ignored (traffic = null) as soon as any of the sources changes.
+TRAFFIC = {
+    # ut_prep 539.0 MB read + 493.2 MB written, chunk_scan 679.6 + 118.3 MB (one launch each)
+    "kda_d128_t8192": {"src_sha": "ec261bf9c0fc7bca", "bytes_per_launch": 1830078976},
+    # recurrent_step, one decode step: 547.4 MB read + 479.2 MB written
+    "kda_decode_b256": {"src_sha": "99a0454504c77460", "bytes_per_launch": 1026655488},
+}
+
+CHUNK_SOURCES = ("chunk_tc.cu", "ut_prep.cu", "sm100_ptx.cuh", "gdr_internal.cuh")
+DECODE_SOURCES = ("recurrent_step.cu", "gdr_internal.cuh")
 
 
 # ----------------------------------------------------------------- helpers
@@ -107,11 +116,17 @@ def roofline(w: W.Workload, seconds_per_launch: float, peaks, kernel_src: str = 
             "peak_source": peaks["source"], "algorithmic_flops": flops}
 
 
-def file_sha(path: str) -> str:
+def file_sha(paths) -> str:
+    """Hash of the concatenated sources (one path or several)."""
+    if isinstance(paths, str):
+        paths = [paths]
+    h = hashlib.sha256()
     try:
-        return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+        for p in paths:
+            h.update(open(p, "rb").read())
     except OSError:
         return ""
+    return h.hexdigest()[:16]
 
 
 def rank_workload(w: W.Workload, rank: int) -> W.Workload:
@@ -428,8 +443,8 @@ def main():
         if w.kind == "decode":
             import dataclasses
             wk = dataclasses.replace(w0, T=1)   # one launch = one decode step
-        src = os.path.join(ROOT, "gated_delta_rule_89_b200", "csrc",
-                           "recurrent_step.cu" if w.kind == "decode" else "chunk_tc.cu")
+        src = [os.path.join(ROOT, "gated_delta_rule_89_b200", "csrc", f)
+               for f in (DECODE_SOURCES if w.kind == "decode" else CHUNK_SOURCES)]
         line = base_line(w0, args, world)
         line.update({
             "value": value,

@@ -135,6 +135,11 @@ def rank_workload(w: W.Workload, rank: int) -> W.Workload:
     return dataclasses.replace(w, seed=w.seed + 1000 * rank)
 
 
+def job_throughput(units_per_rank_step: int, world: int, total_ms_max: float, steps: int) -> float:
+    """Weak scaling: units all ranks processed per second of the slowest rank."""
+    return units_per_rank_step * world / (total_ms_max / steps / 1e3)
+
+
 def reduce_max(x: float, world: int, device) -> float:
     if world <= 1:
         return x
@@ -404,8 +409,7 @@ def main():
     total_ms = reduce_max(total_ms, world, device)
     ms_per_step = total_ms / args.steps
     # chunk: B*T tokens per step; decode: B sequences x T consecutive steps
-    tokens_job = w.B * w.T * world
-    value = tokens_job / (ms_per_step / 1e3)
+    value = job_throughput(w.B * w.T, world, total_ms, args.steps)
 
     # ---- end to end through the public API with host buffers (pinned)
     e2e = None

@@ -40,6 +40,8 @@ _STREAM = 0xD1B54A32D192ED03
 
 # tensor ids: one independent stream per input tensor
 TID_Q, TID_K, TID_V, TID_G, TID_BETA, TID_S0, TID_CHAN = 1, 2, 3, 4, 5, 6, 7
+# raw inputs of the fused gate / normalisation prologue
+TID_QRAW, TID_KRAW, TID_AGATE, TID_ALOG, TID_DTBIAS, TID_BLOGIT = 8, 9, 10, 11, 12, 13
 
 
 def _s64(c: int) -> int:
@@ -298,6 +300,44 @@ def generate(w: Workload, device="cpu", heads: Optional[Sequence[int]] = None,
                    g=shp(g, dk) if w.gate == "per_channel" else shp(g),
                    beta=shp(beta), S0=S0.view(outB, outH, dv, dk))
     return out
+
+
+def generate_prologue(w: Workload, device="cpu", block: int = 1 << 24) -> Dict[str, torch.Tensor]:
+    """Raw inputs of the forward with its gate / normalisation prologue.
+
+    q_raw, k_raw [B,H,T,dk] ~ N(0,1) (not normalised), v [B,H,T,dv] ~ N(0,1)
+    (the same values ``generate`` draws), gate pre-activation a [B,H,T,dk]
+    (per-channel) or [B,H,T] (scalar) ~ N(0,1), A_log [H] ~ U(-1,1),
+    dt_bias [H,dk] (per-channel) or [H] ~ N(0, 0.5^2), beta logits [B,H,T]
+    ~ N(0,1) fp32, S0 as in ``generate``.  q_raw, k_raw, v and a are in the
+    workload dtype; A_log, dt_bias and the logits are fp32.  No prologue
+    arithmetic here: the L2 normalisation, softplus gate and sigmoid belong
+    to the oracle and the kernels.
+    """
+    assert w.kind == "chunk"
+    B, H, T, dk, dv, seed = w.B, w.H, w.T, w.dk, w.dv, w.seed
+
+    def draw(tid, shape, make):
+        n = 1
+        for d in shape:
+            n *= d
+        out = torch.empty(n, dtype=torch.float64, device=device)
+        for s, e in _chunked(n, block):
+            out[s:e] = make(tid, torch.arange(s, e, dtype=torch.int64, device=device))
+        return out.view(*shape)
+
+    nrm = lambda tid, idx: normal(seed, tid, idx)
+    q_raw = to_dtype(draw(TID_QRAW, (B, H, T, dk), nrm), w.dtype)
+    k_raw = to_dtype(draw(TID_KRAW, (B, H, T, dk), nrm), w.dtype)
+    v = to_dtype(draw(TID_V, (B, H, T, dv), nrm), w.dtype)
+    a_shape = (B, H, T, dk) if w.gate == "per_channel" else (B, H, T)
+    a = to_dtype(draw(TID_AGATE, a_shape, nrm), w.dtype)
+    A_log = draw(TID_ALOG, (H,), lambda tid, idx: 2.0 * uniform(seed, tid, idx) - 1.0).to(torch.float32)
+    dt_shape = (H, dk) if w.gate == "per_channel" else (H,)
+    dt_bias = draw(TID_DTBIAS, dt_shape, lambda tid, idx: 0.5 * normal(seed, tid, idx)).to(torch.float32)
+    b_logit = draw(TID_BLOGIT, (B, H, T), nrm).to(torch.float32)
+    S0 = generate(dataclasses.replace(w, T=1), device=device)["S0"]
+    return dict(q_raw=q_raw, k_raw=k_raw, v=v, a=a, A_log=A_log, dt_bias=dt_bias, b_logit=b_logit, S0=S0)
 
 
 def small_chunk_case(B: int, H: int, T: int, dk: int, dv: int, gate: str, dtype: torch.dtype,

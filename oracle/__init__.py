@@ -10,6 +10,9 @@ Contents
   * ``forward``   -- the token-by-token fp64 recurrence (``gdr_oracle.c``),
     the parity reference for the chunked forward and the decode step.
   * ``decode``    -- the same recurrence driven one decode step per token.
+  * ``prologue`` / ``forward_prologue`` -- the input prologue (L2-normalised
+    q, k; softplus gate with the -5 bound; sigmoid beta) and the forward fed
+    by it, the reference of the fused-prologue entry point.
   * ``chunk_form`` (module) -- an fp64 restatement of the chunkwise WY/UT
     equations, used only to pin ``forward`` (it is not a parity reference).
 
@@ -108,6 +111,50 @@ def forward(q, k, v, g, beta, S0=None, gate: str = "per_channel", erase=None, wr
     if rc != 0:
         raise RuntimeError("oracle forward failed")
     return O, ST
+
+
+L2NORM_EPS = 1e-6   # the pages do not give the epsilon of L2Norm; see the reading in the design notes
+
+
+def prologue(q_raw, k_raw, a, A_log, dt_bias, b_logit, gate: str = "per_channel"):
+    """The input prologue of a KDA / Gated DeltaNet layer, in fp64.
+
+    "Token Mixer I", section "Kimi Delta Attention", Neural
+    Parameterization: q and k are L2-normalised per head and token, and
+    beta = Sigmoid(logit).  "Kimi Linear paper notes", gate paragraph: the
+    log-decay is -exp(A_log) * softplus(a + dt_bias), with A_log per head and
+    dt_bias per head and key channel (per head for a scalar gate); KDA bounds
+    the per-channel log-decay below by g_min = -5 ("KDA engineering notes",
+    lower-bounded decay).
+
+    Shapes: q_raw, k_raw [B,H,T,dk]; a [B,H,T,dk] or [B,H,T]; A_log [H];
+    dt_bias [H,dk] or [H]; b_logit [B,H,T].  Returns fp64 (q, k, g, beta).
+    """
+    q = _f64(q_raw)
+    k = _f64(k_raw)
+    q = q / np.sqrt((q * q).sum(-1, keepdims=True) + L2NORM_EPS)
+    k = k / np.sqrt((k * k).sum(-1, keepdims=True) + L2NORM_EPS)
+    A = np.exp(_f64(A_log))                       # [H]
+    z = _f64(a)
+    dtb = _f64(dt_bias)
+    if gate == "per_channel":
+        z = z + dtb[None, :, None, :]
+        sp = np.logaddexp(0.0, z)                 # softplus(z) = log(1 + e^z)
+        g = np.maximum(-A[None, :, None, None] * sp, -5.0)
+    elif gate == "scalar":
+        z = z + dtb[None, :, None]
+        g = -A[None, :, None] * np.logaddexp(0.0, z)
+    else:
+        raise ValueError(gate)
+    beta = 1.0 / (1.0 + np.exp(-_f64(b_logit)))
+    return q, k, g, beta
+
+
+def forward_prologue(q_raw, k_raw, v, a, A_log, dt_bias, b_logit, S0=None, gate: str = "per_channel",
+                     threads: int = 0) -> Tuple[np.ndarray, np.ndarray]:
+    """``prologue`` then ``forward``: the reference of the fused-prologue forward."""
+    q, k, g, beta = prologue(q_raw, k_raw, a, A_log, dt_bias, b_logit, gate)
+    return forward(q, k, v, g, beta, S0, gate=gate, clamp=False, threads=threads)
 
 
 def decode(q, k, v, g, beta, S, gate: str = "per_channel", threads: int = 0) -> Tuple[np.ndarray, np.ndarray]:

@@ -68,6 +68,8 @@ def algorithmic_bytes(w: W.Workload) -> int:
     written once (no intermediates)."""
     e = 2 if w.dtype == torch.bfloat16 else 4
     gate = w.dk * 4 if w.gate == "per_channel" else 4
+    if w.g_recipe == "prologue":    # gate pre-activation in the input dtype, beta logits fp32
+        gate = w.dk * e if w.gate == "per_channel" else e
     per_token = 2 * w.dk * e + w.dv * e + gate + 4 + w.dv * e       # q, k, v, g, beta, O
     heads = w.B * w.H
     state = 2 * w.dv * w.dk * 4                                     # S0 read + S_T write
@@ -222,6 +224,14 @@ def gpu_id_for(device) -> str:
 
 # ------------------------------------------------------------ CPU oracle leg
 
+def api_call(gdr, w: W.Workload, x, **kw):
+    """One forward of workload ``w`` through the public Python API."""
+    if w.g_recipe == "prologue":
+        return gdr.chunk_fwd_prologue(x["q_raw"], x["k_raw"], x["v"], x["a"], x["A_log"], x["dt_bias"],
+                                      x["b_logit"], x["S0"], C=w.C, gate=w.gate, **kw)
+    return gdr.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], C=w.C, gate=w.gate, **kw)
+
+
 def oracle_sample(w: W.Workload, budget_s: float, seed_rank: int = 0):
     """Time the fp64 oracle on a bounded sample of workload ``w``.
 
@@ -244,6 +254,15 @@ def oracle_sample(w: W.Workload, budget_s: float, seed_rank: int = 0):
             x = W.generate(w, heads=hl, steps=ntok)
             t = time.perf_counter()
             oracle.decode(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], gate=w.gate, threads=cores)
+            return time.perf_counter() - t
+        if w.g_recipe == "prologue":
+            # the sampled heads laid out as B = 1, H = len(hl), with their own A_log, dt_bias
+            x = W.generate_prologue(w, heads=hl)
+            sl = lambda a: a.transpose(0, 1)[:, :, :ntok].contiguous()
+            args = [sl(x[k]) for k in ("q_raw", "k_raw", "v", "a")]
+            t = time.perf_counter()
+            oracle.forward_prologue(*args, x["A_log"], x["dt_bias"], sl(x["b_logit"]), x["S0"].transpose(0, 1),
+                                    gate=w.gate, threads=cores)
             return time.perf_counter() - t
         x = W.generate(w, heads=hl)
         sl = lambda a: a[:, :, :ntok].contiguous()
@@ -372,6 +391,13 @@ def main():
         def step():
             for s in range(w.T):
                 gdr.recurrent_step(x["q"][s], x["k"][s], x["v"][s], x["g"][s], x["beta"][s], S, o=o)
+    elif w.g_recipe == "prologue":
+        x = W.generate_prologue(w, device=device)
+        O = torch.empty(w.B, w.H, w.T, w.dv, dtype=w.dtype, device=device)
+        S_T = torch.empty(w.B, w.H, w.dv, w.dk, dtype=torch.float32, device=device)
+
+        def step():
+            api_call(gdr, w, x, O=O, S_T=S_T)
     else:
         x = W.generate(w, device=device)
         O = torch.empty(w.B, w.H, w.T, w.dv, dtype=w.dtype, device=device)
@@ -417,14 +443,14 @@ def main():
         hx = {k: v.to("cpu").pin_memory() for k, v in x.items()}
         h2d = sum(v.numel() * v.element_size() for v in hx.values())
         d2h = O.numel() * O.element_size() + S_T.numel() * S_T.element_size()
-        gdr.chunk_fwd(hx["q"], hx["k"], hx["v"], hx["g"], hx["beta"], hx["S0"], C=w.C, gate=w.gate)  # warm
+        api_call(gdr, w, hx)  # warm
         torch.cuda.synchronize(device)
         if world > 1:
             dist.barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(args.e2e_steps):
-            Oh, Sh = gdr.chunk_fwd(hx["q"], hx["k"], hx["v"], hx["g"], hx["beta"], hx["S0"], C=w.C, gate=w.gate)
+            Oh, Sh = api_call(gdr, w, hx)
         e1.record(stream)
         torch.cuda.synchronize(device)
         e2e_ms = reduce_max(e0.elapsed_time(e1), world, device) / args.e2e_steps

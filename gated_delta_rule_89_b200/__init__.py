@@ -51,6 +51,8 @@ def lib() -> ctypes.CDLL:
         P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
         L.gdr_chunk_fwd.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P, Z, P]
         L.gdr_chunk_fwd.restype = I
+        L.gdr_chunk_fwd_prologue.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P, Z, P]
+        L.gdr_chunk_fwd_prologue.restype = I
         L.gdr_recurrent_step.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, P]
         L.gdr_recurrent_step.restype = I
         L.gdr_chunk_fwd_workspace_size.argtypes = [I, I, I, I, I, I, I, I]
@@ -170,6 +172,70 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor
                          B, H, T, dk, dv, C, gm, _DTYPES[dt],
                          _ptr(workspace) if ws_bytes else None, ws_bytes, _stream_handle(dev, stream))
     _check(st, "gdr_chunk_fwd")
+    if host:
+        O = O.to("cpu")
+        S_T = None if S_T is None else S_T.to("cpu")
+    return O, S_T
+
+
+def chunk_fwd_prologue(q_raw: torch.Tensor, k_raw: torch.Tensor, v: torch.Tensor, a: torch.Tensor,
+                       A_log: torch.Tensor, dt_bias: torch.Tensor, b_logit: torch.Tensor,
+                       S0: Optional[torch.Tensor] = None, C: int = 64, gate: Optional[str] = None,
+                       O: Optional[torch.Tensor] = None, S_T: Optional[torch.Tensor] = None,
+                       final_state: bool = True, workspace: Optional[torch.Tensor] = None,
+                       stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Chunkwise forward with the input prologue fused in (``gdr_chunk_fwd_prologue``).
+
+    q_raw, k_raw [B,H,T,dk] and v [B,H,T,dv] bf16 (q, k not normalised);
+    gate pre-activation a bf16 [B,H,T,dk] (per-channel) or [B,H,T] (scalar);
+    A_log fp32 [H]; dt_bias fp32 [H,dk] or [H]; b_logit fp32 [B,H,T]; S0 fp32
+    [B,H,dv,dk] or None.  Returns (O [B,H,T,dv] bf16, S_T fp32 or None).
+    """
+    host = not q_raw.is_cuda
+    if host:
+        dev = torch.device("cuda", torch.cuda.current_device())
+        q_raw, k_raw, v, a, A_log, dt_bias, b_logit, S0 = (_to_device(x, dev) for x in
+                                                           (q_raw, k_raw, v, a, A_log, dt_bias, b_logit, S0))
+    dev = q_raw.device
+    if gate is None:
+        gate = "per_channel" if a.dim() == 4 else "scalar"
+    B, H, T, dk = q_raw.shape
+    dv = v.shape[-1]
+    dt = q_raw.dtype
+    if dt != torch.bfloat16:
+        raise TypeError("the prologue forward takes bf16 q, k, v, a")
+    for t, n in ((q_raw, "q_raw"), (k_raw, "k_raw"), (v, "v"), (a, "a")):
+        _need(t, n, dt, dev)
+    for t, n in ((A_log, "A_log"), (dt_bias, "dt_bias"), (b_logit, "b_logit")):
+        _need(t, n, torch.float32, dev)
+    if tuple(k_raw.shape) != (B, H, T, dk) or tuple(v.shape[:3]) != (B, H, T) or tuple(b_logit.shape) != (B, H, T):
+        raise ValueError("inconsistent shapes")
+    if tuple(A_log.shape) != (H,):
+        raise ValueError("A_log must be [H]")
+    if gate == "per_channel" and (tuple(a.shape) != (B, H, T, dk) or tuple(dt_bias.shape) != (H, dk)):
+        raise ValueError("per-channel gate: a [B,H,T,dk], dt_bias [H,dk]")
+    if gate == "scalar" and (tuple(a.shape) != (B, H, T) or tuple(dt_bias.shape) != (H,)):
+        raise ValueError("scalar gate: a [B,H,T], dt_bias [H]")
+    if S0 is not None:
+        _need(S0, "S0", torch.float32, dev)
+        if tuple(S0.shape) != (B, H, dv, dk):
+            raise ValueError("S0 must be [B,H,dv,dk]")
+    if O is None:
+        O = torch.empty(B, H, T, dv, dtype=dt, device=dev)
+    _need(O, "O", dt, dev)
+    if S_T is None and final_state:
+        S_T = torch.empty(B, H, dv, dk, dtype=torch.float32, device=dev)
+    if S_T is not None:
+        _need(S_T, "S_T", torch.float32, dev)
+    gm = GATE_PER_CHANNEL if gate == "per_channel" else GATE_SCALAR
+    L = lib()
+    ws_bytes = int(L.gdr_chunk_fwd_workspace_size(B, H, T, dk, dv, C, gm, _DTYPES[dt]))
+    if ws_bytes and (workspace is None or workspace.numel() * workspace.element_size() < ws_bytes):
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    st = L.gdr_chunk_fwd_prologue(_ptr(q_raw), _ptr(k_raw), _ptr(v), _ptr(a), _ptr(A_log), _ptr(dt_bias),
+                                  _ptr(b_logit), _ptr(S0), _ptr(O), _ptr(S_T), B, H, T, dk, dv, C, gm, _DTYPES[dt],
+                                  _ptr(workspace) if ws_bytes else None, ws_bytes, _stream_handle(dev, stream))
+    _check(st, "gdr_chunk_fwd_prologue")
     if host:
         O = O.to("cpu")
         S_T = None if S_T is None else S_T.to("cpu")

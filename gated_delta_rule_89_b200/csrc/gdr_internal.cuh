@@ -17,6 +17,12 @@ struct ChunkArgs {
     bool scalar_gate;
     bool bf16;
     void *workspace;   // device scratch of chunk_tc_workspace_bytes() bytes (tensor-core path)
+    // Input prologue (tensor-core path only): q, k are raw and L2-normalised
+    // in-kernel, g holds the bf16 gate pre-activation a (reinterpreted), the
+    // log-decay is -exp(A_log[h]) * softplus(a + dt_bias) (bounded below by -5
+    // per channel) and beta holds the logits of beta = sigmoid(logit).
+    bool prologue = false;
+    const float *A_log = nullptr, *dt_bias = nullptr;
 };
 
 // Arguments of one decode step, already validated.

@@ -82,7 +82,9 @@ constexpr uint32_t OFF_AQ = OFF_A + kC * kLdA * 4; // Aqk, then Nt / X'
 constexpr uint32_t OFF_U = OFF_AQ + kC * kLdA * 4; // U_10, U_21, U_20 [3][16][24]
 constexpr uint32_t OFF_BETA = OFF_U + 3 * 16 * kLdD * 4;   // beta, two buffers by chunk parity
 constexpr uint32_t OFF_GC = OFF_BETA + 512;        // scalar gate: inclusive cumulative sum
-constexpr uint32_t SMEM_USED = OFF_GC + 256;
+constexpr uint32_t OFF_NRM = OFF_GC + 256;         // prologue: row sums of q^2, k^2 per warp half [8][2][16]
+constexpr uint32_t OFF_INV = OFF_NRM + 1024;       // prologue: 1 / L2 norm of those rows [8][2][16]
+constexpr uint32_t SMEM_USED = OFF_INV + 1024;
 constexpr uint32_t SMEM_ALLOC = SMEM_USED + 1024;  // alignment slack
 static_assert(2 * (SMEM_ALLOC + 1024) <= 233472, "two CTAs per SM must fit in shared memory");
 
@@ -190,12 +192,23 @@ __device__ __forceinline__ float2 pair_factor(const float *bd, int R, int I, int
     return make_float2(a.x * b.x, a.y * b.y);
 }
 
-template <bool SCALAR>
+// softplus(z) = log(1 + e^z) = max(z, 0) + log(1 + e^-|z|), without overflow
+__device__ __forceinline__ float softplus_f(float z) { return fmaxf(z, 0.f) + __logf(1.f + __expf(-fabsf(z))); }
+
+// PRO: the input prologue.  q, k arrive raw and are L2-normalised here
+// (q / sqrt(sum q^2 + 1e-6) per row), gin holds the bf16 gate
+// pre-activation a, the log-decay is g = -exp(A_log[h]) * softplus(a +
+// dt_bias) (per channel: bounded below by -5), and betag holds the logits of
+// beta = sigmoid(logit).  Otherwise gin holds the fp32 log-decay g and betag
+// beta itself.
+template <bool SCALAR, bool PRO>
 __global__ void __launch_bounds__(kThreads, 2)
 ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__restrict__ qg,
-               const float *__restrict__ gg, const float *__restrict__ betag, __nv_bfloat16 *__restrict__ Tout,
+               const void *__restrict__ gin, const float *__restrict__ betag,
+               const float *__restrict__ A_log, const float *__restrict__ dt_bias, __nv_bfloat16 *__restrict__ Tout,
                __nv_bfloat16 *__restrict__ Aqout, __nv_bfloat16 *__restrict__ Wout, __nv_bfloat16 *__restrict__ Qlo,
-               __nv_bfloat16 *__restrict__ Kto, float *__restrict__ gamo, int T_len, int nchunks, int total)
+               __nv_bfloat16 *__restrict__ Kto, float *__restrict__ gamo, int T_len, int nchunks, int total,
+               int n_heads)
 {
     extern __shared__ unsigned char prep_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(prep_raw) + 1023) &
@@ -206,6 +219,8 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
     float *sBd = reinterpret_cast<float *>(sm + OFF_BD);              // [4][128] bd, then [4][128] 1/bd
     float(*sD)[16][kLdD] = reinterpret_cast<float(*)[16][kLdD]>(sm + OFF_D);
     float *sGc = reinterpret_cast<float *>(sm + OFF_GC);
+    const float *gg = static_cast<const float *>(gin);
+    const __nv_bfloat16 *ag = static_cast<const __nv_bfloat16 *>(gin);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -231,6 +246,11 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
         uint2 kr[8], qr[8];
         float4 gv[8];                       // g, then alpha = exp(max(g, -5))
         float2 oa = make_float2(1.f, 1.f), ob = oa;   // alpha product of the other half block
+        // 1 / L2 norm of the rows of q, k (prologue; 1 otherwise), kept in
+        // shared memory: iq(rr), ik(rr) for this thread's row rbase + rr
+        const float *sinv = reinterpret_cast<const float *>(sm + OFF_INV) + (warp * 2 + half) * 16;
+        auto iq = [&](int rr) { return PRO ? sinv[rr] : 1.f; };
+        auto ik = [&](int rr) { return PRO ? sinv[8 + rr] : 1.f; };
         {
             // Unconditional loads from rows clamped into the chunk (a
             // conditional load makes the compiler wait for each one before the
@@ -240,7 +260,15 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
                 const size_t e = (row0 + min(rbase + rr, nrows - 1)) * kDK + c;
                 kr[rr] = __ldg(reinterpret_cast<const uint2 *>(kg + e));
                 qr[rr] = __ldg(reinterpret_cast<const uint2 *>(qg + e));
-                if (!SCALAR) gv[rr] = __ldg(reinterpret_cast<const float4 *>(gg + e));
+                if (!SCALAR) {
+                    if (PRO) {   // a as four bf16, widened; the gate is formed below
+                        const uint2 av = __ldg(reinterpret_cast<const uint2 *>(ag + e));
+                        gv[rr] = make_float4(__uint_as_float(av.x << 16), __uint_as_float(av.x & 0xffff0000u),
+                                             __uint_as_float(av.y << 16), __uint_as_float(av.y & 0xffff0000u));
+                    } else {
+                        gv[rr] = __ldg(reinterpret_cast<const float4 *>(gg + e));
+                    }
+                }
             }
 #pragma unroll
             for (int rr = 0; rr < 8; ++rr) {
@@ -250,11 +278,75 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
                     if (!SCALAR) gv[rr] = make_float4(0.f, 0.f, 0.f, 0.f);
                 }
             }
-            if (tid < kC) sBeta[tid] = tid < nrows ? __ldg(betag + row0 + tid) : 0.f;
+            if (PRO) {
+                // per-channel log-decay from the pre-activation (rows past T keep g = 0)
+                const int hh = head % n_heads;   // A_log, dt_bias are per head h of [B, H]
+                if (!SCALAR) {
+                    const float A = __expf(__ldg(A_log + hh));
+                    const float4 db = __ldg(reinterpret_cast<const float4 *>(dt_bias + (size_t)hh * kDK + c));
+#pragma unroll
+                    for (int rr = 0; rr < 8; ++rr) {
+                        if (rbase + rr < nrows) {
+                            gv[rr].x = -A * softplus_f(gv[rr].x + db.x);
+                            gv[rr].y = -A * softplus_f(gv[rr].y + db.y);
+                            gv[rr].z = -A * softplus_f(gv[rr].z + db.z);
+                            gv[rr].w = -A * softplus_f(gv[rr].w + db.w);
+                        }
+                    }
+                }
+                // L2 norms of q and k per row: this thread's 4 channels, then the
+                // 16 lanes of its half (transpose-reduce: lane v ends with row v & 7
+                // of q (v < 8) or k), then the partner warp holding the other 64
+                // channels (named barrier of the two warps).
+                float ps[16];
+#pragma unroll
+                for (int rr = 0; rr < 8; ++rr) {
+                    const float q0 = __uint_as_float(qr[rr].x << 16), q1 = __uint_as_float(qr[rr].x & 0xffff0000u);
+                    const float q2 = __uint_as_float(qr[rr].y << 16), q3 = __uint_as_float(qr[rr].y & 0xffff0000u);
+                    const float k0 = __uint_as_float(kr[rr].x << 16), k1 = __uint_as_float(kr[rr].x & 0xffff0000u);
+                    const float k2 = __uint_as_float(kr[rr].y << 16), k3 = __uint_as_float(kr[rr].y & 0xffff0000u);
+                    ps[rr] = q0 * q0 + q1 * q1 + q2 * q2 + q3 * q3;
+                    ps[8 + rr] = k0 * k0 + k1 * k1 + k2 * k2 + k3 * k3;
+                }
+                const int v = lane & 15;
+#pragma unroll
+                for (int w = 8; w >= 1; w >>= 1) {
+                    // keep the half of the values whose index has bit w equal to this lane's
+#pragma unroll
+                    for (int j = 0; j < w; ++j) {
+                        const bool up = (v & w) != 0;
+                        const float send = up ? ps[j] : ps[j + w];
+                        const float got = __shfl_xor_sync(0xffffffffu, send, w);
+                        ps[j] = (up ? ps[j + w] : ps[j]) + got;
+                    }
+                }
+                float *nrm = reinterpret_cast<float *>(sm + OFF_NRM);
+                nrm[(warp * 2 + half) * 16 + v] = ps[0];
+                switch (R) {   // the two warps of row block R: literal barrier ids 1..4
+                case 0: asm volatile("bar.sync 1, 64;" ::: "memory"); break;
+                case 1: asm volatile("bar.sync 2, 64;" ::: "memory"); break;
+                case 2: asm volatile("bar.sync 3, 64;" ::: "memory"); break;
+                default: asm volatile("bar.sync 4, 64;" ::: "memory"); break;
+                }
+                const float tot = nrm[(warp * 2 + half) * 16 + v] + nrm[((warp ^ 1) * 2 + half) * 16 + v];
+                reinterpret_cast<float *>(sm + OFF_INV)[(warp * 2 + half) * 16 + v] = rsqrtf(tot + 1e-6f);
+                __syncwarp();
+            }
+            if (tid < kC) {
+                const float bl = tid < nrows ? __ldg(betag + row0 + tid) : 0.f;
+                sBeta[tid] = tid < nrows ? (PRO ? 1.f / (1.f + __expf(-bl)) : bl) : 0.f;
+            }
             if (SCALAR && warp == 0) {
                 // inclusive scan of the scalar log-decay over the chunk (2 values per lane)
-                const float a0 = (2 * lane < nrows) ? __ldg(gg + row0 + 2 * lane) : 0.f;
-                const float a1 = (2 * lane + 1 < nrows) ? __ldg(gg + row0 + 2 * lane + 1) : 0.f;
+                auto gate_at = [&](int t) -> float {
+                    if (t >= nrows) return 0.f;
+                    if (!PRO) return __ldg(gg + row0 + t);
+                    const int hh = head % n_heads;
+                    const float z = __bfloat162float(ag[row0 + t]) + __ldg(dt_bias + hh);
+                    return -__expf(__ldg(A_log + hh)) * softplus_f(z);
+                };
+                const float a0 = gate_at(2 * lane);
+                const float a1 = gate_at(2 * lane + 1);
                 float sum = a0 + a1;
 #pragma unroll
                 for (int off = 1; off < 32; off <<= 1) {
@@ -268,8 +360,14 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
 #pragma unroll
                 for (int rr = 0; rr < 8; ++rr) {
                     const uint32_t off = tile_off(rbase + rr, c);
-                    *reinterpret_cast<uint2 *>(sm + OFF_K + off) = kr[rr];
-                    *reinterpret_cast<uint2 *>(sm + OFF_Q + off) = qr[rr];
+                    if (PRO) {
+                        const float2 fk = make_float2(ik(rr), ik(rr)), fq = make_float2(iq(rr), iq(rr));
+                        *reinterpret_cast<uint2 *>(sm + OFF_K + off) = make_uint2(scale2p(kr[rr].x, fk), scale2p(kr[rr].y, fk));
+                        *reinterpret_cast<uint2 *>(sm + OFF_Q + off) = make_uint2(scale2p(qr[rr].x, fq), scale2p(qr[rr].y, fq));
+                    } else {
+                        *reinterpret_cast<uint2 *>(sm + OFF_K + off) = kr[rr];
+                        *reinterpret_cast<uint2 *>(sm + OFF_Q + off) = qr[rr];
+                    }
                 }
             } else {
                 // alpha = exp(max(g, -5)) and the product over this thread's 8 rows
@@ -293,8 +391,11 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
                     const uint32_t off = tile_off(rbase + rr, c);
                     pa = fmul2(pa, make_float2(gv[rr].x, gv[rr].y));
                     pb = fmul2(pb, make_float2(gv[rr].z, gv[rr].w));
-                    *reinterpret_cast<uint2 *>(sm + OFF_K + off) = make_uint2(scale2p(kr[rr].x, pa), scale2p(kr[rr].y, pb));
-                    *reinterpret_cast<uint2 *>(sm + OFF_Q + off) = make_uint2(scale2p(qr[rr].x, pa), scale2p(qr[rr].y, pb));
+                    const float2 nk = make_float2(ik(rr), ik(rr)), nq = make_float2(iq(rr), iq(rr));
+                    *reinterpret_cast<uint2 *>(sm + OFF_K + off) =
+                        make_uint2(scale2p(kr[rr].x, PRO ? fmul2(pa, nk) : pa), scale2p(kr[rr].y, PRO ? fmul2(pb, nk) : pb));
+                    *reinterpret_cast<uint2 *>(sm + OFF_Q + off) =
+                        make_uint2(scale2p(qr[rr].x, PRO ? fmul2(pa, nq) : pa), scale2p(qr[rr].y, PRO ? fmul2(pb, nq) : pb));
                 }
                 if (half) {   // pa, pb now hold bd_R
                     *reinterpret_cast<float4 *>(sBd + R * kDK + c) = make_float4(pa.x, pa.y, pb.x, pb.y);
@@ -307,7 +408,9 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
 #pragma unroll
                 for (int rr = 7; rr >= 0; --rr) {
                     const uint32_t off = tile_off(rbase + rr, c);
-                    *reinterpret_cast<uint2 *>(sm + OFF_KC + off) = make_uint2(scale2p(kr[rr].x, pa), scale2p(kr[rr].y, pb));
+                    const float2 nk = make_float2(ik(rr), ik(rr));
+                    *reinterpret_cast<uint2 *>(sm + OFF_KC + off) =
+                        make_uint2(scale2p(kr[rr].x, PRO ? fmul2(pa, nk) : pa), scale2p(kr[rr].y, PRO ? fmul2(pb, nk) : pb));
                     pa = fmul2(pa, make_float2(gv[rr].x, gv[rr].y));
                     pb = fmul2(pb, make_float2(gv[rr].z, gv[rr].w));
                 }
@@ -343,7 +446,9 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
                     pb = fmul2(pb, make_float2(gv[rr].z, gv[rr].w));
                     if (rbase + rr < nrows) {
                         const size_t e = e0 + (size_t)(rbase + rr) * kDK;
-                        *reinterpret_cast<uint2 *>(Qlo + e) = make_uint2(scale2p(qr[rr].x, pa), scale2p(qr[rr].y, pb));
+                        const float2 nq = make_float2(iq(rr), iq(rr));
+                        *reinterpret_cast<uint2 *>(Qlo + e) =
+                            make_uint2(scale2p(qr[rr].x, PRO ? fmul2(pa, nq) : pa), scale2p(qr[rr].y, PRO ? fmul2(pb, nq) : pb));
                     }
                 }
                 if (R == 0 && half == 0) {   // gamma_C = product of the four block decays
@@ -357,7 +462,9 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
                 for (int rr = 7; rr >= 0; --rr) {
                     if (rbase + rr < nrows) {
                         const size_t e = e0 + (size_t)(rbase + rr) * kDK;
-                        *reinterpret_cast<uint2 *>(Kto + e) = make_uint2(scale2p(kr[rr].x, pa), scale2p(kr[rr].y, pb));
+                        const float2 nk = make_float2(ik(rr), ik(rr));
+                        *reinterpret_cast<uint2 *>(Kto + e) =
+                            make_uint2(scale2p(kr[rr].x, PRO ? fmul2(pa, nk) : pa), scale2p(kr[rr].y, PRO ? fmul2(pb, nk) : pb));
                     }
                     pa = fmul2(pa, make_float2(gv[rr].x, gv[rr].y));
                     pb = fmul2(pb, make_float2(gv[rr].z, gv[rr].w));
@@ -369,7 +476,7 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
                     const int r = rbase + rr;
                     if (r < nrows) {
                         const float ef = __expf(sGc[r]), et = __expf(Gl - sGc[r]);
-                        const float2 fe = make_float2(ef, ef), ft = make_float2(et, et);
+                        const float2 fe = make_float2(ef * iq(rr), ef * iq(rr)), ft = make_float2(et * ik(rr), et * ik(rr));
                         const size_t e = e0 + (size_t)r * kDK;
                         *reinterpret_cast<uint2 *>(Qlo + e) = make_uint2(scale2p(qr[rr].x, fe), scale2p(qr[rr].y, fe));
                         *reinterpret_cast<uint2 *>(Kto + e) = make_uint2(scale2p(kr[rr].x, ft), scale2p(kr[rr].y, ft));
@@ -667,12 +774,14 @@ cudaError_t launch_ut_prep(const ChunkArgs &a, const TcWorkspace &w, cudaStream_
     if (total > 0x7fffffffLL) return cudaErrorInvalidValue;
     const long long slots = 2LL * sm_count();   // two resident CTAs per SM
     const int grid = (int)(total < slots ? total : slots);
-    auto kern = a.scalar_gate ? ut_prep_kernel<true> : ut_prep_kernel<false>;
+    auto kern = a.prologue ? (a.scalar_gate ? ut_prep_kernel<true, true> : ut_prep_kernel<false, true>)
+                           : (a.scalar_gate ? ut_prep_kernel<true, false> : ut_prep_kernel<false, false>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_ALLOC);
     if (e != cudaSuccess) return e;
-    kern<<<grid, kThreads, SMEM_ALLOC, stream>>>((const __nv_bfloat16 *)a.k, (const __nv_bfloat16 *)a.q, a.g,
-                                                 a.beta, w.T, w.Aqk, w.W, w.Ql, w.Kt, w.gam, a.T, nchunks,
-                                                 (int)total);
+    kern<<<grid, kThreads, SMEM_ALLOC, stream>>>((const __nv_bfloat16 *)a.k, (const __nv_bfloat16 *)a.q,
+                                                 (const void *)a.g, a.beta, a.A_log, a.dt_bias, w.T, w.Aqk, w.W,
+                                                 w.Ql, w.Kt, w.gam, a.T, nchunks,
+                                                 (int)total, a.H);
     return cudaGetLastError();
 }
 

@@ -148,6 +148,11 @@ WORKLOADS: Dict[str, Workload] = {
         "kda_d128_t8192", "chunk", 2, 32, 8192, 128, 128, 64, "per_channel", torch.bfloat16,
         "softplus_n02_clamp5", "normal002", 2,
         "KDA forward at head dim 128: B2 H32 T8192 d128 C64 bf16"),
+    "kda_d128_t8192_prologue": Workload(
+        "kda_d128_t8192_prologue", "chunk", 2, 32, 8192, 128, 128, 64, "per_channel", torch.bfloat16,
+        "prologue", "normal002", 2,
+        "KDA forward with the input prologue fused in (raw q, k; bf16 gate pre-activation; beta "
+        "logits): B2 H32 T8192 d128 C64 bf16"),
     "kda_long_t65536": Workload(
         "kda_long_t65536", "chunk", 1, 32, 65536, 128, 128, 64, "per_channel", torch.bfloat16,
         "long_context_mix", "normal002", 3,
@@ -228,6 +233,8 @@ def generate(w: Workload, device="cpu", heads: Optional[Sequence[int]] = None,
         head_ids = torch.as_tensor(list(heads), dtype=torch.int64, device=device)
         outB, outH = len(heads), 1
     nh = head_ids.numel()
+    if w.g_recipe == "prologue":
+        raise ValueError(f"{w.name} takes raw inputs: use generate_prologue")
     fast = {"mask": fast_channel_mask(w, device)} if w.g_recipe == "long_context_mix" else None
     seed = w.seed
     decode = w.kind == "decode"
@@ -302,7 +309,8 @@ def generate(w: Workload, device="cpu", heads: Optional[Sequence[int]] = None,
     return out
 
 
-def generate_prologue(w: Workload, device="cpu", block: int = 1 << 24) -> Dict[str, torch.Tensor]:
+def generate_prologue(w: Workload, device="cpu", heads: Optional[Sequence[int]] = None,
+                      block: int = 1 << 24) -> Dict[str, torch.Tensor]:
     """Raw inputs of the forward with its gate / normalisation prologue.
 
     q_raw, k_raw [B,H,T,dk] ~ N(0,1) (not normalised), v [B,H,T,dv] ~ N(0,1)
@@ -310,33 +318,50 @@ def generate_prologue(w: Workload, device="cpu", block: int = 1 << 24) -> Dict[s
     (per-channel) or [B,H,T] (scalar) ~ N(0,1), A_log [H] ~ U(-1,1),
     dt_bias [H,dk] (per-channel) or [H] ~ N(0, 0.5^2), beta logits [B,H,T]
     ~ N(0,1) fp32, S0 as in ``generate``.  q_raw, k_raw, v and a are in the
-    workload dtype; A_log, dt_bias and the logits are fp32.  No prologue
-    arithmetic here: the L2 normalisation, softplus gate and sigmoid belong
-    to the oracle and the kernels.
+    workload dtype; A_log, dt_bias and the logits are fp32.  ``heads`` selects
+    flat head ids (b*H + h) as in ``generate``: tensors come back as
+    [len(heads), 1, ...] with the values the full tensors hold there, and
+    A_log, dt_bias as [len(heads)], [len(heads), ...] (the parameters of each
+    selected head, so a sample can be laid out as B = 1, H = len(heads)).
+    No prologue arithmetic here: the L2 normalisation,
+    softplus gate and sigmoid belong to the oracle and the kernels.
     """
     assert w.kind == "chunk"
     B, H, T, dk, dv, seed = w.B, w.H, w.T, w.dk, w.dv, w.seed
+    head_ids = torch.arange(B * H, dtype=torch.int64, device=device) if heads is None else \
+        torch.as_tensor(list(heads), dtype=torch.int64, device=device)
+    nh = head_ids.numel()
+    outB, outH = (B, H) if heads is None else (nh, 1)
 
-    def draw(tid, shape, make):
-        n = 1
-        for d in shape:
-            n *= d
-        out = torch.empty(n, dtype=torch.float64, device=device)
-        for s, e in _chunked(n, block):
-            out[s:e] = make(tid, torch.arange(s, e, dtype=torch.int64, device=device))
-        return out.view(*shape)
+    def per_head(tid, width, make):
+        # element (head, t, j) of the full [B*H, T, width] tensor
+        per = T * width
+        out = torch.empty(nh * per, dtype=torch.float64, device=device)
+        for s, e in _chunked(nh * per, block):
+            lin = torch.arange(s, e, dtype=torch.int64, device=device)
+            out[s:e] = make(tid, head_ids[lin // per] * per + lin % per)
+        return out
+
+    def draw(tid, n, make):
+        return make(tid, torch.arange(n, dtype=torch.int64, device=device))
 
     nrm = lambda tid, idx: normal(seed, tid, idx)
-    q_raw = to_dtype(draw(TID_QRAW, (B, H, T, dk), nrm), w.dtype)
-    k_raw = to_dtype(draw(TID_KRAW, (B, H, T, dk), nrm), w.dtype)
-    v = to_dtype(draw(TID_V, (B, H, T, dv), nrm), w.dtype)
-    a_shape = (B, H, T, dk) if w.gate == "per_channel" else (B, H, T)
-    a = to_dtype(draw(TID_AGATE, a_shape, nrm), w.dtype)
-    A_log = draw(TID_ALOG, (H,), lambda tid, idx: 2.0 * uniform(seed, tid, idx) - 1.0).to(torch.float32)
-    dt_shape = (H, dk) if w.gate == "per_channel" else (H,)
-    dt_bias = draw(TID_DTBIAS, dt_shape, lambda tid, idx: 0.5 * normal(seed, tid, idx)).to(torch.float32)
-    b_logit = draw(TID_BLOGIT, (B, H, T), nrm).to(torch.float32)
-    S0 = generate(dataclasses.replace(w, T=1), device=device)["S0"]
+    q_raw = to_dtype(per_head(TID_QRAW, dk, nrm), w.dtype).view(outB, outH, T, dk)
+    k_raw = to_dtype(per_head(TID_KRAW, dk, nrm), w.dtype).view(outB, outH, T, dk)
+    v = to_dtype(per_head(TID_V, dv, nrm), w.dtype).view(outB, outH, T, dv)
+    if w.gate == "per_channel":
+        a = to_dtype(per_head(TID_AGATE, dk, nrm), w.dtype).view(outB, outH, T, dk)
+        dt_bias = (0.5 * draw(TID_DTBIAS, H * dk, nrm)).to(torch.float32).view(H, dk)
+    else:
+        a = to_dtype(per_head(TID_AGATE, 1, nrm), w.dtype).view(outB, outH, T)
+        dt_bias = (0.5 * draw(TID_DTBIAS, H, nrm)).to(torch.float32)
+    A_log = (2.0 * draw(TID_ALOG, H, lambda tid, idx: uniform(seed, tid, idx)) - 1.0).to(torch.float32)
+    b_logit = per_head(TID_BLOGIT, 1, nrm).to(torch.float32).view(outB, outH, T)
+    if heads is not None:   # per-head parameters of the selected heads
+        hsel = head_ids % H
+        A_log, dt_bias = A_log[hsel], dt_bias[hsel]
+    S0 = generate(dataclasses.replace(w, T=1, g_recipe="softplus_n01_plus1_clamp5"), device=device,
+                  heads=heads)["S0"]
     return dict(q_raw=q_raw, k_raw=k_raw, v=v, a=a, A_log=A_log, dt_bias=dt_bias, b_logit=b_logit, S0=S0)
 
 

@@ -121,6 +121,34 @@ int gdr_recurrent_step(const void *q, const void *k, const void *v, const float 
                        void *stream);
 
 /*
+ * Chunkwise-parallel forward with the layer's input prologue fused in:
+ *   q = L2Norm(q_raw), k = L2Norm(k_raw)          per head and token,
+ *                                                 L2Norm(x) = x / sqrt(sum x^2 + 1e-6)
+ *   g = max(-exp(A_log[h]) * softplus(a + dt_bias[h][c]), -5)   (per-channel gate)
+ *   g = -exp(A_log[h]) * softplus(a + dt_bias[h])               (scalar gate)
+ *   beta = sigmoid(b_logit)
+ * then the same forward as gdr_chunk_fwd.  "Token Mixer I", section "Kimi
+ * Delta Attention", Neural Parameterization (L2Norm of q, k; Sigmoid beta);
+ * the gate of the Kimi Linear notes (-exp(A_log) softplus(. + dt_bias), A_log
+ * of shape [H], dt_bias [H * d_k]); the lower bound g_min = -5 of KDA.
+ *
+ * Arguments as gdr_chunk_fwd, except:
+ *   q_raw, k_raw   [B,H,T,d_k]  not normalised
+ *   a              [B,H,T,d_k] (per-channel) or [B,H,T] (scalar), dtype as q
+ *   A_log          [H] fp32; dt_bias [H,d_k] (per-channel) or [H] (scalar) fp32
+ *   b_logit        [B,H,T] fp32
+ * Only the tensor-core configuration (bf16, d_k = d_v = 128, C = 64) runs;
+ * anything else returns GDR_ERR_UNSUPPORTED.  Same workspace as
+ * gdr_chunk_fwd (gdr_chunk_fwd_workspace_size).  a and dt_bias must be
+ * 16-byte aligned like the other tensors; A_log and b_logit 4-byte aligned.
+ */
+int gdr_chunk_fwd_prologue(const void *q_raw, const void *k_raw, const void *v, const void *a,
+                           const float *A_log, const float *dt_bias, const float *b_logit,
+                           const float *S0, void *O, float *S_T,
+                           int B, int H, int T, int dk, int dv, int C, int gate_mode, int dtype,
+                           void *workspace, size_t ws_bytes, void *stream);
+
+/*
  * Chunked forward that allocates nothing, for callers that cannot allocate
  * device memory or pass a workspace at the point of the call: serving or
  * real-time loops that forbid allocator calls on their hot path, code that

@@ -77,6 +77,29 @@ def test_chunk_argument_validation(L):
     assert chunk(L, T=0) == OK          # no S_T requested: nothing to do
 
 
+def prologue(L, B=1, H=1, T=64, dk=128, dv=128, C=64, gate=0, dtype=1, ptr=GOOD, a=GOOD, alog=GOOD,
+             blog=GOOD, ST=None, ws=1 << 40, wsp=GOOD):
+    return L.gdr_chunk_fwd_prologue(ptr, ptr, ptr, a, alog, ptr, blog, None, ptr, ST, B, H, T, dk, dv, C, gate,
+                                    dtype, wsp, ws, None)
+
+
+def test_prologue_argument_validation(L):
+    assert prologue(L, B=-1) == INVALID
+    assert prologue(L, gate=3) == INVALID
+    # the fused prologue runs on the tensor-core configuration only
+    assert prologue(L, dtype=0) == UNSUPPORTED
+    assert prologue(L, dk=64, dv=64) == UNSUPPORTED
+    assert prologue(L, C=32) == UNSUPPORTED
+    assert prologue(L, a=None) == INVALID
+    assert prologue(L, alog=None) == INVALID
+    assert prologue(L, blog=None) == INVALID
+    assert prologue(L, a=ODD) == ALIGN
+    assert prologue(L, alog=P(0x100002)) == ALIGN
+    assert prologue(L, wsp=None) == INVALID
+    assert prologue(L, B=0) == OK and L.gdr_last_launch_count() == 0
+    assert prologue(L, T=0) == OK
+
+
 def test_step_argument_validation(L):
     def step(B=2, H=2, dk=128, dv=128, gate=0, dtype=1, ptr=GOOD):
         return L.gdr_recurrent_step(ptr, ptr, ptr, ptr, ptr, ptr, ptr, B, H, dk, dv, gate, dtype, None)

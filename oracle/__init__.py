@@ -10,6 +10,9 @@ Contents
   * ``forward``   -- the token-by-token fp64 recurrence (``gdr_oracle.c``),
     the parity reference for the chunked forward and the decode step.
   * ``decode``    -- the same recurrence driven one decode step per token.
+  * ``forward_gdr2`` / ``decode_gdr2`` -- Gated Delta Rule-2 (per-channel erase
+    gate b on the key side, write gate w on the value side), the reference of
+    the GDR-2 entry points.
   * ``prologue`` / ``forward_prologue`` -- the input prologue (L2-normalised
     q, k; softplus gate with the -5 bound; sigmoid beta) and the forward fed
     by it, the reference of the fused-prologue entry point.
@@ -56,6 +59,8 @@ def _load():
             I = ctypes.c_int
             lib.gdr_oracle_forward.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I]
             lib.gdr_oracle_forward.restype = I
+            lib.gdr2_oracle_forward.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I]
+            lib.gdr2_oracle_forward.restype = I
             lib.gdr_oracle_online_cores.restype = I
             _lib = lib
     return _lib
@@ -113,6 +118,41 @@ def forward(q, k, v, g, beta, S0=None, gate: str = "per_channel", erase=None, wr
     return O, ST
 
 
+def forward_gdr2(q, k, v, g, b, w, S0=None, gate: str = "per_channel", clamp: bool = True,
+                 threads: int = 0) -> Tuple[np.ndarray, np.ndarray]:
+    """fp64 Gated Delta Rule-2 over T tokens ("Token Mixer I", section "Gated
+    DeltaNet-2: Decoupling Erase and Write in Linear Attention", eq. (10)):
+    the state is read along b_t * k_t and the delta w_t * v_t - S~ (b_t * k_t)
+    is written along k_t.
+
+    Shapes: q, k, b [B,H,T,dk]; v, w [B,H,T,dv]; g as in ``forward``.  The
+    -5 bound applies to a per-channel gate when ``clamp`` (as in ``forward``).
+    Returns (O [B,H,T,dv], S_T [B,H,dv,dk]) as fp64 numpy arrays.
+    """
+    qa, ka, va, ga, ba, wa = _f64(q), _f64(k), _f64(v), _f64(g), _f64(b), _f64(w)
+    B, H, T, dk = qa.shape
+    dv = va.shape[-1]
+    assert ka.shape == (B, H, T, dk) and ba.shape == (B, H, T, dk)
+    assert va.shape == (B, H, T, dv) and wa.shape == (B, H, T, dv)
+    if gate == "per_channel":
+        assert ga.shape == (B, H, T, dk)
+    elif gate == "scalar":
+        assert ga.shape == (B, H, T)
+    else:
+        raise ValueError(gate)
+    s0 = _f64(S0)
+    if s0 is not None:
+        assert s0.shape == (B, H, dv, dk)
+    O = np.empty((B, H, T, dv), dtype=np.float64)
+    ST = np.empty((B, H, dv, dk), dtype=np.float64)
+    rc = _load().gdr2_oracle_forward(_ptr(qa), _ptr(ka), _ptr(va), _ptr(ga), _ptr(ba), _ptr(wa), _ptr(s0),
+                                     _ptr(O), _ptr(ST), B, H, T, dk, dv, 1 if gate == "scalar" else 0,
+                                     1 if clamp else 0, int(threads))
+    if rc != 0:
+        raise RuntimeError("oracle forward_gdr2 failed")
+    return O, ST
+
+
 L2NORM_EPS = 1e-6   # the pages do not give the epsilon of L2Norm; see the reading in the design notes
 
 
@@ -167,4 +207,13 @@ def decode(q, k, v, g, beta, S, gate: str = "per_channel", threads: int = 0) -> 
     """
     mv = lambda x: _f64(x).transpose(1, 2, 0, *range(3, _f64(x).ndim)).copy()
     O, ST = forward(mv(q), mv(k), mv(v), mv(g), mv(beta), S0=S, gate=gate, threads=threads)
+    return O.transpose(2, 0, 1, 3).copy(), ST
+
+
+def decode_gdr2(q, k, v, g, b, w, S, gate: str = "per_channel", threads: int = 0) -> Tuple[np.ndarray, np.ndarray]:
+    """``steps`` consecutive Gated Delta Rule-2 single-token updates: q, k, b
+    [steps,B,H,dk]; v, w [steps,B,H,dv]; g [steps,B,H,dk] or [steps,B,H];
+    S [B,H,dv,dk].  Returns (o [steps,B,H,dv], S_final)."""
+    mv = lambda x: _f64(x).transpose(1, 2, 0, *range(3, _f64(x).ndim)).copy()
+    O, ST = forward_gdr2(mv(q), mv(k), mv(v), mv(g), mv(b), mv(w), S0=S, gate=gate, threads=threads)
     return O.transpose(2, 0, 1, 3).copy(), ST

@@ -56,3 +56,51 @@ def chunk_forward(q, k, v, g, beta, S0=None, C: int = 64, gate: str = "per_chann
         gC = Gam[-1]
         S = S * gC[None, :] + (Vnew.T @ Kr) * gC[None, :]
     return O, S
+
+
+def chunk_forward_gdr2(q, k, v, g, b, w, S0=None, C: int = 64, gate: str = "per_channel", clamp: bool = True):
+    """Gated Delta Rule-2 in chunk form, one head, fp64: the equations of
+    "Token Mixer I", section "Gated DeltaNet-2", subsection "Chunkwise parallel
+    training", in the d_v x d_k orientation.  Per chunk, with the state
+    normalised by the cumulative decay (S_r = S^_r Diag(gamma_r)):
+        E- = B * K * Gamma (erase-side keys),  K-> = K / Gamma,  Z = W * V
+        T  = StrictTril(E- K->^T),  A = (I + T)^{-1}   (forward substitution)
+        Y  = A E-  (erase side),    U = A Z  (write side)
+        Delta  = U - Y S^T
+        S_next = S Diag(gamma_C) + Delta^T K_tail,   K_tail_r = k_r * gamma_C / gamma_r
+        O      = Q_gamma S^T + (Q_gamma K->^T * M) Delta   (M: lower incl. diagonal)
+    b, q, k [T,dk]; w, v [T,dv]; g [T,dk] or [T]; S0 [dv,dk]."""
+    q, k, v, g, b, w = (np.asarray(x, np.float64) for x in (q, k, v, g, b, w))
+    T, dk = q.shape
+    dv = v.shape[1]
+    if gate == "per_channel":
+        logalpha = np.maximum(g, -5.0) if clamp else g.copy()
+    else:
+        logalpha = np.repeat(g[:, None], dk, axis=1)
+    S = np.zeros((dv, dk)) if S0 is None else np.array(S0, np.float64)
+    O = np.zeros((T, dv))
+    for s in range(0, T, C):
+        e = min(T, s + C)
+        n = e - s
+        G = np.cumsum(logalpha[s:e], axis=0)
+        Gam = np.exp(G)
+        Ebar = b[s:e] * k[s:e] * Gam
+        Kbar = k[s:e] / Gam
+        Z = w[s:e] * v[s:e]
+        Tm = np.tril(Ebar @ Kbar.T, -1)
+        # A = (I + T)^{-1}: forward substitution, column by column
+        A = np.zeros((n, n))
+        for j in range(n):
+            x = np.zeros(n)
+            x[j] = 1.0
+            for r in range(j + 1, n):
+                x[r] = -Tm[r, j:r] @ x[j:r]
+            A[:, j] = x
+        Y = A @ Ebar
+        U = A @ Z
+        Delta = U - Y @ S.T
+        Qg = q[s:e] * Gam
+        O[s:e] = Qg @ S.T + ((Qg @ Kbar.T) * np.tril(np.ones((n, n)))) @ Delta
+        Ktail = k[s:e] * (Gam[-1][None, :] / Gam)
+        S = S * Gam[-1][None, :] + Delta.T @ Ktail
+    return O, S

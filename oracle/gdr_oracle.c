@@ -31,10 +31,23 @@
  * erase and write"): delta = w_t v_t - e_t (S~ k_t).  With e = w = beta it is
  * the method itself; e = 0, w = 1 gives (gated) linear attention.
  *
+ * Gated Delta Rule-2 (gdr2_oracle_forward): the erase gate b_t in [0,1]^dk
+ * and the write gate w_t in [0,1]^dv of "Token Mixer I", section "Gated
+ * DeltaNet-2: Decoupling Erase and Write in Linear Attention", eq. (10).  The
+ * state is read along e_t = b_t * k_t (elementwise) and the written target is
+ * z_t = w_t * v_t; the write direction stays k_t.  In this orientation:
+ *
+ *     S~ = S_{t-1} Diag(alpha_t),   delta = w_t * v_t - S~ (b_t * k_t),
+ *     S_t = S~ + delta k_t^T,       o_t = S_t q_t,
+ *
+ * the residual z_t - S~^T e_t of the section's fast-weight paragraph, taken
+ * in the same order as above (decay, read, delta, write, read out).
+ *
  * Layouts (row-major, contiguous, fp64):
  *   q, k   [B,H,T,dk]      v, O [B,H,T,dv]
  *   g      [B,H,T,dk] (per-channel) or [B,H,T] (scalar)
  *   beta, erase, write  [B,H,T]      (erase / write may be NULL -> beta)
+ *   GDR-2: b [B,H,T,dk], w [B,H,T,dv] (in place of beta)
  *   S0, S_T [B,H,dv,dk]              (S0 NULL -> zeros, S_T NULL -> not written)
  * Heads are independent; they are spread over nthreads POSIX threads
  * (nthreads <= 0 -> all online cores).  Returns 0, or -1 on a bad argument
@@ -48,13 +61,14 @@
 
 typedef struct {
     const double *q, *k, *v, *g, *beta, *erase, *write, *S0;
+    const double *eb, *ww;   /* GDR-2 erase gate [B,H,T,dk] and write gate [B,H,T,dv], or NULL */
     double *O, *S_T;
     int B, H, T, dk, dv, per_channel, clamp;
     int head_begin, head_end;
     int status;
 } oracle_job;
 
-static void run_head(const oracle_job *J, int head, double *S, double *a, double *delta)
+static void run_head(const oracle_job *J, int head, double *S, double *a, double *delta, double *ek)
 {
     const int T = J->T, dk = J->dk, dv = J->dv;
     const size_t hk = (size_t)head * T * dk, hv = (size_t)head * T * dv, hs = (size_t)head * T;
@@ -81,18 +95,34 @@ static void run_head(const oracle_job *J, int head, double *S, double *a, double
             const double as = exp(J->g[hs + t]);
             for (int c = 0; c < dk; ++c) a[c] = as;
         }
-        const double e = J->erase ? J->erase[hs + t] : J->beta[hs + t];
-        const double w = J->write ? J->write[hs + t] : J->beta[hs + t];
-
-        /* decay, then predict from the decayed state: p = S~ k */
-        for (int i = 0; i < dv; ++i) {
-            double *row = S + (size_t)i * dk;
-            double p = 0.0;
-            for (int c = 0; c < dk; ++c) {
-                row[c] *= a[c];
-                p += row[c] * kt[c];
+        if (J->eb) {
+            /* GDR-2: decay, read along e = b * k, delta = w * v - S~ e */
+            const double *bt = J->eb + hk + (size_t)t * dk;
+            const double *wt = J->ww + hv + (size_t)t * dv;
+            for (int c = 0; c < dk; ++c) ek[c] = bt[c] * kt[c];
+            for (int i = 0; i < dv; ++i) {
+                double *row = S + (size_t)i * dk;
+                double p = 0.0;
+                for (int c = 0; c < dk; ++c) {
+                    row[c] *= a[c];
+                    p += row[c] * ek[c];
+                }
+                delta[i] = wt[i] * vt[i] - p;
             }
-            delta[i] = w * vt[i] - e * p;
+        } else {
+            const double e = J->erase ? J->erase[hs + t] : J->beta[hs + t];
+            const double w = J->write ? J->write[hs + t] : J->beta[hs + t];
+
+            /* decay, then predict from the decayed state: p = S~ k */
+            for (int i = 0; i < dv; ++i) {
+                double *row = S + (size_t)i * dk;
+                double p = 0.0;
+                for (int c = 0; c < dk; ++c) {
+                    row[c] *= a[c];
+                    p += row[c] * kt[c];
+                }
+                delta[i] = w * vt[i] - e * p;
+            }
         }
         /* write the delta along k, then read with q: o = S_t q */
         for (int i = 0; i < dv; ++i) {
@@ -114,25 +144,26 @@ static void *worker(void *arg)
     double *S = (double *)malloc(sizeof(double) * (size_t)J->dv * J->dk);
     double *a = (double *)malloc(sizeof(double) * (size_t)J->dk);
     double *delta = (double *)malloc(sizeof(double) * (size_t)J->dv);
-    if (!S || !a || !delta) {
+    double *ek = (double *)malloc(sizeof(double) * (size_t)J->dk);
+    if (!S || !a || !delta || !ek) {
         J->status = -1;
     } else {
-        for (int h = J->head_begin; h < J->head_end; ++h) run_head(J, h, S, a, delta);
+        for (int h = J->head_begin; h < J->head_end; ++h) run_head(J, h, S, a, delta, ek);
     }
+    free(ek);
     free(S);
     free(a);
     free(delta);
     return NULL;
 }
 
-int gdr_oracle_forward(const double *q, const double *k, const double *v, const double *g,
-                       const double *beta, const double *erase, const double *write,
-                       const double *S0, double *O, double *S_T,
-                       int B, int H, int T, int dk, int dv,
-                       int gate_scalar, int clamp, int nthreads)
+static int run_jobs(const double *q, const double *k, const double *v, const double *g,
+                    const double *beta, const double *erase, const double *write,
+                    const double *eb, const double *ww,
+                    const double *S0, double *O, double *S_T,
+                    int B, int H, int T, int dk, int dv,
+                    int gate_scalar, int clamp, int nthreads)
 {
-    if (!q || !k || !v || !g || !O || B < 0 || H < 0 || T < 0 || dk <= 0 || dv <= 0) return -1;
-    if (!beta && (!erase || !write)) return -1;
     const int heads = B * H;
     if (heads == 0) return 0;
     if (nthreads <= 0) nthreads = (int)sysconf(_SC_NPROCESSORS_ONLN);
@@ -151,6 +182,7 @@ int gdr_oracle_forward(const double *q, const double *k, const double *v, const 
         oracle_job *J = &jobs[j];
         J->q = q; J->k = k; J->v = v; J->g = g; J->beta = beta;
         J->erase = erase; J->write = write; J->S0 = S0; J->O = O; J->S_T = S_T;
+        J->eb = eb; J->ww = ww;
         J->B = B; J->H = H; J->T = T; J->dk = dk; J->dv = dv;
         J->per_channel = !gate_scalar;
         J->clamp = clamp;
@@ -177,6 +209,27 @@ int gdr_oracle_forward(const double *q, const double *k, const double *v, const 
     free(jobs);
     free(tid);
     return status;
+}
+
+int gdr_oracle_forward(const double *q, const double *k, const double *v, const double *g,
+                       const double *beta, const double *erase, const double *write,
+                       const double *S0, double *O, double *S_T,
+                       int B, int H, int T, int dk, int dv,
+                       int gate_scalar, int clamp, int nthreads)
+{
+    if (!q || !k || !v || !g || !O || B < 0 || H < 0 || T < 0 || dk <= 0 || dv <= 0) return -1;
+    if (!beta && (!erase || !write)) return -1;
+    return run_jobs(q, k, v, g, beta, erase, write, NULL, NULL, S0, O, S_T, B, H, T, dk, dv, gate_scalar, clamp,
+                    nthreads);
+}
+
+/* Gated Delta Rule-2: b [B,H,T,dk] erase gate, w [B,H,T,dv] write gate (both required). */
+int gdr2_oracle_forward(const double *q, const double *k, const double *v, const double *g,
+                        const double *b, const double *w, const double *S0, double *O, double *S_T,
+                        int B, int H, int T, int dk, int dv, int gate_scalar, int clamp, int nthreads)
+{
+    if (!q || !k || !v || !g || !b || !w || !O || B < 0 || H < 0 || T < 0 || dk <= 0 || dv <= 0) return -1;
+    return run_jobs(q, k, v, g, NULL, NULL, NULL, b, w, S0, O, S_T, B, H, T, dk, dv, gate_scalar, clamp, nthreads);
 }
 
 int gdr_oracle_online_cores(void)

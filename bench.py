@@ -51,8 +51,10 @@ DEFAULT_WORKLOAD = "kda_d128_t8192"
 # workload with the hash of the sources those kernels are built from; an
 # entry is ignored (traffic = null) as soon as any of the sources changes.
 TRAFFIC = {
-    # ut_prep 539.0 MB read + 493.2 MB written, chunk_scan 679.6 + 118.3 MB (one launch each)
-    "kda_d128_t8192": {"src_sha": "ec261bf9c0fc7bca", "bytes_per_launch": 1830078976},
+    # ut_prep 539.0 MB read + 493.4 MB written, chunk_scan 679.5 + 117.7 MB (one launch each)
+    "kda_d128_t8192": {"src_sha": "0c9f0d70d986ac6f", "bytes_per_launch": 1829669120},
+    # Gated Delta Rule-2: ut_prep 939.6 + 634.4 MB (reads b, v, w; writes w * v), chunk_scan 679.5 + 117.9 MB
+    "gdr2_d128_t8192": {"src_sha": "0c9f0d70d986ac6f", "bytes_per_launch": 2371415040},
     # recurrent_step, one decode step: 547.4 MB read + 479.2 MB written
     "kda_decode_b256": {"src_sha": "99a0454504c77460", "bytes_per_launch": 1026655488},
 }
@@ -70,7 +72,10 @@ def algorithmic_bytes(w: W.Workload) -> int:
     gate = w.dk * 4 if w.gate == "per_channel" else 4
     if w.g_recipe == "prologue":    # gate pre-activation in the input dtype, beta logits fp32
         gate = w.dk * e if w.gate == "per_channel" else e
-    per_token = 2 * w.dk * e + w.dv * e + gate + 4 + w.dv * e       # q, k, v, g, beta, O
+    strength = 4                                                    # beta
+    if w.rule == "gdr2":            # erase gate [dk] and write gate [dv] in the input dtype
+        strength = (w.dk + w.dv) * e
+    per_token = 2 * w.dk * e + w.dv * e + gate + strength + w.dv * e   # q, k, v, g, beta, O
     heads = w.B * w.H
     state = 2 * w.dv * w.dk * 4                                     # S0 read + S_T write
     if w.kind == "decode":
@@ -229,6 +234,8 @@ def api_call(gdr, w: W.Workload, x, **kw):
     if w.g_recipe == "prologue":
         return gdr.chunk_fwd_prologue(x["q_raw"], x["k_raw"], x["v"], x["a"], x["A_log"], x["dt_bias"],
                                       x["b_logit"], x["S0"], C=w.C, gate=w.gate, **kw)
+    if w.rule == "gdr2":
+        return gdr.chunk_fwd_gdr2(x["q"], x["k"], x["v"], x["g"], x["b"], x["w"], x["S0"], C=w.C, gate=w.gate, **kw)
     return gdr.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], C=w.C, gate=w.gate, **kw)
 
 
@@ -253,7 +260,11 @@ def oracle_sample(w: W.Workload, budget_s: float, seed_rank: int = 0):
         if w.kind == "decode":
             x = W.generate(w, heads=hl, steps=ntok)
             t = time.perf_counter()
-            oracle.decode(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], gate=w.gate, threads=cores)
+            if w.rule == "gdr2":
+                oracle.decode_gdr2(x["q"], x["k"], x["v"], x["g"], x["b"], x["w"], x["S0"], gate=w.gate,
+                                   threads=cores)
+            else:
+                oracle.decode(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], gate=w.gate, threads=cores)
             return time.perf_counter() - t
         if w.g_recipe == "prologue":
             # the sampled heads laid out as B = 1, H = len(hl), with their own A_log, dt_bias
@@ -266,6 +277,11 @@ def oracle_sample(w: W.Workload, budget_s: float, seed_rank: int = 0):
             return time.perf_counter() - t
         x = W.generate(w, heads=hl)
         sl = lambda a: a[:, :, :ntok].contiguous()
+        if w.rule == "gdr2":
+            args = [sl(x[k]) for k in ("q", "k", "v", "g", "b", "w")]
+            t = time.perf_counter()
+            oracle.forward_gdr2(*args, x["S0"], gate=w.gate, threads=cores)
+            return time.perf_counter() - t
         args = [sl(x[k]) for k in ("q", "k", "v", "g", "beta")]
         t = time.perf_counter()
         oracle.forward(*args, x["S0"], gate=w.gate, threads=cores)
@@ -388,9 +404,15 @@ def main():
         S = x["S0"].clone()
         o = torch.empty(w.B, w.H, w.dv, dtype=w.dtype, device=device)
 
-        def step():
-            for s in range(w.T):
-                gdr.recurrent_step(x["q"][s], x["k"][s], x["v"][s], x["g"][s], x["beta"][s], S, o=o)
+        if w.rule == "gdr2":
+            def step():
+                for s in range(w.T):
+                    gdr.recurrent_step_gdr2(x["q"][s], x["k"][s], x["v"][s], x["g"][s], x["b"][s], x["w"][s], S,
+                                            o=o)
+        else:
+            def step():
+                for s in range(w.T):
+                    gdr.recurrent_step(x["q"][s], x["k"][s], x["v"][s], x["g"][s], x["beta"][s], S, o=o)
     elif w.g_recipe == "prologue":
         x = W.generate_prologue(w, device=device)
         O = torch.empty(w.B, w.H, w.T, w.dv, dtype=w.dtype, device=device)
@@ -400,12 +422,13 @@ def main():
             api_call(gdr, w, x, O=O, S_T=S_T)
     else:
         x = W.generate(w, device=device)
+        if w.rule == "gdr2":
+            del x["beta"]           # the erase and write gates take its place
         O = torch.empty(w.B, w.H, w.T, w.dv, dtype=w.dtype, device=device)
         S_T = torch.empty(w.B, w.H, w.dv, w.dk, dtype=torch.float32, device=device)
 
         def step():
-            gdr.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], C=w.C, gate=w.gate,
-                          O=O, S_T=S_T)
+            api_call(gdr, w, x, O=O, S_T=S_T)
     torch.cuda.synchronize(device)
 
     sampler = ClockSampler(gpu_id_for(device)) if rank == 0 else None

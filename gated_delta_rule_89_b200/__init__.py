@@ -19,7 +19,8 @@ from typing import Optional, Tuple
 
 import torch
 
-__all__ = ["chunk_fwd", "recurrent_step", "chunk_fwd_workspace_size", "GDRError", "library_path",
+__all__ = ["chunk_fwd", "recurrent_step", "chunk_fwd_workspace_size", "chunk_fwd_prologue", "chunk_fwd_gdr2",
+           "recurrent_step_gdr2", "GDRError", "library_path",
            "last_launch_count", "device_status", "GATE_PER_CHANNEL", "GATE_SCALAR"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -57,6 +58,12 @@ def lib() -> ctypes.CDLL:
         L.gdr_recurrent_step.restype = I
         L.gdr_chunk_fwd_workspace_size.argtypes = [I, I, I, I, I, I, I, I]
         L.gdr_chunk_fwd_workspace_size.restype = Z
+        L.gdr2_chunk_fwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P, Z, P]
+        L.gdr2_chunk_fwd.restype = I
+        L.gdr2_chunk_fwd_workspace_size.argtypes = [I, I, I, I, I, I, I, I]
+        L.gdr2_chunk_fwd_workspace_size.restype = Z
+        L.gdr2_recurrent_step.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, P]
+        L.gdr2_recurrent_step.restype = I
         L.gdr_status_string.argtypes = [I]
         L.gdr_status_string.restype = ctypes.c_char_p
         L.gdr_last_cuda_error.restype = I
@@ -272,4 +279,95 @@ def recurrent_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.T
     st = lib().gdr_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(o),
                                   B, H, dk, dv, gm, _DTYPES[dt], _stream_handle(dev, stream))
     _check(st, "gdr_recurrent_step")
+    return o
+
+
+def chunk_fwd_gdr2(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor, b: torch.Tensor,
+                   w: torch.Tensor, S0: Optional[torch.Tensor] = None, C: int = 64, gate: Optional[str] = None,
+                   O: Optional[torch.Tensor] = None, S_T: Optional[torch.Tensor] = None,
+                   final_state: bool = True, workspace: Optional[torch.Tensor] = None,
+                   stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Chunkwise Gated Delta Rule-2 forward (``gdr2_chunk_fwd``).
+
+    q, k, b [B,H,T,dk] and v, w [B,H,T,dv] bf16 (b: erase gate, w: write
+    gate); g fp32 [B,H,T,dk] (per-channel) or [B,H,T] (scalar); S0 fp32
+    [B,H,dv,dk] or None.  Returns (O [B,H,T,dv] bf16, S_T fp32 or None).
+    """
+    host = not q.is_cuda
+    if host:
+        dev = torch.device("cuda", torch.cuda.current_device())
+        q, k, v, g, b, w, S0 = (_to_device(x, dev) for x in (q, k, v, g, b, w, S0))
+    dev = q.device
+    if gate is None:
+        gate = "per_channel" if g.dim() == 4 else "scalar"
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    if dt != torch.bfloat16:
+        raise TypeError("the Gated Delta Rule-2 forward takes bf16 q, k, v, b, w")
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (b, "b"), (w, "w")):
+        _need(t, n, dt, dev)
+    _need(g, "g", torch.float32, dev)
+    if tuple(k.shape) != (B, H, T, dk) or tuple(b.shape) != (B, H, T, dk) or tuple(v.shape[:3]) != (B, H, T) \
+            or tuple(w.shape) != (B, H, T, dv):
+        raise ValueError("inconsistent shapes")
+    if gate == "per_channel" and tuple(g.shape) != (B, H, T, dk):
+        raise ValueError("per-channel g must be [B,H,T,dk]")
+    if gate == "scalar" and tuple(g.shape) != (B, H, T):
+        raise ValueError("scalar g must be [B,H,T]")
+    if S0 is not None:
+        _need(S0, "S0", torch.float32, dev)
+        if tuple(S0.shape) != (B, H, dv, dk):
+            raise ValueError("S0 must be [B,H,dv,dk]")
+    if O is None:
+        O = torch.empty(B, H, T, dv, dtype=dt, device=dev)
+    _need(O, "O", dt, dev)
+    if S_T is None and final_state:
+        S_T = torch.empty(B, H, dv, dk, dtype=torch.float32, device=dev)
+    if S_T is not None:
+        _need(S_T, "S_T", torch.float32, dev)
+    gm = GATE_PER_CHANNEL if gate == "per_channel" else GATE_SCALAR
+    L = lib()
+    ws_bytes = int(L.gdr2_chunk_fwd_workspace_size(B, H, T, dk, dv, C, gm, _DTYPES[dt]))
+    if ws_bytes and (workspace is None or workspace.numel() * workspace.element_size() < ws_bytes):
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    st = L.gdr2_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b), _ptr(w), _ptr(S0), _ptr(O), _ptr(S_T),
+                          B, H, T, dk, dv, C, gm, _DTYPES[dt],
+                          _ptr(workspace) if ws_bytes else None, ws_bytes, _stream_handle(dev, stream))
+    _check(st, "gdr2_chunk_fwd")
+    if host:
+        O = O.to("cpu")
+        S_T = None if S_T is None else S_T.to("cpu")
+    return O, S_T
+
+
+def recurrent_step_gdr2(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor, b: torch.Tensor,
+                        w: torch.Tensor, S: torch.Tensor, o: Optional[torch.Tensor] = None,
+                        gate: Optional[str] = None, stream=None) -> torch.Tensor:
+    """One Gated Delta Rule-2 decode step (``gdr2_recurrent_step``); S is updated in place.
+
+    q, k, b [B,H,dk], v, w [B,H,dv] (fp32 or bf16, one dtype); g fp32
+    [B,H,dk] or [B,H].  Returns o [B,H,dv] in v's dtype.
+    """
+    dev = S.device
+    if gate is None:
+        gate = "per_channel" if g.dim() == 3 else "scalar"
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    if dt not in _DTYPES:
+        raise TypeError("q, k, v, b, w must be float32 or bfloat16")
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (b, "b"), (w, "w")):
+        _need(t, n, dt, dev)
+    _need(g, "g", torch.float32, dev)
+    _need(S, "S", torch.float32, dev)
+    if tuple(S.shape) != (B, H, dv, dk) or tuple(b.shape) != (B, H, dk) or tuple(w.shape) != (B, H, dv):
+        raise ValueError("inconsistent shapes")
+    if o is None:
+        o = torch.empty(B, H, dv, dtype=dt, device=dev)
+    _need(o, "o", dt, dev)
+    gm = GATE_PER_CHANNEL if gate == "per_channel" else GATE_SCALAR
+    st = lib().gdr2_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b), _ptr(w), _ptr(S), _ptr(o),
+                                   B, H, dk, dv, gm, _DTYPES[dt], _stream_handle(dev, stream))
+    _check(st, "gdr2_recurrent_step")
     return o

@@ -515,20 +515,21 @@ bool chunk_tc_supports(const ChunkArgs &a)
     return a.bf16 && a.dk == kD && a.dv == kD && a.C == kC;
 }
 
-size_t chunk_tc_workspace_bytes(int B, int H, int T) { return tc_workspace_bytes(B, H, T); }
+size_t chunk_tc_workspace_bytes(int B, int H, int T, bool gdr2) { return tc_workspace_bytes(B, H, T, gdr2); }
 
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream, int *launches)
 {
     const int BH = a.B * a.H;
     const int nchunks = (a.T + kC - 1) / kC;
-    const TcWorkspace w = carve_tc_workspace(a.workspace, a.B, a.H, a.T);
+    const TcWorkspace w = carve_tc_workspace(a.workspace, a.B, a.H, a.T, a.gdr2);
 
     Maps maps;
     {
         const cuuint64_t dims3[3] = {(cuuint64_t)kD, (cuuint64_t)a.T, (cuuint64_t)BH};
         const cuuint64_t str_bf[2] = {(cuuint64_t)kD * 2, (cuuint64_t)a.T * kD * 2};
         const cuuint32_t box_bf[3] = {64, 64, 1};
-        void *tiles[4] = {w.Ql, w.Kt, const_cast<void *>(a.v), a.O};
+        // Gated Delta Rule-2: U = T' Z with Z = w * v, formed by the prep kernel
+        void *tiles[4] = {w.Ql, w.Kt, a.gdr2 ? static_cast<void *>(w.Z) : const_cast<void *>(a.v), a.O};
         CUtensorMap *dst[4] = {&maps.q, &maps.kt, &maps.v, &maps.o};
         for (int i = 0; i < 4; ++i)
             if (!make_map(dst[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, tiles[i], dims3, str_bf, box_bf,

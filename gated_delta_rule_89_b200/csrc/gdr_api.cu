@@ -167,6 +167,96 @@ GDR_API int gdr_chunk_fwd_prologue(const void *q_raw, const void *k_raw, const v
     return finish(e, launches);
 }
 
+GDR_API size_t gdr2_chunk_fwd_workspace_size(int B, int H, int T, int dk, int dv, int C, int gate_mode, int dtype)
+{
+    if (B <= 0 || H <= 0 || T <= 0) return 0;
+    if (gate_mode != GDR_GATE_PER_CHANNEL && gate_mode != GDR_GATE_SCALAR) return 0;
+    gdr::ChunkArgs a = {};
+    a.dk = dk; a.dv = dv; a.C = C;
+    a.bf16 = (dtype == GDR_BF16);
+    return gdr::chunk_tc_supports(a) ? gdr::chunk_tc_workspace_bytes(B, H, T, true) : 0;
+}
+
+GDR_API int gdr2_chunk_fwd(const void *q, const void *k, const void *v, const float *g, const void *b,
+                           const void *w, const float *S0, void *O, float *S_T,
+                           int B, int H, int T, int dk, int dv, int C, int gate_mode, int dtype,
+                           void *workspace, size_t ws_bytes, void *stream)
+{
+    if (B < 0 || H < 0 || T < 0) return GDR_ERR_INVALID_ARG;
+    if (gate_mode != GDR_GATE_PER_CHANNEL && gate_mode != GDR_GATE_SCALAR) return GDR_ERR_INVALID_ARG;
+    if (dtype != GDR_F32 && dtype != GDR_BF16) return GDR_ERR_INVALID_ARG;
+    if (dk <= 0 || dv <= 0 || C <= 0) return GDR_ERR_INVALID_ARG;
+    gdr::ChunkArgs a_;
+    a_.dk = dk; a_.dv = dv; a_.C = C; a_.bf16 = (dtype == GDR_BF16);
+    if (!gdr::chunk_tc_supports(a_)) return GDR_ERR_UNSUPPORTED;   // bf16, d_k = d_v = 128, C = 64 only
+    if ((long long)B * H * T * 128 >= (1LL << 40)) return GDR_ERR_UNSUPPORTED;
+    const size_t ws_need = gdr2_chunk_fwd_workspace_size(B, H, T, dk, dv, C, gate_mode, dtype);
+    if (ws_bytes < ws_need || (ws_need && !workspace)) return GDR_ERR_INVALID_ARG;
+    const long long heads = (long long)B * H;
+    if (heads == 0) {
+        tl_last_launches = 0;
+        return GDR_OK;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (T == 0) {
+        if (S_T && !aligned16(S_T)) return GDR_ERR_ALIGNMENT;
+        if (S0 && !aligned16(S0)) return GDR_ERR_ALIGNMENT;
+        cudaError_t e = cudaSuccess;
+        const size_t bytes = sizeof(float) * (size_t)heads * dv * dk;
+        if (S_T && S0 && S_T != S0) e = cudaMemcpyAsync(S_T, S0, bytes, cudaMemcpyDeviceToDevice, st);
+        else if (S_T && !S0) e = cudaMemsetAsync(S_T, 0, bytes, st);
+        return finish(e, 0);
+    }
+    if (!q || !k || !v || !g || !b || !w || !O) return GDR_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, g, b, w, S0, O, S_T, workspace};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return GDR_ERR_ALIGNMENT;
+
+    gdr::ChunkArgs c;
+    c.q = q; c.k = k; c.v = v; c.g = g; c.beta = nullptr; c.S0 = S0; c.O = O; c.S_T = S_T;
+    c.B = B; c.H = H; c.T = T; c.dk = dk; c.dv = dv; c.C = C;
+    c.scalar_gate = (gate_mode == GDR_GATE_SCALAR);
+    c.bf16 = true;
+    c.workspace = workspace;
+    c.gdr2 = true;
+    c.erase = b;
+    c.write = w;
+    int launches = 0;
+    cudaError_t e = gdr::launch_chunk_tc(c, st, &launches);
+    return finish(e, launches);
+}
+
+GDR_API int gdr2_recurrent_step(const void *q, const void *k, const void *v, const float *g, const void *b,
+                                const void *w, float *S, void *o, int B, int H, int dk, int dv, int gate_mode,
+                                int dtype, void *stream)
+{
+    if (B < 0 || H < 0) return GDR_ERR_INVALID_ARG;
+    if (gate_mode != GDR_GATE_PER_CHANNEL && gate_mode != GDR_GATE_SCALAR) return GDR_ERR_INVALID_ARG;
+    if (dtype != GDR_F32 && dtype != GDR_BF16) return GDR_ERR_INVALID_ARG;
+    if (dk <= 0 || dv <= 0) return GDR_ERR_INVALID_ARG;
+    if (!size_ok(dk) || !size_ok(dv)) return GDR_ERR_UNSUPPORTED;
+    if ((long long)B * H * dv * dk >= (1LL << 40)) return GDR_ERR_UNSUPPORTED;
+    if ((long long)B * H == 0) {
+        tl_last_launches = 0;
+        return GDR_OK;
+    }
+    if (!q || !k || !v || !g || !b || !w || !S || !o) return GDR_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, g, b, w, S, o};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return GDR_ERR_ALIGNMENT;
+    gdr::StepArgs a;
+    a.q = q; a.k = k; a.v = v; a.g = g; a.beta = nullptr; a.S = S; a.o = o;
+    a.B = B; a.H = H; a.dk = dk; a.dv = dv;
+    a.scalar_gate = (gate_mode == GDR_GATE_SCALAR);
+    a.bf16 = (dtype == GDR_BF16);
+    a.gdr2 = true;
+    a.erase = b;
+    a.write = w;
+    int launches = 0;
+    cudaError_t e = gdr::launch_recurrent_step(a, static_cast<cudaStream_t>(stream), &launches);
+    return finish(e, launches);
+}
+
 GDR_API int gdr_recurrent_step(const void *q, const void *k, const void *v, const float *g, const float *beta,
                                float *S, void *o, int B, int H, int dk, int dv, int gate_mode, int dtype,
                                void *stream)

@@ -23,6 +23,11 @@ struct ChunkArgs {
     // per channel) and beta holds the logits of beta = sigmoid(logit).
     bool prologue = false;
     const float *A_log = nullptr, *dt_bias = nullptr;
+    // Gated Delta Rule-2 (tensor-core path only): beta is unused; erase
+    // [B, H, T, d_k] and write [B, H, T, d_v] are the per-channel erase and
+    // write gates, in the dtype of q, k, v.
+    bool gdr2 = false;
+    const void *erase = nullptr, *write = nullptr;
 };
 
 // Arguments of one decode step, already validated.
@@ -34,6 +39,10 @@ struct StepArgs {
     int B, H, dk, dv;
     bool scalar_gate;
     bool bf16;
+    // Gated Delta Rule-2: erase [B, H, d_k] and write [B, H, d_v] gates in
+    // the dtype of q, k, v (beta unused)
+    bool gdr2 = false;
+    const void *erase = nullptr, *write = nullptr;
 };
 
 // The tensor-core path's scratch, carved out of ChunkArgs::workspace (every
@@ -42,16 +51,19 @@ struct StepArgs {
 //   W        [B*H*chunks][128][64] bf16   W^T, W = T' K<- (key channel rows)
 //   Ql, Kt   [B, H, T, 128] bf16          Q<-, K_tail (chunk-relative decays)
 //   gam      [B*H*chunks][128] fp32       gamma_C per key channel
+//   Z        [B, H, T, 128] bf16          Gated Delta Rule-2 only: w * v
 struct TcWorkspace {
     __nv_bfloat16 *T, *Aqk, *W, *Ql, *Kt;
     float *gam;
+    __nv_bfloat16 *Z;
 };
-inline size_t tc_workspace_bytes(int B, int H, int T)
+inline size_t tc_workspace_bytes(int B, int H, int T, bool gdr2 = false)
 {
     const size_t bh = (size_t)B * H, nch = (size_t)(T + 63) / 64;
-    return 2 * bh * nch * 64 * 64 * 2 + bh * nch * 128 * 64 * 2 + 2 * bh * (size_t)T * 128 * 2 + bh * nch * 128 * 4;
+    return 2 * bh * nch * 64 * 64 * 2 + bh * nch * 128 * 64 * 2 + 2 * bh * (size_t)T * 128 * 2 + bh * nch * 128 * 4 +
+           (gdr2 ? bh * (size_t)T * 128 * 2 : 0);
 }
-inline TcWorkspace carve_tc_workspace(void *ws, int B, int H, int T)
+inline TcWorkspace carve_tc_workspace(void *ws, int B, int H, int T, bool gdr2 = false)
 {
     const size_t bh = (size_t)B * H, nch = (size_t)(T + 63) / 64;
     unsigned char *p = static_cast<unsigned char *>(ws);
@@ -67,6 +79,8 @@ inline TcWorkspace carve_tc_workspace(void *ws, int B, int H, int T)
     w.Kt = reinterpret_cast<__nv_bfloat16 *>(p);
     p += bh * (size_t)T * 128 * 2;
     w.gam = reinterpret_cast<float *>(p);
+    p += bh * nch * 128 * 4;
+    w.Z = gdr2 ? reinterpret_cast<__nv_bfloat16 *>(p) : nullptr;
     return w;
 }
 
@@ -76,7 +90,7 @@ cudaError_t launch_recurrent_step(const StepArgs &a, cudaStream_t stream, int *l
 cudaError_t launch_chunk_simt(const ChunkArgs &a, cudaStream_t stream, int *launches);
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream, int *launches);
 bool chunk_tc_supports(const ChunkArgs &a);
-size_t chunk_tc_workspace_bytes(int B, int H, int T);
+size_t chunk_tc_workspace_bytes(int B, int H, int T, bool gdr2 = false);
 // Synchronizes `stream`, then reads and clears the device status word.
 cudaError_t read_device_status(cudaStream_t stream, int *status);
 

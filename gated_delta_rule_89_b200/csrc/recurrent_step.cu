@@ -8,6 +8,12 @@
 // orientation (o = S q, S in R^{dv x dk}) is that of "Reading notes: Kimi
 // Delta Attention" (mzeromiko), section 4.
 //
+// Gated Delta Rule-2 ("Token Mixer I", section "Gated DeltaNet-2: Decoupling
+// Erase and Write in Linear Attention", eq. (10)): the prediction reads along
+// the erase-gated key and the target is the write-gated value,
+//   p = S~ (b * k),  delta = w * v - p,
+// with the write along k and the readout unchanged.
+//
 // The step is bound by HBM traffic: the state is read once and written once
 // (2 * 4 * dv * dk bytes per head) and everything else is a few hundred
 // bytes.  One warp owns one state row at a time: each lane holds dk/32
@@ -44,10 +50,11 @@ template <> struct VecF<2> {
     }
 };
 
-template <int DK, int RPW, typename T, bool SCALAR>
+template <int DK, int RPW, typename T, bool SCALAR, bool GDR2>
 __global__ void __launch_bounds__(kStepThreads)
 recurrent_step_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
                       const float *__restrict__ g, const float *__restrict__ beta,
+                      const T *__restrict__ erase, const T *__restrict__ write,
                       float *__restrict__ S, T *__restrict__ o, int dv, int blocks_per_head)
 {
     constexpr int VEC = DK / 32;
@@ -62,12 +69,13 @@ recurrent_step_kernel(const T *__restrict__ q, const T *__restrict__ k, const T 
 #pragma unroll
     for (int r = 0; r < RPW; ++r) VecF<VEC>::load(Srow + (size_t)r * DK, s[r]);
 
-    float kv[VEC], qv[VEC], av[VEC];
+    float kv[VEC], qv[VEC], av[VEC], ev[VEC];   // ev: the key the state is read along
     const size_t hk = (size_t)head * DK + lane * VEC;
 #pragma unroll
     for (int j = 0; j < VEC; ++j) {
         kv[j] = to_f32<T>(k[hk + j]);
         qv[j] = to_f32<T>(q[hk + j]);
+        ev[j] = GDR2 ? to_f32<T>(erase[hk + j]) * kv[j] : kv[j];
     }
     if (SCALAR) {
         const float a = expf(g[head]);
@@ -77,10 +85,13 @@ recurrent_step_kernel(const T *__restrict__ q, const T *__restrict__ k, const T 
 #pragma unroll
         for (int j = 0; j < VEC; ++j) av[j] = expf(fmaxf(g[hk + j], kGateMin));
     }
-    const float b = beta[head];
-    float vr[RPW];
+    const float b = GDR2 ? 1.f : beta[head];
+    float vr[RPW];   // the write target: beta v, or w * v for GDR-2
 #pragma unroll
-    for (int r = 0; r < RPW; ++r) vr[r] = to_f32<T>(v[(size_t)head * dv + row0 + r]);
+    for (int r = 0; r < RPW; ++r) {
+        const size_t iv = (size_t)head * dv + row0 + r;
+        vr[r] = GDR2 ? to_f32<T>(write[iv]) * to_f32<T>(v[iv]) : to_f32<T>(v[iv]);
+    }
 
     // k . q (identical in every warp)
     float kq = 0.f;
@@ -95,7 +106,7 @@ recurrent_step_kernel(const T *__restrict__ q, const T *__restrict__ k, const T 
 #pragma unroll
         for (int j = 0; j < VEC; ++j) {
             s[r][j] *= av[j];
-            p[r] = fmaf(s[r][j], kv[j], p[r]);
+            p[r] = fmaf(s[r][j], ev[j], p[r]);
             rq[r] = fmaf(s[r][j], qv[j], rq[r]);
         }
     }
@@ -118,7 +129,7 @@ recurrent_step_kernel(const T *__restrict__ q, const T *__restrict__ k, const T 
     }
 }
 
-template <int DK, typename T, bool SCALAR>
+template <int DK, typename T, bool SCALAR, bool GDR2>
 cudaError_t launch_typed(const StepArgs &a, cudaStream_t stream)
 {
     constexpr int RPW = 4;
@@ -126,17 +137,18 @@ cudaError_t launch_typed(const StepArgs &a, cudaStream_t stream)
     const int blocks_per_head = a.dv / rows_per_block;
     const long long blocks = (long long)a.B * a.H * blocks_per_head;
     if (blocks == 0) return cudaSuccess;
-    recurrent_step_kernel<DK, RPW, T, SCALAR><<<(unsigned)blocks, kStepThreads, 0, stream>>>(
-        (const T *)a.q, (const T *)a.k, (const T *)a.v, a.g, a.beta, a.S, (T *)a.o, a.dv, blocks_per_head);
+    recurrent_step_kernel<DK, RPW, T, SCALAR, GDR2><<<(unsigned)blocks, kStepThreads, 0, stream>>>(
+        (const T *)a.q, (const T *)a.k, (const T *)a.v, a.g, a.beta, (const T *)a.erase, (const T *)a.write, a.S,
+        (T *)a.o, a.dv, blocks_per_head);
     return cudaGetLastError();
 }
 
-template <int DK>
+template <int DK, bool GDR2>
 cudaError_t launch_dk(const StepArgs &a, cudaStream_t s)
 {
-    if (a.bf16) return a.scalar_gate ? launch_typed<DK, __nv_bfloat16, true>(a, s)
-                                     : launch_typed<DK, __nv_bfloat16, false>(a, s);
-    return a.scalar_gate ? launch_typed<DK, float, true>(a, s) : launch_typed<DK, float, false>(a, s);
+    if (a.bf16) return a.scalar_gate ? launch_typed<DK, __nv_bfloat16, true, GDR2>(a, s)
+                                     : launch_typed<DK, __nv_bfloat16, false, GDR2>(a, s);
+    return a.scalar_gate ? launch_typed<DK, float, true, GDR2>(a, s) : launch_typed<DK, float, false, GDR2>(a, s);
 }
 
 }  // namespace
@@ -144,7 +156,8 @@ cudaError_t launch_dk(const StepArgs &a, cudaStream_t s)
 cudaError_t launch_recurrent_step(const StepArgs &a, cudaStream_t stream, int *launches)
 {
     if ((long long)a.B * a.H == 0) return cudaSuccess;
-    cudaError_t e = (a.dk == 128) ? launch_dk<128>(a, stream) : launch_dk<64>(a, stream);
+    cudaError_t e = a.gdr2 ? ((a.dk == 128) ? launch_dk<128, true>(a, stream) : launch_dk<64, true>(a, stream))
+                           : ((a.dk == 128) ? launch_dk<128, false>(a, stream) : launch_dk<64, false>(a, stream));
     if (e == cudaSuccess) *launches += 1;
     return e;
 }

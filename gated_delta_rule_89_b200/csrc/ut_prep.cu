@@ -125,6 +125,12 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi)
     return *reinterpret_cast<uint32_t *>(&o);
 }
 
+// bf16 pair (packed) widened to an fp32 pair
+__device__ __forceinline__ float2 unpack2(uint32_t v)
+{
+    return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
+}
+
 // bf16 pair (packed) times an fp32 pair, rounded back to a bf16 pair
 __device__ __forceinline__ uint32_t scale2p(uint32_t v, float2 f)
 {
@@ -201,15 +207,28 @@ __device__ __forceinline__ float softplus_f(float z) { return fmaxf(z, 0.f) + __
 // dt_bias) (per channel: bounded below by -5), and betag holds the logits of
 // beta = sigmoid(logit).  Otherwise gin holds the fp32 log-decay g and betag
 // beta itself.
-template <bool SCALAR, bool PRO>
+//
+// GDR2: Gated Delta Rule-2 ("Token Mixer I", section "Gated DeltaNet-2",
+// subsection "Chunkwise parallel training").  The erase gate b (bf16, layout
+// of k) replaces beta on the key side: A[r][i] = sum_c b_rc k_rc k_ic
+// exp(G_rc - G_ic), T' = (I + A)^{-1} (no column scaling) and W = T' (b * K<-)
+// (the erase-side auxiliary Y); the write gate w (layout of v) gives the
+// write-side target Z = w * v, written here for the scan's U = T' Z.  So the
+// left operand of A and of W becomes b * Khat; Aqk, Q<-, K_tail and gamma_C
+// are those of KDA.
+template <bool SCALAR, bool PRO, bool GDR2>
 __global__ void __launch_bounds__(kThreads, 2)
 ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__restrict__ qg,
                const void *__restrict__ gin, const float *__restrict__ betag,
-               const float *__restrict__ A_log, const float *__restrict__ dt_bias, __nv_bfloat16 *__restrict__ Tout,
+               const float *__restrict__ A_log, const float *__restrict__ dt_bias,
+               const __nv_bfloat16 *__restrict__ erg, const __nv_bfloat16 *__restrict__ vg,
+               const __nv_bfloat16 *__restrict__ wrg, __nv_bfloat16 *__restrict__ Zout,
+               __nv_bfloat16 *__restrict__ Tout,
                __nv_bfloat16 *__restrict__ Aqout, __nv_bfloat16 *__restrict__ Wout, __nv_bfloat16 *__restrict__ Qlo,
                __nv_bfloat16 *__restrict__ Kto, float *__restrict__ gamo, int T_len, int nchunks, int total,
                int n_heads)
 {
+    static_assert(!(PRO && GDR2), "the fused prologue is for the tied-gate rule");
     extern __shared__ unsigned char prep_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(prep_raw) + 1023) &
                                                           ~static_cast<uintptr_t>(1023));
@@ -244,6 +263,7 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
         const uint32_t c = 64u * (warp & 1) + 4u * (lane & 15);
         const int rbase = 16 * R + 8 * half;
         uint2 kr[8], qr[8];
+        uint2 br[GDR2 ? 8 : 1];             // GDR-2 erase gate b
         float4 gv[8];                       // g, then alpha = exp(max(g, -5))
         float2 oa = make_float2(1.f, 1.f), ob = oa;   // alpha product of the other half block
         // 1 / L2 norm of the rows of q, k (prologue; 1 otherwise), kept in
@@ -260,6 +280,7 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
                 const size_t e = (row0 + min(rbase + rr, nrows - 1)) * kDK + c;
                 kr[rr] = __ldg(reinterpret_cast<const uint2 *>(kg + e));
                 qr[rr] = __ldg(reinterpret_cast<const uint2 *>(qg + e));
+                if (GDR2) br[rr] = __ldg(reinterpret_cast<const uint2 *>(erg + e));
                 if (!SCALAR) {
                     if (PRO) {   // a as four bf16, widened; the gate is formed below
                         const uint2 av = __ldg(reinterpret_cast<const uint2 *>(ag + e));
@@ -275,6 +296,7 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
                 if (rbase + rr >= nrows) {
                     kr[rr] = make_uint2(0u, 0u);
                     qr[rr] = make_uint2(0u, 0u);
+                    if (GDR2) br[rr] = make_uint2(0u, 0u);
                     if (!SCALAR) gv[rr] = make_float4(0.f, 0.f, 0.f, 0.f);
                 }
             }
@@ -333,8 +355,12 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
                 __syncwarp();
             }
             if (tid < kC) {
-                const float bl = tid < nrows ? __ldg(betag + row0 + tid) : 0.f;
-                sBeta[tid] = tid < nrows ? (PRO ? 1.f / (1.f + __expf(-bl)) : bl) : 0.f;
+                if (GDR2) {   // the gates sit in the operands; T' is (I + A)^{-1} itself
+                    sBeta[tid] = tid < nrows ? 1.f : 0.f;
+                } else {
+                    const float bl = tid < nrows ? __ldg(betag + row0 + tid) : 0.f;
+                    sBeta[tid] = tid < nrows ? (PRO ? 1.f / (1.f + __expf(-bl)) : bl) : 0.f;
+                }
             }
             if (SCALAR && warp == 0) {
                 // inclusive scan of the scalar log-decay over the chunk (2 values per lane)
@@ -364,6 +390,11 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
                         const float2 fk = make_float2(ik(rr), ik(rr)), fq = make_float2(iq(rr), iq(rr));
                         *reinterpret_cast<uint2 *>(sm + OFF_K + off) = make_uint2(scale2p(kr[rr].x, fk), scale2p(kr[rr].y, fk));
                         *reinterpret_cast<uint2 *>(sm + OFF_Q + off) = make_uint2(scale2p(qr[rr].x, fq), scale2p(qr[rr].y, fq));
+                    } else if (GDR2) {   // left operand b * k, right operand k
+                        *reinterpret_cast<uint2 *>(sm + OFF_K + off) =
+                            make_uint2(scale2p(kr[rr].x, unpack2(br[rr].x)), scale2p(kr[rr].y, unpack2(br[rr].y)));
+                        *reinterpret_cast<uint2 *>(sm + OFF_KC + off) = kr[rr];
+                        *reinterpret_cast<uint2 *>(sm + OFF_Q + off) = qr[rr];
                     } else {
                         *reinterpret_cast<uint2 *>(sm + OFF_K + off) = kr[rr];
                         *reinterpret_cast<uint2 *>(sm + OFF_Q + off) = qr[rr];
@@ -392,8 +423,13 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
                     pa = fmul2(pa, make_float2(gv[rr].x, gv[rr].y));
                     pb = fmul2(pb, make_float2(gv[rr].z, gv[rr].w));
                     const float2 nk = make_float2(ik(rr), ik(rr)), nq = make_float2(iq(rr), iq(rr));
-                    *reinterpret_cast<uint2 *>(sm + OFF_K + off) =
-                        make_uint2(scale2p(kr[rr].x, PRO ? fmul2(pa, nk) : pa), scale2p(kr[rr].y, PRO ? fmul2(pb, nk) : pb));
+                    if (GDR2)   // Ehat = b * Khat
+                        *reinterpret_cast<uint2 *>(sm + OFF_K + off) =
+                            make_uint2(scale2p(kr[rr].x, fmul2(pa, unpack2(br[rr].x))),
+                                       scale2p(kr[rr].y, fmul2(pb, unpack2(br[rr].y))));
+                    else
+                        *reinterpret_cast<uint2 *>(sm + OFF_K + off) =
+                            make_uint2(scale2p(kr[rr].x, PRO ? fmul2(pa, nk) : pa), scale2p(kr[rr].y, PRO ? fmul2(pb, nk) : pb));
                     *reinterpret_cast<uint2 *>(sm + OFF_Q + off) =
                         make_uint2(scale2p(qr[rr].x, PRO ? fmul2(pa, nq) : pa), scale2p(qr[rr].y, PRO ? fmul2(pb, nq) : pb));
                 }
@@ -487,13 +523,26 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
                     *reinterpret_cast<float4 *>(gamo + (size_t)ci * kDK + c) = make_float4(gl, gl, gl, gl);
                 }
             }
+            if (GDR2) {
+                // write-side target Z = w * v (d_v = 128 channels, the layout of v)
+#pragma unroll
+                for (int rr = 0; rr < 8; ++rr) {
+                    if (rbase + rr < nrows) {
+                        const size_t e = e0 + (size_t)(rbase + rr) * kDK;
+                        const uint2 vv = __ldg(reinterpret_cast<const uint2 *>(vg + e));
+                        const uint2 ww = __ldg(reinterpret_cast<const uint2 *>(wrg + e));
+                        *reinterpret_cast<uint2 *>(Zout + e) =
+                            make_uint2(scale2p(vv.x, unpack2(ww.x)), scale2p(vv.y, unpack2(ww.y)));
+                    }
+                }
+            }
         }
 
         // ---- block products on tensor cores: 10 block pairs over 8 warps, each
         // pair gives both A and Aqk (the right operand and its scaling are shared)
         {
             const uint32_t left_k = smem_u32(sm + OFF_K), left_q = smem_u32(sm + OFF_Q);
-            const uint32_t right = SCALAR ? left_k : smem_u32(sm + OFF_KC);
+            const uint32_t right = (SCALAR && !GDR2) ? left_k : smem_u32(sm + OFF_KC);
             for (int p = warp; p < 10; p += 8) {
                 // pairs (R, I), I <= R, in row-major order of the lower block triangle
                 const int R = p < 1 ? 0 : p < 3 ? 1 : p < 6 ? 2 : 3;
@@ -774,12 +823,15 @@ cudaError_t launch_ut_prep(const ChunkArgs &a, const TcWorkspace &w, cudaStream_
     if (total > 0x7fffffffLL) return cudaErrorInvalidValue;
     const long long slots = 2LL * sm_count();   // two resident CTAs per SM
     const int grid = (int)(total < slots ? total : slots);
-    auto kern = a.prologue ? (a.scalar_gate ? ut_prep_kernel<true, true> : ut_prep_kernel<false, true>)
-                           : (a.scalar_gate ? ut_prep_kernel<true, false> : ut_prep_kernel<false, false>);
+    auto kern = a.gdr2       ? (a.scalar_gate ? ut_prep_kernel<true, false, true> : ut_prep_kernel<false, false, true>)
+                : a.prologue ? (a.scalar_gate ? ut_prep_kernel<true, true, false> : ut_prep_kernel<false, true, false>)
+                             : (a.scalar_gate ? ut_prep_kernel<true, false, false> : ut_prep_kernel<false, false, false>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_ALLOC);
     if (e != cudaSuccess) return e;
     kern<<<grid, kThreads, SMEM_ALLOC, stream>>>((const __nv_bfloat16 *)a.k, (const __nv_bfloat16 *)a.q,
-                                                 (const void *)a.g, a.beta, a.A_log, a.dt_bias, w.T, w.Aqk, w.W,
+                                                 (const void *)a.g, a.beta, a.A_log, a.dt_bias,
+                                                 (const __nv_bfloat16 *)a.erase, (const __nv_bfloat16 *)a.v,
+                                                 (const __nv_bfloat16 *)a.write, w.Z, w.T, w.Aqk, w.W,
                                                  w.Ql, w.Kt, w.gam, a.T, nchunks,
                                                  (int)total, a.H);
     return cudaGetLastError();

@@ -42,6 +42,7 @@ _STREAM = 0xD1B54A32D192ED03
 TID_Q, TID_K, TID_V, TID_G, TID_BETA, TID_S0, TID_CHAN = 1, 2, 3, 4, 5, 6, 7
 # raw inputs of the fused gate / normalisation prologue
 TID_QRAW, TID_KRAW, TID_AGATE, TID_ALOG, TID_DTBIAS, TID_BLOGIT = 8, 9, 10, 11, 12, 13
+TID_ERASE, TID_WRITE = 14, 15   # Gated Delta Rule-2 erase and write gates
 
 
 def _s64(c: int) -> int:
@@ -128,6 +129,7 @@ class Workload:
     s0: str              # "zero" or "normal002"
     seed: int
     description: str
+    rule: str = "gdr"    # "gdr" (tied beta: KDA / Gated DeltaNet) or "gdr2" (erase and write gates)
 
     @property
     def tokens(self) -> int:
@@ -153,6 +155,15 @@ WORKLOADS: Dict[str, Workload] = {
         "prologue", "normal002", 2,
         "KDA forward with the input prologue fused in (raw q, k; bf16 gate pre-activation; beta "
         "logits): B2 H32 T8192 d128 C64 bf16"),
+    "gdr2_d128_t8192": Workload(
+        "gdr2_d128_t8192", "chunk", 2, 32, 8192, 128, 128, 64, "per_channel", torch.bfloat16,
+        "softplus_n02_clamp5", "normal002", 5,
+        "Gated Delta Rule-2 forward (per-channel decay, erase and write gates): B2 H32 T8192 d128 C64 bf16",
+        rule="gdr2"),
+    "gdr2_decode_b256": Workload(
+        "gdr2_decode_b256", "decode", 256, 32, 1000, 128, 128, 1, "per_channel", torch.bfloat16,
+        "softplus_n01_plus1_clamp5", "normal002", 6,
+        "Gated Delta Rule-2 recurrent decode: B256 H32 d128, 1000 steps, fp32 state", rule="gdr2"),
     "kda_long_t65536": Workload(
         "kda_long_t65536", "chunk", 1, 32, 65536, 128, 128, 64, "per_channel", torch.bfloat16,
         "long_context_mix", "normal002", 3,
@@ -224,6 +235,8 @@ def generate(w: Workload, device="cpu", heads: Optional[Sequence[int]] = None,
     Chunk workloads return q, k [B,H,T,dk], v [B,H,T,dv], g [B,H,T,dk] or
     [B,H,T], beta [B,H,T], S0 [B,H,dv,dk] (fp32).  Decode returns the same
     keys with a leading steps axis: q [S,B,H,dk] ... and S0 [B,H,dv,dk].
+    Gated Delta Rule-2 workloads add the erase gate b (shape of k) and the
+    write gate w (shape of v), sigmoid(N(0,1)) in the workload dtype.
     """
     B, H, dk, dv = w.B, w.H, w.dk, w.dv
     if heads is None:
@@ -283,6 +296,11 @@ def generate(w: Workload, device="cpu", heads: Optional[Sequence[int]] = None,
                   torch.float64).to(torch.float32)
     beta = field(TID_BETA, 0, lambda tid_, full, b, h, c, t: _sigmoid64(normal(seed, tid_, full)),
                  torch.float64).to(torch.float32)
+    gates2 = {}
+    if w.rule == "gdr2":
+        sig = lambda tid_, full, b, h, c, t: _sigmoid64(normal(seed, tid_, full))
+        gates2 = dict(b=(to_dtype(field(TID_ERASE, dk, sig, torch.float64), w.dtype), dk),
+                      w=(to_dtype(field(TID_WRITE, dv, sig, torch.float64), w.dtype), dv))
 
     # initial state: [head, dv, dk], flat index over the full [B,H,dv,dk]
     if w.s0 == "zero":
@@ -306,6 +324,8 @@ def generate(w: Workload, device="cpu", heads: Optional[Sequence[int]] = None,
         out = dict(q=shp(q, dk), k=shp(k, dk), v=shp(v, dv),
                    g=shp(g, dk) if w.gate == "per_channel" else shp(g),
                    beta=shp(beta), S0=S0.view(outB, outH, dv, dk))
+    for name, (x, width) in gates2.items():
+        out[name] = shp(x, width)
     return out
 
 
@@ -367,7 +387,7 @@ def generate_prologue(w: Workload, device="cpu", heads: Optional[Sequence[int]] 
 
 def small_chunk_case(B: int, H: int, T: int, dk: int, dv: int, gate: str, dtype: torch.dtype,
                      g_recipe: str = "softplus_n01_plus1_clamp5", s0: str = "normal002",
-                     seed: int = 11, C: int = 64) -> Workload:
+                     seed: int = 11, C: int = 64, rule: str = "gdr") -> Workload:
     """An ad-hoc chunk workload with the same value recipes (parity tests)."""
-    return Workload(f"case_B{B}H{H}T{T}d{dk}x{dv}_{gate}", "chunk", B, H, T, dk, dv, C, gate, dtype,
-                    g_recipe, s0, seed, "parity case")
+    return Workload(f"case_B{B}H{H}T{T}d{dk}x{dv}_{gate}_{rule}", "chunk", B, H, T, dk, dv, C, gate, dtype,
+                    g_recipe, s0, seed, "parity case", rule=rule)

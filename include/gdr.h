@@ -149,6 +149,47 @@ int gdr_chunk_fwd_prologue(const void *q_raw, const void *k_raw, const void *v, 
                            void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * Gated Delta Rule-2: the erase and write decisions of the delta rule get
+ * their own per-channel gates ("Token Mixer I", section "Gated DeltaNet-2:
+ * Decoupling Erase and Write in Linear Attention", eq. (10)).  With
+ * S~ = S_{t-1} Diag(alpha_t), in the d_v x d_k orientation of gdr_chunk_fwd:
+ *   delta = w_t * v_t - S~ (b_t * k_t),   S_t = S~ + delta k_t^T,   o_t = S_t q_t
+ * b_t in [0,1]^d_k is the erase gate (the key coordinates the old content is
+ * read along), w_t in [0,1]^d_v the write gate (the value coordinates
+ * written).  b = w = beta 1 gives gdr_chunk_fwd / gdr_recurrent_step.  The
+ * chunked form follows the section's "Chunkwise parallel training": T' =
+ * (I + StrictTril((b * K<-) K->^T))^{-1}, Y = T' (b * K<-), U = T' (w * V).
+ *
+ * gdr2_chunk_fwd: arguments as gdr_chunk_fwd, with beta replaced by
+ *   b   [B,H,T,d_k]   dtype (as q, k)     erase gate
+ *   w   [B,H,T,d_v]   dtype (as v)        write gate
+ * Only the tensor-core configuration (bf16, d_k = d_v = 128, C = 64) runs;
+ * anything else returns GDR_ERR_UNSUPPORTED.  The -5 lower bound applies to
+ * a per-channel gate as in gdr_chunk_fwd.  Its workspace is larger than
+ * gdr_chunk_fwd's (it also holds w * v): size it with
+ * gdr2_chunk_fwd_workspace_size (0 for unsupported arguments).
+ */
+size_t gdr2_chunk_fwd_workspace_size(int B, int H, int T, int dk, int dv, int C,
+                                     int gate_mode, int dtype);
+
+int gdr2_chunk_fwd(const void *q, const void *k, const void *v, const float *g, const void *b, const void *w,
+                   const float *S0, void *O, float *S_T,
+                   int B, int H, int T, int dk, int dv, int C, int gate_mode, int dtype,
+                   void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * gdr2_recurrent_step: one Gated Delta Rule-2 decode step, arguments as
+ * gdr_recurrent_step with beta replaced by
+ *   b   [B,H,d_k]   dtype     erase gate
+ *   w   [B,H,d_v]   dtype     write gate
+ * Same sizes and dtypes as gdr_recurrent_step (d_k, d_v in {64, 128}; fp32
+ * or bf16); S is updated in place.
+ */
+int gdr2_recurrent_step(const void *q, const void *k, const void *v, const float *g, const void *b, const void *w,
+                        float *S, void *o, int B, int H, int dk, int dv, int gate_mode, int dtype,
+                        void *stream);
+
+/*
  * Chunked forward that allocates nothing, for callers that cannot allocate
  * device memory or pass a workspace at the point of the call: serving or
  * real-time loops that forbid allocator calls on their hot path, code that

@@ -100,6 +100,31 @@ def test_prologue_argument_validation(L):
     assert prologue(L, T=0) == OK
 
 
+def gdr2(L, B=1, H=1, T=64, dk=128, dv=128, C=64, gate=0, dtype=1, ptr=GOOD, b=GOOD, w=GOOD, ws=1 << 40, wsp=GOOD):
+    return L.gdr2_chunk_fwd(ptr, ptr, ptr, ptr, b, w, None, ptr, None, B, H, T, dk, dv, C, gate, dtype, wsp, ws, None)
+
+
+def test_gdr2_argument_validation(L):
+    assert gdr2(L, B=-1) == INVALID
+    assert gdr2(L, gate=2) == INVALID
+    assert gdr2(L, dtype=0) == UNSUPPORTED          # the tensor-core configuration only
+    assert gdr2(L, dk=64, dv=64) == UNSUPPORTED
+    assert gdr2(L, b=None) == INVALID
+    assert gdr2(L, w=None) == INVALID
+    assert gdr2(L, w=ODD) == ALIGN
+    need = L.gdr2_chunk_fwd_workspace_size(1, 1, 64, 128, 128, 64, 0, 1)
+    assert need == _tc_workspace(1, 1, 64) + 64 * 128 * 2   # plus w * v, bf16 per token
+    assert gdr2(L, ws=need - 1) == INVALID
+    assert gdr2(L, B=0) == OK and L.gdr_last_launch_count() == 0
+    assert gdr2(L, T=0) == OK
+
+    def step(dk=128, dv=128, b=GOOD, w=GOOD, ptr=GOOD):
+        return L.gdr2_recurrent_step(ptr, ptr, ptr, ptr, b, w, ptr, ptr, 2, 2, dk, dv, 0, 1, None)
+    assert step(dk=32) == UNSUPPORTED
+    assert step(b=None) == INVALID
+    assert step(w=ODD) == ALIGN
+
+
 def test_step_argument_validation(L):
     def step(B=2, H=2, dk=128, dv=128, gate=0, dtype=1, ptr=GOOD):
         return L.gdr_recurrent_step(ptr, ptr, ptr, ptr, ptr, ptr, ptr, B, H, dk, dv, gate, dtype, None)
@@ -124,6 +149,9 @@ def test_workspace_query(L):
     # fp32 inputs or other sizes run on the CUDA-core path, which needs none
     assert L.gdr_chunk_fwd_workspace_size(1, 2, 256, 64, 64, 64, 0, 0) == 0
     assert L.gdr_chunk_fwd_workspace_size(1, 2, 256, 128, 128, 32, 0, 1) == 0
+    assert L.gdr2_chunk_fwd_workspace_size(2, 32, 8192, 128, 128, 64, 0, 1) == \
+        _tc_workspace(2, 32, 8192) + 2 * 32 * 8192 * 128 * 2
+    assert L.gdr2_chunk_fwd_workspace_size(1, 2, 256, 64, 64, 64, 0, 0) == 0
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):

@@ -16,6 +16,9 @@ Contents
   * ``prologue`` / ``forward_prologue`` -- the input prologue (L2-normalised
     q, k; softplus gate with the -5 bound; sigmoid beta) and the forward fed
     by it, the reference of the fused-prologue entry point.
+  * ``output_gate`` / ``forward_gated`` -- the output epilogue of the layer
+    (per-head RMSNorm of o_t, times a sigmoid output gate), the reference of
+    the gated-output entry point.
   * ``chunk_form`` (module) -- an fp64 restatement of the chunkwise WY/UT
     equations, used only to pin ``forward`` (it is not a parity reference).
 
@@ -217,3 +220,29 @@ def decode_gdr2(q, k, v, g, b, w, S, gate: str = "per_channel", threads: int = 0
     mv = lambda x: _f64(x).transpose(1, 2, 0, *range(3, _f64(x).ndim)).copy()
     O, ST = forward_gdr2(mv(q), mv(k), mv(v), mv(g), mv(b), mv(w), S0=S, gate=gate, threads=threads)
     return O.transpose(2, 0, 1, 3).copy(), ST
+
+
+def output_gate(O, gate, norm_w, eps: float):
+    """The output epilogue of a KDA layer, in fp64: "Token Mixer I", section
+    "The Kimi Linear Model Architecture" -- before the output projection W_o,
+    each head's output o_t is normalised by a per-head RMSNorm and multiplied
+    by a data-dependent sigmoid gate:
+
+        y_t = Sigmoid(gate_t) * RMSNorm(o_t),
+        RMSNorm(x) = x / sqrt(mean_c x_c^2 + eps) * norm_w      (over the d_v channels)
+
+    O, gate [B,H,T,dv]; norm_w [dv] (one weight vector shared by the heads).
+    Returns y [B,H,T,dv] (fp64).
+    """
+    o = _f64(O)
+    z = _f64(gate)
+    wv = _f64(norm_w)
+    ms = (o * o).mean(-1, keepdims=True)
+    return o / np.sqrt(ms + eps) * wv * (1.0 / (1.0 + np.exp(-z)))
+
+
+def forward_gated(q, k, v, g, beta, gate, norm_w, eps: float, S0=None, gate_mode: str = "per_channel",
+                  threads: int = 0) -> Tuple[np.ndarray, np.ndarray]:
+    """``forward`` then ``output_gate``: returns (y [B,H,T,dv], S_T)."""
+    O, ST = forward(q, k, v, g, beta, S0, gate=gate_mode, threads=threads)
+    return output_gate(O, gate, norm_w, eps), ST

@@ -51,10 +51,12 @@ DEFAULT_WORKLOAD = "kda_d128_t8192"
 # workload with the hash of the sources those kernels are built from; an
 # entry is ignored (traffic = null) as soon as any of the sources changes.
 TRAFFIC = {
-    # ut_prep 539.0 MB read + 493.4 MB written, chunk_scan 679.5 + 117.7 MB (one launch each)
-    "kda_d128_t8192": {"src_sha": "0c9f0d70d986ac6f", "bytes_per_launch": 1829669120},
-    # Gated Delta Rule-2: ut_prep 939.6 + 634.4 MB (reads b, v, w; writes w * v), chunk_scan 679.5 + 117.9 MB
-    "gdr2_d128_t8192": {"src_sha": "0c9f0d70d986ac6f", "bytes_per_launch": 2371415040},
+    # ut_prep 539.0 MB read + 493.3 MB written, chunk_scan 679.6 + 118.4 MB (one launch each)
+    "kda_d128_t8192": {"src_sha": "5fc857a143f498dc", "bytes_per_launch": 1830330112},
+    # gated output: the scan also reads the gate tiles (813.9 + 121.6 MB); ut_prep 539.0 + 493.8 MB
+    "kda_d128_t8192_gated": {"src_sha": "5fc857a143f498dc", "bytes_per_launch": 1968358144},
+    # Gated Delta Rule-2: ut_prep 939.6 + 633.4 MB (reads b, v, w; writes w * v), chunk_scan 679.6 + 118.4 MB
+    "gdr2_d128_t8192": {"src_sha": "5fc857a143f498dc", "bytes_per_launch": 2371053824},
     # recurrent_step, one decode step: 547.4 MB read + 479.2 MB written
     "kda_decode_b256": {"src_sha": "99a0454504c77460", "bytes_per_launch": 1026655488},
 }
@@ -76,6 +78,8 @@ def algorithmic_bytes(w: W.Workload) -> int:
     if w.rule == "gdr2":            # erase gate [dk] and write gate [dv] in the input dtype
         strength = (w.dk + w.dv) * e
     per_token = 2 * w.dk * e + w.dv * e + gate + strength + w.dv * e   # q, k, v, g, beta, O
+    if w.out == "gated":            # the output gate pre-activation is read too
+        per_token += w.dv * e
     heads = w.B * w.H
     state = 2 * w.dv * w.dk * 4                                     # S0 read + S_T write
     if w.kind == "decode":
@@ -234,6 +238,9 @@ def api_call(gdr, w: W.Workload, x, **kw):
     if w.g_recipe == "prologue":
         return gdr.chunk_fwd_prologue(x["q_raw"], x["k_raw"], x["v"], x["a"], x["A_log"], x["dt_bias"],
                                       x["b_logit"], x["S0"], C=w.C, gate=w.gate, **kw)
+    if w.out == "gated":
+        return gdr.chunk_fwd_gated(x["q"], x["k"], x["v"], x["g"], x["beta"], x["ogate"], x["norm_w"], 1e-6,
+                                   x["S0"], C=w.C, gate_mode=w.gate, **{("Y" if k == "O" else k): v for k, v in kw.items()})
     if w.rule == "gdr2":
         return gdr.chunk_fwd_gdr2(x["q"], x["k"], x["v"], x["g"], x["b"], x["w"], x["S0"], C=w.C, gate=w.gate, **kw)
     return gdr.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], C=w.C, gate=w.gate, **kw)
@@ -284,7 +291,10 @@ def oracle_sample(w: W.Workload, budget_s: float, seed_rank: int = 0):
             return time.perf_counter() - t
         args = [sl(x[k]) for k in ("q", "k", "v", "g", "beta")]
         t = time.perf_counter()
-        oracle.forward(*args, x["S0"], gate=w.gate, threads=cores)
+        if w.out == "gated":
+            oracle.forward_gated(*args, sl(x["ogate"]), x["norm_w"], 1e-6, x["S0"], gate_mode=w.gate, threads=cores)
+        else:
+            oracle.forward(*args, x["S0"], gate=w.gate, threads=cores)
         return time.perf_counter() - t
 
     # calibrate on one head per core

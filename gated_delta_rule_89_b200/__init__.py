@@ -20,6 +20,7 @@ from typing import Optional, Tuple
 import torch
 
 __all__ = ["chunk_fwd", "recurrent_step", "chunk_fwd_workspace_size", "chunk_fwd_prologue", "chunk_fwd_gdr2",
+           "chunk_fwd_gated",
            "recurrent_step_gdr2", "GDRError", "library_path",
            "last_launch_count", "device_status", "GATE_PER_CHANNEL", "GATE_SCALAR"]
 
@@ -58,6 +59,9 @@ def lib() -> ctypes.CDLL:
         L.gdr_recurrent_step.restype = I
         L.gdr_chunk_fwd_workspace_size.argtypes = [I, I, I, I, I, I, I, I]
         L.gdr_chunk_fwd_workspace_size.restype = Z
+        L.gdr_chunk_fwd_gated.argtypes = [P, P, P, P, P, P, P, ctypes.c_float, P, P, P, I, I, I, I, I, I, I, I,
+                                          P, Z, P]
+        L.gdr_chunk_fwd_gated.restype = I
         L.gdr2_chunk_fwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P, Z, P]
         L.gdr2_chunk_fwd.restype = I
         L.gdr2_chunk_fwd_workspace_size.argtypes = [I, I, I, I, I, I, I, I]
@@ -371,3 +375,64 @@ def recurrent_step_gdr2(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: to
                                    B, H, dk, dv, gm, _DTYPES[dt], _stream_handle(dev, stream))
     _check(st, "gdr2_recurrent_step")
     return o
+
+
+def chunk_fwd_gated(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor, beta: torch.Tensor,
+                    gate: torch.Tensor, norm_w: torch.Tensor, eps: float = 1e-6,
+                    S0: Optional[torch.Tensor] = None, C: int = 64, gate_mode: Optional[str] = None,
+                    Y: Optional[torch.Tensor] = None, S_T: Optional[torch.Tensor] = None,
+                    final_state: bool = True, workspace: Optional[torch.Tensor] = None,
+                    stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Chunkwise forward with the output epilogue fused in (``gdr_chunk_fwd_gated``):
+    Y = Sigmoid(gate) * RMSNorm(o) per head and token.
+
+    q, k [B,H,T,dk], v and gate [B,H,T,dv] bf16; g, beta, S0 as ``chunk_fwd``;
+    norm_w fp32 [dv].  Returns (Y [B,H,T,dv] bf16, S_T fp32 or None).
+    """
+    host = not q.is_cuda
+    if host:
+        dev = torch.device("cuda", torch.cuda.current_device())
+        q, k, v, g, beta, gate, norm_w, S0 = (_to_device(x, dev) for x in (q, k, v, g, beta, gate, norm_w, S0))
+    dev = q.device
+    if gate_mode is None:
+        gate_mode = "per_channel" if g.dim() == 4 else "scalar"
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    if dt != torch.bfloat16:
+        raise TypeError("the gated-output forward takes bf16 q, k, v, gate")
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (gate, "gate")):
+        _need(t, n, dt, dev)
+    for t, n in ((g, "g"), (beta, "beta"), (norm_w, "norm_w")):
+        _need(t, n, torch.float32, dev)
+    if tuple(k.shape) != (B, H, T, dk) or tuple(v.shape[:3]) != (B, H, T) or tuple(beta.shape) != (B, H, T) \
+            or tuple(gate.shape) != (B, H, T, dv) or tuple(norm_w.shape) != (dv,):
+        raise ValueError("inconsistent shapes")
+    if gate_mode == "per_channel" and tuple(g.shape) != (B, H, T, dk):
+        raise ValueError("per-channel g must be [B,H,T,dk]")
+    if gate_mode == "scalar" and tuple(g.shape) != (B, H, T):
+        raise ValueError("scalar g must be [B,H,T]")
+    if S0 is not None:
+        _need(S0, "S0", torch.float32, dev)
+        if tuple(S0.shape) != (B, H, dv, dk):
+            raise ValueError("S0 must be [B,H,dv,dk]")
+    if Y is None:
+        Y = torch.empty(B, H, T, dv, dtype=dt, device=dev)
+    _need(Y, "Y", dt, dev)
+    if S_T is None and final_state:
+        S_T = torch.empty(B, H, dv, dk, dtype=torch.float32, device=dev)
+    if S_T is not None:
+        _need(S_T, "S_T", torch.float32, dev)
+    gm = GATE_PER_CHANNEL if gate_mode == "per_channel" else GATE_SCALAR
+    L = lib()
+    ws_bytes = int(L.gdr_chunk_fwd_workspace_size(B, H, T, dk, dv, C, gm, _DTYPES[dt]))
+    if ws_bytes and (workspace is None or workspace.numel() * workspace.element_size() < ws_bytes):
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    st = L.gdr_chunk_fwd_gated(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(gate), _ptr(norm_w), float(eps),
+                               _ptr(S0), _ptr(Y), _ptr(S_T), B, H, T, dk, dv, C, gm, _DTYPES[dt],
+                               _ptr(workspace) if ws_bytes else None, ws_bytes, _stream_handle(dev, stream))
+    _check(st, "gdr_chunk_fwd_gated")
+    if host:
+        Y = Y.to("cpu")
+        S_T = None if S_T is None else S_T.to("cpu")
+    return Y, S_T

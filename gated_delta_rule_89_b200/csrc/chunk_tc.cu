@@ -23,18 +23,25 @@
 //      into double-buffered tiles, and the same tiles serve as K-major or
 //      MN-major operands.
 //
-// Warp roles (320 threads):
+// Warp roles (448 threads):
 //   warp 0      TMA producer (lane 0): all tiles of a chunk land in one of
 //               two stages and complete one barrier; gamma_C in two slots.
-//               Lane 1 issues the TMA stores of the output tiles.
+//               Lane 1 issues the TMA stores of the output tiles (and, for
+//               the gated output, the loads of the gate tiles).
 //   warp 1      TMEM allocation and the MMA issuer (one lane), in the order
 //               X^T(n), O^T(n), dS(n), O(n), U^T(n+1), so the products that do
 //               not depend on the state run while the state is updated
-//   warps 2-9   every conversion, split by columns between warps 2-5 and
-//               6-9: on the sequential path S (TMEM) -> bf16 smem and
+//   warps 2-9   the state conversions, split by columns between warps 2-5
+//               and 6-9: on the sequential path S (TMEM) -> bf16 smem and
 //               V_new^T (TMEM) -> bf16 smem; off it, in the gaps while the
-//               tensor core runs, S *= gamma_C in TMEM and the output
-//               epilogue O^T (TMEM) -> bf16 smem tile -> TMA store.
+//               tensor core runs, S *= gamma_C in TMEM.
+//   warps 10-13 the output epilogue, one chunk behind the MMAs (the O^T
+//               accumulator is double-buffered): O^T (TMEM) -> bf16 staging
+//               tile -> TMA store.  With OEPI the layer's gated output is
+//               fused in: y_t = Sigmoid(gate_t) * RMSNorm(o_t) per head
+//               ("Token Mixer I", section "The Kimi Linear Model
+//               Architecture", the output equation before W_o), RMSNorm over
+//               the d_v channels in fp32 straight from the accumulator.
 // The sequential chain per chunk is dS -> S to bf16 -> X^T -> V_new -> dS.
 // Every wait is bounded (about a second); on timeout the kernel records
 // GDR_ERR_TIMEOUT in a device status word, lets the copies and MMAs it
@@ -57,7 +64,7 @@ using namespace sm100;
 
 constexpr int kC = 64;
 constexpr int kD = 128;
-constexpr int kThreads = 320;   // 10 warps: TMA, MMA, 4 x E, 4 x M
+constexpr int kThreads = 448;   // 14 warps: TMA, MMA, 8 conversion warps, 4 output-epilogue warps
 constexpr long long kWaitBudget = 2000000000LL;   // clock cycles per wait (~1 s)
 
 // shared memory map (bytes from a 1024-aligned base).  The input tiles of a
@@ -76,7 +83,9 @@ constexpr uint32_t OFF_S = OFF_OST + 16384;        // bf16 S (2 panels x 16 KB) 
 constexpr uint32_t OFF_VN = OFF_S + 32768;         // V_new^T (1 panel, 128 rows)           16 KB
 constexpr uint32_t OFF_GAM = OFF_VN + 16384;       // gamma_C of each stage, [2][128] fp32   1 KB
 constexpr uint32_t OFF_BAR = OFF_GAM + 1024;       // mbarriers, TMEM slot, abort flag
-constexpr uint32_t SMEM_USED = OFF_BAR + 256;
+constexpr uint32_t OFF_RED = OFF_BAR + 256;        // gated output: partial sums [4 warps][32 tokens] fp32
+constexpr uint32_t OFF_RSTD = OFF_RED + 512;       // gated output: 1 / RMS of the 64 tokens
+constexpr uint32_t SMEM_USED = OFF_RSTD + 256;
 constexpr uint32_t SMEM_ALLOC = SMEM_USED + 1024;  // alignment slack
 static_assert(SMEM_ALLOC <= 232448, "dynamic shared memory above the 227 KB per-block limit");
 
@@ -99,6 +108,7 @@ enum Bar {
     B_OACC_EMPTY, B_OACC_EMPTY1,   // O^T accumulator drained by the epilogue
     B_EPI_FULL,               // O^T staging tile written (warps 2-9)
     B_EPI_FREE,               // O^T staging tile free again (the previous store has read it)
+    B_GATE_FULL,              // gated output: the gate tile of the next chunk landed in the staging tile
     B_FINAL,
     B_COUNT
 };
@@ -107,6 +117,7 @@ static_assert(8 * B_COUNT + 8 <= 256, "barrier area");
 struct Maps {
     CUtensorMap w, q, kt, v, t, aq, o;   // Q<-, K_tail, v, O: [BH][T][128]; T', Aqk: [chunks*64][64];
                                          // W^T: [chunks*128][64]
+    CUtensorMap og;                      // output gate [BH][T][128] (gated output only)
 };
 
 __device__ __forceinline__ void record_error(int code) { atomicCAS(&g_device_status, 0, code); }
@@ -123,6 +134,12 @@ __device__ long long g_trace[16][1024];
     do {                    \
     } while (0)
 #endif
+
+__device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi)
+{
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
 {
@@ -143,11 +160,30 @@ __device__ __forceinline__ void pack16(const uint32_t (&r)[16], uint4 &lo, uint4
     hi.w = pack_bf16(__uint_as_float(r[14]), __uint_as_float(r[15]));
 }
 
-template <bool SCALAR>
+// One barrier of the 128 threads of the output-epilogue warps that also
+// returns whether every one of them passed ok (so they leave together).
+__device__ __forceinline__ bool epi_all(bool ok)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, 1, 128, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)ok)
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+template <bool SCALAR, bool OEPI>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ gamma_c,
                   const float *__restrict__ S0, __nv_bfloat16 *__restrict__ O, float *__restrict__ ST,
-                  int T_len, int nchunks)
+                  int T_len, int nchunks, const __nv_bfloat16 *__restrict__ ogate,
+                  const float *__restrict__ norm_w, float eps)
 {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -159,7 +195,6 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
     const int head = blockIdx.x;
-    const size_t tok0 = (size_t)head * T_len;
 
     if (tid == 0) {
         const uint32_t counts[B_COUNT] = {
@@ -167,8 +202,9 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
             1, 1, 256, 256,   // gamma full (TMA), gamma empty (warps 2-9)
             256, 1, 256,      // sw ready (warps 2-9), x full (MMA), vn ready (warps 2-9)
             1,                // s full (MMA)
-            1, 1, 256, 256,   // o full (MMA) x2, oacc empty (warps 2-9) x2
-            256, 1,           // epilogue tile written (warps 2-9), free (warp 0 lane 1)
+            1, 1, 128, 128,   // o full (MMA) x2, oacc empty (epilogue warps) x2
+            128, 1,  // epilogue tile written (epilogue warps), free (warp 0 lane 1)
+            1,                // gate tile landed (TMA)
             1};
         for (int i = 0; i < B_COUNT; ++i) mbar_init(&bar[i], counts[i]);
         *abort_flag = 0;
@@ -207,9 +243,39 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
 
     if (warp == 0) {
         // ================================================================ TMA producer, output stores
-        if (lane == 1) {
-            // Output tile m: stored once the conversion warps have written it;
-            // the tile is handed back once the store has read it.
+        if (lane == 1 && OEPI) {
+            // Gated output: the staging tile first receives the gate tile of chunk m
+            // (TMA), the epilogue overwrites it with y(m), the tile is stored, and as
+            // soon as the store has read it the gate tile of chunk m + 1 goes in.
+            auto load_gate = [&](int m) {
+                mbar_arrive_expect_tx(&bar[B_GATE_FULL], 16384);
+                tma_load_3d(sm + OFF_OST, &maps.og, &bar[B_GATE_FULL], 0, m * kC, head);
+                tma_load_3d(sm + OFF_OST + 8192, &maps.og, &bar[B_GATE_FULL], 64, m * kC, head);
+            };
+            int loaded = 0;
+            if (nchunks > 0) {
+                load_gate(0);
+                loaded = 1;
+            }
+            for (int m = 0; m < nchunks; ++m) {
+                if (!wait(B_EPI_FULL, (uint32_t)(m & 1))) break;
+                tma_store_3d(&maps.o, sm + OFF_OST, 0, m * kC, head);
+                tma_store_3d(&maps.o, sm + OFF_OST + 8192, 64, m * kC, head);
+                bulk_commit_group();
+                bulk_wait_read_all();
+                if (m + 1 < nchunks) {
+                    load_gate(m + 1);
+                    loaded = m + 2;
+                }
+            }
+            bulk_wait_all();   // the last store has completed before the CTA exits
+            if (*abort_flag && loaded > 0)   // a gate tile still in flight lands before exit
+                mbar_wait(&bar[B_GATE_FULL], (uint32_t)((loaded - 1) & 1), kWaitBudget / 4);
+        }
+        if (lane == 1 && !OEPI) {
+            // Output tile m: stored once the epilogue has written it; the tile
+            // is handed back once the store has read it.  (The gated output is
+            // written by the epilogue warps themselves.)
             mbar_arrive(&bar[B_EPI_FREE]);
             for (int m = 0; m < nchunks; ++m) {
                 if (!wait(B_EPI_FULL, (uint32_t)(m & 1))) break;
@@ -223,6 +289,7 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
         }
         if (lane == 0) {
             for (int i = 0; i < 6; ++i) tma_prefetch_desc(&maps.w + i);
+            if (OEPI) tma_prefetch_desc(&maps.og);
             int issued = 0;
             for (int n = 0; n < nchunks; ++n) {
                 const int t0 = n * kC;
@@ -242,6 +309,10 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
                 tma_load_3d(st + ST_KT, &maps.kt, full, 0, t0, head);
                 tma_load_3d(st + ST_KT + 8192, &maps.kt, full, 64, t0, head);
                 tma_load_2d(st + ST_AQ, &maps.aq, full, 0, crow);
+                if (OEPI) {   // the epilogue's gate tile, warmed in L2 a chunk ahead of its load
+                    tma_prefetch_l2_3d(&maps.og, 0, t0, head);
+                    tma_prefetch_l2_3d(&maps.og, 64, t0, head);
+                }
                 // gamma_C has its own slots, released by the state update, so the
                 // stage itself only waits for the MMAs that read it
                 if (!wait(B_GEMPTY + b, upar ^ 1)) break;
@@ -325,7 +396,7 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
             mma_commit(&bar[B_FINAL]);
             mbar_wait(&bar[B_FINAL], 0, kWaitBudget);
         }
-    } else {
+    } else if (warp < 10) {
         // ================================================================ state update, conversions, epilogue
         // The state S_n lives at TM_S.  At chunk n these warps copy it to bf16
         // smem for the MMAs of chunk n (on the sequential path), then scale it
@@ -391,34 +462,6 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
             mbar_arrive(&bar[B_GEMPTY + (n & 1)]);
             return true;
         };
-        // Output of chunk m: O^T (TMEM, rows d_v) -> bf16 into the staging tile
-        // laid out as the TMA store wants it ([64 tokens x 64 d_v] panels,
-        // 128-byte swizzle), then one thread stores it.  The staging tile is
-        // reused only after the previous store has finished reading it.
-        auto epilogue = [&](int m) -> bool {
-            const int bb = m & 1;
-            if (!waitw(B_EPI_FREE, (uint32_t)(m & 1)) || !waitw(B_O_FULL + bb, (uint32_t)((m >> 1) & 1))) return false;
-            tc_fence_after();
-            // row t of a panel, column i & 63: t * 128 + (((i & 63) / 8) ^ (t % 8)) * 16 + (i % 8) * 2
-            unsigned char *ost = sm + OFF_OST + (i >> 6) * 8192 + (i & 7) * 2 + vc0 * 128;
-            const uint32_t c8 = (uint32_t)((i & 63) >> 3);
-#pragma unroll 2
-            for (int cb = 0; cb < 4; ++cb) {   // 8 tokens per step: rows vc0 + 8 cb + j, j = t % 8
-                uint32_t r[8];
-                tmem_ld8(trow + TM_O + 64 * bb + vc0 + 8 * cb, r);
-                tmem_ld_wait8(r);
-                unsigned char *rowp = ost + cb * 1024;
-#pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    *reinterpret_cast<__nv_bfloat16 *>(rowp + j * 128 + ((c8 ^ (uint32_t)j) << 4)) =
-                        __float2bfloat16_rn(__uint_as_float(r[j]));
-            }
-            tc_fence_before();
-            mbar_arrive(&bar[B_OACC_EMPTY + bb]);
-            fence_async_smem();
-            mbar_arrive(&bar[B_EPI_FULL]);
-            return true;
-        };
         bool ok = true;
         for (int n = 0; n < nchunks && ok; ++n) {
             const uint32_t par = (uint32_t)(n & 1);
@@ -449,11 +492,7 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
             tc_fence_before();
             mbar_arrive(&bar[B_VN_READY]);   // also: S_n scaled
             if (tid == 192) GDR_TRACE_AT(14, n);
-            // ---- off the sequential path while S += dS runs: last chunk's output
-            if (n > 0 && !epilogue(n - 1)) { ok = false; break; }
-            if (tid == 192) GDR_TRACE_AT(7, n);
         }
-        if (ok && nchunks > 0) ok = epilogue(nchunks - 1);
         // ---- final state S_N: the last accumulation has completed
         if (ok && nchunks > 0 && waitw(B_S_FULL, (uint32_t)((nchunks - 1) & 1))) {
             tc_fence_after();
@@ -469,6 +508,140 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
                         dst[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
                                              __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
                 }
+            }
+        }
+    } else {
+        // ================================================================ output epilogue (warps 10-13)
+        // Warp w holds d_v channels 32 (w & 3) .. + 31 (its TMEM lane quarter)
+        // of all 64 tokens of O^T(m).
+        // Plain: O^T -> bf16 staging tile -> TMA store (warp 0, lane 1).
+        // OEPI: the gate tile of chunk m is TMA-loaded into the staging tile
+        // (same layout as the output); per token the sum of squares over the 128
+        // channels (lanes, then the four warps), then
+        // y = o * rsqrt(mean o^2 + eps) * norm_w * Sigmoid(gate) is stored to
+        // global memory straight from registers (32 consecutive channels per
+        // warp and token), which frees the tile for the next gate load as soon
+        // as it has been read.
+        const uint32_t lq = 32u * (warp & 3);
+        const int i = (int)lq + lane;
+        const uint32_t trow = tmem + (lq << 16);
+        unsigned char *ost = sm + OFF_OST + (i >> 6) * 8192 + (i & 7) * 2;
+        const uint32_t c8 = (uint32_t)((i & 63) >> 3);
+        const float nw = OEPI ? __ldg(norm_w + i) : 1.f;
+        float *red = reinterpret_cast<float *>(sm + OFF_RED);     // [4 warps][32 tokens]
+        float *rstd = reinterpret_cast<float *>(sm + OFF_RSTD);   // [64 tokens]
+        for (int m = 0; m < nchunks; ++m) {
+            const int bb = m & 1;
+            // the gate tile is only needed by pass 2: its load overlaps pass 1
+            bool ok = (OEPI || waitw(B_EPI_FREE, (uint32_t)(m & 1))) && waitw(B_O_FULL + bb, (uint32_t)((m >> 1) & 1));
+            if (OEPI) ok = epi_all(ok);   // the four warps go on (or stop) together
+            if (!ok) break;
+            tc_fence_after();
+            if (tid == 320) GDR_TRACE_AT(4, m);
+            const uint32_t oc = trow + TM_O + 64 * bb;
+            if (!OEPI) {
+#pragma unroll 2
+                for (int cb = 0; cb < 8; ++cb) {
+                    uint32_t r[8];
+                    tmem_ld8(oc + 8 * cb, r);
+                    tmem_ld_wait8(r);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        *reinterpret_cast<__nv_bfloat16 *>(ost + cb * 1024 + j * 128 + ((c8 ^ (uint32_t)j) << 4)) =
+                            __float2bfloat16_rn(__uint_as_float(r[j]));
+                }
+                tc_fence_before();
+                mbar_arrive(&bar[B_OACC_EMPTY + bb]);
+                fence_async_smem();
+                mbar_arrive(&bar[B_EPI_FULL]);
+            } else {
+                // pass 1, per 32 tokens: lane L ends with this warp's partial sum of
+                // token 32 h + L; warp (w & 3) == 0 adds the four up
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    float ps[32];
+                    {
+                        uint32_t r0[8], r1[8], r2[8], r3[8];
+                        tmem_ld8(oc + 32 * h, r0);
+                        tmem_ld8(oc + 32 * h + 8, r1);
+                        tmem_ld8(oc + 32 * h + 16, r2);
+                        tmem_ld8(oc + 32 * h + 24, r3);
+                        tmem_ld_wait8(r0);
+                        reg_touch8(r1);
+                        reg_touch8(r2);
+                        reg_touch8(r3);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            ps[j] = __uint_as_float(r0[j]) * __uint_as_float(r0[j]);
+                            ps[8 + j] = __uint_as_float(r1[j]) * __uint_as_float(r1[j]);
+                            ps[16 + j] = __uint_as_float(r2[j]) * __uint_as_float(r2[j]);
+                            ps[24 + j] = __uint_as_float(r3[j]) * __uint_as_float(r3[j]);
+                        }
+                    }
+                    // transpose-reduce: keep the half of the values whose index has bit w
+                    // equal to this lane's, add the partner's copy of it
+#pragma unroll
+                    for (int w = 16; w >= 1; w >>= 1) {
+#pragma unroll
+                        for (int j = 0; j < w; ++j) {
+                            const bool up = (lane & w) != 0;
+                            const float send = up ? ps[j] : ps[j + w];
+                            const float got = __shfl_xor_sync(0xffffffffu, send, w);
+                            ps[j] = (up ? ps[j + w] : ps[j]) + got;
+                        }
+                    }
+                    red[(warp & 3) * 32 + lane] = ps[0];
+                    epi_sync();
+                    if ((warp & 3) == 0)   // half the reciprocal RMS: Sigmoid(z) = (1 + tanh(z / 2)) / 2
+                        rstd[32 * h + lane] =
+                            0.5f * rsqrtf((red[lane] + red[32 + lane] + red[64 + lane] + red[96 + lane]) * (1.f / kD) + eps);
+                    epi_sync();   // red is free again, rstd of these tokens written
+                }
+                if (tid == 320) GDR_TRACE_AT(5, m);
+                if (!epi_all(waitw(B_GATE_FULL, (uint32_t)(m & 1)))) break;
+                if (tid == 320) GDR_TRACE_AT(9, m);
+                // pass 2: 16 tokens per step; y replaces the gate element it was computed
+                // from, and the tile leaves by TMA store (rows past T are dropped)
+#pragma unroll 1
+                for (int cs = 0; cs < 4; ++cs) {
+                    uint32_t r0[8], r1[8];
+                    tmem_ld8(oc + 16 * cs, r0);
+                    tmem_ld8(oc + 16 * cs + 8, r1);
+                    float f[16], z[16];
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const float4 fv = *reinterpret_cast<const float4 *>(rstd + 16 * cs + 4 * q4);
+                        f[4 * q4] = fv.x;
+                        f[4 * q4 + 1] = fv.y;
+                        f[4 * q4 + 2] = fv.z;
+                        f[4 * q4 + 3] = fv.w;
+                    }
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        z[j] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(
+                            ost + (2 * cs + (j >> 3)) * 1024 + (j & 7) * 128 + ((c8 ^ (uint32_t)(j & 7)) << 4)));
+                    tmem_ld_wait8(r0);
+                    reg_touch8(r1);
+                    // two tokens at a time: a = o * rstd / 2 * norm_w, y = a (1 + tanh(z / 2))
+#pragma unroll
+                    for (int j = 0; j < 16; j += 2) {
+                        const float2 o2 = make_float2(__uint_as_float(j < 8 ? r0[j] : r1[j - 8]),
+                                                      __uint_as_float(j < 8 ? r0[j + 1] : r1[j - 7]));
+                        const float2 a = fmul2(fmul2(o2, make_float2(f[j], f[j + 1])), make_float2(nw, nw));
+                        const float2 hz = fmul2(make_float2(z[j], z[j + 1]), make_float2(0.5f, 0.5f));
+                        const float2 y = ffma2(a, make_float2(tanh_approx(hz.x), tanh_approx(hz.y)), a);
+                        const uint32_t yb = pack2_bf16(y.x, y.y);
+                        *reinterpret_cast<unsigned short *>(ost + (2 * cs + (j >> 3)) * 1024 + (j & 7) * 128 +
+                                                            ((c8 ^ (uint32_t)(j & 7)) << 4)) = (unsigned short)(yb & 0xffffu);
+                        *reinterpret_cast<unsigned short *>(ost + (2 * cs + (j >> 3)) * 1024 + ((j + 1) & 7) * 128 +
+                                                            ((c8 ^ (uint32_t)((j + 1) & 7)) << 4)) = (unsigned short)(yb >> 16);
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(&bar[B_OACC_EMPTY + bb]);
+                fence_async_smem();   // the tile is read next by the TMA store
+                mbar_arrive(&bar[B_EPI_FULL]);
+                if (tid == 320) GDR_TRACE_AT(6, m);
             }
         }
     }
@@ -535,6 +708,9 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream, int *launch
             if (!make_map(dst[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, tiles[i], dims3, str_bf, box_bf,
                           CU_TENSOR_MAP_SWIZZLE_128B))
                 return cudaErrorInvalidValue;
+        if (a.gated_out && !make_map(&maps.og, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(a.ogate), dims3,
+                                     str_bf, box_bf, CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
         const cuuint64_t dims2[2] = {(cuuint64_t)kC, (cuuint64_t)BH * nchunks * kC};
         const cuuint64_t str2[1] = {(cuuint64_t)kC * 2};
         const cuuint32_t box2[2] = {64, 64};
@@ -550,11 +726,13 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream, int *launch
     if (e != cudaSuccess) return e;
     *launches += 1;
 
-    auto kern = a.scalar_gate ? chunk_scan_kernel<true> : chunk_scan_kernel<false>;
+    auto kern = a.gated_out ? (a.scalar_gate ? chunk_scan_kernel<true, true> : chunk_scan_kernel<false, true>)
+                            : (a.scalar_gate ? chunk_scan_kernel<true, false> : chunk_scan_kernel<false, false>);
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_ALLOC);
     if (e != cudaSuccess) return e;
-    kern<<<BH, kThreads, SMEM_ALLOC, stream>>>(maps, w.gam, a.S0, static_cast<__nv_bfloat16 *>(a.O), a.S_T, a.T,
-                                              nchunks);
+    kern<<<BH, kThreads, SMEM_ALLOC, stream>>>(
+        maps, w.gam, a.S0, static_cast<__nv_bfloat16 *>(a.O), a.S_T, a.T, nchunks,
+        static_cast<const __nv_bfloat16 *>(a.ogate), a.norm_w, a.eps);
     e = cudaGetLastError();
     if (e == cudaSuccess) *launches += 1;
     return e;

@@ -167,6 +167,59 @@ GDR_API int gdr_chunk_fwd_prologue(const void *q_raw, const void *k_raw, const v
     return finish(e, launches);
 }
 
+GDR_API int gdr_chunk_fwd_gated(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                                const void *gate, const float *norm_w, float eps,
+                                const float *S0, void *Y, float *S_T,
+                                int B, int H, int T, int dk, int dv, int C, int gate_mode, int dtype,
+                                void *workspace, size_t ws_bytes, void *stream)
+{
+    if (B < 0 || H < 0 || T < 0) return GDR_ERR_INVALID_ARG;
+    if (gate_mode != GDR_GATE_PER_CHANNEL && gate_mode != GDR_GATE_SCALAR) return GDR_ERR_INVALID_ARG;
+    if (dtype != GDR_F32 && dtype != GDR_BF16) return GDR_ERR_INVALID_ARG;
+    if (dk <= 0 || dv <= 0 || C <= 0) return GDR_ERR_INVALID_ARG;
+    if (!(eps >= 0.f) || eps > 1e30f) return GDR_ERR_INVALID_ARG;   // also rejects NaN
+    gdr::ChunkArgs a_;
+    a_.dk = dk; a_.dv = dv; a_.C = C; a_.bf16 = (dtype == GDR_BF16);
+    if (!gdr::chunk_tc_supports(a_)) return GDR_ERR_UNSUPPORTED;   // bf16, d_k = d_v = 128, C = 64 only
+    if ((long long)B * H * T * 128 >= (1LL << 40)) return GDR_ERR_UNSUPPORTED;
+    const size_t ws_need = gdr_chunk_fwd_workspace_size(B, H, T, dk, dv, C, gate_mode, dtype);
+    if (ws_bytes < ws_need || (ws_need && !workspace)) return GDR_ERR_INVALID_ARG;
+    const long long heads = (long long)B * H;
+    if (heads == 0) {
+        tl_last_launches = 0;
+        return GDR_OK;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (T == 0) {
+        if (S_T && !aligned16(S_T)) return GDR_ERR_ALIGNMENT;
+        if (S0 && !aligned16(S0)) return GDR_ERR_ALIGNMENT;
+        cudaError_t e = cudaSuccess;
+        const size_t bytes = sizeof(float) * (size_t)heads * dv * dk;
+        if (S_T && S0 && S_T != S0) e = cudaMemcpyAsync(S_T, S0, bytes, cudaMemcpyDeviceToDevice, st);
+        else if (S_T && !S0) e = cudaMemsetAsync(S_T, 0, bytes, st);
+        return finish(e, 0);
+    }
+    if (!q || !k || !v || !g || !beta || !gate || !norm_w || !Y) return GDR_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, g, beta, gate, S0, Y, S_T, workspace};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return GDR_ERR_ALIGNMENT;
+    if (reinterpret_cast<uintptr_t>(norm_w) % 4) return GDR_ERR_ALIGNMENT;
+
+    gdr::ChunkArgs c;
+    c.q = q; c.k = k; c.v = v; c.g = g; c.beta = beta; c.S0 = S0; c.O = Y; c.S_T = S_T;
+    c.B = B; c.H = H; c.T = T; c.dk = dk; c.dv = dv; c.C = C;
+    c.scalar_gate = (gate_mode == GDR_GATE_SCALAR);
+    c.bf16 = true;
+    c.workspace = workspace;
+    c.gated_out = true;
+    c.ogate = gate;
+    c.norm_w = norm_w;
+    c.eps = eps;
+    int launches = 0;
+    cudaError_t e = gdr::launch_chunk_tc(c, st, &launches);
+    return finish(e, launches);
+}
+
 GDR_API size_t gdr2_chunk_fwd_workspace_size(int B, int H, int T, int dk, int dv, int C, int gate_mode, int dtype)
 {
     if (B <= 0 || H <= 0 || T <= 0) return 0;

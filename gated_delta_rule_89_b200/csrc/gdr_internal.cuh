@@ -28,6 +28,13 @@ struct ChunkArgs {
     // write gates, in the dtype of q, k, v.
     bool gdr2 = false;
     const void *erase = nullptr, *write = nullptr;
+    // Gated output (tensor-core path only): O receives
+    // y = Sigmoid(ogate) * RMSNorm(o) per head and token, RMSNorm over the d_v
+    // channels with weight norm_w [d_v] and epsilon eps; ogate is bf16 [B, H, T, d_v].
+    bool gated_out = false;
+    const void *ogate = nullptr;
+    const float *norm_w = nullptr;
+    float eps = 0.f;
 };
 
 // Arguments of one decode step, already validated.

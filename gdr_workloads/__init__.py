@@ -43,6 +43,7 @@ TID_Q, TID_K, TID_V, TID_G, TID_BETA, TID_S0, TID_CHAN = 1, 2, 3, 4, 5, 6, 7
 # raw inputs of the fused gate / normalisation prologue
 TID_QRAW, TID_KRAW, TID_AGATE, TID_ALOG, TID_DTBIAS, TID_BLOGIT = 8, 9, 10, 11, 12, 13
 TID_ERASE, TID_WRITE = 14, 15   # Gated Delta Rule-2 erase and write gates
+TID_OGATE, TID_NORMW = 16, 17   # output gate pre-activation, RMSNorm weight
 
 
 def _s64(c: int) -> int:
@@ -130,6 +131,7 @@ class Workload:
     seed: int
     description: str
     rule: str = "gdr"    # "gdr" (tied beta: KDA / Gated DeltaNet) or "gdr2" (erase and write gates)
+    out: str = "plain"   # "plain" (o_t) or "gated" (Sigmoid(gate) * RMSNorm(o_t))
 
     @property
     def tokens(self) -> int:
@@ -160,6 +162,11 @@ WORKLOADS: Dict[str, Workload] = {
         "softplus_n02_clamp5", "normal002", 5,
         "Gated Delta Rule-2 forward (per-channel decay, erase and write gates): B2 H32 T8192 d128 C64 bf16",
         rule="gdr2"),
+    "kda_d128_t8192_gated": Workload(
+        "kda_d128_t8192_gated", "chunk", 2, 32, 8192, 128, 128, 64, "per_channel", torch.bfloat16,
+        "softplus_n02_clamp5", "normal002", 2,
+        "KDA forward with the output epilogue fused in (per-head RMSNorm times a sigmoid output gate): "
+        "B2 H32 T8192 d128 C64 bf16", out="gated"),
     "gdr2_decode_b256": Workload(
         "gdr2_decode_b256", "decode", 256, 32, 1000, 128, 128, 1, "per_channel", torch.bfloat16,
         "softplus_n01_plus1_clamp5", "normal002", 6,
@@ -237,6 +244,9 @@ def generate(w: Workload, device="cpu", heads: Optional[Sequence[int]] = None,
     keys with a leading steps axis: q [S,B,H,dk] ... and S0 [B,H,dv,dk].
     Gated Delta Rule-2 workloads add the erase gate b (shape of k) and the
     write gate w (shape of v), sigmoid(N(0,1)) in the workload dtype.
+    Gated-output workloads add the output gate pre-activation ogate (shape of
+    v) ~ N(0,1) in the workload dtype and the RMSNorm weight norm_w [dv] ~
+    1 + 0.1 N(0,1) fp32 (shared by the heads).
     """
     B, H, dk, dv = w.B, w.H, w.dk, w.dv
     if heads is None:
@@ -326,6 +336,10 @@ def generate(w: Workload, device="cpu", heads: Optional[Sequence[int]] = None,
                    beta=shp(beta), S0=S0.view(outB, outH, dv, dk))
     for name, (x, width) in gates2.items():
         out[name] = shp(x, width)
+    if w.out == "gated":
+        out["ogate"] = shp(to_dtype(field(TID_OGATE, dv, lambda tid_, full, b, h, c, t: normal(seed, tid_, full),
+                                          torch.float64), w.dtype), dv)
+        out["norm_w"] = (1.0 + 0.1 * normal(seed, TID_NORMW, torch.arange(dv, device=device))).to(torch.float32)
     return out
 
 
@@ -387,7 +401,7 @@ def generate_prologue(w: Workload, device="cpu", heads: Optional[Sequence[int]] 
 
 def small_chunk_case(B: int, H: int, T: int, dk: int, dv: int, gate: str, dtype: torch.dtype,
                      g_recipe: str = "softplus_n01_plus1_clamp5", s0: str = "normal002",
-                     seed: int = 11, C: int = 64, rule: str = "gdr") -> Workload:
+                     seed: int = 11, C: int = 64, rule: str = "gdr", out: str = "plain") -> Workload:
     """An ad-hoc chunk workload with the same value recipes (parity tests)."""
-    return Workload(f"case_B{B}H{H}T{T}d{dk}x{dv}_{gate}_{rule}", "chunk", B, H, T, dk, dv, C, gate, dtype,
-                    g_recipe, s0, seed, "parity case", rule=rule)
+    return Workload(f"case_B{B}H{H}T{T}d{dk}x{dv}_{gate}_{rule}_{out}", "chunk", B, H, T, dk, dv, C, gate, dtype,
+                    g_recipe, s0, seed, "parity case", rule=rule, out=out)

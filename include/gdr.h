@@ -149,6 +149,31 @@ int gdr_chunk_fwd_prologue(const void *q_raw, const void *k_raw, const void *v, 
                            void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * Chunkwise forward with the layer's output epilogue fused in ("Token Mixer
+ * I", section "The Kimi Linear Model Architecture": before the output
+ * projection W_o, a per-head RMSNorm of the output and a data-dependent
+ * sigmoid gate):
+ *   Y[b,h,t,:] = Sigmoid(gate[b,h,t,:]) * RMSNorm(o_t),
+ *   RMSNorm(x) = x / sqrt(mean_c x_c^2 + eps) * norm_w        (c over the d_v channels)
+ * with o_t the output gdr_chunk_fwd would write.  The normalisation is taken
+ * in fp32 from the accumulator, before any rounding of o_t.
+ *
+ * Arguments as gdr_chunk_fwd, plus
+ *   gate     [B,H,T,d_v]   dtype       pre-activation of the output gate
+ *   norm_w   [d_v]         float       RMSNorm weight (shared by the heads)
+ *   eps      >= 0                      RMSNorm epsilon
+ * and Y [B,H,T,d_v] (dtype) in place of O.  Only the tensor-core
+ * configuration (bf16, d_k = d_v = 128, C = 64) runs; anything else returns
+ * GDR_ERR_UNSUPPORTED.  Same workspace as gdr_chunk_fwd.  norm_w must be
+ * 4-byte aligned, the other tensors 16-byte aligned.
+ */
+int gdr_chunk_fwd_gated(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                        const void *gate, const float *norm_w, float eps,
+                        const float *S0, void *Y, float *S_T,
+                        int B, int H, int T, int dk, int dv, int C, int gate_mode, int dtype,
+                        void *workspace, size_t ws_bytes, void *stream);
+
+/*
  * Gated Delta Rule-2: the erase and write decisions of the delta rule get
  * their own per-channel gates ("Token Mixer I", section "Gated DeltaNet-2:
  * Decoupling Erase and Write in Linear Attention", eq. (10)).  With

@@ -125,6 +125,27 @@ def test_gdr2_argument_validation(L):
     assert step(w=ODD) == ALIGN
 
 
+def gated(L, B=1, H=1, T=64, dk=128, dv=128, C=64, gate=0, dtype=1, ptr=GOOD, og=GOOD, nw=GOOD, eps=1e-6,
+          ws=1 << 40, wsp=GOOD):
+    return L.gdr_chunk_fwd_gated(ptr, ptr, ptr, ptr, ptr, og, nw, eps, None, ptr, None, B, H, T, dk, dv, C, gate,
+                                 dtype, wsp, ws, None)
+
+
+def test_gated_argument_validation(L):
+    assert gated(L, B=-1) == INVALID
+    assert gated(L, eps=-1.0) == INVALID
+    assert gated(L, eps=float("nan")) == INVALID
+    assert gated(L, dtype=0) == UNSUPPORTED
+    assert gated(L, C=32) == UNSUPPORTED
+    assert gated(L, og=None) == INVALID
+    assert gated(L, nw=None) == INVALID
+    assert gated(L, og=ODD) == ALIGN
+    assert gated(L, nw=P(0x100002)) == ALIGN
+    assert gated(L, wsp=None) == INVALID
+    assert gated(L, B=0) == OK and L.gdr_last_launch_count() == 0
+    assert gated(L, T=0) == OK
+
+
 def test_step_argument_validation(L):
     def step(B=2, H=2, dk=128, dv=128, gate=0, dtype=1, ptr=GOOD):
         return L.gdr_recurrent_step(ptr, ptr, ptr, ptr, ptr, ptr, ptr, B, H, dk, dv, gate, dtype, None)

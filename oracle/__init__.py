@@ -16,6 +16,8 @@ Contents
   * ``prologue`` / ``forward_prologue`` -- the input prologue (L2-normalised
     q, k; softplus gate with the -5 bound; sigmoid beta) and the forward fed
     by it, the reference of the fused-prologue entry point.
+  * ``backward``  -- reverse mode through the same token recurrence (the
+    gradients of <dO, O> + <dS_T, S_T>), the reference of the chunked backward.
   * ``output_gate`` / ``forward_gated`` -- the output epilogue of the layer
     (per-head RMSNorm of o_t, times a sigmoid output gate), the reference of
     the gated-output entry point.
@@ -62,6 +64,8 @@ def _load():
             I = ctypes.c_int
             lib.gdr_oracle_forward.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I]
             lib.gdr_oracle_forward.restype = I
+            lib.gdr_oracle_backward.argtypes = [P] * 14 + [I] * 8
+            lib.gdr_oracle_backward.restype = I
             lib.gdr2_oracle_forward.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I]
             lib.gdr2_oracle_forward.restype = I
             lib.gdr_oracle_online_cores.restype = I
@@ -119,6 +123,32 @@ def forward(q, k, v, g, beta, S0=None, gate: str = "per_channel", erase=None, wr
     if rc != 0:
         raise RuntimeError("oracle forward failed")
     return O, ST
+
+
+def backward(q, k, v, g, beta, S0, dO, dS_T=None, gate: str = "per_channel", clamp: bool = True,
+             threads: int = 0):
+    """fp64 gradients of L = <dO, O> + <dS_T, S_T> through the token recurrence
+    of ``forward`` (reverse mode, token by token, states recomputed from
+    checkpoints).  The per-channel -5 bound passes the gradient where
+    g >= -5.  Returns (dq, dk, dv, dg, dbeta, dS0) as fp64 numpy arrays
+    shaped like q, k, v, g, beta and the state.
+    """
+    qa, ka, va, ga, ba, oa = _f64(q), _f64(k), _f64(v), _f64(g), _f64(beta), _f64(dO)
+    B, H, T, dk = qa.shape
+    dv = va.shape[-1]
+    assert ka.shape == qa.shape and oa.shape == va.shape and ba.shape == (B, H, T)
+    assert ga.shape == ((B, H, T, dk) if gate == "per_channel" else (B, H, T))
+    s0, dst = _f64(S0), _f64(dS_T)
+    for x in (s0, dst):
+        assert x is None or x.shape == (B, H, dv, dk)
+    outs = [np.zeros_like(qa), np.zeros_like(ka), np.zeros_like(va), np.zeros_like(ga), np.zeros_like(ba),
+            np.zeros((B, H, dv, dk))]
+    rc = _load().gdr_oracle_backward(_ptr(qa), _ptr(ka), _ptr(va), _ptr(ga), _ptr(ba), _ptr(s0), _ptr(oa), _ptr(dst),
+                                     *[_ptr(o) for o in outs], B, H, T, dk, dv, 1 if gate == "scalar" else 0,
+                                     1 if clamp else 0, int(threads))
+    if rc != 0:
+        raise RuntimeError("oracle backward failed")
+    return tuple(outs)
 
 
 def forward_gdr2(q, k, v, g, b, w, S0=None, gate: str = "per_channel", clamp: bool = True,

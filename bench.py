@@ -82,6 +82,10 @@ def algorithmic_bytes(w: W.Workload) -> int:
         per_token += w.dv * e
     heads = w.B * w.H
     state = 2 * w.dv * w.dk * 4                                     # S0 read + S_T write
+    if w.direction == "bwd":
+        # reads q, k, v, g, beta, dO; writes dq, dk, dv, dg, dbeta; S0 and dS_T read, dS0 written
+        per_token = 2 * w.dk * e + w.dv * e + gate + 4 + w.dv * e + (2 * w.dk * e + w.dv * e + gate + 4)
+        state = 3 * w.dv * w.dk * 4
     if w.kind == "decode":
         return w.T * heads * (per_token + state)                    # the state moves every step
     return heads * w.T * per_token + heads * state
@@ -238,6 +242,9 @@ def api_call(gdr, w: W.Workload, x, **kw):
     if w.g_recipe == "prologue":
         return gdr.chunk_fwd_prologue(x["q_raw"], x["k_raw"], x["v"], x["a"], x["A_log"], x["dt_bias"],
                                       x["b_logit"], x["S0"], C=w.C, gate=w.gate, **kw)
+    if w.direction == "bwd":
+        return gdr.chunk_bwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["dO"], S0=x["S0"], dS_T=x["dS_T"],
+                             C=w.C, gate=w.gate, **kw)
     if w.out == "gated":
         return gdr.chunk_fwd_gated(x["q"], x["k"], x["v"], x["g"], x["beta"], x["ogate"], x["norm_w"], 1e-6,
                                    x["S0"], C=w.C, gate_mode=w.gate, **{("Y" if k == "O" else k): v for k, v in kw.items()})
@@ -284,6 +291,12 @@ def oracle_sample(w: W.Workload, budget_s: float, seed_rank: int = 0):
             return time.perf_counter() - t
         x = W.generate(w, heads=hl)
         sl = lambda a: a[:, :, :ntok].contiguous()
+        if w.direction == "bwd":
+            gr = W.generate_grads(w, heads=hl)
+            args = [sl(x[k]) for k in ("q", "k", "v", "g", "beta")]
+            t = time.perf_counter()
+            oracle.backward(*args, x["S0"], sl(gr["dO"]), gr["dS_T"], gate=w.gate, threads=cores)
+            return time.perf_counter() - t
         if w.rule == "gdr2":
             args = [sl(x[k]) for k in ("q", "k", "v", "g", "b", "w")]
             t = time.perf_counter()
@@ -430,6 +443,16 @@ def main():
 
         def step():
             api_call(gdr, w, x, O=O, S_T=S_T)
+    elif w.direction == "bwd":
+        x = W.generate(w, device=device)
+        x.update(W.generate_grads(w, device=device))
+        bws = torch.empty(gdr.chunk_bwd_workspace_size(w.B, w.H, w.T, w.dk, w.dv, w.C, w.gate, w.dtype),
+                          dtype=torch.uint8, device=device)
+        O = x["dO"]     # the result read back in the end-to-end measurement: dq
+        S_T = x["dS_T"]
+
+        def step():
+            api_call(gdr, w, x, workspace=bws)
     else:
         x = W.generate(w, device=device)
         if w.rule == "gdr2":
@@ -475,7 +498,10 @@ def main():
     if w.kind != "decode" and args.e2e_steps > 0:
         hx = {k: v.to("cpu").pin_memory() for k, v in x.items()}
         h2d = sum(v.numel() * v.element_size() for v in hx.values())
-        d2h = O.numel() * O.element_size() + S_T.numel() * S_T.element_size()
+        if w.direction == "bwd":   # every gradient comes back
+            d2h = sum(x[n].numel() * x[n].element_size() for n in ("q", "k", "v", "g", "beta", "S0"))
+        else:
+            d2h = O.numel() * O.element_size() + S_T.numel() * S_T.element_size()
         api_call(gdr, w, hx)  # warm
         torch.cuda.synchronize(device)
         if world > 1:
@@ -483,7 +509,7 @@ def main():
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(args.e2e_steps):
-            Oh, Sh = api_call(gdr, w, hx)
+            res = api_call(gdr, w, hx)
         e1.record(stream)
         torch.cuda.synchronize(device)
         e2e_ms = reduce_max(e0.elapsed_time(e1), world, device) / args.e2e_steps

@@ -20,7 +20,7 @@ from typing import Optional, Tuple
 import torch
 
 __all__ = ["chunk_fwd", "recurrent_step", "chunk_fwd_workspace_size", "chunk_fwd_prologue", "chunk_fwd_gdr2",
-           "chunk_fwd_gated",
+           "chunk_fwd_gated", "chunk_bwd",
            "recurrent_step_gdr2", "GDRError", "library_path",
            "last_launch_count", "device_status", "GATE_PER_CHANNEL", "GATE_SCALAR"]
 
@@ -59,6 +59,10 @@ def lib() -> ctypes.CDLL:
         L.gdr_recurrent_step.restype = I
         L.gdr_chunk_fwd_workspace_size.argtypes = [I, I, I, I, I, I, I, I]
         L.gdr_chunk_fwd_workspace_size.restype = Z
+        L.gdr_chunk_bwd.argtypes = [P] * 14 + [I] * 8 + [P, Z, P]
+        L.gdr_chunk_bwd.restype = I
+        L.gdr_chunk_bwd_workspace_size.argtypes = [I] * 8
+        L.gdr_chunk_bwd_workspace_size.restype = Z
         L.gdr_chunk_fwd_gated.argtypes = [P, P, P, P, P, P, P, ctypes.c_float, P, P, P, I, I, I, I, I, I, I, I,
                                           P, Z, P]
         L.gdr_chunk_fwd_gated.restype = I
@@ -436,3 +440,62 @@ def chunk_fwd_gated(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.
         Y = Y.to("cpu")
         S_T = None if S_T is None else S_T.to("cpu")
     return Y, S_T
+
+
+def chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor, beta: torch.Tensor,
+              dO: torch.Tensor, S0: Optional[torch.Tensor] = None, dS_T: Optional[torch.Tensor] = None,
+              C: int = 64, gate: Optional[str] = None, want_dS0: bool = True,
+              workspace: Optional[torch.Tensor] = None, stream=None):
+    """Backward of the chunkwise forward (``gdr_chunk_bwd``): the gradients of
+    <dO, O> + <dS_T, S_T> with respect to q, k, v, g, beta and S0.
+
+    Inputs as ``chunk_fwd`` plus dO [B,H,T,dv] (dtype of v) and dS_T fp32
+    [B,H,dv,dk] or None.  Returns (dq, dk, dv, dg, dbeta, dS0 or None).
+    Host tensors are copied to the current device and the gradients back.
+    """
+    host = not q.is_cuda
+    if host:
+        d = torch.device("cuda", torch.cuda.current_device())
+        q, k, v, g, beta, dO, S0, dS_T = (_to_device(x, d) for x in (q, k, v, g, beta, dO, S0, dS_T))
+    dev = q.device
+    if gate is None:
+        gate = "per_channel" if g.dim() == 4 else "scalar"
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    if dt not in _DTYPES:
+        raise TypeError("q, k, v must be float32 or bfloat16")
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (dO, "dO")):
+        _need(t, n, dt, dev)
+    _need(g, "g", torch.float32, dev)
+    _need(beta, "beta", torch.float32, dev)
+    if tuple(k.shape) != (B, H, T, dk) or tuple(v.shape[:3]) != (B, H, T) or tuple(beta.shape) != (B, H, T) \
+            or tuple(dO.shape) != tuple(v.shape):
+        raise ValueError("inconsistent shapes")
+    for t, n in ((S0, "S0"), (dS_T, "dS_T")):
+        if t is not None:
+            _need(t, n, torch.float32, dev)
+            if tuple(t.shape) != (B, H, dv, dk):
+                raise ValueError(f"{n} must be [B,H,dv,dk]")
+    dq, dk_, dv_ = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dg, dbeta = torch.empty_like(g), torch.empty_like(beta)
+    dS0 = torch.empty(B, H, dv, dk, dtype=torch.float32, device=dev) if want_dS0 else None
+    gm = GATE_PER_CHANNEL if gate == "per_channel" else GATE_SCALAR
+    L = lib()
+    ws_bytes = int(L.gdr_chunk_bwd_workspace_size(B, H, T, dk, dv, C, gm, _DTYPES[dt]))
+    if ws_bytes and (workspace is None or workspace.numel() * workspace.element_size() < ws_bytes):
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    st = L.gdr_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(dO), _ptr(dS_T),
+                         _ptr(dq), _ptr(dk_), _ptr(dv_), _ptr(dg), _ptr(dbeta), _ptr(dS0),
+                         B, H, T, dk, dv, C, gm, _DTYPES[dt],
+                         _ptr(workspace) if ws_bytes else None, ws_bytes, _stream_handle(dev, stream))
+    _check(st, "gdr_chunk_bwd")
+    out = (dq, dk_, dv_, dg, dbeta, dS0)
+    if host:
+        out = tuple(None if t is None else t.to("cpu") for t in out)
+    return out
+
+
+def chunk_bwd_workspace_size(B, H, T, dk, dv, C=64, gate="per_channel", dtype=torch.bfloat16) -> int:
+    g = GATE_PER_CHANNEL if gate == "per_channel" else GATE_SCALAR
+    return int(lib().gdr_chunk_bwd_workspace_size(B, H, T, dk, dv, C, g, _DTYPES[dtype]))

@@ -1,0 +1,717 @@
+// Backward pass of the chunkwise gated delta rule, fp32 on CUDA cores.
+//
+// The gradients of L = <dO, O> + <dS_T, S_T> with respect to q, k, v, the
+// log-decay g, beta and S0, for the chunk form the forward computes ("Token
+// Mixer I", section "Kimi Delta Attention: Improving Delta Rule with
+// Fine-grained Gating", the UT transform; "Reading notes: Kimi Delta
+// Attention" (mzeromiko), section 4), d_v x d_k orientation.  Per chunk, with
+// S the state entering it, G_r the inclusive cumulative (bounded) log-decay,
+// gamma_r = exp(G_r), E_ric = exp(G_rc - G_ic) (i <= r):
+//
+//   A_ri = beta_r sum_c k_rc k_ic E_ric (i < r),  M = (I + A)^{-1},  T' = M Diag(beta)
+//   W = T' (K * gamma),  U = T' V,  V_new = U - W S^T
+//   Aqk_ri = sum_c q_rc k_ic E_ric (i <= r)
+//   O = (Q * gamma) S^T + Aqk V_new
+//   S' = S Diag(gamma_C) + V_new^T (K * gamma_C / gamma)
+//
+// Reverse mode, given dO and dS' (the gradient of the state leaving the chunk):
+//   dV_new = Aqk^T dO + K_tail dS'^T
+//   dS     = dO^T Q<- + dS' Diag(gamma_C) - dV_new^T W          (into the previous chunk)
+//   dAqk = (dO V_new^T) masked,   dQ<- = dO S,   dK_tail = V_new dS',
+//   dW = -dV_new S,   dV = T'^T dV_new,   dT' = dV_new V^T + dW K<-^T,
+//   dK<- = T'^T dW,   dbeta_j += sum_i dT'_ij M_ij,   dA = -M^T (dT' Diag(beta)) M^T,
+// then the decay-weighted contractions of dA and dAqk give dq, dk, dbeta and
+// the gradient of G, and dg is its reverse cumulative sum inside the chunk
+// (plus the gamma_C terms at the chunk's last row), masked where the -5 bound
+// is active.
+//
+// Kernels (one call):
+//   1. bwd_prep     every chunk in parallel: G, M, Aqk, W, U -> workspace
+//   2. bwd_fwd_scan (head, 32-row d_v tile), chunks in order: the state at
+//                   every chunk start and V_new -> workspace
+//   3. bwd_rev_scan (head, d_v tile), chunks in reverse: dS at every chunk
+//                   end and dV_new -> workspace; dS0
+//   4. bwd_grads    every chunk in parallel: dq, dk, dv, dg, dbeta
+// Decay ratios are only ever formed as exp of a difference that is <= 0.
+// Rows past the end of a partial last chunk act as identity tokens.
+#include "gdr_internal.cuh"
+
+namespace gdr {
+namespace {
+
+constexpr int kC = 64;
+constexpr int kBT = 256;   // threads per block
+constexpr int kTile = 32;  // d_v rows per scan block
+
+struct BwdWs {
+    float *G, *W, *U, *Vn, *dVn;   // [BH][Tp][D], Tp = chunks * 64 (padded rows)
+    float *M, *Aq;                  // [BH * chunks][64][64]
+    float *Sck, *dSck;              // [BH * chunks][D][D]
+};
+
+inline BwdWs carve(void *ws, int B, int H, int T, int D)
+{
+    const size_t bh = (size_t)B * H, nch = (size_t)(T + kC - 1) / kC, tp = nch * kC;
+    float *p = static_cast<float *>(ws);
+    BwdWs w;
+    w.G = p; p += bh * tp * D;
+    w.W = p; p += bh * tp * D;
+    w.U = p; p += bh * tp * D;
+    w.Vn = p; p += bh * tp * D;
+    w.dVn = p; p += bh * tp * D;
+    w.M = p; p += bh * nch * kC * kC;
+    w.Aq = p; p += bh * nch * kC * kC;
+    w.Sck = p; p += bh * nch * (size_t)D * D;
+    w.dSck = p;
+    return w;
+}
+
+// ------------------------------------------------------------------ 1. prep
+template <int D>
+struct PrepSmem {
+    static constexpr int LD = D + 1;
+    static constexpr int K = 0, Q = K + kC * LD, G = Q + kC * LD, A = G + kC * LD, M = A + kC * 65, B = M + kC * 65;
+    static constexpr int TOTAL = B + kC;
+};
+
+template <int D, typename T, bool SCALAR>
+__global__ void __launch_bounds__(kBT)
+bwd_prep(const T *__restrict__ qg, const T *__restrict__ kg, const T *__restrict__ vg, const float *__restrict__ gg,
+         const float *__restrict__ betag, BwdWs w, int T_len, int nch)
+{
+    using L = PrepSmem<D>;
+    constexpr int LD = L::LD, RS = kBT / D, NR = kC / RS;
+    extern __shared__ float sm[];
+    float *sk = sm + L::K, *sq = sm + L::Q, *sG = sm + L::G, *sA = sm + L::A, *sM = sm + L::M, *sb = sm + L::B;
+    const int tid = threadIdx.x;
+    const int ci = blockIdx.x, head = ci / nch, n = ci - head * nch;
+    const int t0 = n * kC, nrows = min(kC, T_len - t0);
+    const size_t row0 = (size_t)head * T_len + t0, prow0 = (size_t)head * nch * kC + t0;
+
+    for (int idx = tid; idx < kC * D; idx += kBT) {
+        const int r = idx / D, c = idx - r * D;
+        const bool ok = r < nrows;
+        sk[r * LD + c] = ok ? to_f32<T>(kg[(row0 + r) * D + c]) : 0.f;
+        sq[r * LD + c] = ok ? to_f32<T>(qg[(row0 + r) * D + c]) : 0.f;
+        float g = 0.f;
+        if (ok) g = SCALAR ? gg[row0 + r] : fmaxf(gg[(row0 + r) * D + c], kGateMin);
+        sG[r * LD + c] = g;
+    }
+    if (tid < kC) sb[tid] = tid < nrows ? betag[row0 + tid] : 0.f;
+    __syncthreads();
+    if (tid < D) {   // inclusive cumulative sum per channel
+        float acc = 0.f;
+        for (int r = 0; r < kC; ++r) {
+            acc += sG[r * LD + tid];
+            sG[r * LD + tid] = acc;
+            w.G[(prow0 + r) * D + tid] = acc;
+        }
+    }
+    __syncthreads();
+    // A (strictly lower, beta_r in) and Aqk (lower incl. the diagonal)
+    float *Aqo = w.Aq + (size_t)ci * kC * kC;
+    for (int idx = tid; idx < kC * kC; idx += kBT) {
+        const int r = idx >> 6, i = idx & 63;
+        float sa = 0.f, sq_ = 0.f;
+        if (i <= r) {
+            for (int c = 0; c < D; ++c) {
+                const float e = __expf(sG[r * LD + c] - sG[i * LD + c]);
+                const float ki = sk[i * LD + c] * e;
+                sa = fmaf(sk[r * LD + c], ki, sa);
+                sq_ = fmaf(sq[r * LD + c], ki, sq_);
+            }
+        }
+        sA[r * 65 + i] = i < r ? sb[r] * sa : 0.f;
+        Aqo[r * kC + i] = sq_;
+    }
+    __syncthreads();
+    // M = (I + A)^{-1}: column j by forward substitution
+    if (tid < kC) {
+        const int j = tid;
+        for (int r = 0; r < kC; ++r) {
+            float x = 0.f;
+            if (r == j) {
+                x = 1.f;
+            } else if (r > j) {
+                float s = 0.f;
+                for (int m = j; m < r; ++m) s = fmaf(sA[r * 65 + m], sM[m * 65 + j], s);
+                x = -s;
+            }
+            sM[r * 65 + j] = x;
+        }
+    }
+    __syncthreads();
+    float *Mo = w.M + (size_t)ci * kC * kC;
+    for (int idx = tid; idx < kC * kC; idx += kBT) Mo[idx] = sM[(idx >> 6) * 65 + (idx & 63)];
+    // W = M Diag(beta) (K * gamma): the operand beta_i k_ic gamma_ic into sq
+    for (int idx = tid; idx < kC * D; idx += kBT) {
+        const int r = idx / D, c = idx - r * D;
+        sq[r * LD + c] = sb[r] * sk[r * LD + c] * __expf(sG[r * LD + c]);
+    }
+    __syncthreads();
+    const int c = tid % D, h = tid / D;
+    {
+        float acc[NR];
+#pragma unroll
+        for (int m = 0; m < NR; ++m) acc[m] = 0.f;
+        for (int i = 0; i < kC; ++i) {
+            const float b = sq[i * LD + c];
+#pragma unroll
+            for (int m = 0; m < NR; ++m) acc[m] = fmaf(sM[(h + RS * m) * 65 + i], b, acc[m]);
+        }
+#pragma unroll
+        for (int m = 0; m < NR; ++m) w.W[(prow0 + h + RS * m) * D + c] = acc[m];
+    }
+    __syncthreads();
+    // U = M Diag(beta) V (d_v = D)
+    for (int idx = tid; idx < kC * D; idx += kBT) {
+        const int r = idx / D, j = idx - r * D;
+        sq[r * LD + j] = r < nrows ? sb[r] * to_f32<T>(vg[(row0 + r) * D + j]) : 0.f;
+    }
+    __syncthreads();
+    {
+        float acc[NR];
+#pragma unroll
+        for (int m = 0; m < NR; ++m) acc[m] = 0.f;
+        for (int i = 0; i < kC; ++i) {
+            const float b = sq[i * LD + c];
+#pragma unroll
+            for (int m = 0; m < NR; ++m) acc[m] = fmaf(sM[(h + RS * m) * 65 + i], b, acc[m]);
+        }
+#pragma unroll
+        for (int m = 0; m < NR; ++m) w.U[(prow0 + h + RS * m) * D + c] = acc[m];
+    }
+}
+
+// ------------------------------------------------------------------ 2. forward state scan
+template <int D>
+struct FwdSmem {
+    static constexpr int LD = D + 1;
+    static constexpr int S = 0, W = S + kTile * LD, KT = W + kC * LD, VN = KT + kC * LD, GC = VN + kC * (kTile + 1);
+    static constexpr int TOTAL = GC + D;
+};
+
+// K_tail rows of chunk n into kt (k * exp(G_C - G), zero past T), G_C into gc
+template <int D, typename T>
+__device__ __forceinline__ void load_ktail(float *kt, float *gc, const T *kg, const float *G, size_t row0,
+                                           size_t prow0, int nrows, int tid)
+{
+    constexpr int LD = D + 1;
+    for (int c = tid; c < D; c += kBT) gc[c] = G[(prow0 + kC - 1) * D + c];
+    __syncthreads();
+    for (int idx = tid; idx < kC * D; idx += kBT) {
+        const int r = idx / D, c = idx - r * D;
+        kt[r * LD + c] = r < nrows ? to_f32<T>(kg[(row0 + r) * D + c]) * __expf(gc[c] - G[(prow0 + r) * D + c]) : 0.f;
+    }
+}
+
+template <int D, typename T>
+__global__ void __launch_bounds__(kBT)
+bwd_fwd_scan(const T *__restrict__ kg, const float *__restrict__ S0, BwdWs w, int T_len, int nch)
+{
+    using L = FwdSmem<D>;
+    constexpr int LD = L::LD, RS = kBT / D, NJ = kTile / RS;
+    extern __shared__ float sm[];
+    float *sS = sm + L::S, *sW = sm + L::W, *sKt = sm + L::KT, *sVn = sm + L::VN, *gc = sm + L::GC;
+    const int tid = threadIdx.x;
+    const int head = blockIdx.x, i0 = blockIdx.y * kTile;
+    for (int idx = tid; idx < kTile * D; idx += kBT) {
+        const int j = idx / D, c = idx - j * D;
+        sS[j * LD + c] = S0 ? S0[((size_t)head * D + i0 + j) * D + c] : 0.f;
+    }
+    const int c = tid % D, h = tid / D;
+    const int vj = tid & 31, vr = tid >> 5;   // V_new: column (state row) vj, rows vr + 8 m
+    for (int n = 0; n < nch; ++n) {
+        const int t0 = n * kC, nrows = min(kC, T_len - t0);
+        const size_t row0 = (size_t)head * T_len + t0, prow0 = (size_t)head * nch * kC + t0;
+        __syncthreads();
+        float *ck = w.Sck + ((size_t)(head * nch + n) * D + i0) * D;
+        for (int idx = tid; idx < kTile * D; idx += kBT) ck[idx] = sS[(idx / D) * LD + idx % D];
+        for (int idx = tid; idx < kC * D; idx += kBT) sW[(idx / D) * LD + idx % D] = w.W[(prow0 + idx / D) * D + idx % D];
+        load_ktail<D, T>(sKt, gc, kg, w.G, row0, prow0, nrows, tid);
+        __syncthreads();
+        // V_new = U - W S^T (this tile's d_v columns)
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+            const int r = vr + 8 * m;
+            float acc = w.U[(prow0 + r) * D + i0 + vj];
+            for (int cc = 0; cc < D; ++cc) acc = fmaf(-sW[r * LD + cc], sS[vj * LD + cc], acc);
+            sVn[r * (kTile + 1) + vj] = acc;
+            w.Vn[(prow0 + r) * D + i0 + vj] = acc;
+        }
+        __syncthreads();
+        // S <- S Diag(gamma_C) + V_new^T K_tail
+        float acc[NJ];
+        const float gcc = __expf(gc[c]);
+#pragma unroll
+        for (int m = 0; m < NJ; ++m) acc[m] = sS[(h + RS * m) * LD + c] * gcc;
+        for (int r = 0; r < kC; ++r) {
+            const float kt = sKt[r * LD + c];
+#pragma unroll
+            for (int m = 0; m < NJ; ++m) acc[m] = fmaf(sVn[r * (kTile + 1) + h + RS * m], kt, acc[m]);
+        }
+        __syncthreads();
+#pragma unroll
+        for (int m = 0; m < NJ; ++m) sS[(h + RS * m) * LD + c] = acc[m];
+    }
+}
+
+// ------------------------------------------------------------------ 3. reverse state scan
+template <int D>
+struct RevSmem {
+    static constexpr int LD = D + 1;
+    static constexpr int DS = 0, AQ = DS + kTile * LD, DO = AQ + kC * 65, DVN = DO + kC * (kTile + 1),
+                         KT = DVN + kC * (kTile + 1), GC = KT + kC * LD;
+    static constexpr int TOTAL = GC + D;
+};
+
+template <int D, typename T>
+__global__ void __launch_bounds__(kBT)
+bwd_rev_scan(const T *__restrict__ qg, const T *__restrict__ kg, const T *__restrict__ dOg,
+             const float *__restrict__ dST, float *__restrict__ dS0, BwdWs w, int T_len, int nch)
+{
+    using L = RevSmem<D>;
+    constexpr int LD = L::LD, RS = kBT / D, NJ = kTile / RS, TL = kTile + 1;
+    extern __shared__ float sm[];
+    float *sdS = sm + L::DS, *sAq = sm + L::AQ, *sdO = sm + L::DO, *sdVn = sm + L::DVN, *sKt = sm + L::KT,
+          *gc = sm + L::GC;
+    const int tid = threadIdx.x;
+    const int head = blockIdx.x, i0 = blockIdx.y * kTile;
+    for (int idx = tid; idx < kTile * D; idx += kBT) {
+        const int j = idx / D, c = idx - j * D;
+        sdS[j * LD + c] = dST ? dST[((size_t)head * D + i0 + j) * D + c] : 0.f;
+    }
+    const int c = tid % D, h = tid / D;
+    const int vj = tid & 31, vr = tid >> 5;
+    for (int n = nch - 1; n >= 0; --n) {
+        const int t0 = n * kC, nrows = min(kC, T_len - t0);
+        const size_t row0 = (size_t)head * T_len + t0, prow0 = (size_t)head * nch * kC + t0;
+        __syncthreads();
+        float *ck = w.dSck + ((size_t)(head * nch + n) * D + i0) * D;
+        for (int idx = tid; idx < kTile * D; idx += kBT) ck[idx] = sdS[(idx / D) * LD + idx % D];
+        const float *aq = w.Aq + (size_t)(head * nch + n) * kC * kC;
+        for (int idx = tid; idx < kC * kC; idx += kBT) sAq[(idx >> 6) * 65 + (idx & 63)] = aq[idx];
+        for (int idx = tid; idx < kC * kTile; idx += kBT) {
+            const int r = idx / kTile, j = idx - r * kTile;
+            sdO[r * TL + j] = r < nrows ? to_f32<T>(dOg[(row0 + r) * D + i0 + j]) : 0.f;
+        }
+        load_ktail<D, T>(sKt, gc, kg, w.G, row0, prow0, nrows, tid);
+        __syncthreads();
+        // dV_new = Aqk^T dO + K_tail dS^T
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+            const int r = vr + 8 * m;
+            float acc = 0.f;
+            for (int i = r; i < kC; ++i) acc = fmaf(sAq[i * 65 + r], sdO[i * TL + vj], acc);
+            for (int cc = 0; cc < D; ++cc) acc = fmaf(sKt[r * LD + cc], sdS[vj * LD + cc], acc);
+            sdVn[r * TL + vj] = acc;
+            w.dVn[(prow0 + r) * D + i0 + vj] = acc;
+        }
+        __syncthreads();
+        // dS <- dS Diag(gamma_C) + dO^T Q<- - dV_new^T W  (Q<-, then W, staged in the K_tail buffer)
+        float acc[NJ];
+        const float gcc = __expf(gc[c]);
+#pragma unroll
+        for (int m = 0; m < NJ; ++m) acc[m] = sdS[(h + RS * m) * LD + c] * gcc;
+        for (int idx = tid; idx < kC * D; idx += kBT) {
+            const int r = idx / D, cc = idx - r * D;
+            sKt[r * LD + cc] =
+                r < nrows ? to_f32<T>(qg[(row0 + r) * D + cc]) * __expf(w.G[(prow0 + r) * D + cc]) : 0.f;
+        }
+        __syncthreads();
+        for (int r = 0; r < kC; ++r) {
+            const float ql = sKt[r * LD + c];
+#pragma unroll
+            for (int m = 0; m < NJ; ++m) acc[m] = fmaf(sdO[r * TL + h + RS * m], ql, acc[m]);
+        }
+        __syncthreads();
+        for (int idx = tid; idx < kC * D; idx += kBT) sKt[(idx / D) * LD + idx % D] = w.W[(prow0 + idx / D) * D + idx % D];
+        __syncthreads();
+        for (int r = 0; r < kC; ++r) {
+            const float wv = sKt[r * LD + c];
+#pragma unroll
+            for (int m = 0; m < NJ; ++m) acc[m] = fmaf(-sdVn[r * TL + h + RS * m], wv, acc[m]);
+        }
+        __syncthreads();
+#pragma unroll
+        for (int m = 0; m < NJ; ++m) sdS[(h + RS * m) * LD + c] = acc[m];
+    }
+    __syncthreads();
+    if (dS0)
+        for (int idx = tid; idx < kTile * D; idx += kBT)
+            dS0[((size_t)head * D + i0 + idx / D) * D + idx % D] = sdS[(idx / D) * LD + idx % D];
+}
+
+// ------------------------------------------------------------------ 4. per-chunk gradients
+template <int D>
+struct GradSmem {
+    static constexpr int LD = D + 1;
+    static constexpr int Q = 0, K = Q + kC * LD, G = K + kC * LD, X = G + kC * LD, Y = X + kC * LD, M = Y + kC * LD,
+                         P = M + kC * 65, R = P + kC * 65, B = R + kC * 65, DB = B + kC, GCP = DB + kC,
+                         RED = GCP + (kBT / D) * D;
+    static constexpr int TOTAL = RED + (kBT / 32) * (kC / (kBT / D));
+};
+
+template <int D, typename T, bool SCALAR>
+__global__ void __launch_bounds__(kBT, 1)
+bwd_grads(const T *__restrict__ qg, const T *__restrict__ kg, const T *__restrict__ vg, const float *__restrict__ gg,
+          const float *__restrict__ betag, const T *__restrict__ dOg, T *__restrict__ dqg, T *__restrict__ dkg,
+          T *__restrict__ dvg, float *__restrict__ dgg, float *__restrict__ dbg, BwdWs w, int T_len, int nch)
+{
+    using L = GradSmem<D>;
+    constexpr int LD = L::LD, RS = kBT / D, NR = kC / RS;
+    extern __shared__ float sm[];
+    float *sq = sm + L::Q, *sk = sm + L::K, *sG = sm + L::G, *sX = sm + L::X, *sY = sm + L::Y;
+    float *sM = sm + L::M, *sP = sm + L::P, *sR = sm + L::R, *sb = sm + L::B, *sdb = sm + L::DB;
+    float *sgcp = sm + L::GCP, *sred = sm + L::RED;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int ci = blockIdx.x, head = ci / nch, n = ci - head * nch;
+    const int t0 = n * kC, nrows = min(kC, T_len - t0);
+    const size_t row0 = (size_t)head * T_len + t0, prow0 = (size_t)head * nch * kC + t0;
+    const float *Sn = w.Sck + (size_t)ci * D * D;    // state entering the chunk
+    const float *dSn = w.dSck + (size_t)ci * D * D;  // gradient of the state leaving it
+    const int c = tid % D, h = tid / D;              // this thread: channel c, rows h + RS m
+    const int pi = tid & 63, pr = tid >> 6;          // 64 x 64 outputs: column pi, rows pr + 4 m
+
+    for (int idx = tid; idx < kC * D; idx += kBT) {
+        const int r = idx / D, cc = idx - r * D;
+        const bool ok = r < nrows;
+        sq[r * LD + cc] = ok ? to_f32<T>(qg[(row0 + r) * D + cc]) : 0.f;
+        sk[r * LD + cc] = ok ? to_f32<T>(kg[(row0 + r) * D + cc]) : 0.f;
+        sG[r * LD + cc] = w.G[(prow0 + r) * D + cc];
+        sX[r * LD + cc] = ok ? to_f32<T>(dOg[(row0 + r) * D + cc]) : 0.f;   // dO
+        sY[r * LD + cc] = w.Vn[(prow0 + r) * D + cc];                         // V_new
+    }
+    const float *Mg = w.M + (size_t)ci * kC * kC;
+    for (int idx = tid; idx < kC * kC; idx += kBT) sM[(idx >> 6) * 65 + (idx & 63)] = Mg[idx];
+    if (tid < kC) {
+        sb[tid] = tid < nrows ? betag[row0 + tid] : 0.f;
+        sdb[tid] = 0.f;
+    }
+    __syncthreads();
+
+    float dq[NR], dk[NR], dG[NR];
+#pragma unroll
+    for (int m = 0; m < NR; ++m) dq[m] = dk[m] = dG[m] = 0.f;
+    const float gcl = sG[(kC - 1) * LD + c];   // G at the chunk end
+    float dgc = 0.f;                           // this thread's share of d G_C (channel c)
+
+    // dQ<- = dO S  ->  dq += dQ<- gamma,  dG += dQ<- q gamma
+    {
+        float acc[NR];
+#pragma unroll
+        for (int m = 0; m < NR; ++m) acc[m] = 0.f;
+#pragma unroll 8
+        for (int i = 0; i < D; ++i) {
+            const float s = Sn[(size_t)i * D + c];
+#pragma unroll
+            for (int m = 0; m < NR; ++m) acc[m] = fmaf(sX[(h + RS * m) * LD + i], s, acc[m]);
+        }
+#pragma unroll
+        for (int m = 0; m < NR; ++m) {
+            const int r = h + RS * m;
+            const float ga = __expf(sG[r * LD + c]);
+            dq[m] = fmaf(acc[m], ga, dq[m]);
+            dG[m] = fmaf(acc[m] * sq[r * LD + c], ga, dG[m]);
+        }
+    }
+    // dAqk = (dO V_new^T) on the lower triangle incl. the diagonal  -> sR
+#pragma unroll
+    for (int m = 0; m < kC / 4; ++m) {
+        const int r = pr + 4 * m;
+        float acc = 0.f;
+        if (pi <= r)
+            for (int j = 0; j < D; ++j) acc = fmaf(sX[r * LD + j], sY[pi * LD + j], acc);
+        sR[r * 65 + pi] = acc;
+    }
+    // dK_tail = V_new dS'  ->  dk += dK_tail gamma_C / gamma,  dG -= (same) k, dG_C += (same) k
+    {
+        float acc[NR];
+#pragma unroll
+        for (int m = 0; m < NR; ++m) acc[m] = 0.f;
+#pragma unroll 8
+        for (int j = 0; j < D; ++j) {
+            const float s = dSn[(size_t)j * D + c];
+#pragma unroll
+            for (int m = 0; m < NR; ++m) acc[m] = fmaf(sY[(h + RS * m) * LD + j], s, acc[m]);
+        }
+#pragma unroll
+        for (int m = 0; m < NR; ++m) {
+            const int r = h + RS * m;
+            const float e = __expf(gcl - sG[r * LD + c]);
+            const float t = acc[m] * e;
+            dk[m] = fmaf(t, 1.f, dk[m]);
+            const float tk = t * sk[r * LD + c];
+            dG[m] -= tk;
+            dgc += tk;
+        }
+    }
+    // d gamma_C = sum_j dS'_jc S_jc  ->  dG_C += d gamma_C gamma_C
+    {
+        float s = 0.f;
+#pragma unroll 8
+        for (int j = h; j < D; j += RS) s = fmaf(dSn[(size_t)j * D + c], Sn[(size_t)j * D + c], s);
+        dgc = fmaf(s, __expf(gcl), dgc);
+    }
+    sgcp[h * D + c] = dgc;
+    __syncthreads();   // dO, V_new done
+    // dV_new -> sX;  dV = T'^T dV_new = Diag(beta) M^T dV_new  -> output
+    for (int idx = tid; idx < kC * D; idx += kBT) sX[(idx / D) * LD + idx % D] = w.dVn[(prow0 + idx / D) * D + idx % D];
+    for (int idx = tid; idx < kC * D; idx += kBT) {
+        const int r = idx / D, j = idx - r * D;
+        sY[r * LD + j] = r < nrows ? to_f32<T>(vg[(row0 + r) * D + j]) : 0.f;   // V
+    }
+    __syncthreads();
+    {
+        float acc[NR];
+#pragma unroll
+        for (int m = 0; m < NR; ++m) acc[m] = 0.f;
+        for (int i = 0; i < kC; ++i) {
+            const float x = sX[i * LD + c];
+#pragma unroll
+            for (int m = 0; m < NR; ++m) acc[m] = fmaf(sM[i * 65 + h + RS * m], x, acc[m]);
+        }
+#pragma unroll
+        for (int m = 0; m < NR; ++m) {
+            const int r = h + RS * m;
+            if (r < nrows) dvg[(row0 + r) * D + c] = from_f32<T>(sb[r] * acc[m]);
+        }
+    }
+    // dT' = dV_new V^T  -> sP
+#pragma unroll
+    for (int m = 0; m < kC / 4; ++m) {
+        const int r = pr + 4 * m;
+        float acc = 0.f;
+        for (int j = 0; j < D; ++j) acc = fmaf(sX[r * LD + j], sY[pi * LD + j], acc);
+        sP[r * 65 + pi] = acc;
+    }
+    __syncthreads();   // V read
+    // dW = -dV_new S  -> sY
+    {
+        float acc[NR];
+#pragma unroll
+        for (int m = 0; m < NR; ++m) acc[m] = 0.f;
+#pragma unroll 8
+        for (int j = 0; j < D; ++j) {
+            const float s = Sn[(size_t)j * D + c];
+#pragma unroll
+            for (int m = 0; m < NR; ++m) acc[m] = fmaf(sX[(h + RS * m) * LD + j], s, acc[m]);
+        }
+#pragma unroll
+        for (int m = 0; m < NR; ++m) sY[(h + RS * m) * LD + c] = -acc[m];
+    }
+    __syncthreads();
+    // dT' += dW K<-^T
+#pragma unroll
+    for (int m = 0; m < kC / 4; ++m) {
+        const int r = pr + 4 * m;
+        float acc = 0.f;
+        for (int cc = 0; cc < D; ++cc)
+            acc = fmaf(sY[r * LD + cc], sk[pi * LD + cc] * __expf(sG[pi * LD + cc]), acc);
+        sP[r * 65 + pi] += acc;
+    }
+    // dK<- = T'^T dW = Diag(beta) M^T dW  ->  dk += dK<- gamma,  dG += dK<- k gamma
+    {
+        float acc[NR];
+#pragma unroll
+        for (int m = 0; m < NR; ++m) acc[m] = 0.f;
+        for (int i = 0; i < kC; ++i) {
+            const float x = sY[i * LD + c];
+#pragma unroll
+            for (int m = 0; m < NR; ++m) acc[m] = fmaf(sM[i * 65 + h + RS * m], x, acc[m]);
+        }
+#pragma unroll
+        for (int m = 0; m < NR; ++m) {
+            const int r = h + RS * m;
+            const float t = sb[r] * acc[m] * __expf(sG[r * LD + c]);
+            dk[m] += t;
+            dG[m] = fmaf(t, sk[r * LD + c], dG[m]);
+        }
+    }
+    __syncthreads();   // dT' complete
+    // dbeta_j += sum_i dT'_ij M_ij;  dM = dT' Diag(beta) (in place)
+    if (tid < kC) {
+        float s = 0.f;
+        for (int i = 0; i < kC; ++i) s = fmaf(sP[i * 65 + tid], sM[i * 65 + tid], s);
+        sdb[tid] = s;
+    }
+    __syncthreads();
+    for (int idx = tid; idx < kC * kC; idx += kBT) sP[(idx >> 6) * 65 + (idx & 63)] *= sb[idx & 63];
+    __syncthreads();
+    // dA = -M^T dM M^T on the strict lower triangle: first Z = dM M^T -> sY (as 64 x 65)
+    float *sZ = sY;
+#pragma unroll
+    for (int m = 0; m < kC / 4; ++m) {
+        const int r = pr + 4 * m;
+        float acc = 0.f;
+        for (int kk = 0; kk < kC; ++kk) acc = fmaf(sP[r * 65 + kk], sM[pi * 65 + kk], acc);
+        sZ[r * 65 + pi] = acc;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int m = 0; m < kC / 4; ++m) {
+        const int r = pr + 4 * m;
+        float acc = 0.f;
+        if (pi < r)
+            for (int kk = 0; kk < kC; ++kk) acc = fmaf(sM[kk * 65 + r], sZ[kk * 65 + pi], acc);
+        sP[r * 65 + pi] = -acc;   // dA (zero on and above the diagonal)
+    }
+    __syncthreads();
+    // decay-weighted contractions of dA (A_ri = beta_r sum_c k_rc k_ic E) and dAqk
+    // row side: (r, c) collects over i <= r
+    float xb[NR];
+#pragma unroll
+    for (int m = 0; m < NR; ++m) {
+        const int r = h + RS * m;
+        const float gr = sG[r * LD + c], kr = sk[r * LD + c], qr = sq[r * LD + c], br = sb[r];
+        float sdk = 0.f, sdq = 0.f, sx = 0.f, sxq = 0.f;
+        for (int i = 0; i <= r; ++i) {
+            const float kie = sk[i * LD + c] * __expf(gr - sG[i * LD + c]);
+            const float a = sP[r * 65 + i], b = sR[r * 65 + i];
+            sdk = fmaf(a, kie, sdk);
+            sdq = fmaf(b, kie, sdq);
+        }
+        sx = sdk * kr;    // sum_i dA_ri k_rc k_ic E
+        sxq = sdq * qr;   // sum_i dAqk_ri q_rc k_ic E
+        dk[m] = fmaf(br, sdk, dk[m]);
+        dq[m] += sdq;
+        dG[m] += br * sx + sxq;
+        xb[m] = sx;
+    }
+    // column side: (i, c) collects over r >= i
+#pragma unroll
+    for (int m = 0; m < NR; ++m) {
+        const int i = h + RS * m;
+        const float gi = sG[i * LD + c], ki = sk[i * LD + c];
+        float sa = 0.f;
+        for (int r = i; r < kC; ++r) {
+            const float e = __expf(sG[r * LD + c] - gi);
+            sa = fmaf(sb[r] * sP[r * 65 + i] * sk[r * LD + c] + sR[r * 65 + i] * sq[r * LD + c], e, sa);
+        }
+        dk[m] += sa;
+        dG[m] = fmaf(-sa, ki, dG[m]);
+    }
+    // dbeta_r += sum_c xb  (lanes, then the warps that share the rows)
+#pragma unroll
+    for (int m = 0; m < NR; ++m) {
+        float v = xb[m];
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0) sred[warp * NR + m] = v;
+    }
+    __syncthreads();
+    if (tid < kC) {
+        const int r = tid, hh = r % RS, m = r / RS;
+        float s = 0.f;
+        for (int wq = 0; wq < D / 32; ++wq) s += sred[(hh * (D / 32) + wq) * NR + m];
+        if (r < nrows) dbg[row0 + r] = sdb[r] + s;
+    }
+    // G_C: the chunk's last row collects every share of d G_C
+    if (h == (kC - 1) % RS) {
+        float s = 0.f;
+        for (int hh = 0; hh < RS; ++hh) s += sgcp[hh * D + c];
+        dG[(kC - 1) / RS] += s;
+    }
+    // dq, dk out; dG -> sX for the reverse cumulative sum
+    __syncthreads();
+#pragma unroll
+    for (int m = 0; m < NR; ++m) {
+        const int r = h + RS * m;
+        if (r < nrows) {
+            dqg[(row0 + r) * D + c] = from_f32<T>(dq[m]);
+            dkg[(row0 + r) * D + c] = from_f32<T>(dk[m]);
+        }
+        sX[r * LD + c] = dG[m];
+    }
+    __syncthreads();
+    // dg_t = sum_{r >= t} dG_r, where the -5 bound passes (per channel); a scalar
+    // gate sums the channels
+    if (tid < D) {
+        float acc = 0.f;
+        for (int r = kC - 1; r >= 0; --r) {
+            acc += sX[r * LD + tid];
+            if (SCALAR) {
+                sX[r * LD + tid] = acc;
+            } else if (r < nrows) {
+                const float graw = gg[(row0 + r) * D + tid];
+                dgg[(row0 + r) * D + tid] = graw >= kGateMin ? acc : 0.f;
+            }
+        }
+    }
+    if (SCALAR) {
+        __syncthreads();
+        if (tid < nrows) {
+            float s = 0.f;
+            for (int cc = 0; cc < D; ++cc) s += sX[tid * LD + cc];
+            dgg[row0 + tid] = s;
+        }
+    }
+}
+
+template <int D, typename T, bool SCALAR>
+cudaError_t launch_typed(const BwdArgs &a, cudaStream_t st, int *launches)
+{
+    const int BH = a.B * a.H, nch = (a.T + kC - 1) / kC;
+    const BwdWs w = carve(a.workspace, a.B, a.H, a.T, D);
+    const T *q = static_cast<const T *>(a.q), *k = static_cast<const T *>(a.k), *v = static_cast<const T *>(a.v);
+    const T *dO = static_cast<const T *>(a.dO);
+    cudaError_t e;
+    {
+        auto kern = bwd_prep<D, T, SCALAR>;
+        const size_t bytes = sizeof(float) * PrepSmem<D>::TOTAL;
+        if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes))) return e;
+        kern<<<BH * nch, kBT, bytes, st>>>(q, k, v, a.g, a.beta, w, a.T, nch);
+        if ((e = cudaGetLastError())) return e;
+        ++*launches;
+    }
+    {
+        auto kern = bwd_fwd_scan<D, T>;
+        const size_t bytes = sizeof(float) * FwdSmem<D>::TOTAL;
+        if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes))) return e;
+        kern<<<dim3(BH, D / kTile), kBT, bytes, st>>>(k, a.S0, w, a.T, nch);
+        if ((e = cudaGetLastError())) return e;
+        ++*launches;
+    }
+    {
+        auto kern = bwd_rev_scan<D, T>;
+        const size_t bytes = sizeof(float) * RevSmem<D>::TOTAL;
+        if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes))) return e;
+        kern<<<dim3(BH, D / kTile), kBT, bytes, st>>>(q, k, dO, a.dS_T, a.dS0, w, a.T, nch);
+        if ((e = cudaGetLastError())) return e;
+        ++*launches;
+    }
+    {
+        auto kern = bwd_grads<D, T, SCALAR>;
+        const size_t bytes = sizeof(float) * GradSmem<D>::TOTAL;
+        if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes))) return e;
+        kern<<<BH * nch, kBT, bytes, st>>>(q, k, v, a.g, a.beta, dO, static_cast<T *>(a.dq), static_cast<T *>(a.dk),
+                                           static_cast<T *>(a.dv), a.dg, a.dbeta, w, a.T, nch);
+        if ((e = cudaGetLastError())) return e;
+        ++*launches;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace
+
+size_t chunk_bwd_workspace_bytes(int B, int H, int T, int D)
+{
+    const size_t bh = (size_t)B * H, nch = (size_t)(T + kC - 1) / kC, tp = nch * kC;
+    return sizeof(float) * (5 * bh * tp * D + 2 * bh * nch * kC * kC + 2 * bh * nch * (size_t)D * D);
+}
+
+cudaError_t launch_chunk_bwd(const BwdArgs &a, cudaStream_t st, int *launches)
+{
+    if ((long long)a.B * a.H == 0 || a.T == 0) return cudaSuccess;
+    if (a.D == 128)
+        return a.bf16 ? (a.scalar_gate ? launch_typed<128, __nv_bfloat16, true>(a, st, launches)
+                                       : launch_typed<128, __nv_bfloat16, false>(a, st, launches))
+                      : (a.scalar_gate ? launch_typed<128, float, true>(a, st, launches)
+                                       : launch_typed<128, float, false>(a, st, launches));
+    return a.bf16 ? (a.scalar_gate ? launch_typed<64, __nv_bfloat16, true>(a, st, launches)
+                                   : launch_typed<64, __nv_bfloat16, false>(a, st, launches))
+                  : (a.scalar_gate ? launch_typed<64, float, true>(a, st, launches)
+                                   : launch_typed<64, float, false>(a, st, launches));
+}
+
+}  // namespace gdr

@@ -220,6 +220,61 @@ GDR_API int gdr_chunk_fwd_gated(const void *q, const void *k, const void *v, con
     return finish(e, launches);
 }
 
+GDR_API size_t gdr_chunk_bwd_workspace_size(int B, int H, int T, int dk, int dv, int C, int gate_mode, int dtype)
+{
+    if (B <= 0 || H <= 0 || T <= 0) return 0;
+    if (gate_mode != GDR_GATE_PER_CHANNEL && gate_mode != GDR_GATE_SCALAR) return 0;
+    if (dtype != GDR_F32 && dtype != GDR_BF16) return 0;
+    if (dk != dv || !size_ok(dk) || C != 64) return 0;
+    return gdr::chunk_bwd_workspace_bytes(B, H, T, dk);
+}
+
+GDR_API int gdr_chunk_bwd(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                          const float *S0, const void *dO, const float *dS_T,
+                          void *dq, void *dk, void *dv, float *dg, float *dbeta, float *dS0,
+                          int B, int H, int T, int dk_, int dv_, int C, int gate_mode, int dtype,
+                          void *workspace, size_t ws_bytes, void *stream)
+{
+    if (B < 0 || H < 0 || T < 0) return GDR_ERR_INVALID_ARG;
+    if (gate_mode != GDR_GATE_PER_CHANNEL && gate_mode != GDR_GATE_SCALAR) return GDR_ERR_INVALID_ARG;
+    if (dtype != GDR_F32 && dtype != GDR_BF16) return GDR_ERR_INVALID_ARG;
+    if (dk_ <= 0 || dv_ <= 0 || C <= 0) return GDR_ERR_INVALID_ARG;
+    if (dk_ != dv_ || !size_ok(dk_) || C != 64) return GDR_ERR_UNSUPPORTED;
+    if ((long long)B * H * T * dk_ >= (1LL << 40)) return GDR_ERR_UNSUPPORTED;
+    const long long heads = (long long)B * H;
+    if (heads == 0) {
+        tl_last_launches = 0;
+        return GDR_OK;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (T == 0) {
+        // no tokens: S_T = S0, so dS0 = dS_T
+        if (dS0 && !aligned16(dS0)) return GDR_ERR_ALIGNMENT;
+        if (dS_T && !aligned16(dS_T)) return GDR_ERR_ALIGNMENT;
+        cudaError_t e = cudaSuccess;
+        const size_t bytes = sizeof(float) * (size_t)heads * dv_ * dk_;
+        if (dS0 && dS_T && dS0 != dS_T) e = cudaMemcpyAsync(dS0, dS_T, bytes, cudaMemcpyDeviceToDevice, st);
+        else if (dS0 && !dS_T) e = cudaMemsetAsync(dS0, 0, bytes, st);
+        return finish(e, 0);
+    }
+    const size_t ws_need = gdr_chunk_bwd_workspace_size(B, H, T, dk_, dv_, C, gate_mode, dtype);
+    if (ws_bytes < ws_need || !workspace) return GDR_ERR_INVALID_ARG;
+    if (!q || !k || !v || !g || !beta || !dO || !dq || !dk || !dv || !dg || !dbeta) return GDR_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, g, beta, S0, dO, dS_T, dq, dk, dv, dg, dbeta, dS0, workspace};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return GDR_ERR_ALIGNMENT;
+    gdr::BwdArgs a;
+    a.q = q; a.k = k; a.v = v; a.dO = dO; a.g = g; a.beta = beta; a.S0 = S0; a.dS_T = dS_T;
+    a.dq = dq; a.dk = dk; a.dv = dv; a.dg = dg; a.dbeta = dbeta; a.dS0 = dS0;
+    a.B = B; a.H = H; a.T = T; a.D = dk_;
+    a.scalar_gate = (gate_mode == GDR_GATE_SCALAR);
+    a.bf16 = (dtype == GDR_BF16);
+    a.workspace = workspace;
+    int launches = 0;
+    cudaError_t e = gdr::launch_chunk_bwd(a, st, &launches);
+    return finish(e, launches);
+}
+
 GDR_API size_t gdr2_chunk_fwd_workspace_size(int B, int H, int T, int dk, int dv, int C, int gate_mode, int dtype)
 {
     if (B <= 0 || H <= 0 || T <= 0) return 0;

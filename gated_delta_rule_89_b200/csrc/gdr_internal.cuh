@@ -91,6 +91,21 @@ inline TcWorkspace carve_tc_workspace(void *ws, int B, int H, int T, bool gdr2 =
     return w;
 }
 
+// Arguments of one chunked backward, already validated (d_k = d_v = D).
+struct BwdArgs {
+    const void *q, *k, *v, *dO;
+    const float *g, *beta, *S0, *dS_T;
+    void *dq, *dk, *dv;
+    float *dg, *dbeta, *dS0;
+    int B, H, T;
+    int D;   // d_k = d_v
+    bool scalar_gate;
+    bool bf16;
+    void *workspace;   // chunk_bwd_workspace_bytes()
+};
+size_t chunk_bwd_workspace_bytes(int B, int H, int T, int D);
+cudaError_t launch_chunk_bwd(const BwdArgs &a, cudaStream_t stream, int *launches);
+
 // Each launcher enqueues its kernels on `stream`, adds the number of kernels
 // it launched to *launches and returns the first launch error.
 cudaError_t launch_recurrent_step(const StepArgs &a, cudaStream_t stream, int *launches);

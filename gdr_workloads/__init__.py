@@ -44,6 +44,7 @@ TID_Q, TID_K, TID_V, TID_G, TID_BETA, TID_S0, TID_CHAN = 1, 2, 3, 4, 5, 6, 7
 TID_QRAW, TID_KRAW, TID_AGATE, TID_ALOG, TID_DTBIAS, TID_BLOGIT = 8, 9, 10, 11, 12, 13
 TID_ERASE, TID_WRITE = 14, 15   # Gated Delta Rule-2 erase and write gates
 TID_OGATE, TID_NORMW = 16, 17   # output gate pre-activation, RMSNorm weight
+TID_DO, TID_DST = 18, 19         # gradients fed to the backward pass
 
 
 def _s64(c: int) -> int:
@@ -132,6 +133,7 @@ class Workload:
     description: str
     rule: str = "gdr"    # "gdr" (tied beta: KDA / Gated DeltaNet) or "gdr2" (erase and write gates)
     out: str = "plain"   # "plain" (o_t) or "gated" (Sigmoid(gate) * RMSNorm(o_t))
+    direction: str = "fwd"   # "fwd" or "bwd" (the gradients of <dO, O> + <dS_T, S_T>)
 
     @property
     def tokens(self) -> int:
@@ -167,6 +169,11 @@ WORKLOADS: Dict[str, Workload] = {
         "softplus_n02_clamp5", "normal002", 2,
         "KDA forward with the output epilogue fused in (per-head RMSNorm times a sigmoid output gate): "
         "B2 H32 T8192 d128 C64 bf16", out="gated"),
+    "kda_d128_t8192_bwd": Workload(
+        "kda_d128_t8192_bwd", "chunk", 2, 32, 8192, 128, 128, 64, "per_channel", torch.bfloat16,
+        "softplus_n02_clamp5", "normal002", 2,
+        "KDA backward (gradients of q, k, v, g, beta, S0 from dO, dS_T): B2 H32 T8192 d128 C64 bf16",
+        direction="bwd"),
     "gdr2_decode_b256": Workload(
         "gdr2_decode_b256", "decode", 256, 32, 1000, 128, 128, 1, "per_channel", torch.bfloat16,
         "softplus_n01_plus1_clamp5", "normal002", 6,
@@ -397,6 +404,30 @@ def generate_prologue(w: Workload, device="cpu", heads: Optional[Sequence[int]] 
     S0 = generate(dataclasses.replace(w, T=1, g_recipe="softplus_n01_plus1_clamp5"), device=device,
                   heads=heads)["S0"]
     return dict(q_raw=q_raw, k_raw=k_raw, v=v, a=a, A_log=A_log, dt_bias=dt_bias, b_logit=b_logit, S0=S0)
+
+
+def generate_grads(w: Workload, device="cpu", heads: Optional[Sequence[int]] = None,
+                   block: int = 1 << 24) -> Dict[str, torch.Tensor]:
+    """Output-side gradients for the backward pass of chunk workload ``w``:
+    dO [B,H,T,dv] ~ N(0,1) in the workload dtype and dS_T [B,H,dv,dk] ~ N(0,1)
+    fp32, with the same head selection rule as ``generate``."""
+    assert w.kind == "chunk"
+    B, H, T, dk, dv, seed = w.B, w.H, w.T, w.dk, w.dv, w.seed
+    head_ids = torch.arange(B * H, dtype=torch.int64, device=device) if heads is None else \
+        torch.as_tensor(list(heads), dtype=torch.int64, device=device)
+    nh = head_ids.numel()
+    outB, outH = (B, H) if heads is None else (nh, 1)
+
+    def per_head(tid, per):
+        out = torch.empty(nh * per, dtype=torch.float64, device=device)
+        for s, e in _chunked(nh * per, block):
+            lin = torch.arange(s, e, dtype=torch.int64, device=device)
+            out[s:e] = normal(seed, tid, head_ids[lin // per] * per + lin % per)
+        return out
+
+    dO = to_dtype(per_head(TID_DO, T * dv), w.dtype).view(outB, outH, T, dv)
+    dST = per_head(TID_DST, dv * dk).to(torch.float32).view(outB, outH, dv, dk)
+    return dict(dO=dO, dS_T=dST)
 
 
 def small_chunk_case(B: int, H: int, T: int, dk: int, dv: int, gate: str, dtype: torch.dtype,

@@ -174,6 +174,40 @@ int gdr_chunk_fwd_gated(const void *q, const void *k, const void *v, const float
                         void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * Backward pass of the chunkwise forward: the gradients of
+ *   L = <dO, O> + <dS_T, S_T>
+ * with respect to q, k, v, g, beta and S0, where (O, S_T) is what
+ * gdr_chunk_fwd returns for the same inputs.  It differentiates the same
+ * chunk form (UT transform, chunk state recurrence and output: "Token Mixer
+ * I", section "Kimi Delta Attention: Improving Delta Rule with Fine-grained
+ * Gating"; the training path of the section "Gated Delta Networks"): the
+ * states at chunk boundaries are recomputed, the state gradient runs through
+ * the chunks in reverse, and the rest is parallel over chunks.  fp32
+ * arithmetic throughout.  The -5 bound on a per-channel g passes the gradient
+ * where g >= -5 and blocks it below.
+ *
+ *   q, k, v, g, beta, S0   as gdr_chunk_fwd (S0 NULL -> zeros)
+ *   dO     [B,H,T,d_v]   dtype                  gradient of O
+ *   dS_T   [B,H,d_v,d_k] float or NULL (zeros)  gradient of S_T
+ *   dq, dk [B,H,T,d_k], dv [B,H,T,d_v]   dtype  (written)
+ *   dg     layout of g, float                   (written)
+ *   dbeta  [B,H,T] float                        (written)
+ *   dS0    [B,H,d_v,d_k] float or NULL          (written if given)
+ * Supported: d_k = d_v in {64, 128}, C = 64, fp32 or bf16; anything else
+ * returns GDR_ERR_UNSUPPORTED.  The workspace (device, >=
+ * gdr_chunk_bwd_workspace_size() bytes, 16-byte aligned) holds the
+ * recomputed chunk quantities and the per-chunk states and state gradients:
+ * about 320 KB per 64-token chunk at d = 128.
+ */
+size_t gdr_chunk_bwd_workspace_size(int B, int H, int T, int dk, int dv, int C, int gate_mode, int dtype);
+
+int gdr_chunk_bwd(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                  const float *S0, const void *dO, const float *dS_T,
+                  void *dq, void *dk, void *dv, float *dg, float *dbeta, float *dS0,
+                  int B, int H, int T, int dk_, int dv_, int C, int gate_mode, int dtype,
+                  void *workspace, size_t ws_bytes, void *stream);
+
+/*
  * Gated Delta Rule-2: the erase and write decisions of the delta rule get
  * their own per-channel gates ("Token Mixer I", section "Gated DeltaNet-2:
  * Decoupling Erase and Write in Linear Attention", eq. (10)).  With

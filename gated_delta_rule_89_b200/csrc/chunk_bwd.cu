@@ -45,6 +45,7 @@ constexpr int kTile = 32;  // d_v rows per scan block
 
 struct BwdWs {
     float *G, *W, *U, *Vn, *dVn;   // [BH][Tp][D], Tp = chunks * 64 (padded rows)
+    float *Kt, *Ql;                 // K_tail = k exp(G_C - G), Q<- = q exp(G), same layout
     float *M, *Aq;                  // [BH * chunks][64][64]
     float *Sck, *dSck;              // [BH * chunks][D][D]
 };
@@ -59,6 +60,8 @@ inline BwdWs carve(void *ws, int B, int H, int T, int D)
     w.U = p; p += bh * tp * D;
     w.Vn = p; p += bh * tp * D;
     w.dVn = p; p += bh * tp * D;
+    w.Kt = p; p += bh * tp * D;
+    w.Ql = p; p += bh * tp * D;
     w.M = p; p += bh * nch * kC * kC;
     w.Aq = p; p += bh * nch * kC * kC;
     w.Sck = p; p += bh * nch * (size_t)D * D;
@@ -88,6 +91,7 @@ bwd_prep(const T *__restrict__ qg, const T *__restrict__ kg, const T *__restrict
     const int t0 = n * kC, nrows = min(kC, T_len - t0);
     const size_t row0 = (size_t)head * T_len + t0, prow0 = (size_t)head * nch * kC + t0;
 
+#pragma unroll 8
     for (int idx = tid; idx < kC * D; idx += kBT) {
         const int r = idx / D, c = idx - r * D;
         const bool ok = r < nrows;
@@ -108,8 +112,17 @@ bwd_prep(const T *__restrict__ qg, const T *__restrict__ kg, const T *__restrict
         }
     }
     __syncthreads();
+    // the scans' operands K_tail = k exp(G_C - G) and Q<- = q exp(G)
+#pragma unroll 8
+    for (int idx = tid; idx < kC * D; idx += kBT) {
+        const int r = idx / D, c = idx - r * D;
+        const float gr = sG[r * LD + c];
+        w.Kt[(prow0 + r) * D + c] = sk[r * LD + c] * __expf(sG[(kC - 1) * LD + c] - gr);
+        w.Ql[(prow0 + r) * D + c] = sq[r * LD + c] * __expf(gr);
+    }
     // A (strictly lower, beta_r in) and Aqk (lower incl. the diagonal)
     float *Aqo = w.Aq + (size_t)ci * kC * kC;
+#pragma unroll 8
     for (int idx = tid; idx < kC * kC; idx += kBT) {
         const int r = idx >> 6, i = idx & 63;
         float sa = 0.f, sq_ = 0.f;
@@ -142,8 +155,10 @@ bwd_prep(const T *__restrict__ qg, const T *__restrict__ kg, const T *__restrict
     }
     __syncthreads();
     float *Mo = w.M + (size_t)ci * kC * kC;
+#pragma unroll 8
     for (int idx = tid; idx < kC * kC; idx += kBT) Mo[idx] = sM[(idx >> 6) * 65 + (idx & 63)];
     // W = M Diag(beta) (K * gamma): the operand beta_i k_ic gamma_ic into sq
+#pragma unroll 8
     for (int idx = tid; idx < kC * D; idx += kBT) {
         const int r = idx / D, c = idx - r * D;
         sq[r * LD + c] = sb[r] * sk[r * LD + c] * __expf(sG[r * LD + c]);
@@ -164,6 +179,7 @@ bwd_prep(const T *__restrict__ qg, const T *__restrict__ kg, const T *__restrict
     }
     __syncthreads();
     // U = M Diag(beta) V (d_v = D)
+#pragma unroll 8
     for (int idx = tid; idx < kC * D; idx += kBT) {
         const int r = idx / D, j = idx - r * D;
         sq[r * LD + j] = r < nrows ? sb[r] * to_f32<T>(vg[(row0 + r) * D + j]) : 0.f;
@@ -191,23 +207,19 @@ struct FwdSmem {
     static constexpr int TOTAL = GC + D;
 };
 
-// K_tail rows of chunk n into kt (k * exp(G_C - G), zero past T), G_C into gc
-template <int D, typename T>
-__device__ __forceinline__ void load_ktail(float *kt, float *gc, const T *kg, const float *G, size_t row0,
-                                           size_t prow0, int nrows, int tid)
+// K_tail rows of chunk n into kt (zero past T: k is), G_C into gc
+template <int D>
+__device__ __forceinline__ void load_ktail(float *kt, float *gc, const BwdWs &w, size_t prow0, int tid)
 {
     constexpr int LD = D + 1;
-    for (int c = tid; c < D; c += kBT) gc[c] = G[(prow0 + kC - 1) * D + c];
-    __syncthreads();
-    for (int idx = tid; idx < kC * D; idx += kBT) {
-        const int r = idx / D, c = idx - r * D;
-        kt[r * LD + c] = r < nrows ? to_f32<T>(kg[(row0 + r) * D + c]) * __expf(gc[c] - G[(prow0 + r) * D + c]) : 0.f;
-    }
+    for (int c = tid; c < D; c += kBT) gc[c] = w.G[(prow0 + kC - 1) * D + c];
+#pragma unroll 8
+    for (int idx = tid; idx < kC * D; idx += kBT) kt[(idx / D) * LD + idx % D] = w.Kt[(prow0 + idx / D) * D + idx % D];
 }
 
-template <int D, typename T>
+template <int D>
 __global__ void __launch_bounds__(kBT)
-bwd_fwd_scan(const T *__restrict__ kg, const float *__restrict__ S0, BwdWs w, int T_len, int nch)
+bwd_fwd_scan(const float *__restrict__ S0, BwdWs w, int nch)
 {
     using L = FwdSmem<D>;
     constexpr int LD = L::LD, RS = kBT / D, NJ = kTile / RS;
@@ -215,6 +227,7 @@ bwd_fwd_scan(const T *__restrict__ kg, const float *__restrict__ S0, BwdWs w, in
     float *sS = sm + L::S, *sW = sm + L::W, *sKt = sm + L::KT, *sVn = sm + L::VN, *gc = sm + L::GC;
     const int tid = threadIdx.x;
     const int head = blockIdx.x, i0 = blockIdx.y * kTile;
+#pragma unroll 8
     for (int idx = tid; idx < kTile * D; idx += kBT) {
         const int j = idx / D, c = idx - j * D;
         sS[j * LD + c] = S0 ? S0[((size_t)head * D + i0 + j) * D + c] : 0.f;
@@ -222,13 +235,14 @@ bwd_fwd_scan(const T *__restrict__ kg, const float *__restrict__ S0, BwdWs w, in
     const int c = tid % D, h = tid / D;
     const int vj = tid & 31, vr = tid >> 5;   // V_new: column (state row) vj, rows vr + 8 m
     for (int n = 0; n < nch; ++n) {
-        const int t0 = n * kC, nrows = min(kC, T_len - t0);
-        const size_t row0 = (size_t)head * T_len + t0, prow0 = (size_t)head * nch * kC + t0;
+        const size_t prow0 = (size_t)head * nch * kC + (size_t)n * kC;
         __syncthreads();
         float *ck = w.Sck + ((size_t)(head * nch + n) * D + i0) * D;
+#pragma unroll 8
         for (int idx = tid; idx < kTile * D; idx += kBT) ck[idx] = sS[(idx / D) * LD + idx % D];
+#pragma unroll 8
         for (int idx = tid; idx < kC * D; idx += kBT) sW[(idx / D) * LD + idx % D] = w.W[(prow0 + idx / D) * D + idx % D];
-        load_ktail<D, T>(sKt, gc, kg, w.G, row0, prow0, nrows, tid);
+        load_ktail<D>(sKt, gc, w, prow0, tid);
         __syncthreads();
         // V_new = U - W S^T (this tile's d_v columns)
 #pragma unroll
@@ -267,8 +281,8 @@ struct RevSmem {
 
 template <int D, typename T>
 __global__ void __launch_bounds__(kBT)
-bwd_rev_scan(const T *__restrict__ qg, const T *__restrict__ kg, const T *__restrict__ dOg,
-             const float *__restrict__ dST, float *__restrict__ dS0, BwdWs w, int T_len, int nch)
+bwd_rev_scan(const T *__restrict__ dOg, const float *__restrict__ dST, float *__restrict__ dS0, BwdWs w, int T_len,
+             int nch)
 {
     using L = RevSmem<D>;
     constexpr int LD = L::LD, RS = kBT / D, NJ = kTile / RS, TL = kTile + 1;
@@ -277,6 +291,7 @@ bwd_rev_scan(const T *__restrict__ qg, const T *__restrict__ kg, const T *__rest
           *gc = sm + L::GC;
     const int tid = threadIdx.x;
     const int head = blockIdx.x, i0 = blockIdx.y * kTile;
+#pragma unroll 8
     for (int idx = tid; idx < kTile * D; idx += kBT) {
         const int j = idx / D, c = idx - j * D;
         sdS[j * LD + c] = dST ? dST[((size_t)head * D + i0 + j) * D + c] : 0.f;
@@ -288,14 +303,17 @@ bwd_rev_scan(const T *__restrict__ qg, const T *__restrict__ kg, const T *__rest
         const size_t row0 = (size_t)head * T_len + t0, prow0 = (size_t)head * nch * kC + t0;
         __syncthreads();
         float *ck = w.dSck + ((size_t)(head * nch + n) * D + i0) * D;
+#pragma unroll 8
         for (int idx = tid; idx < kTile * D; idx += kBT) ck[idx] = sdS[(idx / D) * LD + idx % D];
         const float *aq = w.Aq + (size_t)(head * nch + n) * kC * kC;
+#pragma unroll 8
         for (int idx = tid; idx < kC * kC; idx += kBT) sAq[(idx >> 6) * 65 + (idx & 63)] = aq[idx];
+#pragma unroll 8
         for (int idx = tid; idx < kC * kTile; idx += kBT) {
             const int r = idx / kTile, j = idx - r * kTile;
             sdO[r * TL + j] = r < nrows ? to_f32<T>(dOg[(row0 + r) * D + i0 + j]) : 0.f;
         }
-        load_ktail<D, T>(sKt, gc, kg, w.G, row0, prow0, nrows, tid);
+        load_ktail<D>(sKt, gc, w, prow0, tid);
         __syncthreads();
         // dV_new = Aqk^T dO + K_tail dS^T
 #pragma unroll
@@ -313,11 +331,8 @@ bwd_rev_scan(const T *__restrict__ qg, const T *__restrict__ kg, const T *__rest
         const float gcc = __expf(gc[c]);
 #pragma unroll
         for (int m = 0; m < NJ; ++m) acc[m] = sdS[(h + RS * m) * LD + c] * gcc;
-        for (int idx = tid; idx < kC * D; idx += kBT) {
-            const int r = idx / D, cc = idx - r * D;
-            sKt[r * LD + cc] =
-                r < nrows ? to_f32<T>(qg[(row0 + r) * D + cc]) * __expf(w.G[(prow0 + r) * D + cc]) : 0.f;
-        }
+#pragma unroll 8
+        for (int idx = tid; idx < kC * D; idx += kBT) sKt[(idx / D) * LD + idx % D] = w.Ql[(prow0 + idx / D) * D + idx % D];
         __syncthreads();
         for (int r = 0; r < kC; ++r) {
             const float ql = sKt[r * LD + c];
@@ -325,6 +340,7 @@ bwd_rev_scan(const T *__restrict__ qg, const T *__restrict__ kg, const T *__rest
             for (int m = 0; m < NJ; ++m) acc[m] = fmaf(sdO[r * TL + h + RS * m], ql, acc[m]);
         }
         __syncthreads();
+#pragma unroll 8
         for (int idx = tid; idx < kC * D; idx += kBT) sKt[(idx / D) * LD + idx % D] = w.W[(prow0 + idx / D) * D + idx % D];
         __syncthreads();
         for (int r = 0; r < kC; ++r) {
@@ -338,6 +354,7 @@ bwd_rev_scan(const T *__restrict__ qg, const T *__restrict__ kg, const T *__rest
     }
     __syncthreads();
     if (dS0)
+#pragma unroll 8
         for (int idx = tid; idx < kTile * D; idx += kBT)
             dS0[((size_t)head * D + i0 + idx / D) * D + idx % D] = sdS[(idx / D) * LD + idx % D];
 }
@@ -373,6 +390,7 @@ bwd_grads(const T *__restrict__ qg, const T *__restrict__ kg, const T *__restric
     const int c = tid % D, h = tid / D;              // this thread: channel c, rows h + RS m
     const int pi = tid & 63, pr = tid >> 6;          // 64 x 64 outputs: column pi, rows pr + 4 m
 
+#pragma unroll 8
     for (int idx = tid; idx < kC * D; idx += kBT) {
         const int r = idx / D, cc = idx - r * D;
         const bool ok = r < nrows;
@@ -383,6 +401,7 @@ bwd_grads(const T *__restrict__ qg, const T *__restrict__ kg, const T *__restric
         sY[r * LD + cc] = w.Vn[(prow0 + r) * D + cc];                         // V_new
     }
     const float *Mg = w.M + (size_t)ci * kC * kC;
+#pragma unroll 8
     for (int idx = tid; idx < kC * kC; idx += kBT) sM[(idx >> 6) * 65 + (idx & 63)] = Mg[idx];
     if (tid < kC) {
         sb[tid] = tid < nrows ? betag[row0 + tid] : 0.f;
@@ -456,7 +475,9 @@ bwd_grads(const T *__restrict__ qg, const T *__restrict__ kg, const T *__restric
     sgcp[h * D + c] = dgc;
     __syncthreads();   // dO, V_new done
     // dV_new -> sX;  dV = T'^T dV_new = Diag(beta) M^T dV_new  -> output
+#pragma unroll 8
     for (int idx = tid; idx < kC * D; idx += kBT) sX[(idx / D) * LD + idx % D] = w.dVn[(prow0 + idx / D) * D + idx % D];
+#pragma unroll 8
     for (int idx = tid; idx < kC * D; idx += kBT) {
         const int r = idx / D, j = idx - r * D;
         sY[r * LD + j] = r < nrows ? to_f32<T>(vg[(row0 + r) * D + j]) : 0.f;   // V
@@ -500,14 +521,19 @@ bwd_grads(const T *__restrict__ qg, const T *__restrict__ kg, const T *__restric
 #pragma unroll
         for (int m = 0; m < NR; ++m) sY[(h + RS * m) * LD + c] = -acc[m];
     }
+    __syncthreads();   // dV_new no longer needed: K<- = k exp(G) into sX
+#pragma unroll 8
+    for (int idx = tid; idx < kC * D; idx += kBT) {
+        const int r = idx / D, cc = idx - r * D;
+        sX[r * LD + cc] = sk[r * LD + cc] * __expf(sG[r * LD + cc]);
+    }
     __syncthreads();
     // dT' += dW K<-^T
 #pragma unroll
     for (int m = 0; m < kC / 4; ++m) {
         const int r = pr + 4 * m;
         float acc = 0.f;
-        for (int cc = 0; cc < D; ++cc)
-            acc = fmaf(sY[r * LD + cc], sk[pi * LD + cc] * __expf(sG[pi * LD + cc]), acc);
+        for (int cc = 0; cc < D; ++cc) acc = fmaf(sY[r * LD + cc], sX[pi * LD + cc], acc);
         sP[r * 65 + pi] += acc;
     }
     // dK<- = T'^T dW = Diag(beta) M^T dW  ->  dk += dK<- gamma,  dG += dK<- k gamma
@@ -536,6 +562,7 @@ bwd_grads(const T *__restrict__ qg, const T *__restrict__ kg, const T *__restric
         sdb[tid] = s;
     }
     __syncthreads();
+#pragma unroll 8
     for (int idx = tid; idx < kC * kC; idx += kBT) sP[(idx >> 6) * 65 + (idx & 63)] *= sb[idx & 63];
     __syncthreads();
     // dA = -M^T dM M^T on the strict lower triangle: first Z = dM M^T -> sY (as 64 x 65)
@@ -665,10 +692,10 @@ cudaError_t launch_typed(const BwdArgs &a, cudaStream_t st, int *launches)
         ++*launches;
     }
     {
-        auto kern = bwd_fwd_scan<D, T>;
+        auto kern = bwd_fwd_scan<D>;
         const size_t bytes = sizeof(float) * FwdSmem<D>::TOTAL;
         if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes))) return e;
-        kern<<<dim3(BH, D / kTile), kBT, bytes, st>>>(k, a.S0, w, a.T, nch);
+        kern<<<dim3(BH, D / kTile), kBT, bytes, st>>>(a.S0, w, nch);
         if ((e = cudaGetLastError())) return e;
         ++*launches;
     }
@@ -676,7 +703,7 @@ cudaError_t launch_typed(const BwdArgs &a, cudaStream_t st, int *launches)
         auto kern = bwd_rev_scan<D, T>;
         const size_t bytes = sizeof(float) * RevSmem<D>::TOTAL;
         if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes))) return e;
-        kern<<<dim3(BH, D / kTile), kBT, bytes, st>>>(q, k, dO, a.dS_T, a.dS0, w, a.T, nch);
+        kern<<<dim3(BH, D / kTile), kBT, bytes, st>>>(dO, a.dS_T, a.dS0, w, a.T, nch);
         if ((e = cudaGetLastError())) return e;
         ++*launches;
     }
@@ -697,7 +724,7 @@ cudaError_t launch_typed(const BwdArgs &a, cudaStream_t st, int *launches)
 size_t chunk_bwd_workspace_bytes(int B, int H, int T, int D)
 {
     const size_t bh = (size_t)B * H, nch = (size_t)(T + kC - 1) / kC, tp = nch * kC;
-    return sizeof(float) * (5 * bh * tp * D + 2 * bh * nch * kC * kC + 2 * bh * nch * (size_t)D * D);
+    return sizeof(float) * (7 * bh * tp * D + 2 * bh * nch * kC * kC + 2 * bh * nch * (size_t)D * D);
 }
 
 cudaError_t launch_chunk_bwd(const BwdArgs &a, cudaStream_t st, int *launches)

@@ -49,10 +49,11 @@
 //   U_20 = -Nt_20 D_0 - Nt_21 U_10,   U_31 = -Nt_31 D_1 - Nt_32 U_21,
 //   U_30 = -Nt_30 D_0 - Nt_31 U_10 - Nt_32 U_20,
 // (from N N^{-1} = I, left-multiplied by D_i).  These 16 products of 16 x 16
-// fp32 blocks run on mma.sync (m16n8k8, tf32) with each operand split into a
-// high and a low tf32 part (x = hi + lo) and the product taken as
-// hi*hi + hi*lo + lo*hi, the three-pass tf32 error compensation of
-// Ootomo and Yokota (2022), which keeps fp32-level accuracy.
+// fp32 blocks run on mma.sync (m16n8k8, tf32 operands, fp32 accumulation).
+// T' leaves this kernel in bf16 (8-bit mantissa), so the 10-bit tf32
+// operands add well under the final rounding; a three-pass hi/lo split
+// (Ootomo and Yokota, 2022) measured the same end-to-end error and was
+// slower.
 
 #include <mutex>
 
@@ -138,11 +139,11 @@ __device__ __forceinline__ uint32_t scale2p(uint32_t v, float2 f)
     return pack2(r.x, r.y);
 }
 
-__device__ __forceinline__ void split_tf32(float x, uint32_t &hi, uint32_t &lo)
+__device__ __forceinline__ uint32_t to_tf32(float x)
 {
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(hi) : "f"(x));
-    const float r = x - __uint_as_float(hi);
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(lo) : "f"(r));
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
 }
 
 __device__ __forceinline__ void mma1688(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
@@ -154,8 +155,8 @@ __device__ __forceinline__ void mma1688(float (&d)[4], const uint32_t (&a)[4], u
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// One warp: c[16x16] -= A[16x16] B[16x16] in fp32 accuracy (three tf32
-// passes).  A, B row-major in shared memory with row strides lda, ldb.
+// One warp: c[16x16] -= A[16x16] B[16x16] (tf32 operands, fp32 accumulation).
+// A, B row-major in shared memory with row strides lda, ldb.
 // Fragment of c: c[nt][e] is row g + 8 (e >> 1), column 8 nt + 2 t + (e & 1),
 // with g = lane / 4, t = lane % 4.
 __device__ __forceinline__ void mm16_sub(float (&c)[2][4], const float *A, int lda, const float *B, int ldb, int g,
@@ -163,20 +164,14 @@ __device__ __forceinline__ void mm16_sub(float (&c)[2][4], const float *A, int l
 {
 #pragma unroll
     for (int ks = 0; ks < 2; ++ks) {
-        uint32_t ah[4], al[4];
-        split_tf32(-A[g * lda + 8 * ks + t], ah[0], al[0]);
-        split_tf32(-A[(g + 8) * lda + 8 * ks + t], ah[1], al[1]);
-        split_tf32(-A[g * lda + 8 * ks + t + 4], ah[2], al[2]);
-        split_tf32(-A[(g + 8) * lda + 8 * ks + t + 4], ah[3], al[3]);
+        uint32_t a[4];
+        a[0] = to_tf32(-A[g * lda + 8 * ks + t]);
+        a[1] = to_tf32(-A[(g + 8) * lda + 8 * ks + t]);
+        a[2] = to_tf32(-A[g * lda + 8 * ks + t + 4]);
+        a[3] = to_tf32(-A[(g + 8) * lda + 8 * ks + t + 4]);
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            uint32_t bh0, bl0, bh1, bl1;
-            split_tf32(B[(8 * ks + t) * ldb + 8 * nt + g], bh0, bl0);
-            split_tf32(B[(8 * ks + t + 4) * ldb + 8 * nt + g], bh1, bl1);
-            mma1688(c[nt], al, bh0, bh1);
-            mma1688(c[nt], ah, bl0, bl1);
-            mma1688(c[nt], ah, bh0, bh1);
-        }
+        for (int nt = 0; nt < 2; ++nt)
+            mma1688(c[nt], a, to_tf32(B[(8 * ks + t) * ldb + 8 * nt + g]), to_tf32(B[(8 * ks + t + 4) * ldb + 8 * nt + g]));
     }
 }
 

@@ -163,6 +163,14 @@ __device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap *map, int c
                  : "memory");
 }
 
+// Bulk prefetch of a contiguous global range into L2 (address and size
+// multiples of 16 bytes; no completion to wait for).
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes)
+                 : "memory");
+}
+
 // hardware tanh approximation (MUFU), about 2^-11 relative error
 __device__ __forceinline__ float tanh_approx(float x)
 {

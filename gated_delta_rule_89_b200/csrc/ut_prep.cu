@@ -246,6 +246,23 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
         const int t0 = (ci - head * nchunks) * kC;
         const int nrows = min(kC, T_len - t0);
         const size_t row0 = (size_t)head * T_len + t0;   // first token row of this chunk
+        if (tid == 0 && ci + (int)gridDim.x < total) {
+            // warm L2 with the next chunk's inputs while this one is processed
+            const int cn = ci + gridDim.x, hn = cn / nchunks, tn = (cn - hn * nchunks) * kC;
+            const int rn = min(kC, T_len - tn);
+            const size_t rown = (size_t)hn * T_len + tn;
+            bulk_prefetch_l2(kg + rown * kDK, (uint32_t)rn * kDK * 2);
+            bulk_prefetch_l2(qg + rown * kDK, (uint32_t)rn * kDK * 2);
+            if (!SCALAR) {
+                if (PRO) bulk_prefetch_l2(static_cast<const __nv_bfloat16 *>(gin) + rown * kDK, (uint32_t)rn * kDK * 2);
+                else bulk_prefetch_l2(static_cast<const float *>(gin) + rown * kDK, (uint32_t)rn * kDK * 4);
+            }
+            if (GDR2) {
+                bulk_prefetch_l2(erg + rown * kDK, (uint32_t)rn * kDK * 2);
+                bulk_prefetch_l2(vg + rown * kDK, (uint32_t)rn * kDK * 2);
+                bulk_prefetch_l2(wrg + rown * kDK, (uint32_t)rn * kDK * 2);
+            }
+        }
         const size_t cbase = (size_t)ci * kC * kC;       // this chunk's T' and Aqk
         // beta alternates between two buffers: the last T' stores of the
         // previous chunk may still read theirs while this chunk starts

@@ -51,18 +51,24 @@ DEFAULT_WORKLOAD = "kda_d128_t8192"
 # workload with the hash of the sources those kernels are built from; an
 # entry is ignored (traffic = null) as soon as any of the sources changes.
 TRAFFIC = {
-    # ut_prep 539.0 MB read + 493.3 MB written, chunk_scan 679.6 + 118.4 MB (one launch each)
-    "kda_d128_t8192": {"src_sha": "5fc857a143f498dc", "bytes_per_launch": 1830330112},
-    # gated output: the scan also reads the gate tiles (813.9 + 121.6 MB); ut_prep 539.0 + 493.8 MB
-    "kda_d128_t8192_gated": {"src_sha": "5fc857a143f498dc", "bytes_per_launch": 1968358144},
-    # Gated Delta Rule-2: ut_prep 939.6 + 633.4 MB (reads b, v, w; writes w * v), chunk_scan 679.6 + 118.4 MB
-    "gdr2_d128_t8192": {"src_sha": "5fc857a143f498dc", "bytes_per_launch": 2371053824},
-    # recurrent_step, one decode step: 547.4 MB read + 479.2 MB written
-    "kda_decode_b256": {"src_sha": "99a0454504c77460", "bytes_per_launch": 1026655488},
+    # ut_prep 558.8 MB read + 494.9 MB written, chunk_scan 679.6 + 118.8 MB (one launch each)
+    "kda_d128_t8192": {"src_sha": "fe8676200985376b", "bytes_per_launch": 1852187392},
+    # fused input prologue: ut_prep 409.8 + 488.6 MB, chunk_scan 679.6 + 118.9 MB
+    "kda_d128_t8192_prologue": {"src_sha": "fe8676200985376b", "bytes_per_launch": 1696968960},
+    # gated output: the scan also reads the gate tiles (813.9 + 120.4 MB); ut_prep 558.5 + 493.8 MB
+    "kda_d128_t8192_gated": {"src_sha": "fe8676200985376b", "bytes_per_launch": 1986628864},
+    # Gated Delta Rule-2: ut_prep 1394.0 + 634.1 MB (reads b, v, w; writes w * v), chunk_scan 679.6 + 118.5 MB
+    "gdr2_d128_t8192": {"src_sha": "fe8676200985376b", "bytes_per_launch": 2826130432},
+    # backward: bwd_prep 675.0 + 1553.2, bwd_fwd_scan 1521.9 + 777.1, bwd_rev_scan 2449.8 + 789.2,
+    # bwd_grads 2827.1 + 651.4 MB
+    "kda_d128_t8192_bwd": {"src_sha": "79812d6152006030", "bytes_per_launch": 11244719872},
+    # recurrent_step, one decode step: 547.4 MB read + 477.8 MB written
+    "kda_decode_b256": {"src_sha": "13bedf0248f32e59", "bytes_per_launch": 1025204480},
 }
 
 CHUNK_SOURCES = ("chunk_tc.cu", "ut_prep.cu", "sm100_ptx.cuh", "gdr_internal.cuh")
 DECODE_SOURCES = ("recurrent_step.cu", "gdr_internal.cuh")
+BWD_SOURCES = ("chunk_bwd.cu", "gdr_internal.cuh")
 
 
 # ----------------------------------------------------------------- helpers
@@ -533,7 +539,8 @@ def main():
             import dataclasses
             wk = dataclasses.replace(w0, T=1)   # one launch = one decode step
         src = [os.path.join(ROOT, "gated_delta_rule_89_b200", "csrc", f)
-               for f in (DECODE_SOURCES if w.kind == "decode" else CHUNK_SOURCES)]
+               for f in (DECODE_SOURCES if w.kind == "decode" else BWD_SOURCES if w.direction == "bwd"
+                         else CHUNK_SOURCES)]
         line = base_line(w0, args, world)
         line.update({
             "value": value,

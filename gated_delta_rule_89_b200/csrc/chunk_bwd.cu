@@ -200,21 +200,72 @@ bwd_prep(const T *__restrict__ qg, const T *__restrict__ kg, const T *__restrict
 }
 
 // ------------------------------------------------------------------ 2. forward state scan
+// Both scans hold a 32-row d_v tile of the state (or its gradient) in shared
+// memory and walk the chunks in order (reverse order).  Their small products
+// are register-tiled: a thread computes 4 rows x 2 state rows of V_new (or
+// dV_new) and 2 state rows x 8 channels of the state update, reading 16-byte
+// operand vectors (rows padded to D + 4 floats).
 template <int D>
 struct FwdSmem {
-    static constexpr int LD = D + 1;
-    static constexpr int S = 0, W = S + kTile * LD, KT = W + kC * LD, VN = KT + kC * LD, GC = VN + kC * (kTile + 1);
+    static constexpr int L4 = D + 4;
+    static constexpr int S = 0, W = S + kTile * L4, KT = W + kC * L4, VN = KT + kC * L4, GC = VN + kC * (kTile + 1);
     static constexpr int TOTAL = GC + D;
 };
 
-// K_tail rows of chunk n into kt (zero past T: k is), G_C into gc
+// K_tail rows of chunk n into kt, G_C into gc
 template <int D>
 __device__ __forceinline__ void load_ktail(float *kt, float *gc, const BwdWs &w, size_t prow0, int tid)
 {
-    constexpr int LD = D + 1;
+    constexpr int L4 = D + 4;
     for (int c = tid; c < D; c += kBT) gc[c] = w.G[(prow0 + kC - 1) * D + c];
-#pragma unroll 8
-    for (int idx = tid; idx < kC * D; idx += kBT) kt[(idx / D) * LD + idx % D] = w.Kt[(prow0 + idx / D) * D + idx % D];
+#pragma unroll 4
+    for (int idx = tid; idx < kC * D / 4; idx += kBT) {
+        const int r = idx / (D / 4), c4 = idx - r * (D / 4);
+        *reinterpret_cast<float4 *>(kt + r * L4 + 4 * c4) = *reinterpret_cast<const float4 *>(w.Kt + (prow0 + r) * D + 4 * c4);
+    }
+}
+
+// acc[a][b] += sum_c A[(r0 + a) * L4 + c] * B[(j_b) * L4 + c] for 4 rows of A and 2 rows of B
+template <int D>
+__device__ __forceinline__ void dot_4x2(float (&acc)[4][2], const float *A, int r0, const float *B, int j0, int j1)
+{
+    constexpr int L4 = D + 4;
+#pragma unroll 4
+    for (int c = 0; c < D; c += 4) {
+        const float4 b0 = *reinterpret_cast<const float4 *>(B + j0 * L4 + c);
+        const float4 b1 = *reinterpret_cast<const float4 *>(B + j1 * L4 + c);
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+            const float4 x = *reinterpret_cast<const float4 *>(A + (r0 + a) * L4 + c);
+            acc[a][0] = fmaf(x.x, b0.x, fmaf(x.y, b0.y, fmaf(x.z, b0.z, fmaf(x.w, b0.w, acc[a][0]))));
+            acc[a][1] = fmaf(x.x, b1.x, fmaf(x.y, b1.y, fmaf(x.z, b1.z, fmaf(x.w, b1.w, acc[a][1]))));
+        }
+    }
+}
+
+// acc[b][e] += sgn * sum_r X[r * XL + j_b] * Y[r * L4 + c0 + e] for the thread's state rows j_b
+template <int D, int JPT>
+__device__ __forceinline__ void outer_rows(float (&acc)[JPT][8], const float *X, int XL, const float *Y, int jb0,
+                                           int c0, float sgn)
+{
+    constexpr int L4 = D + 4;
+#pragma unroll 4
+    for (int r = 0; r < kC; ++r) {
+        const float4 y0 = *reinterpret_cast<const float4 *>(Y + r * L4 + c0);
+        const float4 y1 = *reinterpret_cast<const float4 *>(Y + r * L4 + c0 + 4);
+#pragma unroll
+        for (int b = 0; b < JPT; ++b) {
+            const float x = sgn * X[r * XL + jb0 + b];
+            acc[b][0] = fmaf(x, y0.x, acc[b][0]);
+            acc[b][1] = fmaf(x, y0.y, acc[b][1]);
+            acc[b][2] = fmaf(x, y0.z, acc[b][2]);
+            acc[b][3] = fmaf(x, y0.w, acc[b][3]);
+            acc[b][4] = fmaf(x, y1.x, acc[b][4]);
+            acc[b][5] = fmaf(x, y1.y, acc[b][5]);
+            acc[b][6] = fmaf(x, y1.z, acc[b][6]);
+            acc[b][7] = fmaf(x, y1.w, acc[b][7]);
+        }
+    }
 }
 
 template <int D>
@@ -222,60 +273,66 @@ __global__ void __launch_bounds__(kBT)
 bwd_fwd_scan(const float *__restrict__ S0, BwdWs w, int nch)
 {
     using L = FwdSmem<D>;
-    constexpr int LD = L::LD, RS = kBT / D, NJ = kTile / RS;
+    constexpr int L4 = D + 4, TL = kTile + 1;
+    constexpr int NCG = D / 8, JPT = kTile * NCG / kBT;   // state update: 8 channels x JPT state rows per thread
     extern __shared__ float sm[];
     float *sS = sm + L::S, *sW = sm + L::W, *sKt = sm + L::KT, *sVn = sm + L::VN, *gc = sm + L::GC;
     const int tid = threadIdx.x;
     const int head = blockIdx.x, i0 = blockIdx.y * kTile;
-#pragma unroll 8
     for (int idx = tid; idx < kTile * D; idx += kBT) {
         const int j = idx / D, c = idx - j * D;
-        sS[j * LD + c] = S0 ? S0[((size_t)head * D + i0 + j) * D + c] : 0.f;
+        sS[j * L4 + c] = S0 ? S0[((size_t)head * D + i0 + j) * D + c] : 0.f;
     }
-    const int c = tid % D, h = tid / D;
-    const int vj = tid & 31, vr = tid >> 5;   // V_new: column (state row) vj, rows vr + 8 m
+    const int vj = tid & 15, vr = 4 * (tid >> 4);               // V_new: rows vr..vr+3, state rows vj, vj+16
+    const int cg = tid % NCG, jb0 = JPT * (tid / NCG), c0 = 8 * cg;   // update: channels c0..c0+7
     for (int n = 0; n < nch; ++n) {
         const size_t prow0 = (size_t)head * nch * kC + (size_t)n * kC;
         __syncthreads();
         float *ck = w.Sck + ((size_t)(head * nch + n) * D + i0) * D;
-#pragma unroll 8
-        for (int idx = tid; idx < kTile * D; idx += kBT) ck[idx] = sS[(idx / D) * LD + idx % D];
-#pragma unroll 8
-        for (int idx = tid; idx < kC * D; idx += kBT) sW[(idx / D) * LD + idx % D] = w.W[(prow0 + idx / D) * D + idx % D];
+        for (int idx = tid; idx < kTile * D; idx += kBT) ck[idx] = sS[(idx / D) * L4 + idx % D];
+#pragma unroll 4
+        for (int idx = tid; idx < kC * D / 4; idx += kBT) {
+            const int r = idx / (D / 4), c4 = idx - r * (D / 4);
+            *reinterpret_cast<float4 *>(sW + r * L4 + 4 * c4) = *reinterpret_cast<const float4 *>(w.W + (prow0 + r) * D + 4 * c4);
+        }
         load_ktail<D>(sKt, gc, w, prow0, tid);
         __syncthreads();
         // V_new = U - W S^T (this tile's d_v columns)
+        {
+            float acc[4][2] = {};
+            dot_4x2<D>(acc, sW, vr, sS, vj, vj + 16);
 #pragma unroll
-        for (int m = 0; m < 8; ++m) {
-            const int r = vr + 8 * m;
-            float acc = w.U[(prow0 + r) * D + i0 + vj];
-            for (int cc = 0; cc < D; ++cc) acc = fmaf(-sW[r * LD + cc], sS[vj * LD + cc], acc);
-            sVn[r * (kTile + 1) + vj] = acc;
-            w.Vn[(prow0 + r) * D + i0 + vj] = acc;
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int b = 0; b < 2; ++b) {
+                    const int r = vr + a, j = vj + 16 * b;
+                    const float x = w.U[(prow0 + r) * D + i0 + j] - acc[a][b];
+                    sVn[r * TL + j] = x;
+                    w.Vn[(prow0 + r) * D + i0 + j] = x;
+                }
         }
         __syncthreads();
         // S <- S Diag(gamma_C) + V_new^T K_tail
-        float acc[NJ];
-        const float gcc = __expf(gc[c]);
+        float acc[JPT][8];
 #pragma unroll
-        for (int m = 0; m < NJ; ++m) acc[m] = sS[(h + RS * m) * LD + c] * gcc;
-        for (int r = 0; r < kC; ++r) {
-            const float kt = sKt[r * LD + c];
+        for (int b = 0; b < JPT; ++b)
 #pragma unroll
-            for (int m = 0; m < NJ; ++m) acc[m] = fmaf(sVn[r * (kTile + 1) + h + RS * m], kt, acc[m]);
-        }
+            for (int e = 0; e < 8; ++e) acc[b][e] = sS[(jb0 + b) * L4 + c0 + e] * __expf(gc[c0 + e]);
+        outer_rows<D, JPT>(acc, sVn, TL, sKt, jb0, c0, 1.f);
         __syncthreads();
 #pragma unroll
-        for (int m = 0; m < NJ; ++m) sS[(h + RS * m) * LD + c] = acc[m];
+        for (int b = 0; b < JPT; ++b)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) sS[(jb0 + b) * L4 + c0 + e] = acc[b][e];
     }
 }
 
 // ------------------------------------------------------------------ 3. reverse state scan
 template <int D>
 struct RevSmem {
-    static constexpr int LD = D + 1;
-    static constexpr int DS = 0, AQ = DS + kTile * LD, DO = AQ + kC * 65, DVN = DO + kC * (kTile + 1),
-                         KT = DVN + kC * (kTile + 1), GC = KT + kC * LD;
+    static constexpr int L4 = D + 4;
+    static constexpr int DS = 0, AQ = DS + kTile * L4, DO = AQ + kC * 68, DVN = DO + kC * (kTile + 1),
+                         KT = DVN + kC * (kTile + 1), GC = KT + kC * L4;
     static constexpr int TOTAL = GC + D;
 };
 
@@ -285,29 +342,29 @@ bwd_rev_scan(const T *__restrict__ dOg, const float *__restrict__ dST, float *__
              int nch)
 {
     using L = RevSmem<D>;
-    constexpr int LD = L::LD, RS = kBT / D, NJ = kTile / RS, TL = kTile + 1;
+    constexpr int L4 = D + 4, TL = kTile + 1;
+    constexpr int NCG = D / 8, JPT = kTile * NCG / kBT;
     extern __shared__ float sm[];
     float *sdS = sm + L::DS, *sAq = sm + L::AQ, *sdO = sm + L::DO, *sdVn = sm + L::DVN, *sKt = sm + L::KT,
           *gc = sm + L::GC;
     const int tid = threadIdx.x;
     const int head = blockIdx.x, i0 = blockIdx.y * kTile;
-#pragma unroll 8
     for (int idx = tid; idx < kTile * D; idx += kBT) {
         const int j = idx / D, c = idx - j * D;
-        sdS[j * LD + c] = dST ? dST[((size_t)head * D + i0 + j) * D + c] : 0.f;
+        sdS[j * L4 + c] = dST ? dST[((size_t)head * D + i0 + j) * D + c] : 0.f;
     }
-    const int c = tid % D, h = tid / D;
-    const int vj = tid & 31, vr = tid >> 5;
+    const int vj = tid & 15, vr = 4 * (tid >> 4);
+    const int cg = tid % NCG, jb0 = JPT * (tid / NCG), c0 = 8 * cg;
     for (int n = nch - 1; n >= 0; --n) {
         const int t0 = n * kC, nrows = min(kC, T_len - t0);
         const size_t row0 = (size_t)head * T_len + t0, prow0 = (size_t)head * nch * kC + t0;
         __syncthreads();
         float *ck = w.dSck + ((size_t)(head * nch + n) * D + i0) * D;
-#pragma unroll 8
-        for (int idx = tid; idx < kTile * D; idx += kBT) ck[idx] = sdS[(idx / D) * LD + idx % D];
+        for (int idx = tid; idx < kTile * D; idx += kBT) ck[idx] = sdS[(idx / D) * L4 + idx % D];
         const float *aq = w.Aq + (size_t)(head * nch + n) * kC * kC;
-#pragma unroll 8
-        for (int idx = tid; idx < kC * kC; idx += kBT) sAq[(idx >> 6) * 65 + (idx & 63)] = aq[idx];
+#pragma unroll 4
+        for (int idx = tid; idx < kC * kC / 4; idx += kBT)
+            *reinterpret_cast<float4 *>(sAq + (idx >> 4) * 68 + 4 * (idx & 15)) = *reinterpret_cast<const float4 *>(aq + 4 * idx);
 #pragma unroll 8
         for (int idx = tid; idx < kC * kTile; idx += kBT) {
             const int r = idx / kTile, j = idx - r * kTile;
@@ -315,48 +372,63 @@ bwd_rev_scan(const T *__restrict__ dOg, const float *__restrict__ dST, float *__
         }
         load_ktail<D>(sKt, gc, w, prow0, tid);
         __syncthreads();
-        // dV_new = Aqk^T dO + K_tail dS^T
+        // dV_new = Aqk^T dO + K_tail dS^T  (Aqk is zero above the diagonal)
+        {
+            float acc[4][2] = {};
+            dot_4x2<D>(acc, sKt, vr, sdS, vj, vj + 16);
+            for (int i = vr; i < kC; ++i) {
+                const float4 aqv = *reinterpret_cast<const float4 *>(sAq + i * 68 + vr);
+                const float d0 = sdO[i * TL + vj], d1 = sdO[i * TL + vj + 16];
+                acc[0][0] = fmaf(aqv.x, d0, acc[0][0]);
+                acc[0][1] = fmaf(aqv.x, d1, acc[0][1]);
+                acc[1][0] = fmaf(aqv.y, d0, acc[1][0]);
+                acc[1][1] = fmaf(aqv.y, d1, acc[1][1]);
+                acc[2][0] = fmaf(aqv.z, d0, acc[2][0]);
+                acc[2][1] = fmaf(aqv.z, d1, acc[2][1]);
+                acc[3][0] = fmaf(aqv.w, d0, acc[3][0]);
+                acc[3][1] = fmaf(aqv.w, d1, acc[3][1]);
+            }
 #pragma unroll
-        for (int m = 0; m < 8; ++m) {
-            const int r = vr + 8 * m;
-            float acc = 0.f;
-            for (int i = r; i < kC; ++i) acc = fmaf(sAq[i * 65 + r], sdO[i * TL + vj], acc);
-            for (int cc = 0; cc < D; ++cc) acc = fmaf(sKt[r * LD + cc], sdS[vj * LD + cc], acc);
-            sdVn[r * TL + vj] = acc;
-            w.dVn[(prow0 + r) * D + i0 + vj] = acc;
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int b = 0; b < 2; ++b) {
+                    const int r = vr + a, j = vj + 16 * b;
+                    sdVn[r * TL + j] = acc[a][b];
+                    w.dVn[(prow0 + r) * D + i0 + j] = acc[a][b];
+                }
         }
         __syncthreads();
         // dS <- dS Diag(gamma_C) + dO^T Q<- - dV_new^T W  (Q<-, then W, staged in the K_tail buffer)
-        float acc[NJ];
-        const float gcc = __expf(gc[c]);
+        float acc[JPT][8];
 #pragma unroll
-        for (int m = 0; m < NJ; ++m) acc[m] = sdS[(h + RS * m) * LD + c] * gcc;
-#pragma unroll 8
-        for (int idx = tid; idx < kC * D; idx += kBT) sKt[(idx / D) * LD + idx % D] = w.Ql[(prow0 + idx / D) * D + idx % D];
-        __syncthreads();
-        for (int r = 0; r < kC; ++r) {
-            const float ql = sKt[r * LD + c];
+        for (int b = 0; b < JPT; ++b)
 #pragma unroll
-            for (int m = 0; m < NJ; ++m) acc[m] = fmaf(sdO[r * TL + h + RS * m], ql, acc[m]);
+            for (int e = 0; e < 8; ++e) acc[b][e] = sdS[(jb0 + b) * L4 + c0 + e] * __expf(gc[c0 + e]);
+#pragma unroll 4
+        for (int idx = tid; idx < kC * D / 4; idx += kBT) {
+            const int r = idx / (D / 4), c4 = idx - r * (D / 4);
+            *reinterpret_cast<float4 *>(sKt + r * L4 + 4 * c4) = *reinterpret_cast<const float4 *>(w.Ql + (prow0 + r) * D + 4 * c4);
         }
         __syncthreads();
-#pragma unroll 8
-        for (int idx = tid; idx < kC * D; idx += kBT) sKt[(idx / D) * LD + idx % D] = w.W[(prow0 + idx / D) * D + idx % D];
+        outer_rows<D, JPT>(acc, sdO, TL, sKt, jb0, c0, 1.f);
         __syncthreads();
-        for (int r = 0; r < kC; ++r) {
-            const float wv = sKt[r * LD + c];
-#pragma unroll
-            for (int m = 0; m < NJ; ++m) acc[m] = fmaf(-sdVn[r * TL + h + RS * m], wv, acc[m]);
+#pragma unroll 4
+        for (int idx = tid; idx < kC * D / 4; idx += kBT) {
+            const int r = idx / (D / 4), c4 = idx - r * (D / 4);
+            *reinterpret_cast<float4 *>(sKt + r * L4 + 4 * c4) = *reinterpret_cast<const float4 *>(w.W + (prow0 + r) * D + 4 * c4);
         }
         __syncthreads();
+        outer_rows<D, JPT>(acc, sdVn, TL, sKt, jb0, c0, -1.f);
+        __syncthreads();
 #pragma unroll
-        for (int m = 0; m < NJ; ++m) sdS[(h + RS * m) * LD + c] = acc[m];
+        for (int b = 0; b < JPT; ++b)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) sdS[(jb0 + b) * L4 + c0 + e] = acc[b][e];
     }
     __syncthreads();
     if (dS0)
-#pragma unroll 8
         for (int idx = tid; idx < kTile * D; idx += kBT)
-            dS0[((size_t)head * D + i0 + idx / D) * D + idx % D] = sdS[(idx / D) * LD + idx % D];
+            dS0[((size_t)head * D + i0 + idx / D) * D + idx % D] = sdS[(idx / D) * L4 + idx % D];
 }
 
 // ------------------------------------------------------------------ 4. per-chunk gradients

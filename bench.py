@@ -59,9 +59,9 @@ TRAFFIC = {
     "kda_d128_t8192_gated": {"src_sha": "fe8676200985376b", "bytes_per_launch": 1986628864},
     # Gated Delta Rule-2: ut_prep 1394.0 + 634.1 MB (reads b, v, w; writes w * v), chunk_scan 679.6 + 118.5 MB
     "gdr2_d128_t8192": {"src_sha": "fe8676200985376b", "bytes_per_launch": 2826130432},
-    # backward: bwd_prep 675.0 + 1553.2, bwd_fwd_scan 1521.9 + 777.1, bwd_rev_scan 2449.8 + 789.2,
-    # bwd_grads 2827.1 + 651.4 MB
-    "kda_d128_t8192_bwd": {"src_sha": "79812d6152006030", "bytes_per_launch": 11244719872},
+    # backward: bwd_prep 674.2 + 1553.4, bwd_fwd_scan 1142.5 + 771.5, bwd_rev_scan 1645.5 + 780.4,
+    # bwd_grads 2826.6 + 651.5 MB
+    "kda_d128_t8192_bwd": {"src_sha": "6be716bedd859aa1", "bytes_per_launch": 10045581824},
     # recurrent_step, one decode step: 547.4 MB read + 477.8 MB written
     "kda_decode_b256": {"src_sha": "13bedf0248f32e59", "bytes_per_launch": 1025204480},
 }

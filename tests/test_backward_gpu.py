@@ -86,3 +86,22 @@ def test_full_size_sampled():
                           sel(gr["dO"]), sel(gr["dS_T"]))
     errs = {n: relerr(sel(a), b) for n, a, b in zip(NAMES, got, ref)}
     assert all(e <= 2e-2 for e in errs.values()), errs
+
+
+def test_empty_problems():
+    dev = torch.device("cuda")
+    # T = 0: S_T = S0, so dS0 = dS_T (zeros without dS_T)
+    e = torch.empty(1, 2, 0, 128, dtype=torch.bfloat16, device=dev)
+    g = torch.empty(1, 2, 0, 128, device=dev)
+    b = torch.empty(1, 2, 0, device=dev)
+    dST = torch.randn(1, 2, 128, 128, device=dev)
+    out = gdr.chunk_bwd(e, e, e, g, b, e, dS_T=dST)
+    torch.cuda.synchronize()
+    assert torch.equal(out[5], dST) and out[0].numel() == 0
+    out = gdr.chunk_bwd(e, e, e, g, b, e)
+    torch.cuda.synchronize()
+    assert float(out[5].abs().max()) == 0.0
+    # B = 0
+    z = torch.empty(0, 2, 64, 128, dtype=torch.bfloat16, device=dev)
+    out = gdr.chunk_bwd(z, z, z, torch.empty(0, 2, 64, 128, device=dev), torch.empty(0, 2, 64, device=dev), z)
+    assert out[0].shape == (0, 2, 64, 128)

@@ -153,3 +153,12 @@ def test_decode_full_size_sampled():
                                       pick(d0["S0"]).cpu()[:, None])
     assert relerr(torch.stack(hist["o"]), o_ref[:, :, 0]) <= 2e-2
     assert relerr(pick(S).cpu(), S_ref[:, 0]) <= 2e-2
+
+
+def test_empty_problems():
+    dev = torch.device("cuda")
+    S0 = torch.randn(1, 2, 128, 128, device=dev)
+    e = torch.empty(1, 2, 0, 128, dtype=torch.bfloat16, device=dev)
+    O, S = gdr.chunk_fwd_gdr2(e, e, e, torch.empty(1, 2, 0, 128, device=dev), e, e, S0)
+    torch.cuda.synchronize()
+    assert O.numel() == 0 and torch.equal(S, S0)

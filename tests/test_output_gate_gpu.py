@@ -111,3 +111,13 @@ def test_full_size_sampled():
     ey = gated_err(sel(Y), Y_ref, O_ref, sel(d["ogate"]), d["norm_w"], 1e-6)
     es = relerr(sel(S), S_ref)
     assert ey <= 2e-2 and es <= 2e-2, (ey, es, relerr(sel(Y), Y_ref))
+
+
+def test_empty_problems():
+    dev = torch.device("cuda")
+    S0 = torch.randn(1, 2, 128, 128, device=dev)
+    e = torch.empty(1, 2, 0, 128, dtype=torch.bfloat16, device=dev)
+    Y, S = gdr.chunk_fwd_gated(e, e, e, torch.empty(1, 2, 0, 128, device=dev), torch.empty(1, 2, 0, device=dev), e,
+                               torch.ones(128, device=dev), 1e-6, S0)
+    torch.cuda.synchronize()
+    assert Y.numel() == 0 and torch.equal(S, S0)

@@ -44,6 +44,7 @@ import gdr_workloads as W  # noqa: E402
 
 METRIC = "tokens/s (device-timed) of gated-delta-rule chunk fwd; % of roofline"
 METRIC_DECODE = "tokens/s (device-timed) of gated-delta-rule recurrent decode step; % of HBM roofline"
+METRIC_BWD = "tokens/s (device-timed) of gated-delta-rule chunk backward; % of roofline"
 DEFAULT_WORKLOAD = "kda_d128_t8192"
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per call of the
@@ -364,7 +365,7 @@ def parse():
 
 def base_line(w: W.Workload, args, world: int):
     return {
-        "metric": METRIC_DECODE if w.kind == "decode" else METRIC,
+        "metric": METRIC_DECODE if w.kind == "decode" else METRIC_BWD if w.direction == "bwd" else METRIC,
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,

@@ -52,14 +52,14 @@ DEFAULT_WORKLOAD = "kda_d128_t8192"
 # workload with the hash of the sources those kernels are built from; an
 # entry is ignored (traffic = null) as soon as any of the sources changes.
 TRAFFIC = {
-    # ut_prep 558.8 MB read + 494.9 MB written, chunk_scan 679.6 + 118.8 MB (one launch each)
-    "kda_d128_t8192": {"src_sha": "fe8676200985376b", "bytes_per_launch": 1852187392},
-    # fused input prologue: ut_prep 409.8 + 488.6 MB, chunk_scan 679.6 + 118.9 MB
-    "kda_d128_t8192_prologue": {"src_sha": "fe8676200985376b", "bytes_per_launch": 1696968960},
-    # gated output: the scan also reads the gate tiles (813.9 + 120.4 MB); ut_prep 558.5 + 493.8 MB
-    "kda_d128_t8192_gated": {"src_sha": "fe8676200985376b", "bytes_per_launch": 1986628864},
-    # Gated Delta Rule-2: ut_prep 1394.0 + 634.1 MB (reads b, v, w; writes w * v), chunk_scan 679.6 + 118.5 MB
-    "gdr2_d128_t8192": {"src_sha": "fe8676200985376b", "bytes_per_launch": 2826130432},
+    # ut_prep 559.9 MB read + 494.0 MB written, chunk_scan 679.7 + 118.2 MB (one launch each)
+    "kda_d128_t8192": {"src_sha": "8246377c36975a52", "bytes_per_launch": 1851855360},
+    # fused input prologue: ut_prep 408.0 + 488.7 MB, chunk_scan 679.6 + 118.8 MB
+    "kda_d128_t8192_prologue": {"src_sha": "8246377c36975a52", "bytes_per_launch": 1695170816},
+    # gated output: the scan also reads the gate tiles (813.9 + 120.5 MB); ut_prep 558.8 + 493.7 MB
+    "kda_d128_t8192_gated": {"src_sha": "8246377c36975a52", "bytes_per_launch": 1986893312},
+    # Gated Delta Rule-2: ut_prep 1115.3 + 634.3 MB (reads b, v, w; writes w * v), chunk_scan 679.6 + 118.3 MB
+    "gdr2_d128_t8192": {"src_sha": "8246377c36975a52", "bytes_per_launch": 2547477760},
     # backward: bwd_prep 674.2 + 1553.4, bwd_fwd_scan 1142.5 + 771.5, bwd_rev_scan 1645.5 + 780.4,
     # bwd_grads 2826.6 + 651.5 MB
     "kda_d128_t8192_bwd": {"src_sha": "6be716bedd859aa1", "bytes_per_launch": 10045581824},

@@ -257,11 +257,7 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
                 if (PRO) bulk_prefetch_l2(static_cast<const __nv_bfloat16 *>(gin) + rown * kDK, (uint32_t)rn * kDK * 2);
                 else bulk_prefetch_l2(static_cast<const float *>(gin) + rown * kDK, (uint32_t)rn * kDK * 4);
             }
-            if (GDR2) {
-                bulk_prefetch_l2(erg + rown * kDK, (uint32_t)rn * kDK * 2);
-                bulk_prefetch_l2(vg + rown * kDK, (uint32_t)rn * kDK * 2);
-                bulk_prefetch_l2(wrg + rown * kDK, (uint32_t)rn * kDK * 2);
-            }
+            if (GDR2) bulk_prefetch_l2(erg + rown * kDK, (uint32_t)rn * kDK * 2);   // (v, w are read later, once)
         }
         const size_t cbase = (size_t)ci * kC * kC;       // this chunk's T' and Aqk
         // beta alternates between two buffers: the last T' stores of the

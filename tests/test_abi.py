@@ -146,6 +146,31 @@ def test_gated_argument_validation(L):
     assert gated(L, T=0) == OK
 
 
+def bwd(L, B=1, H=1, T=64, d=128, C=64, gate=0, dtype=1, ptr=GOOD, dST=None, dS0=None, ws=1 << 40, wsp=GOOD):
+    return L.gdr_chunk_bwd(ptr, ptr, ptr, ptr, ptr, None, ptr, dST, ptr, ptr, ptr, ptr, ptr, dS0,
+                           B, H, T, d, d, C, gate, dtype, wsp, ws, None)
+
+
+def test_backward_argument_validation(L):
+    assert bwd(L, B=-1) == INVALID
+    assert bwd(L, gate=2) == INVALID
+    assert bwd(L, dtype=3) == INVALID
+    assert bwd(L, d=96) == UNSUPPORTED
+    assert bwd(L, C=32) == UNSUPPORTED
+    assert L.gdr_chunk_bwd(GOOD, GOOD, GOOD, GOOD, GOOD, None, GOOD, None, GOOD, GOOD, GOOD, GOOD, GOOD, None,
+                           1, 1, 64, 128, 64, 64, 0, 1, GOOD, 1 << 40, None) == UNSUPPORTED   # d_k != d_v
+    assert bwd(L, ptr=ODD) == ALIGN
+    assert bwd(L, dS0=ODD) == ALIGN
+    assert bwd(L, wsp=None) == INVALID
+    need = L.gdr_chunk_bwd_workspace_size(1, 1, 64, 128, 128, 64, 0, 1)
+    # per 64-token chunk: G, W, U, V_new, dV_new, K_tail, Q<- (64 x 128 fp32 each),
+    # (I + A)^{-1} and Aqk (64 x 64 fp32), the state and its gradient (128 x 128 fp32)
+    assert need == 4 * (7 * 64 * 128 + 2 * 64 * 64 + 2 * 128 * 128)
+    assert bwd(L, ws=need - 1) == INVALID
+    assert L.gdr_chunk_bwd_workspace_size(1, 1, 64, 128, 128, 32, 0, 1) == 0
+    assert bwd(L, B=0) == OK and L.gdr_last_launch_count() == 0
+
+
 def test_step_argument_validation(L):
     def step(B=2, H=2, dk=128, dv=128, gate=0, dtype=1, ptr=GOOD):
         return L.gdr_recurrent_step(ptr, ptr, ptr, ptr, ptr, ptr, ptr, B, H, dk, dv, gate, dtype, None)

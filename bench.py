@@ -60,9 +60,9 @@ TRAFFIC = {
     "kda_d128_t8192_gated": {"src_sha": "8246377c36975a52", "bytes_per_launch": 1986893312},
     # Gated Delta Rule-2: ut_prep 1115.3 + 634.3 MB (reads b, v, w; writes w * v), chunk_scan 679.6 + 118.3 MB
     "gdr2_d128_t8192": {"src_sha": "8246377c36975a52", "bytes_per_launch": 2547477760},
-    # backward: bwd_prep 674.2 + 1553.4, bwd_fwd_scan 1142.5 + 771.5, bwd_rev_scan 1645.5 + 780.4,
-    # bwd_grads 2826.6 + 651.5 MB
-    "kda_d128_t8192_bwd": {"src_sha": "6be716bedd859aa1", "bytes_per_launch": 10045581824},
+    # backward: bwd_prep 675.1 + 1553.3, bwd_fwd_scan 1126.1 + 771.1, bwd_rev_scan 1643.4 + 779.4,
+    # bwd_grads 2825.2 + 653.2 MB
+    "kda_d128_t8192_bwd": {"src_sha": "767fb4d511b44a85", "bytes_per_launch": 10026771200},
     # recurrent_step, one decode step: 547.4 MB read + 477.8 MB written
     "kda_decode_b256": {"src_sha": "13bedf0248f32e59", "bytes_per_launch": 1025204480},
 }

@@ -656,39 +656,66 @@ bwd_grads(const T *__restrict__ qg, const T *__restrict__ kg, const T *__restric
         sP[r * 65 + pi] = -acc;   // dA (zero on and above the diagonal)
     }
     __syncthreads();
-    // decay-weighted contractions of dA (A_ri = beta_r sum_c k_rc k_ic E) and dAqk
+    // decay-weighted contractions of dA (A_ri = beta_r sum_c k_rc k_ic E) and dAqk,
+    // four of the thread's rows at a time so the per-channel operands are read once
+    // for all four.  A row's terms past its own r are dropped (a select, so an
+    // exponential that overflows there never meets the zero it is multiplied by).
     // row side: (r, c) collects over i <= r
     float xb[NR];
 #pragma unroll
-    for (int m = 0; m < NR; ++m) {
-        const int r = h + RS * m;
-        const float gr = sG[r * LD + c], kr = sk[r * LD + c], qr = sq[r * LD + c], br = sb[r];
-        float sdk = 0.f, sdq = 0.f, sx = 0.f, sxq = 0.f;
-        for (int i = 0; i <= r; ++i) {
-            const float kie = sk[i * LD + c] * __expf(gr - sG[i * LD + c]);
-            const float a = sP[r * 65 + i], b = sR[r * 65 + i];
-            sdk = fmaf(a, kie, sdk);
-            sdq = fmaf(b, kie, sdq);
+    for (int m0 = 0; m0 < NR; m0 += 4) {
+        float gr[4], sdk[4], sdq[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            gr[u] = sG[(h + RS * (m0 + u)) * LD + c];
+            sdk[u] = sdq[u] = 0.f;
         }
-        sx = sdk * kr;    // sum_i dA_ri k_rc k_ic E
-        sxq = sdq * qr;   // sum_i dAqk_ri q_rc k_ic E
-        dk[m] = fmaf(br, sdk, dk[m]);
-        dq[m] += sdq;
-        dG[m] += br * sx + sxq;
-        xb[m] = sx;
+        const int rmax = h + RS * (m0 + 3);
+        for (int i = 0; i <= rmax; ++i) {
+            const float ki = sk[i * LD + c], gi = sG[i * LD + c];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int r = h + RS * (m0 + u);
+                const float kie = i <= r ? ki * __expf(gr[u] - gi) : 0.f;
+                sdk[u] = fmaf(sP[r * 65 + i], kie, sdk[u]);
+                sdq[u] = fmaf(sR[r * 65 + i], kie, sdq[u]);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int m = m0 + u, r = h + RS * m;
+            const float sx = sdk[u] * sk[r * LD + c];    // sum_i dA_ri k_rc k_ic E
+            const float sxq = sdq[u] * sq[r * LD + c];   // sum_i dAqk_ri q_rc k_ic E
+            dk[m] = fmaf(sb[r], sdk[u], dk[m]);
+            dq[m] += sdq[u];
+            dG[m] += sb[r] * sx + sxq;
+            xb[m] = sx;
+        }
     }
     // column side: (i, c) collects over r >= i
 #pragma unroll
-    for (int m = 0; m < NR; ++m) {
-        const int i = h + RS * m;
-        const float gi = sG[i * LD + c], ki = sk[i * LD + c];
-        float sa = 0.f;
-        for (int r = i; r < kC; ++r) {
-            const float e = __expf(sG[r * LD + c] - gi);
-            sa = fmaf(sb[r] * sP[r * 65 + i] * sk[r * LD + c] + sR[r * 65 + i] * sq[r * LD + c], e, sa);
+    for (int m0 = 0; m0 < NR; m0 += 4) {
+        float gi[4], sa[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            gi[u] = sG[(h + RS * (m0 + u)) * LD + c];
+            sa[u] = 0.f;
         }
-        dk[m] += sa;
-        dG[m] = fmaf(-sa, ki, dG[m]);
+        for (int r = h + RS * m0; r < kC; ++r) {
+            const float gr = sG[r * LD + c], bk = sb[r] * sk[r * LD + c], qr = sq[r * LD + c];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = h + RS * (m0 + u);
+                const float e = r >= i ? __expf(gr - gi[u]) : 0.f;
+                sa[u] = fmaf(bk * sP[r * 65 + i] + sR[r * 65 + i] * qr, e, sa[u]);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int m = m0 + u;
+            dk[m] += sa[u];
+            dG[m] = fmaf(-sa[u], sk[(h + RS * m) * LD + c], dG[m]);
+        }
     }
     // dbeta_r += sum_c xb  (lanes, then the warps that share the rows)
 #pragma unroll

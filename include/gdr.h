@@ -197,7 +197,7 @@ int gdr_chunk_fwd_gated(const void *q, const void *k, const void *v, const float
  * returns GDR_ERR_UNSUPPORTED.  The workspace (device, >=
  * gdr_chunk_bwd_workspace_size() bytes, 16-byte aligned) holds the
  * recomputed chunk quantities and the per-chunk states and state gradients:
- * about 320 KB per 64-token chunk at d = 128.
+ * 384 KB per 64-token chunk at d = 128.
  */
 size_t gdr_chunk_bwd_workspace_size(int B, int H, int T, int dk, int dv, int C, int gate_mode, int dtype);
 

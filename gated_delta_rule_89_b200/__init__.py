@@ -133,6 +133,18 @@ def _to_device(x, device):
     return None if x is None else x.to(device, non_blocking=True)
 
 
+def _to_host(x):
+    """Device tensor -> page-locked host tensor.  The device is synchronized
+    first (the kernels may run on a stream other than the current one); the
+    copy into pinned memory then runs at the full DMA rate."""
+    if x is None:
+        return None
+    torch.cuda.synchronize(x.device)
+    h = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+    h.copy_(x)
+    return h
+
+
 def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor, beta: torch.Tensor,
               S0: Optional[torch.Tensor] = None, C: int = 64, gate: Optional[str] = None,
               O: Optional[torch.Tensor] = None, S_T: Optional[torch.Tensor] = None,
@@ -188,8 +200,8 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor
                          _ptr(workspace) if ws_bytes else None, ws_bytes, _stream_handle(dev, stream))
     _check(st, "gdr_chunk_fwd")
     if host:
-        O = O.to("cpu")
-        S_T = None if S_T is None else S_T.to("cpu")
+        O = _to_host(O)
+        S_T = _to_host(S_T)
     return O, S_T
 
 
@@ -252,8 +264,8 @@ def chunk_fwd_prologue(q_raw: torch.Tensor, k_raw: torch.Tensor, v: torch.Tensor
                                   _ptr(workspace) if ws_bytes else None, ws_bytes, _stream_handle(dev, stream))
     _check(st, "gdr_chunk_fwd_prologue")
     if host:
-        O = O.to("cpu")
-        S_T = None if S_T is None else S_T.to("cpu")
+        O = _to_host(O)
+        S_T = _to_host(S_T)
     return O, S_T
 
 
@@ -344,8 +356,8 @@ def chunk_fwd_gdr2(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.T
                           _ptr(workspace) if ws_bytes else None, ws_bytes, _stream_handle(dev, stream))
     _check(st, "gdr2_chunk_fwd")
     if host:
-        O = O.to("cpu")
-        S_T = None if S_T is None else S_T.to("cpu")
+        O = _to_host(O)
+        S_T = _to_host(S_T)
     return O, S_T
 
 
@@ -437,8 +449,8 @@ def chunk_fwd_gated(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.
                                _ptr(workspace) if ws_bytes else None, ws_bytes, _stream_handle(dev, stream))
     _check(st, "gdr_chunk_fwd_gated")
     if host:
-        Y = Y.to("cpu")
-        S_T = None if S_T is None else S_T.to("cpu")
+        Y = _to_host(Y)
+        S_T = _to_host(S_T)
     return Y, S_T
 
 
@@ -492,7 +504,7 @@ def chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor
     _check(st, "gdr_chunk_bwd")
     out = (dq, dk_, dv_, dg, dbeta, dS0)
     if host:
-        out = tuple(None if t is None else t.to("cpu") for t in out)
+        out = tuple(_to_host(t) for t in out)
     return out
 
 

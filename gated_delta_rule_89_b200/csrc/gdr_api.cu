@@ -26,6 +26,25 @@ int finish(cudaError_t e, int launches)
 
 bool size_ok(int d) { return d == 64 || d == 128; }
 
+// Debug mode only: GDR_ERR_GATE_RANGE when an element of g is positive or not
+// finite (n elements), GDR_ERR_CUDA when the check itself failed, else GDR_OK.
+int gate_guard(const float *g, size_t n, cudaStream_t st)
+{
+    if (!gdr::debug_checks_enabled()) return GDR_OK;
+    bool bad = false;
+    const cudaError_t e = gdr::check_gate_range(g, n, st, &bad);
+    if (e != cudaSuccess) {
+        tl_last_cuda_error = (int)e;
+        return GDR_ERR_CUDA;
+    }
+    return bad ? GDR_ERR_GATE_RANGE : GDR_OK;
+}
+
+size_t gate_elems(long long heads, int T, int dk, int gate_mode)
+{
+    return (size_t)heads * (size_t)T * (gate_mode == GDR_GATE_PER_CHANNEL ? (size_t)dk : 1u);
+}
+
 }  // namespace
 
 GDR_API const char *gdr_status_string(int status)
@@ -108,6 +127,7 @@ GDR_API int gdr_chunk_fwd(const void *q, const void *k, const void *v, const flo
     a.scalar_gate = (gate_mode == GDR_GATE_SCALAR);
     a.bf16 = (dtype == GDR_BF16);
     a.workspace = workspace;
+    if (const int gs = gate_guard(g, gate_elems(heads, T, dk, gate_mode), st)) return gs;
     int launches = 0;
     cudaError_t e = gdr::chunk_tc_supports(a) ? gdr::launch_chunk_tc(a, st, &launches)
                                               : gdr::launch_chunk_simt(a, st, &launches);
@@ -215,6 +235,7 @@ GDR_API int gdr_chunk_fwd_gated(const void *q, const void *k, const void *v, con
     c.ogate = gate;
     c.norm_w = norm_w;
     c.eps = eps;
+    if (const int gs = gate_guard(g, gate_elems(heads, T, dk, gate_mode), st)) return gs;
     int launches = 0;
     cudaError_t e = gdr::launch_chunk_tc(c, st, &launches);
     return finish(e, launches);
@@ -270,6 +291,7 @@ GDR_API int gdr_chunk_bwd(const void *q, const void *k, const void *v, const flo
     a.scalar_gate = (gate_mode == GDR_GATE_SCALAR);
     a.bf16 = (dtype == GDR_BF16);
     a.workspace = workspace;
+    if (const int gs = gate_guard(g, gate_elems(heads, T, dk_, gate_mode), st)) return gs;
     int launches = 0;
     cudaError_t e = gdr::launch_chunk_bwd(a, st, &launches);
     return finish(e, launches);
@@ -329,6 +351,7 @@ GDR_API int gdr2_chunk_fwd(const void *q, const void *k, const void *v, const fl
     c.gdr2 = true;
     c.erase = b;
     c.write = w;
+    if (const int gs = gate_guard(g, gate_elems(heads, T, dk, gate_mode), st)) return gs;
     int launches = 0;
     cudaError_t e = gdr::launch_chunk_tc(c, st, &launches);
     return finish(e, launches);
@@ -360,8 +383,10 @@ GDR_API int gdr2_recurrent_step(const void *q, const void *k, const void *v, con
     a.gdr2 = true;
     a.erase = b;
     a.write = w;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (const int gs = gate_guard(g, gate_elems((long long)B * H, 1, dk, gate_mode), st)) return gs;
     int launches = 0;
-    cudaError_t e = gdr::launch_recurrent_step(a, static_cast<cudaStream_t>(stream), &launches);
+    cudaError_t e = gdr::launch_recurrent_step(a, st, &launches);
     return finish(e, launches);
 }
 
@@ -388,7 +413,9 @@ GDR_API int gdr_recurrent_step(const void *q, const void *k, const void *v, cons
     a.B = B; a.H = H; a.dk = dk; a.dv = dv;
     a.scalar_gate = (gate_mode == GDR_GATE_SCALAR);
     a.bf16 = (dtype == GDR_BF16);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (const int gs = gate_guard(g, gate_elems((long long)B * H, 1, dk, gate_mode), st)) return gs;
     int launches = 0;
-    cudaError_t e = gdr::launch_recurrent_step(a, static_cast<cudaStream_t>(stream), &launches);
+    cudaError_t e = gdr::launch_recurrent_step(a, st, &launches);
     return finish(e, launches);
 }

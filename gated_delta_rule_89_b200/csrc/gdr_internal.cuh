@@ -115,6 +115,11 @@ bool chunk_tc_supports(const ChunkArgs &a);
 size_t chunk_tc_workspace_bytes(int B, int H, int T, bool gdr2 = false);
 // Synchronizes `stream`, then reads and clears the device status word.
 cudaError_t read_device_status(cudaStream_t stream, int *status);
+// Debug mode (GDR_DEBUG set in the environment, read once): the entry points
+// that take a log-decay gate check its n elements first (finite and <= 0);
+// *bad is set when one is not.  Synchronizes `stream`.
+bool debug_checks_enabled();
+cudaError_t check_gate_range(const float *g, size_t n, cudaStream_t stream, bool *bad);
 
 // The KDA lower bound on the per-channel log-decay.
 constexpr float kGateMin = -5.0f;

@@ -1,9 +1,9 @@
 // gdr_chunk_fwd_noalloc: the chunked forward for callers that cannot
 // allocate device memory.
 //
-// The tensor-core forward needs device scratch between its two kernels (the
-// per-chunk T' and Aqk matrices, 16 KiB per chunk of 64 tokens).  The normal
-// entry point asks the caller for it.  Some callers cannot provide it:
+// The tensor-core forward needs device scratch for what its UT-transform
+// stage hands to its state scan (see gdr_chunk_fwd_workspace_size).  The
+// normal entry point asks the caller for it.  Some callers cannot provide it:
 // real-time or serving loops that forbid allocator calls on their hot path,
 // code that keeps allocator calls out of a region it records as a CUDA graph,
 // and hosts whose device memory is owned by another runtime or a custom pool

@@ -30,6 +30,15 @@
  *   - Supported sizes: d_k, d_v in {64, 128}; chunk C in {16, 32, 64};
  *     any T >= 0, B >= 0, H >= 0.  Other sizes return GDR_ERR_UNSUPPORTED.
  *   - Functions return a gdr_status value as int.
+ *   - Debug mode: when the environment variable GDR_DEBUG is set (to
+ *     anything but "" or "0") at the library's first call, every entry point
+ *     that takes a log-decay g first checks it on the device: a valid gate is
+ *     a finite value <= 0 (alpha = exp(g) in (0, 1]).  The check synchronizes
+ *     `stream`; if an element is positive, NaN or infinite the call returns
+ *     GDR_ERR_GATE_RANGE and launches nothing else.  Per-channel values below
+ *     -5 are legal (the -5 bound clamps them).  Debug mode adds a pass over g
+ *     and a host synchronization per call, so it is not for timed or
+ *     graph-captured code.
  */
 #ifndef GDR_H_
 #define GDR_H_
@@ -46,8 +55,8 @@ typedef enum gdr_status {
     GDR_ERR_UNSUPPORTED = 2,  /* valid but unsupported size (d_k, d_v, C) */
     GDR_ERR_ALIGNMENT = 3,    /* a tensor pointer is not 16-byte aligned */
     GDR_ERR_CUDA = 4,         /* a CUDA call failed; see gdr_last_cuda_error() */
-    GDR_ERR_GATE_RANGE = 5,   /* reserved: gate outside its domain */
-    GDR_ERR_TIMEOUT = 6       /* reserved: a bounded device wait ran out */
+    GDR_ERR_GATE_RANGE = 5,   /* debug mode (GDR_DEBUG): an element of g is > 0, NaN or infinite */
+    GDR_ERR_TIMEOUT = 6       /* a bounded device wait ran out (see gdr_device_status) */
 } gdr_status;
 
 typedef enum gdr_dtype { GDR_F32 = 0, GDR_BF16 = 1 } gdr_dtype;

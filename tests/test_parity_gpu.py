@@ -5,7 +5,10 @@ oracle reads the exact bf16 / fp32 values the device receives).  Metric:
 max|X - X_ref| / max|X_ref| over every element of O and S_T, with the
 tolerances the workloads state: 1e-5 for fp32 inputs, 2e-2 for bf16 inputs
 with an fp32 state.  Full-size workloads run exactly as bench.py launches
-them and are compared on sampled heads, plus finiteness everywhere.
+them and are compared over every element (the oracle runs over batches of
+heads).  The special cases the pages reduce the method to (no decay with
+beta = 1 and orthonormal keys, the -5 gate bound on every channel, beta = 1)
+run on the device too.
 """
 import numpy as np
 import pytest
@@ -113,6 +116,70 @@ def test_empty_and_degenerate():
     assert relerr(O, O_ref) <= 2e-2 and relerr(S, S_ref) <= 2e-2
 
 
+def _orthonormal_keys(n, dk, seed):
+    """n <= dk orthonormal rows (fp64 QR of a seeded Gaussian matrix)."""
+    gen = torch.Generator().manual_seed(seed)
+    m = torch.randn(dk, dk, generator=gen, dtype=torch.float64)
+    qm, _ = torch.linalg.qr(m)
+    return qm[:n]
+
+
+# The reductions the pages state, on the device.  "retrieval": no decay
+# (g = 0), beta = 1, orthonormal keys and S0 = 0, so every write overwrites its
+# own key direction and S_T k_i returns v_i ("Token Mixer I", the DeltaNet
+# section, and the overwrite property of "Gated DeltaNet-2", Preliminary).
+# "gmin": every channel and token at the KDA bound g = -5 (and below it,
+# clamped), the largest decay spread a 16-token sub-block can see.  "beta1":
+# full-strength writes.  "alpha1": no decay with random writes, so the state
+# carries across every chunk.
+EDGE = [
+    # name, B, H, T, dk, dtype, gate
+    ("retrieval", 1, 2, 128, 128, torch.bfloat16, "per_channel"),
+    ("retrieval", 1, 2, 100, 128, torch.bfloat16, "scalar"),
+    ("retrieval", 1, 1, 64, 64, torch.float32, "per_channel"),
+    ("retrieval", 1, 1, 128, 128, torch.float32, "scalar"),
+    ("gmin", 1, 2, 293, 128, torch.bfloat16, "per_channel"),
+    ("gmin_below", 1, 2, 256, 128, torch.bfloat16, "per_channel"),
+    ("gmin", 1, 1, 150, 64, torch.float32, "per_channel"),
+    ("beta1", 1, 2, 200, 128, torch.bfloat16, "per_channel"),
+    ("beta1", 1, 2, 200, 128, torch.bfloat16, "scalar"),
+    ("alpha1", 2, 1, 300, 128, torch.bfloat16, "per_channel"),
+    ("alpha1", 1, 2, 300, 128, torch.bfloat16, "scalar"),
+]
+
+
+@pytest.mark.parametrize("case", EDGE, ids=lambda c: f"{c[0]}-B{c[1]}H{c[2]}T{c[3]}d{c[4]}-{str(c[5])[6:]}-{c[6]}")
+def test_reductions_on_device(case):
+    kind, B, H, T, dk, dt, gate = case
+    recipe = "softplus_n02_clamp5" if gate == "per_channel" else "scalar_softplus_n01_plus2"
+    w = W.small_chunk_case(B, H, T, dk, dk, gate, dt, g_recipe=recipe, seed=41)
+    x = W.generate(w)
+    if kind == "retrieval":
+        keys = torch.stack([_orthonormal_keys(T, dk, 100 + h) for h in range(B * H)]).view(B, H, T, dk)
+        x["k"] = W.to_dtype(keys, dt)
+        x["g"].zero_()
+        x["beta"].fill_(1.0)
+        x["S0"].zero_()
+    elif kind in ("gmin", "gmin_below"):
+        x["g"].fill_(-5.0 if kind == "gmin" else -9.0)
+    elif kind == "beta1":
+        x["beta"].fill_(1.0)
+    elif kind == "alpha1":
+        x["g"].zero_()
+    O_ref, S_ref = oracle.forward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], gate=gate)
+    d = to_dev(x)
+    O, S = gdr.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], C=64, gate=gate)
+    torch.cuda.synchronize()
+    assert gdr.device_status() == 0
+    tol = TOL[dt]
+    eo, es = relerr(O, O_ref), relerr(S, S_ref)
+    assert eo <= tol and es <= tol, (case, eo, es)
+    if kind == "retrieval" and dt == torch.float32:
+        # S_T k_i = v_i for every written key, to the fp32 tolerance
+        got = torch.einsum("bhvk,bhtk->bhtv", S.double().cpu(), x["k"].double())
+        assert relerr(got, x["v"].double().numpy()) <= 1e-5
+
+
 def test_in_place_state_and_guard_bands():
     w = W.small_chunk_case(1, 2, 150, 128, 128, "per_channel", torch.bfloat16)
     x = W.generate(w)
@@ -143,22 +210,37 @@ def test_host_buffers_round_trip():
     assert relerr(O, O_ref) <= 2e-2 and relerr(S, S_ref) <= 2e-2
 
 
-@pytest.mark.parametrize("name,heads", [("gdn_scalar_t4096", [0, 17, 40, 63]),
-                                        ("kda_d128_t8192", [0, 31, 50]),
-                                        ("kda_long_t65536", [5, 30])])
-def test_full_size_sampled(name, heads):
+def _parity_accumulate(acc, x, ref):
+    """Running max|X - X_ref| and max|X_ref| over batches of heads."""
+    x = np.asarray(x.detach().double().cpu() if isinstance(x, torch.Tensor) else x, np.float64)
+    ref = np.asarray(ref, np.float64)
+    acc[0] = max(acc[0], float(np.max(np.abs(x - ref))))
+    acc[1] = max(acc[1], float(np.max(np.abs(ref))))
+
+
+# Every element of the three full-size chunk workloads, launched exactly as
+# bench.py launches them.  The oracle runs over batches of heads (one thread
+# per head) so that its fp64 copies stay a few GB.
+@pytest.mark.parametrize("name,batch", [("gdn_scalar_t4096", 64), ("kda_d128_t8192", 64),
+                                        ("kda_long_t65536", 16)])
+def test_full_size_every_element(name, batch):
     w = W.WORKLOADS[name]
     d = W.generate(w, device="cuda")
     O, S = gdr.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], C=w.C, gate=w.gate)
     torch.cuda.synchronize()
     assert gdr.device_status() == 0
-    assert bool(torch.isfinite(O).all()) and bool(torch.isfinite(S).all())
-    H = w.H
-    sel = lambda t: torch.stack([t[h // H, h % H] for h in heads])[:, None].cpu()
-    O_ref, S_ref = oracle.forward(sel(d["q"]), sel(d["k"]), sel(d["v"]), sel(d["g"]), sel(d["beta"]),
-                                  sel(d["S0"]), gate=w.gate)
-    eo, es = relerr(sel(O), O_ref), relerr(sel(S), S_ref)
-    assert eo <= 2e-2 and es <= 2e-2, (name, eo, es)
+    BH = w.B * w.H
+    flat = lambda t: t.reshape(BH, 1, *t.shape[2:])
+    eo, es = [0.0, 0.0], [0.0, 0.0]
+    for h0 in range(0, BH, batch):
+        sl = lambda t: flat(t)[h0:h0 + batch].cpu()
+        O_ref, S_ref = oracle.forward(sl(d["q"]), sl(d["k"]), sl(d["v"]), sl(d["g"]), sl(d["beta"]),
+                                      sl(d["S0"]), gate=w.gate)
+        _parity_accumulate(eo, sl(O), O_ref)
+        _parity_accumulate(es, sl(S), S_ref)
+        del O_ref, S_ref
+    ro, rs = eo[0] / eo[1], es[0] / es[1]
+    assert ro <= 2e-2 and rs <= 2e-2, (name, ro, rs)
 
 
 # ---------------------------------------------------------------- decode step
@@ -187,28 +269,35 @@ def test_decode_small(dk, dv, gate, dt):
     assert relerr(O, O_ref) <= tol and relerr(S, S_ref) <= tol
 
 
-def test_decode_full_size_sampled():
+def test_decode_full_size_every_element():
+    """All 8192 heads of the decode workload over its 1000 steps: every o_t and
+    the final state against the oracle (heads in batches on the host)."""
     w = W.WORKLOADS["kda_decode_b256"]
-    heads = [0, 1, 777, 4096, 8191]
-    steps = w.T
+    steps, BH = w.T, w.B * w.H
     d0 = W.generate(w, device="cuda", steps=1, step0=0)
     S = d0["S0"].clone()
-    sel_hist = {k: [] for k in ("q", "k", "v", "g", "beta", "o")}
-    H = w.H
-    pick = lambda t: torch.stack([t[h // H, h % H] for h in heads])
+    outs = torch.empty(steps, w.B, w.H, w.dv, dtype=w.dtype, device="cuda")
     for s in range(steps):
         x = W.generate(w, device="cuda", steps=1, step0=s)
-        o = gdr.recurrent_step(x["q"][0], x["k"][0], x["v"][0], x["g"][0], x["beta"][0], S)
-        for key in ("q", "k", "v", "g", "beta"):
-            sel_hist[key].append(pick(x[key][0]))
-        sel_hist["o"].append(pick(o))
+        gdr.recurrent_step(x["q"][0], x["k"][0], x["v"][0], x["g"][0], x["beta"][0], S, o=outs[s])
     torch.cuda.synchronize()
-    assert bool(torch.isfinite(S).all())
-    st = lambda key: torch.stack(sel_hist[key])[:, :, None].cpu()   # [steps, nh, 1, ...]
-    o_ref, S_ref = oracle.decode(st("q"), st("k"), st("v"), st("g"), st("beta"), pick(d0["S0"])[:, None].cpu())
-    eo = relerr(torch.stack(sel_hist["o"]), o_ref[:, :, 0])
-    es = relerr(pick(S), S_ref[:, 0])
-    assert eo <= 2e-2 and es <= 2e-2, (eo, es)
+    assert gdr.device_status() == 0
+    S0 = d0["S0"].reshape(BH, 1, w.dv, w.dk)
+    outs = outs.reshape(steps, BH, 1, w.dv)
+    Sf = S.reshape(BH, 1, w.dv, w.dk)
+    eo, es = [0.0, 0.0], [0.0, 0.0]
+    batch = 512
+    for h0 in range(0, BH, batch):
+        heads = list(range(h0, min(BH, h0 + batch)))
+        x = W.generate(w, device="cuda", heads=heads, steps=steps, step0=0)   # [steps, nh, 1, ...]
+        cpu = lambda t: t.cpu()
+        o_ref, S_ref = oracle.decode(cpu(x["q"]), cpu(x["k"]), cpu(x["v"]), cpu(x["g"]), cpu(x["beta"]),
+                                     S0[h0:h0 + batch].cpu())
+        _parity_accumulate(eo, outs[:, h0:h0 + batch].cpu(), o_ref)
+        _parity_accumulate(es, Sf[h0:h0 + batch].cpu(), S_ref)
+        del x, o_ref, S_ref
+    ro, rs = eo[0] / eo[1], es[0] / es[1]
+    assert ro <= 2e-2 and rs <= 2e-2, (ro, rs)
 
 
 # A slowly decaying gate keeps the state alive across chunks, so a wrong state

@@ -118,6 +118,13 @@ def load_peaks():
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+# B200 datasheet peaks (HBM3e bandwidth, dense bf16 tensor throughput): the
+# contract's `frac` is taken against the measured peaks above; `frac_vs_spec`
+# states the same achievement against these.
+SPEC_HBM_GBS = 8000.0
+SPEC_BF16_TFLOPS = 2250.0
+
+
 def roofline(w: W.Workload, seconds_per_launch: float, peaks, kernel_src: str = None):
     byts = algorithmic_bytes(w)
     flops = dense_flops(w)
@@ -131,11 +138,13 @@ def roofline(w: W.Workload, seconds_per_launch: float, peaks, kernel_src: str = 
         ach = byts / seconds_per_launch / 1e9
         return {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(ach / peaks["hbm_gbs"], 4), "traffic": traffic,
-                "peak_source": peaks["source"] + " (copy bandwidth)", "algorithmic_bytes": byts}
+                "peak_source": peaks["source"] + " (copy bandwidth)", "algorithmic_bytes": byts,
+                "frac_vs_spec": round(ach / SPEC_HBM_GBS, 4), "spec_peak": SPEC_HBM_GBS}
     ach = flops / seconds_per_launch / 1e12
     return {"bound": "tensor", "achieved": round(ach, 2), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
             "frac": round(ach / peaks["bf16_tflops"], 4), "traffic": traffic,
-            "peak_source": peaks["source"], "algorithmic_flops": flops}
+            "peak_source": peaks["source"], "algorithmic_flops": flops,
+            "frac_vs_spec": round(ach / SPEC_BF16_TFLOPS, 4), "spec_peak": SPEC_BF16_TFLOPS}
 
 
 def file_sha(paths) -> str:
@@ -174,6 +183,61 @@ def reduce_max(x: float, world: int, device) -> float:
 # ------------------------------------------------------------ clock sampler
 
 _REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+
+class NvmlClockSampler:
+    """SM clock, max SM clock and active clock-event reasons read through NVML
+    (the library nvidia-smi reports from) every ~1 ms in a background thread,
+    so that even a timed region of a few milliseconds holds several samples.
+    Only reads settings."""
+
+    _BITS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40, "sw_power_cap": 0x4}
+
+    def __init__(self, device_index: int, period_s: float = 0.001):
+        import pynvml
+        pynvml.nvmlInit()
+        self.nv = pynvml
+        self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+        self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+        self.samples = []
+        self.period = period_s
+        self.running = True
+        self.proc = True
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
+
+    def _run(self):
+        nv = self.nv
+        while self.running:
+            try:
+                mhz = float(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((time.time(), mhz, self.max_mhz, [r for r, b in self._BITS.items() if bits & b]))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def wait_first(self, timeout_s: float = 5.0):
+        t0 = time.time()
+        while not self.samples and time.time() - t0 < timeout_s:
+            time.sleep(0.001)
+
+    def stop(self):
+        self.running = False
+        self.thread.join(timeout=2)
+
+    def summary(self, t0: float, t1: float):
+        return ClockSampler.summary(self, t0, t1)
+
+    def window(self, t0: float, t1: float):
+        return self.summary(t0, t1)
+
+
+def make_sampler(device):
+    try:
+        return NvmlClockSampler(device.index if device.index is not None else 0)
+    except Exception:
+        return ClockSampler(gpu_id_for(device))
 
 
 class ClockSampler:
@@ -360,6 +424,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the other configurations timed after the headline (one GPU only)")
     return ap.parse_args()
 
 
@@ -406,6 +472,90 @@ def run_reference(args, w: W.Workload, rank: int, world: int):
     return 0
 
 
+def build_step(gdr, w: W.Workload, device):
+    """Inputs of workload ``w`` resident in HBM and the step that runs it:
+    returns (step, x, O, S_T) with O, S_T the buffers the step writes."""
+    if w.kind == "decode":
+        x = W.generate(w, device=device, steps=w.T)
+        S = x["S0"].clone()
+        o = torch.empty(w.B, w.H, w.dv, dtype=w.dtype, device=device)
+
+        if w.rule == "gdr2":
+            def step():
+                for s in range(w.T):
+                    gdr.recurrent_step_gdr2(x["q"][s], x["k"][s], x["v"][s], x["g"][s], x["b"][s], x["w"][s], S,
+                                            o=o)
+        else:
+            def step():
+                for s in range(w.T):
+                    gdr.recurrent_step(x["q"][s], x["k"][s], x["v"][s], x["g"][s], x["beta"][s], S, o=o)
+        return step, x, o, S
+    if w.g_recipe == "prologue":
+        x = W.generate_prologue(w, device=device)
+        O = torch.empty(w.B, w.H, w.T, w.dv, dtype=w.dtype, device=device)
+        S_T = torch.empty(w.B, w.H, w.dv, w.dk, dtype=torch.float32, device=device)
+        return (lambda: api_call(gdr, w, x, O=O, S_T=S_T)), x, O, S_T
+    if w.direction == "bwd":
+        x = W.generate(w, device=device)
+        x.update(W.generate_grads(w, device=device))
+        bws = torch.empty(gdr.chunk_bwd_workspace_size(w.B, w.H, w.T, w.dk, w.dv, w.C, w.gate, w.dtype),
+                          dtype=torch.uint8, device=device)
+        # the result read back in the end-to-end measurement: dq (shape of q) and dS0
+        return (lambda: api_call(gdr, w, x, workspace=bws)), x, x["dO"], x["dS_T"]
+    x = W.generate(w, device=device)
+    if w.rule == "gdr2":
+        del x["beta"]           # the erase and write gates take its place
+    O = torch.empty(w.B, w.H, w.T, w.dv, dtype=w.dtype, device=device)
+    S_T = torch.empty(w.B, w.H, w.dv, w.dk, dtype=torch.float32, device=device)
+    return (lambda: api_call(gdr, w, x, O=O, S_T=S_T)), x, O, S_T
+
+
+def time_steps(step, steps: int, warmup: int, stream, device, world: int):
+    """W untimed steps, then K steps between barriers and synchronizes, each
+    bracketed by CUDA events on the launching stream.  Returns the per-step
+    device times (ms) and the wall-clock window of the timed region."""
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    t_wall0 = time.time()
+    for i in range(steps):
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize(device)
+    t_wall1 = time.time()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    return [a.elapsed_time(b) for a, b in ev], t_wall0, t_wall1
+
+
+def kernel_sources(w: W.Workload):
+    return [os.path.join(ROOT, "gated_delta_rule_89_b200", "csrc", f)
+            for f in (DECODE_SOURCES if w.kind == "decode" else BWD_SOURCES if w.direction == "bwd"
+                      else CHUNK_SOURCES)]
+
+
+def roofline_for(w: W.Workload, step_ms, peaks):
+    """Roofline of one launch of the dominant path: one chunked call, or one
+    decode step (a decode workload step is w.T launches)."""
+    import dataclasses
+    per_launch_s = statistics.mean(step_ms) / 1e3 / (w.T if w.kind == "decode" else 1)
+    wk = dataclasses.replace(w, T=1) if w.kind == "decode" else w
+    return roofline(wk, per_launch_s, peaks, kernel_sources(w))
+
+
+# the other configurations of the method's workload list, timed in the same
+# process after the headline (one GPU only)
+EXTRA_WORKLOADS = ("gdn_scalar_t4096", "kda_long_t65536", "kda_decode_b256")
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
@@ -428,77 +578,20 @@ def main():
     stream = torch.cuda.current_stream(device)
 
     # ---- inputs resident in HBM before timing
-    if w.kind == "decode":
-        steps_needed = w.T
-        x = W.generate(w, device=device, steps=steps_needed)
-        S = x["S0"].clone()
-        o = torch.empty(w.B, w.H, w.dv, dtype=w.dtype, device=device)
-
-        if w.rule == "gdr2":
-            def step():
-                for s in range(w.T):
-                    gdr.recurrent_step_gdr2(x["q"][s], x["k"][s], x["v"][s], x["g"][s], x["b"][s], x["w"][s], S,
-                                            o=o)
-        else:
-            def step():
-                for s in range(w.T):
-                    gdr.recurrent_step(x["q"][s], x["k"][s], x["v"][s], x["g"][s], x["beta"][s], S, o=o)
-    elif w.g_recipe == "prologue":
-        x = W.generate_prologue(w, device=device)
-        O = torch.empty(w.B, w.H, w.T, w.dv, dtype=w.dtype, device=device)
-        S_T = torch.empty(w.B, w.H, w.dv, w.dk, dtype=torch.float32, device=device)
-
-        def step():
-            api_call(gdr, w, x, O=O, S_T=S_T)
-    elif w.direction == "bwd":
-        x = W.generate(w, device=device)
-        x.update(W.generate_grads(w, device=device))
-        bws = torch.empty(gdr.chunk_bwd_workspace_size(w.B, w.H, w.T, w.dk, w.dv, w.C, w.gate, w.dtype),
-                          dtype=torch.uint8, device=device)
-        O = x["dO"]     # the result read back in the end-to-end measurement: dq
-        S_T = x["dS_T"]
-
-        def step():
-            api_call(gdr, w, x, workspace=bws)
-    else:
-        x = W.generate(w, device=device)
-        if w.rule == "gdr2":
-            del x["beta"]           # the erase and write gates take its place
-        O = torch.empty(w.B, w.H, w.T, w.dv, dtype=w.dtype, device=device)
-        S_T = torch.empty(w.B, w.H, w.dv, w.dk, dtype=torch.float32, device=device)
-
-        def step():
-            api_call(gdr, w, x, O=O, S_T=S_T)
+    step, x, O, S_T = build_step(gdr, w, device)
     torch.cuda.synchronize(device)
 
-    sampler = ClockSampler(gpu_id_for(device)) if rank == 0 else None
+    sampler = make_sampler(device) if rank == 0 else None
     if sampler is not None:
         sampler.wait_first()
-    for _ in range(args.warmup):
-        step()
+    step()
     launches_per_step = gdr.last_launch_count() * (w.T if w.kind == "decode" else 1)
-    torch.cuda.synchronize(device)
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-    torch.cuda.synchronize(device)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    t_wall0 = time.time()
-    for i in range(args.steps):
-        ev[i][0].record(stream)
-        step()
-        ev[i][1].record(stream)
-    torch.cuda.synchronize(device)
-    t_wall1 = time.time()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize(device)
-    step_ms = [a.elapsed_time(b) for a, b in ev]
-    total_ms = sum(step_ms)
-    total_ms = reduce_max(total_ms, world, device)
+    step_ms, t_wall0, t_wall1 = time_steps(step, args.steps, max(0, args.warmup - 1), stream, device, world)
+    total_ms = reduce_max(sum(step_ms), world, device)
     ms_per_step = total_ms / args.steps
     # chunk: B*T tokens per step; decode: B sequences x T consecutive steps
     value = job_throughput(w.B * w.T, world, total_ms, args.steps)
+    clocks = sampler.summary(t_wall0, t_wall1) if sampler is not None else None
 
     # ---- end to end through the public API with host buffers (pinned)
     e2e = None
@@ -527,26 +620,14 @@ def main():
         e2e = {"value": None, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0,
                "note": "not measured for the decode workload"}
 
-    clocks = None
-    if sampler is not None:
-        sampler.stop()
-        clocks = sampler.summary(t_wall0, t_wall1)
-
+    line = None
     if rank == 0:
         peaks = load_peaks()
-        per_launch_s = statistics.mean(step_ms) / 1e3 / (w.T if w.kind == "decode" else 1)
-        wk = w0
-        if w.kind == "decode":
-            import dataclasses
-            wk = dataclasses.replace(w0, T=1)   # one launch = one decode step
-        src = [os.path.join(ROOT, "gated_delta_rule_89_b200", "csrc", f)
-               for f in (DECODE_SOURCES if w.kind == "decode" else BWD_SOURCES if w.direction == "bwd"
-                         else CHUNK_SOURCES)]
         line = base_line(w0, args, world)
         line.update({
             "value": value,
             "ms_per_step": round(ms_per_step, 4),
-            "roofline": roofline(wk, per_launch_s, peaks, src),
+            "roofline": roofline_for(w0, step_ms, peaks),
             "gpu_launches": launches_per_step * args.steps,
             "e2e": e2e,
             "clocks": clocks,
@@ -554,6 +635,40 @@ def main():
         if world == 1 and not args.no_cpu_baseline:
             v, desc = oracle_sample(w0, args.cpu_budget)
             line["cpu_baseline"] = dict(desc, value=v, unit="tokens/s")
+
+    # ---- the other configurations, same process, same steps (one GPU only)
+    if world == 1 and not args.no_extra:
+        del step, x, O, S_T
+        torch.cuda.empty_cache()
+        extra = {}
+        for name in EXTRA_WORKLOADS:
+            if name == w0.name:
+                continue
+            we = W.WORKLOADS[name]
+            st, xe, Oe, Se = build_step(gdr, we, device)
+            torch.cuda.synchronize(device)
+            st()
+            lp = gdr.last_launch_count() * (we.T if we.kind == "decode" else 1)
+            ms, a0, a1 = time_steps(st, args.steps, max(0, args.warmup - 1), stream, device, 1)
+            extra[name] = {
+                "metric": METRIC_DECODE if we.kind == "decode" else METRIC,
+                "config": {"B": we.B, "H": we.H, "T": we.T, "dk": we.dk, "dv": we.dv, "C": we.C, "gate": we.gate,
+                           "description": we.description},
+                "ms_per_step": round(statistics.mean(ms), 4),
+                "value": we.B * we.T / (statistics.mean(ms) / 1e3),
+                "unit": "tokens/s",
+                "roofline": roofline_for(we, ms, load_peaks()),
+                "gpu_launches": lp * args.steps,
+                "clocks": sampler.summary(a0, a1) if sampler is not None else None,
+            }
+            del st, xe, Oe, Se
+            torch.cuda.empty_cache()
+        if line is not None:
+            line["workloads"] = extra
+
+    if sampler is not None:
+        sampler.stop()
+    if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

@@ -78,6 +78,8 @@ def lib() -> ctypes.CDLL:
         L.gdr_last_launch_count.restype = I
         L.gdr_device_status.argtypes = [P]
         L.gdr_device_status.restype = I
+        L.gdr_debug_set_wait_budget.argtypes = [ctypes.c_longlong]
+        L.gdr_debug_set_wait_budget.restype = None
         _lib = L
     return _lib
 

@@ -47,6 +47,7 @@
 // GDR_ERR_TIMEOUT in a device status word, lets the copies and MMAs it
 // issued finish, frees its tensor memory and returns.
 #include <cuda.h>
+#include <atomic>
 #include <mutex>
 
 #include "gdr_internal.cuh"
@@ -65,7 +66,8 @@ using namespace sm100;
 constexpr int kC = 64;
 constexpr int kD = 128;
 constexpr int kThreads = 448;   // 14 warps: TMA, MMA, 8 conversion warps, 4 output-epilogue warps
-constexpr long long kWaitBudget = 2000000000LL;   // clock cycles per wait (~1 s)
+constexpr long long kWaitBudget = 2000000000LL;   // default clock cycles per wait (~1 s)
+constexpr long long kDrainBudget = 500000000LL;   // waits for copies and MMAs already issued, on the way out
 
 // shared memory map (bytes from a 1024-aligned base).  The input tiles of a
 // chunk form one stage (gamma_C in a slot of its own); two stages alternate
@@ -122,19 +124,6 @@ struct Maps {
 
 __device__ __forceinline__ void record_error(int code) { atomicCAS(&g_device_status, 0, code); }
 
-// Optional phase timestamps of block 0 (SM clock), compiled only with -DGDR_TRACE.
-#ifdef GDR_TRACE
-__device__ long long g_trace[16][1024];
-#define GDR_TRACE_AT(ev, n)                                                   \
-    do {                                                                      \
-        if (blockIdx.x == 0 && (n) < 1024) g_trace[(ev)][(n)] = clock64();    \
-    } while (0)
-#else
-#define GDR_TRACE_AT(ev, n) \
-    do {                    \
-    } while (0)
-#endif
-
 __device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi)
 {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
@@ -183,11 +172,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ gamma_c,
                   const float *__restrict__ S0, __nv_bfloat16 *__restrict__ O, float *__restrict__ ST,
                   int T_len, int nchunks, const __nv_bfloat16 *__restrict__ ogate,
-                  const float *__restrict__ norm_w, float eps)
+                  const float *__restrict__ norm_w, float eps, long long wait_budget)
 {
     extern __shared__ unsigned char smem_raw[];
-    unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                          ~static_cast<uintptr_t>(1023));
+    // aligned by an offset into the __shared__ array itself, so that the
+    // compiler keeps every access through `sm` in the shared state space
+    unsigned char *sm = smem_raw + ((1024u - (sm100::smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_BAR + 8 * B_COUNT);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + OFF_BAR + 8 * B_COUNT + 4);
@@ -225,7 +215,7 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
     auto wait = [&](int b, uint32_t parity) -> bool {
         if (mbar_try_wait(&bar[b], parity)) return true;
         if (*abort_flag) return false;
-        if (mbar_wait(&bar[b], parity, kWaitBudget)) return true;
+        if (mbar_wait(&bar[b], parity, wait_budget)) return true;
         record_error(6 /* GDR_ERR_TIMEOUT */);
         *abort_flag = 1;
         return false;
@@ -270,7 +260,7 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
             }
             bulk_wait_all();   // the last store has completed before the CTA exits
             if (*abort_flag && loaded > 0)   // a gate tile still in flight lands before exit
-                mbar_wait(&bar[B_GATE_FULL], (uint32_t)((loaded - 1) & 1), kWaitBudget / 4);
+                mbar_wait(&bar[B_GATE_FULL], (uint32_t)((loaded - 1) & 1), kDrainBudget);
         }
         if (lane == 1 && !OEPI) {
             // Output tile m: stored once the epilogue has written it; the tile
@@ -318,14 +308,15 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
                 if (!wait(B_GEMPTY + b, upar ^ 1)) break;
                 mbar_arrive_expect_tx(&bar[B_GFULL + b], 512);
                 bulk_load(sm + OFF_GAM + b * 512, gamma_c + (size_t)(head * nchunks + n) * kD, 512, &bar[B_GFULL + b]);
-                GDR_TRACE_AT(0, n);
                 issued = n + 1;
             }
-            if (*abort_flag && issued > 0) {
-                // let the copies of the last issued chunk land before the CTA exits
-                const int n = issued - 1;
-                mbar_wait(&bar[B_FULL + (n & 1)], (uint32_t)((n >> 1) & 1), kWaitBudget / 4);
-                mbar_wait(&bar[B_GFULL + (n & 1)], (uint32_t)((n >> 1) & 1), kWaitBudget / 4);
+            if (*abort_flag) {
+                // let the copies of the (at most two) stages still in flight land
+                // before the CTA exits
+                for (int n = issued - 1; n >= 0 && n >= issued - 2; --n) {
+                    mbar_wait(&bar[B_FULL + (n & 1)], (uint32_t)((n >> 1) & 1), kDrainBudget);
+                    mbar_wait(&bar[B_GFULL + (n & 1)], (uint32_t)((n >> 1) & 1), kDrainBudget);
+                }
             }
         }
     } else if (warp == 1) {
@@ -335,60 +326,54 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
             constexpr uint32_t ID_X = idesc_bf16(128, 64, false, true, true);    // -A, B (W) MN-major
             constexpr uint32_t ID_O = idesc_bf16(128, 64, false, false);
             constexpr uint32_t ID_S = idesc_bf16(128, 128, false, true);         // B MN-major
+            // descriptors of the two operand layouts at the base of shared memory:
+            // the address field counts 16-byte units, so a byte offset adds directly
+            const uint64_t d16 = sdesc_sw128(sbase, 16, 1024), d8k = sdesc_sw128(sbase, 8192, 1024);
+            auto K16 = [&](uint32_t off) { return d16 + (uint64_t)(off >> 4); };   // K-major tile
+            auto MN = [&](uint32_t off) { return d8k + (uint64_t)(off >> 4); };    // MN-major tile, panels 8 KB apart
             // U^T = V^T T'^T of chunk n (stage n & 1); it has to wait until
             // V_new^T of the previous chunk has left TM_V
             auto mma_u = [&](int n) {
-                const uint32_t st = sbase + (n & 1) * STAGE;
+                const uint32_t st = (n & 1) * STAGE;
 #pragma unroll
-                for (int s = 0; s < 4; ++s)
-                    mma_bf16(tmem + TM_V, sdesc_sw128(st + ST_V + s * 2048, 8192, 1024),
-                             sdesc_sw128(st + ST_T + s * 32, 16, 1024), ID_WU, s > 0);
+                for (int s = 0; s < 4; ++s) mma_bf16(tmem + TM_V, MN(st + ST_V + s * 2048), K16(st + ST_T + s * 32), ID_WU, s > 0);
             };
             bool ok = nchunks > 0 && wait(B_FULL, 0);
             if (ok) {
                 tc_fence_after();
-                GDR_TRACE_AT(1, 0);
                 mma_u(0);
             }
             for (int n = 0; n < nchunks && ok; ++n) {
                 const int b = n & 1;
                 const uint32_t par = (uint32_t)(n & 1), upar = (uint32_t)((n >> 1) & 1);
-                const uint32_t st = sbase + b * STAGE;
+                const uint32_t st = b * STAGE;
                 // ---- V_new^T += -S W^T ; O^T = S Q<-^T
                 if (!wait(B_SW_READY, par) || !wait(B_OACC_EMPTY + b, upar ^ 1)) break;
                 tc_fence_after();
-                GDR_TRACE_AT(2, n);
 #pragma unroll
                 for (int s = 0; s < 8; ++s)
-                    mma_bf16(tmem + TM_V, sdesc_sw128(sbase + OFF_S + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024),
-                             sdesc_sw128(st + ST_W + s * 2048, 8192, 1024), ID_X, 1);
+                    mma_bf16(tmem + TM_V, K16(OFF_S + (s >> 2) * 16384 + (s & 3) * 32), MN(st + ST_W + s * 2048), ID_X, 1);
                 mma_commit(&bar[B_X_FULL]);
 #pragma unroll
                 for (int s = 0; s < 8; ++s)
-                    mma_bf16(tmem + TM_O + 64 * b,
-                             sdesc_sw128(sbase + OFF_S + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024),
-                             sdesc_sw128(st + ST_Q + (s >> 2) * 8192 + (s & 3) * 32, 16, 1024), ID_O, s > 0);
+                    mma_bf16(tmem + TM_O + 64 * b, K16(OFF_S + (s >> 2) * 16384 + (s & 3) * 32),
+                             K16(st + ST_Q + (s >> 2) * 8192 + (s & 3) * 32), ID_O, s > 0);
                 // ---- S += V_new^T K_tail (the sequential path; S already scaled by
                 // gamma_C); O^T += V_new^T Aqk^T
                 if (!wait(B_VN_READY, par)) break;
                 tc_fence_after();
-                GDR_TRACE_AT(3, n);
 #pragma unroll
-                for (int s = 0; s < 4; ++s)
-                    mma_bf16(tmem + TM_S, sdesc_sw128(sbase + OFF_VN + s * 32, 16, 1024),
-                             sdesc_sw128(st + ST_KT + s * 2048, 8192, 1024), ID_S, 1);
+                for (int s = 0; s < 4; ++s) mma_bf16(tmem + TM_S, K16(OFF_VN + s * 32), MN(st + ST_KT + s * 2048), ID_S, 1);
                 mma_commit(&bar[B_S_FULL]);
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
-                    mma_bf16(tmem + TM_O + 64 * b, sdesc_sw128(sbase + OFF_VN + s * 32, 16, 1024),
-                             sdesc_sw128(st + ST_AQ + s * 32, 16, 1024), ID_O, 1);
+                    mma_bf16(tmem + TM_O + 64 * b, K16(OFF_VN + s * 32), K16(st + ST_AQ + s * 32), ID_O, 1);
                 mma_commit(&bar[B_O_FULL + b]);
                 mma_commit(&bar[B_EMPTY + b]);   // every read of this stage is issued
                 // ---- U^T of the next chunk
                 if (n + 1 < nchunks) {
                     if (!wait(B_FULL + (b ^ 1), (uint32_t)(((n + 1) >> 1) & 1))) break;
                     tc_fence_after();
-                    GDR_TRACE_AT(1, n + 1);
                     mma_u(n + 1);
                 }
             }
@@ -443,7 +428,6 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
             fence_async_smem();
             tc_fence_before();
             mbar_arrive(&bar[B_SW_READY]);
-            if (tid == 192) GDR_TRACE_AT(12, n);
             if (!waitw(B_GFULL + (n & 1), (uint32_t)((n >> 1) & 1))) return false;
             const float4 *gm = reinterpret_cast<const float4 *>(sm + OFF_GAM + (n & 1) * 512) + (sc0 >> 2);
 #pragma unroll
@@ -471,13 +455,11 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
                 if (!waitw(B_S_FULL, par ^ 1)) { ok = false; break; }
                 tc_fence_after();
             }
-            if (tid == 192) GDR_TRACE_AT(11, n);
             if (!state_pass(n)) { ok = false; break; }
             // ---- V_new^T (TMEM) -> bf16 smem (the MMAs of chunk n - 1 that read
             // the old copy completed before X_FULL(n))
             if (!waitw(B_X_FULL, par)) { ok = false; break; }
             tc_fence_after();
-            if (tid == 192) GDR_TRACE_AT(13, n);
 #pragma unroll
             for (int cb = 0; cb < 2; ++cb) {
                 uint32_t r[16];
@@ -491,7 +473,6 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
             fence_async_smem();
             tc_fence_before();
             mbar_arrive(&bar[B_VN_READY]);   // also: S_n scaled
-            if (tid == 192) GDR_TRACE_AT(14, n);
         }
         // ---- final state S_N: the last accumulation has completed
         if (ok && nchunks > 0 && waitw(B_S_FULL, (uint32_t)((nchunks - 1) & 1))) {
@@ -537,7 +518,6 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
             if (OEPI) ok = epi_all(ok);   // the four warps go on (or stop) together
             if (!ok) break;
             tc_fence_after();
-            if (tid == 320) GDR_TRACE_AT(4, m);
             const uint32_t oc = trow + TM_O + 64 * bb;
             if (!OEPI) {
 #pragma unroll 2
@@ -597,9 +577,7 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
                             0.5f * rsqrtf((red[lane] + red[32 + lane] + red[64 + lane] + red[96 + lane]) * (1.f / kD) + eps);
                     epi_sync();   // red is free again, rstd of these tokens written
                 }
-                if (tid == 320) GDR_TRACE_AT(5, m);
                 if (!epi_all(waitw(B_GATE_FULL, (uint32_t)(m & 1)))) break;
-                if (tid == 320) GDR_TRACE_AT(9, m);
                 // pass 2: 16 tokens per step; y replaces the gate element it was computed
                 // from, and the tile leaves by TMA store (rows past T are dropped)
 #pragma unroll 1
@@ -641,7 +619,6 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
                 mbar_arrive(&bar[B_OACC_EMPTY + bb]);
                 fence_async_smem();   // the tile is read next by the TMA store
                 mbar_arrive(&bar[B_EPI_FULL]);
-                if (tid == 320) GDR_TRACE_AT(6, m);
             }
         }
     }
@@ -682,6 +659,17 @@ bool make_map(CUtensorMap *m, CUtensorMapDataType dt, int rank, void *ptr, const
 }
 
 }  // namespace
+
+namespace {
+std::atomic<long long> g_wait_budget{0};   // 0: the default budget
+long long wait_budget_now()
+{
+    const long long v = g_wait_budget.load(std::memory_order_relaxed);
+    return v > 0 ? v : kWaitBudget;
+}
+}  // namespace
+
+void set_wait_budget(long long cycles) { g_wait_budget.store(cycles > 0 ? cycles : 0, std::memory_order_relaxed); }
 
 bool chunk_tc_supports(const ChunkArgs &a)
 {
@@ -732,18 +720,11 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream, int *launch
     if (e != cudaSuccess) return e;
     kern<<<BH, kThreads, SMEM_ALLOC, stream>>>(
         maps, w.gam, a.S0, static_cast<__nv_bfloat16 *>(a.O), a.S_T, a.T, nchunks,
-        static_cast<const __nv_bfloat16 *>(a.ogate), a.norm_w, a.eps);
+        static_cast<const __nv_bfloat16 *>(a.ogate), a.norm_w, a.eps, wait_budget_now());
     e = cudaGetLastError();
     if (e == cudaSuccess) *launches += 1;
     return e;
 }
-
-#ifdef GDR_TRACE
-extern "C" __attribute__((visibility("default"))) int gdr_trace_dump(long long *host)
-{
-    return (int)cudaMemcpyFromSymbol(host, g_trace, sizeof(g_trace));
-}
-#endif
 
 cudaError_t read_device_status(cudaStream_t stream, int *status)
 {
@@ -755,9 +736,10 @@ cudaError_t read_device_status(cudaStream_t stream, int *status)
     if (v != 0) {
         const int zero = 0;
         e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int));
+        if (e != cudaSuccess) return e;
     }
     *status = v;
-    return e;
+    return cudaSuccess;
 }
 
 }  // namespace gdr

@@ -65,6 +65,8 @@ GDR_API int gdr_last_cuda_error(void) { return tl_last_cuda_error; }
 
 GDR_API int gdr_last_launch_count(void) { return tl_last_launches; }
 
+GDR_API void gdr_debug_set_wait_budget(long long cycles) { gdr::set_wait_budget(cycles); }
+
 GDR_API size_t gdr_chunk_fwd_workspace_size(int B, int H, int T, int dk, int dv, int C, int gate_mode, int dtype)
 {
     if (B <= 0 || H <= 0 || T <= 0) return 0;

@@ -115,6 +115,9 @@ bool chunk_tc_supports(const ChunkArgs &a);
 size_t chunk_tc_workspace_bytes(int B, int H, int T, bool gdr2 = false);
 // Synchronizes `stream`, then reads and clears the device status word.
 cudaError_t read_device_status(cudaStream_t stream, int *status);
+// Clock cycles each bounded device wait of later launches may take (0: the
+// default, about a second); for tests of the timeout path.
+void set_wait_budget(long long cycles);
 // Debug mode (GDR_DEBUG set in the environment, read once): the entry points
 // that take a log-decay gate check its n elements first (finite and <= 0);
 // *bad is set when one is not.  Synchronizes `stream`.

@@ -86,11 +86,14 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t pari
 
 // Wait for the phase with the given parity to complete, giving up after
 // `budget` clock cycles.  Returns false on timeout (the caller reports it).
+// The suspend hint of each try is at most 20 us, and shorter for a short
+// budget (about half a nanosecond per cycle), so that the budget holds.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, long long budget)
 {
     if (mbar_try_wait(bar, parity)) return true;
+    const uint32_t hint = budget >= 40000 ? 20000u : (uint32_t)(budget > 64 ? budget / 2 : 32);
     const long long t0 = clock64();
-    while (!mbar_try_wait_sleep(bar, parity, 20000u)) {
+    while (!mbar_try_wait_sleep(bar, parity, hint)) {
         if (clock64() - t0 > budget) return false;
     }
     return true;

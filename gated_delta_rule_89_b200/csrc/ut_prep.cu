@@ -225,8 +225,9 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
 {
     static_assert(!(PRO && GDR2), "the fused prologue is for the tied-gate rule");
     extern __shared__ unsigned char prep_raw[];
-    unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(prep_raw) + 1023) &
-                                                          ~static_cast<uintptr_t>(1023));
+    // aligned by an offset into the __shared__ array itself, so that the
+    // compiler keeps every access through `sm` in the shared state space
+    unsigned char *sm = prep_raw + ((1024u - (sm100::smem_u32(prep_raw) & 1023u)) & 1023u);
     float(*sA)[kLdA] = reinterpret_cast<float(*)[kLdA]>(sm + OFF_A);
     float(*sQ)[kLdA] = reinterpret_cast<float(*)[kLdA]>(sm + OFF_AQ);   // Aqk, later Nt
     float(*sU)[16][kLdD] = reinterpret_cast<float(*)[16][kLdD]>(sm + OFF_U);

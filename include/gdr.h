@@ -301,6 +301,18 @@ int gdr_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const flo
  */
 int gdr_device_status(void *stream);
 
+/*
+ * Testing aid for the timeout path: the number of SM clock cycles each
+ * bounded device wait of the kernels launched after this call may take
+ * before it gives up (process-wide; cycles <= 0 restores the default of
+ * about two billion cycles, about a second).  With a budget far below the
+ * time the pipeline's hand-offs take, a call's waits run out: the kernel
+ * records GDR_ERR_TIMEOUT (read it with gdr_device_status), lets the copies
+ * and tensor-core operations it issued finish, frees its tensor memory and
+ * returns; its outputs are undefined.  Not for production use.
+ */
+void gdr_debug_set_wait_budget(long long cycles);
+
 /* Human-readable name of a status value (static string, never NULL). */
 const char *gdr_status_string(int status);
 

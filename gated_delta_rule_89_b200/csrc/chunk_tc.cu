@@ -5,16 +5,17 @@
 //   1. ut_prep (ut_prep.cu): every chunk of every head in parallel -> the
 //      UT-transform matrix T' = (I + A)^{-1} Diag(beta), the masked
 //      intra-chunk matrix Aqk and, with G the cumulative log-decay inside the
-//      chunk, W = T' (K*exp(G)) (stored transposed), Q<- = Q*exp(G),
-//      K_tail = K*exp(G_C - G) and gamma_C = exp(G_C), all into the workspace.
+//      chunk, -W = -T' (K*exp(G)), Q<- = Q*exp(G), K_tail = K*exp(G_C - G)
+//      (stored transposed) and gamma_C = exp(G_C), all into the workspace.
 //   2. chunk_scan (this file): one CTA per (b, h) walks the chunks in order.
 //      The fp32 state S [d_v x d_k] lives in tensor memory for the whole
 //      sequence.  Per chunk:
-//        V_new^T = V^T T'^T - S W^T          (U^T, then -S W^T accumulated)
-//        O^T     = S Q<-^T + V_new^T Aqk^T
-//        S       = S Diag(gamma_C) + V_new^T K_tail   (the scaling in place in
-//                  TMEM, the increment accumulated onto it by the MMA)
-//      which is the chunk state update and chunk output of "Reading notes:
+//        [O^T | V_new^T] = [0 | V^T T'^T] + S [Q<-; -W]^T          (N = 128)
+//        [S   | O^T    ] = [S Diag(gamma_C) | O^T] + V_new^T [K_tail^T; Aqk]^T
+//                                                                   (N = 192)
+//      (the scaling of S by the conversion warps, the increment accumulated
+//      onto it by the MMA; S alternates between two TMEM regions so that each
+//      pair of accumulators is contiguous), which is the chunk state update and chunk output of "Reading notes:
 //      Kimi Delta Attention" (mzeromiko), section 4, and of "Token Mixer I",
 //      section "Kimi Delta Attention: Improving Delta Rule with Fine-grained
 //      Gating", in the d_v x d_k orientation.  Every product is one
@@ -29,20 +30,23 @@
 //               Lane 1 issues the TMA stores of the output tiles (and, for
 //               the gated output, the loads of the gate tiles).
 //   warp 1      TMEM allocation and the MMA issuer (one lane), in the order
-//               X^T(n), O^T(n), dS(n), O(n), U^T(n+1), so the products that do
-//               not depend on the state run while the state is updated
+//               XO(n) = S_n [Q<-; -W]^T (in two halves, each issued once its
+//               half of the bf16 S_n is in smem), SO(n) = V_new^T(n)
+//               [K_tail^T; Aqk]^T, U^T(n+1), so the product that does not
+//               depend on the state runs while the conversion warps work
 //   warps 2-9   the state conversions, split by columns between warps 2-5
 //               and 6-9: on the sequential path S (TMEM) -> bf16 smem and
 //               V_new^T (TMEM) -> bf16 smem; off it, in the gaps while the
 //               tensor core runs, S *= gamma_C in TMEM.
-//   warps 10-13 the output epilogue, one chunk behind the MMAs (the O^T
-//               accumulator is double-buffered): O^T (TMEM) -> bf16 staging
-//               tile -> TMA store.  With OEPI the layer's gated output is
+//   warps 10-13 the output epilogue, one chunk behind the MMAs (the
+//               [V_new^T | O^T] accumulator is double-buffered): O^T (TMEM) ->
+//               bf16 staging tile -> TMA store, then the O^T columns are
+//               zeroed for the chunk after next.  With OEPI the layer's gated output is
 //               fused in: y_t = Sigmoid(gate_t) * RMSNorm(o_t) per head
 //               ("Token Mixer I", section "The Kimi Linear Model
 //               Architecture", the output equation before W_o), RMSNorm over
 //               the d_v channels in fp32 straight from the accumulator.
-// The sequential chain per chunk is dS -> S to bf16 -> X^T -> V_new -> dS.
+// The sequential chain per chunk is SO -> S to bf16 -> XO -> V_new -> SO.
 // Every wait is bounded (about a second); on timeout the kernel records
 // GDR_ERR_TIMEOUT in a device status word, lets the copies and MMAs it
 // issued finish, frees its tensor memory and returns.
@@ -72,12 +76,13 @@ constexpr long long kDrainBudget = 500000000LL;   // waits for copies and MMAs a
 // shared memory map (bytes from a 1024-aligned base).  The input tiles of a
 // chunk form one stage (gamma_C in a slot of its own); two stages alternate
 // by chunk parity.
-constexpr uint32_t ST_W = 0;                       // W^T, MN-major [128 ch x 64 tok]      16 KB
-constexpr uint32_t ST_Q = 16384;                   // Q<-                                  16 KB
-constexpr uint32_t ST_KT = 32768;                  // K_tail                               16 KB
-constexpr uint32_t ST_V = 49152;                   // v                                    16 KB
-constexpr uint32_t ST_T = 65536;                   // T' (1 panel)                          8 KB
-constexpr uint32_t ST_AQ = 73728;                  // Aqk                                   8 KB
+constexpr uint32_t ST_WQ = 0;                      // [Q<-; -W]: per 64-channel panel (16 KB) the 64
+                                                   // token rows of Q<-, then the 64 of -W  32 KB
+constexpr uint32_t ST_V = 32768;                   // v                                    16 KB
+constexpr uint32_t ST_T = 49152;                   // T' (1 panel)                          8 KB
+constexpr uint32_t ST_KT = 57344;                  // [K_tail^T; Aqk]: the 128 key-channel rows of
+                                                   // K_tail^T, then the 64 token rows of Aqk  24 KB
+constexpr uint32_t ST_AQ = 73728;
 constexpr uint32_t STAGE = 81920;                  // stage stride (1024-aligned)
 constexpr uint32_t STAGE_TX = 4 * 16384 + 2 * 8192;   // bytes one stage receives
 constexpr uint32_t OFF_OST = 2 * STAGE;            // O^T staging for the TMA store (2 panels) 16 KB
@@ -91,21 +96,28 @@ constexpr uint32_t SMEM_USED = OFF_RSTD + 256;
 constexpr uint32_t SMEM_ALLOC = SMEM_USED + 1024;  // alignment slack
 static_assert(SMEM_ALLOC <= 232448, "dynamic shared memory above the 227 KB per-block limit");
 
-// TMEM columns (fp32)
-constexpr uint32_t TM_S = 0;      // state S_n, 128 columns: scaled by gamma_C in place, dS accumulated onto it
-constexpr uint32_t TM_V = 128;    // V_new^T accumulator, 64 columns
-constexpr uint32_t TM_O = 192;    // O^T accumulators, 2 x 64 columns
-constexpr uint32_t TM_COLS = 512; // allocation granularity (power of two); 320 used
+// TMEM columns (fp32): one region of 256 columns per chunk parity b, at
+// TM_REG * b.  For chunk n (b = n & 1) the region holds
+//   + TM_S  (128)  gamma_C(n) S_n, written by the conversion warps, onto which
+//                  the MMA accumulates the increment: S_{n+1} stays here while
+//                  chunk n + 1 reads it (and writes its own region)
+//   + TM_O  (64)   O^T(n)      } contiguous, so that [S | O^T] and
+//   + TM_V  (64)   V_new^T(n)  } [O^T | V_new^T] are each one accumulator
+constexpr uint32_t TM_REG = 256;
+constexpr uint32_t TM_S = 0;
+constexpr uint32_t TM_O = 128;
+constexpr uint32_t TM_V = 192;
+constexpr uint32_t TM_COLS = 512;
 
 enum Bar {
     B_FULL, B_FULL1,          // stage landed (TMA transaction bytes)
     B_EMPTY, B_EMPTY1,        // stage released (MMA commit)
     B_GFULL, B_GFULL1,        // gamma_C slot landed
     B_GEMPTY, B_GEMPTY1,      // gamma_C slot read by the state-update threads
-    B_SW_READY,               // S_n (bf16) in smem
-    B_X_FULL,                 // V_new^T(n) in TMEM
-    B_VN_READY,               // V_new^T(n) bf16 in smem, TM_V read, S_n scaled by gamma_C(n)
-    B_S_FULL,                 // S_{n+1} complete in TMEM
+    B_SW_LO, B_SW_HI,         // S_n (bf16) in smem: columns 0-31 and 64-95, then 32-63 and 96-127
+    B_X_FULL,                 // XO(n) done: V_new^T(n) in TMEM, the S Q<-^T part of O^T(n) in place
+    B_VN_READY,               // V_new^T(n) bf16 in smem, V part read, S_n scaled by gamma_C(n)
+    B_S_FULL,                 // S_{n+1} complete in TMEM (and O^T(n))
     B_O_FULL, B_O_FULL1,      // O^T(n) complete
     B_OACC_EMPTY, B_OACC_EMPTY1,   // O^T accumulator drained by the epilogue
     B_EPI_FULL,               // O^T staging tile written (warps 2-9)
@@ -118,7 +130,7 @@ static_assert(8 * B_COUNT + 8 <= 256, "barrier area");
 
 struct Maps {
     CUtensorMap w, q, kt, v, t, aq, o;   // Q<-, K_tail, v, O: [BH][T][128]; T', Aqk: [chunks*64][64];
-                                         // W^T: [chunks*128][64]
+                                         // -W: [chunks*64][128]; K_tail^T: [chunks*128][64]
     CUtensorMap og;                      // output gate [BH][T][128] (gated output only)
 };
 
@@ -189,11 +201,11 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
     if (tid == 0) {
         const uint32_t counts[B_COUNT] = {
             1, 1, 1, 1,       // stage full (TMA), stage empty (MMA commit)
-            1, 1, 256, 256,   // gamma full (TMA), gamma empty (warps 2-9)
-            256, 1, 256,      // sw ready (warps 2-9), x full (MMA), vn ready (warps 2-9)
+            1, 1, 8, 8,       // gamma full (TMA), gamma empty (warps 2-9)
+            8, 8, 1, 8,       // sw ready (warps 2-9, two halves), x full (MMA), vn ready (warps 2-9)
             1,                // s full (MMA)
-            1, 1, 128, 128,   // o full (MMA) x2, oacc empty (epilogue warps) x2
-            128, 1,  // epilogue tile written (epilogue warps), free (warp 0 lane 1)
+            1, 1, 4, 4,       // o full (MMA) x2, oacc empty (epilogue warps) x2
+            4, 1,             // epilogue tile written (epilogue warps), free (warp 0 lane 1)
             1,                // gate tile landed (TMA)
             1};
         for (int i = 0; i < B_COUNT; ++i) mbar_init(&bar[i], counts[i]);
@@ -219,6 +231,14 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
         record_error(6 /* GDR_ERR_TIMEOUT */);
         *abort_flag = 1;
         return false;
+    };
+    // Warp-wide roles arrive once per warp: the warp barrier orders every
+    // lane's prior writes (after its proxy and tcgen05 fences) before lane 0's
+    // arrive.  An arrive is an atomic on one shared word, so 32 of them from a
+    // warp would queue behind each other on the hand-offs of the chain.
+    auto warp_arrive = [&](int b) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[b]);
     };
     // Warp-wide roles wait with `waitw`: every lane acquires the barrier
     // phase, the result is made warp-uniform, and the warp reconverges -- the
@@ -290,14 +310,14 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
                 uint64_t *full = &bar[B_FULL + b];
                 if (!wait(B_EMPTY + b, upar ^ 1)) break;
                 mbar_arrive_expect_tx(full, STAGE_TX);
-                tma_load_2d(st + ST_W, &maps.w, full, 0, (head * nchunks + n) * kD);
-                tma_load_2d(st + ST_T, &maps.t, full, 0, crow);
+                tma_load_3d(st + ST_WQ, &maps.q, full, 0, t0, head);
+                tma_load_3d(st + ST_WQ + 16384, &maps.q, full, 64, t0, head);
+                tma_load_2d(st + ST_WQ + 8192, &maps.w, full, 0, crow);
+                tma_load_2d(st + ST_WQ + 16384 + 8192, &maps.w, full, 64, crow);
                 tma_load_3d(st + ST_V, &maps.v, full, 0, t0, head);
                 tma_load_3d(st + ST_V + 8192, &maps.v, full, 64, t0, head);
-                tma_load_3d(st + ST_Q, &maps.q, full, 0, t0, head);
-                tma_load_3d(st + ST_Q + 8192, &maps.q, full, 64, t0, head);
-                tma_load_3d(st + ST_KT, &maps.kt, full, 0, t0, head);
-                tma_load_3d(st + ST_KT + 8192, &maps.kt, full, 64, t0, head);
+                tma_load_2d(st + ST_T, &maps.t, full, 0, crow);
+                tma_load_2d(st + ST_KT, &maps.kt, full, 0, 2 * crow);   // key-channel rows of this chunk
                 tma_load_2d(st + ST_AQ, &maps.aq, full, 0, crow);
                 if (OEPI) {   // the epilogue's gate tile, warmed in L2 a chunk ahead of its load
                     tma_prefetch_l2_3d(&maps.og, 0, t0, head);
@@ -323,58 +343,67 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
         // ================================================================ MMA issuer
         if (lane == 0) {
             constexpr uint32_t ID_WU = idesc_bf16(128, 64, true, false);         // A (v) MN-major, B K-major
-            constexpr uint32_t ID_X = idesc_bf16(128, 64, false, true, true);    // -A, B (W) MN-major
-            constexpr uint32_t ID_O = idesc_bf16(128, 64, false, false);
-            constexpr uint32_t ID_S = idesc_bf16(128, 128, false, true);         // B MN-major
+            constexpr uint32_t ID_XO = idesc_bf16(128, 128, false, false);       // S [Q<-; -W]^T
+            constexpr uint32_t ID_SO = idesc_bf16(128, 192, false, false);       // V_new^T [K_tail^T; Aqk]^T
             // descriptors of the two operand layouts at the base of shared memory:
             // the address field counts 16-byte units, so a byte offset adds directly
             const uint64_t d16 = sdesc_sw128(sbase, 16, 1024), d8k = sdesc_sw128(sbase, 8192, 1024);
             auto K16 = [&](uint32_t off) { return d16 + (uint64_t)(off >> 4); };   // K-major tile
             auto MN = [&](uint32_t off) { return d8k + (uint64_t)(off >> 4); };    // MN-major tile, panels 8 KB apart
-            // U^T = V^T T'^T of chunk n (stage n & 1); it has to wait until
-            // V_new^T of the previous chunk has left TM_V
-            auto mma_u = [&](int n) {
+            // U^T = V^T T'^T of chunk n into V_new^T of region n & 1, tokens 16 s .. 16 s + 15
+            auto mma_u = [&](int n, int s) {
                 const uint32_t st = (n & 1) * STAGE;
-#pragma unroll
-                for (int s = 0; s < 4; ++s) mma_bf16(tmem + TM_V, MN(st + ST_V + s * 2048), K16(st + ST_T + s * 32), ID_WU, s > 0);
+                mma_bf16(tmem + TM_REG * (n & 1) + TM_V, MN(st + ST_V + s * 2048), K16(st + ST_T + s * 32), ID_WU, s > 0);
+            };
+            // [O^T | V_new^T] += S [Q<-; -W]^T, key channels 16 s .. 16 s + 15
+            auto mma_xo = [&](uint32_t st, uint32_t reg, int s) {
+                mma_bf16(reg + TM_O, K16(OFF_S + (s >> 2) * 16384 + (s & 3) * 32),
+                         K16(st + ST_WQ + (s >> 2) * 16384 + (s & 3) * 32), ID_XO, 1);
             };
             bool ok = nchunks > 0 && wait(B_FULL, 0);
             if (ok) {
                 tc_fence_after();
-                mma_u(0);
+                for (int s = 0; s < 4; ++s) mma_u(0, s);
             }
+            // U^T(n + 1) does not depend on the state; it is issued last, when
+            // the stage of chunk n + 1 (loaded once the MMAs of chunk n - 1 had
+            // released it) has landed, and runs while S_{n+1} is converted.
             for (int n = 0; n < nchunks && ok; ++n) {
                 const int b = n & 1;
                 const uint32_t par = (uint32_t)(n & 1), upar = (uint32_t)((n >> 1) & 1);
                 const uint32_t st = b * STAGE;
-                // ---- V_new^T += -S W^T ; O^T = S Q<-^T
-                if (!wait(B_SW_READY, par) || !wait(B_OACC_EMPTY + b, upar ^ 1)) break;
+                const uint32_t reg = tmem + TM_REG * b;
+                const bool more = n + 1 < nchunks;
+                // ---- O^T = S Q<-^T and V_new^T = U^T - S W^T in one product (the O^T
+                // part was zeroed by the epilogue), the half of S converted first first
+                if (!wait(B_SW_LO, par) || !wait(B_OACC_EMPTY + b, upar ^ 1)) break;
                 tc_fence_after();
-#pragma unroll
-                for (int s = 0; s < 8; ++s)
-                    mma_bf16(tmem + TM_V, K16(OFF_S + (s >> 2) * 16384 + (s & 3) * 32), MN(st + ST_W + s * 2048), ID_X, 1);
+                mma_xo(st, reg, 0);
+                mma_xo(st, reg, 1);
+                mma_xo(st, reg, 4);
+                mma_xo(st, reg, 5);
+                if (!wait(B_SW_HI, par)) break;
+                tc_fence_after();
+                mma_xo(st, reg, 2);
+                mma_xo(st, reg, 3);
+                mma_xo(st, reg, 6);
+                mma_xo(st, reg, 7);
                 mma_commit(&bar[B_X_FULL]);
-#pragma unroll
-                for (int s = 0; s < 8; ++s)
-                    mma_bf16(tmem + TM_O + 64 * b, K16(OFF_S + (s >> 2) * 16384 + (s & 3) * 32),
-                             K16(st + ST_Q + (s >> 2) * 8192 + (s & 3) * 32), ID_O, s > 0);
-                // ---- S += V_new^T K_tail (the sequential path; S already scaled by
-                // gamma_C); O^T += V_new^T Aqk^T
+                // ---- [S | O^T] += V_new^T [K_tail^T; Aqk]^T: the state increment
+                // (the sequential path; S already scaled by gamma_C) and the
+                // intra-chunk part of the output in one product
                 if (!wait(B_VN_READY, par)) break;
                 tc_fence_after();
 #pragma unroll
-                for (int s = 0; s < 4; ++s) mma_bf16(tmem + TM_S, K16(OFF_VN + s * 32), MN(st + ST_KT + s * 2048), ID_S, 1);
+                for (int s = 0; s < 4; ++s) mma_bf16(reg + TM_S, K16(OFF_VN + s * 32), K16(st + ST_KT + s * 32), ID_SO, 1);
                 mma_commit(&bar[B_S_FULL]);
-#pragma unroll
-                for (int s = 0; s < 4; ++s)
-                    mma_bf16(tmem + TM_O + 64 * b, K16(OFF_VN + s * 32), K16(st + ST_AQ + s * 32), ID_O, 1);
                 mma_commit(&bar[B_O_FULL + b]);
                 mma_commit(&bar[B_EMPTY + b]);   // every read of this stage is issued
-                // ---- U^T of the next chunk
-                if (n + 1 < nchunks) {
+                // ---- U^T(n + 1)
+                if (more) {
                     if (!wait(B_FULL + (b ^ 1), (uint32_t)(((n + 1) >> 1) & 1))) break;
                     tc_fence_after();
-                    mma_u(n + 1);
+                    for (int s = 0; s < 4; ++s) mma_u(n + 1, s);
                 }
             }
             // every MMA issued above has completed before TMEM is released
@@ -383,18 +412,18 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
         }
     } else if (warp < 10) {
         // ================================================================ state update, conversions, epilogue
-        // The state S_n lives at TM_S.  At chunk n these warps copy it to bf16
-        // smem for the MMAs of chunk n (on the sequential path), then scale it
-        // in place by gamma_C(n) (off the path, while X^T(n) runs); the MMA of
-        // S += V_new^T K_tail then leaves S_{n+1} in TM_S.  Warps 2-5 take key
-        // channels 64..127 of S and tokens 32..63 of V_new^T, warps 6-9 the
-        // other halves; the same split applies to W^T and O^T.
+        // The state S_n lives in region (n + 1) & 1.  At chunk n these warps copy
+        // it to bf16 smem for the MMAs of chunk n (on the sequential path), then
+        // store gamma_C(n) S_n into region n & 1 (off the path, while XO(n)
+        // runs); the MMA of S += V_new^T K_tail then leaves S_{n+1} there.
+        // Warps 2-5 take key channels 64..127 of S and tokens 32..63 of V_new^T,
+        // warps 6-9 the other halves.
         const bool ga = warp < 6;                     // warps 2-5
         const uint32_t lq = 32u * (warp & 3);         // TMEM lane quarter of this warp
-        const int i = (int)lq + lane;                 // TMEM lane: row of S / V_new^T / O^T, key channel of W^T
+        const int i = (int)lq + lane;                 // TMEM lane: row of S / V_new^T / O^T
         const uint32_t trow = tmem + (lq << 16);
         const int sc0 = ga ? 64 : 0;                  // first state column of this warp
-        const int vc0 = ga ? 32 : 0;                  // first V_new^T / W^T / O^T column (token)
+        const int vc0 = ga ? 32 : 0;                  // first V_new^T / O^T column (token)
         // initial state into TMEM
 #pragma unroll
         for (int cb = 0; cb < 4; ++cb) {
@@ -402,32 +431,46 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
 #pragma unroll
             for (int j = 0; j < 16; ++j)
                 r[j] = __float_as_uint(S0 ? S0[((size_t)head * kD + i) * kD + sc0 + 16 * cb + j] : 0.f);
-            tmem_st16(trow + TM_S + sc0 + 16 * cb, r);
+            tmem_st16(trow + TM_REG + TM_S + sc0 + 16 * cb, r);   // read by chunk 0 from region 1
+        }
+        // the O^T parts of both regions start at zero (the first products
+        // accumulate onto them; later the epilogue zeroes what it drained)
+        {
+            uint32_t z[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) z[j] = 0u;
+#pragma unroll
+            for (int bb = 0; bb < 2; ++bb)
+#pragma unroll
+                for (int cb = 0; cb < 2; ++cb) tmem_st16(trow + TM_REG * bb + TM_O + vc0 + 16 * cb, z);
         }
         tmem_st_wait();
-        // One pass over this warp's 64 columns of S_n (TMEM): the bf16 copy goes
-        // to smem and is released to the MMAs at once (the sequential path);
-        // then S_n *= gamma_C(n) is stored back in place for the accumulation
-        // of chunk n's increment.
+        // One pass over this warp's 64 columns of S_n (TMEM, region (n + 1) & 1):
+        // the bf16 copy goes to smem and is released to the MMAs at once, in two
+        // halves (the sequential path); then gamma_C(n) S_n is stored into
+        // region n & 1 for the accumulation of chunk n's increment.
         auto state_pass = [&](int n) -> bool {
             unsigned char *sp = sm + OFF_S + (sc0 >> 6) * 16384;
             uint32_t r[4][16];
 #pragma unroll
-            for (int cb = 0; cb < 4; ++cb) tmem_ld16(trow + TM_S + sc0 + 16 * cb, r[cb]);
+            for (int cb = 0; cb < 4; ++cb) tmem_ld16(trow + TM_REG * ((n + 1) & 1) + TM_S + sc0 + 16 * cb, r[cb]);
             tmem_ld_wait(r[0]);
             reg_touch(r[1]);
             reg_touch(r[2]);
             reg_touch(r[3]);
 #pragma unroll
-            for (int cb = 0; cb < 4; ++cb) {
-                uint4 lo, hi;
-                pack16(r[cb], lo, hi);
-                *reinterpret_cast<uint4 *>(sp + sw128_off(i, 16 * cb)) = lo;
-                *reinterpret_cast<uint4 *>(sp + sw128_off(i, 16 * cb + 8)) = hi;
+            for (int hf = 0; hf < 2; ++hf) {
+#pragma unroll
+                for (int cb = 2 * hf; cb < 2 * hf + 2; ++cb) {
+                    uint4 lo, hi;
+                    pack16(r[cb], lo, hi);
+                    *reinterpret_cast<uint4 *>(sp + sw128_off(i, 16 * cb)) = lo;
+                    *reinterpret_cast<uint4 *>(sp + sw128_off(i, 16 * cb + 8)) = hi;
+                }
+                fence_async_smem();
+                tc_fence_before();
+                warp_arrive(hf ? B_SW_HI : B_SW_LO);
             }
-            fence_async_smem();
-            tc_fence_before();
-            mbar_arrive(&bar[B_SW_READY]);
             if (!waitw(B_GFULL + (n & 1), (uint32_t)((n >> 1) & 1))) return false;
             const float4 *gm = reinterpret_cast<const float4 *>(sm + OFF_GAM + (n & 1) * 512) + (sc0 >> 2);
 #pragma unroll
@@ -440,10 +483,10 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
                     r[cb][4 * q + 2] = __float_as_uint(__uint_as_float(r[cb][4 * q + 2]) * gv.z);
                     r[cb][4 * q + 3] = __float_as_uint(__uint_as_float(r[cb][4 * q + 3]) * gv.w);
                 }
-                tmem_st16(trow + TM_S + sc0 + 16 * cb, r[cb]);
+                tmem_st16(trow + TM_REG * (n & 1) + TM_S + sc0 + 16 * cb, r[cb]);
             }
             tmem_st_wait();
-            mbar_arrive(&bar[B_GEMPTY + (n & 1)]);
+            warp_arrive(B_GEMPTY + (n & 1));
             return true;
         };
         bool ok = true;
@@ -463,7 +506,7 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
 #pragma unroll
             for (int cb = 0; cb < 2; ++cb) {
                 uint32_t r[16];
-                tmem_ld16(trow + TM_V + vc0 + 16 * cb, r);
+                tmem_ld16(trow + TM_REG * (n & 1) + TM_V + vc0 + 16 * cb, r);
                 tmem_ld_wait(r);
                 uint4 lo, hi;
                 pack16(r, lo, hi);
@@ -472,7 +515,7 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
             }
             fence_async_smem();
             tc_fence_before();
-            mbar_arrive(&bar[B_VN_READY]);   // also: S_n scaled
+            warp_arrive(B_VN_READY);   // also: S_n scaled
         }
         // ---- final state S_N: the last accumulation has completed
         if (ok && nchunks > 0 && waitw(B_S_FULL, (uint32_t)((nchunks - 1) & 1))) {
@@ -481,7 +524,7 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
 #pragma unroll
                 for (int cb = 0; cb < 4; ++cb) {
                     uint32_t r[16];
-                    tmem_ld16(trow + TM_S + sc0 + 16 * cb, r);
+                    tmem_ld16(trow + TM_REG * ((nchunks - 1) & 1) + TM_S + sc0 + 16 * cb, r);
                     tmem_ld_wait(r);
                     float4 *dst = reinterpret_cast<float4 *>(ST + ((size_t)head * kD + i) * kD + sc0 + 16 * cb);
 #pragma unroll
@@ -518,7 +561,17 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
             if (OEPI) ok = epi_all(ok);   // the four warps go on (or stop) together
             if (!ok) break;
             tc_fence_after();
-            const uint32_t oc = trow + TM_O + 64 * bb;
+            const uint32_t oc = trow + TM_REG * bb + TM_O;
+            // after the last read of O^T(m) its columns are zeroed: the next
+            // product into this accumulator adds onto them
+            auto zero_oacc = [&]() {
+                uint32_t z[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) z[j] = 0u;
+#pragma unroll
+                for (int cb = 0; cb < 4; ++cb) tmem_st16(oc + 16 * cb, z);
+                tmem_st_wait();
+            };
             if (!OEPI) {
 #pragma unroll 2
                 for (int cb = 0; cb < 8; ++cb) {
@@ -530,10 +583,11 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
                         *reinterpret_cast<__nv_bfloat16 *>(ost + cb * 1024 + j * 128 + ((c8 ^ (uint32_t)j) << 4)) =
                             __float2bfloat16_rn(__uint_as_float(r[j]));
                 }
+                zero_oacc();
                 tc_fence_before();
-                mbar_arrive(&bar[B_OACC_EMPTY + bb]);
+                warp_arrive(B_OACC_EMPTY + bb);
                 fence_async_smem();
-                mbar_arrive(&bar[B_EPI_FULL]);
+                warp_arrive(B_EPI_FULL);
             } else {
                 // pass 1, per 32 tokens: lane L ends with this warp's partial sum of
                 // token 32 h + L; warp (w & 3) == 0 adds the four up
@@ -615,10 +669,11 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
                                                             ((c8 ^ (uint32_t)((j + 1) & 7)) << 4)) = (unsigned short)(yb >> 16);
                     }
                 }
+                zero_oacc();
                 tc_fence_before();
-                mbar_arrive(&bar[B_OACC_EMPTY + bb]);
+                warp_arrive(B_OACC_EMPTY + bb);
                 fence_async_smem();   // the tile is read next by the TMA store
-                mbar_arrive(&bar[B_EPI_FULL]);
+                warp_arrive(B_EPI_FULL);
             }
         }
     }
@@ -690,9 +745,9 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream, int *launch
         const cuuint64_t str_bf[2] = {(cuuint64_t)kD * 2, (cuuint64_t)a.T * kD * 2};
         const cuuint32_t box_bf[3] = {64, 64, 1};
         // Gated Delta Rule-2: U = T' Z with Z = w * v, formed by the prep kernel
-        void *tiles[4] = {w.Ql, w.Kt, a.gdr2 ? static_cast<void *>(w.Z) : const_cast<void *>(a.v), a.O};
-        CUtensorMap *dst[4] = {&maps.q, &maps.kt, &maps.v, &maps.o};
-        for (int i = 0; i < 4; ++i)
+        void *tiles[3] = {w.Ql, a.gdr2 ? static_cast<void *>(w.Z) : const_cast<void *>(a.v), a.O};
+        CUtensorMap *dst[3] = {&maps.q, &maps.v, &maps.o};
+        for (int i = 0; i < 3; ++i)
             if (!make_map(dst[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, tiles[i], dims3, str_bf, box_bf,
                           CU_TENSOR_MAP_SWIZZLE_128B))
                 return cudaErrorInvalidValue;
@@ -702,9 +757,14 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream, int *launch
         const cuuint64_t dims2[2] = {(cuuint64_t)kC, (cuuint64_t)BH * nchunks * kC};
         const cuuint64_t str2[1] = {(cuuint64_t)kC * 2};
         const cuuint32_t box2[2] = {64, 64};
-        const cuuint64_t dimsw[2] = {(cuuint64_t)kC, (cuuint64_t)BH * nchunks * kD};
-        const cuuint32_t boxw[2] = {64, 128};
-        if (!make_map(&maps.w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w.W, dimsw, str2, boxw, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        // -W: [chunks * 64 token rows][128 channels], boxes of 64 x 64
+        const cuuint64_t dimsw[2] = {(cuuint64_t)kD, (cuuint64_t)BH * nchunks * kC};
+        const cuuint64_t strw[1] = {(cuuint64_t)kD * 2};
+        // K_tail^T: [chunks * 128 key-channel rows][64 tokens], one box of 64 x 128
+        const cuuint64_t dimsk[2] = {(cuuint64_t)kC, (cuuint64_t)BH * nchunks * kD};
+        const cuuint32_t boxk[2] = {64, 128};
+        if (!make_map(&maps.w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w.W, dimsw, strw, box2, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_map(&maps.kt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w.Kt, dimsk, str2, boxk, CU_TENSOR_MAP_SWIZZLE_128B) ||
             !make_map(&maps.t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w.T, dims2, str2, box2, CU_TENSOR_MAP_SWIZZLE_128B) ||
             !make_map(&maps.aq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w.Aqk, dims2, str2, box2, CU_TENSOR_MAP_SWIZZLE_128B))
             return cudaErrorInvalidValue;

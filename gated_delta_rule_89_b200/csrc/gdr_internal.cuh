@@ -55,8 +55,9 @@ struct StepArgs {
 // The tensor-core path's scratch, carved out of ChunkArgs::workspace (every
 // part starts on a 256-byte boundary):
 //   T, Aqk   [B*H*chunks][64][64] bf16    T' = (I + A)^{-1} Diag(beta) and Aqk
-//   W        [B*H*chunks][128][64] bf16   W^T, W = T' K<- (key channel rows)
-//   Ql, Kt   [B, H, T, 128] bf16          Q<-, K_tail (chunk-relative decays)
+//   W        [B*H*chunks][64][128] bf16   -W, W = T' K<- (token rows, the layout of Q<-)
+//   Ql       [B, H, T, 128] bf16          Q<- (chunk-relative decays)
+//   Kt       [B*H*chunks][128][64] bf16   K_tail^T (key channel rows; zeros past T)
 //   gam      [B*H*chunks][128] fp32       gamma_C per key channel
 //   Z        [B, H, T, 128] bf16          Gated Delta Rule-2 only: w * v
 struct TcWorkspace {
@@ -67,7 +68,7 @@ struct TcWorkspace {
 inline size_t tc_workspace_bytes(int B, int H, int T, bool gdr2 = false)
 {
     const size_t bh = (size_t)B * H, nch = (size_t)(T + 63) / 64;
-    return 2 * bh * nch * 64 * 64 * 2 + bh * nch * 128 * 64 * 2 + 2 * bh * (size_t)T * 128 * 2 + bh * nch * 128 * 4 +
+    return 2 * bh * nch * 64 * 64 * 2 + 2 * bh * nch * 128 * 64 * 2 + bh * (size_t)T * 128 * 2 + bh * nch * 128 * 4 +
            (gdr2 ? bh * (size_t)T * 128 * 2 : 0);
 }
 inline TcWorkspace carve_tc_workspace(void *ws, int B, int H, int T, bool gdr2 = false)
@@ -84,7 +85,7 @@ inline TcWorkspace carve_tc_workspace(void *ws, int B, int H, int T, bool gdr2 =
     w.Ql = reinterpret_cast<__nv_bfloat16 *>(p);
     p += bh * (size_t)T * 128 * 2;
     w.Kt = reinterpret_cast<__nv_bfloat16 *>(p);
-    p += bh * (size_t)T * 128 * 2;
+    p += bh * nch * 128 * 64 * 2;
     w.gam = reinterpret_cast<float *>(p);
     p += bh * nch * 128 * 4;
     w.Z = gdr2 ? reinterpret_cast<__nv_bfloat16 *>(p) : nullptr;

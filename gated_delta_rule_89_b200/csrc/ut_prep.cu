@@ -6,7 +6,7 @@
 //   T' = (I + A)^{-1} Diag(beta)
 // and writes T' and Aqk (bf16, row-major 64 x 64) to the workspace, together
 // with the operands of the state scan that do not depend on the state:
-// W = T' K<- (stored transposed), Q<-, K_tail and gamma_C (defined where they
+// -W = -T' K<- (token-major), Q<-, K_tail^T and gamma_C (defined where they
 // are written).  T' is
 // the matrix the UT transform of "Token Mixer I", section "Kimi Delta
 // Attention: Improving Delta Rule with Fine-grained Gating" calls
@@ -73,7 +73,7 @@ constexpr int kLdA = 68;       // fp32 row stride: 16-byte rows, conflict-free f
 // shared memory (offsets from a 1024-byte aligned base)
 constexpr uint32_t OFF_K = 0;                      // Khat (or k), two swizzled panels   16 KB
 constexpr uint32_t OFF_Q = 16384;                  // Qhat (or q); then T' bf16 [64][72]   16 KB
-constexpr uint32_t OFF_KC = 32768;                 // Kchk; then W^T staging, 2 KB/warp   16 KB
+constexpr uint32_t OFF_KC = 32768;                 // Kchk; then -W staging [64][128] bf16  16 KB
 constexpr int kLdT = 72;                           // bf16 row stride of T' (ldmatrix conflict free)
 constexpr uint32_t OFF_BD = 49152;                 // bd[4][128], 1/bd[4][128] fp32         4 KB
 constexpr int kLdD = 24;       // row stride of the 16 x 16 blocks (conflict-free mma B fragments)
@@ -101,14 +101,6 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], uint32_t addr)
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                  : "r"(addr));
-}
-
-// two 8x8 bf16 matrices from mma fragments, stored transposed (lanes 0..15
-// give the row addresses of the transposed matrices)
-__device__ __forceinline__ void stsm_x2_trans(uint32_t addr, uint32_t r0, uint32_t r1)
-{
-    asm volatile("stmatrix.sync.aligned.m8n8.x2.trans.shared.b16 [%0], {%1, %2};" ::"r"(addr), "r"(r0), "r"(r1)
-                 : "memory");
 }
 
 __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
@@ -463,14 +455,16 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
         }
         __syncthreads();
 
-        // ---- chunk-relative operands of the state scan, to global memory in
-        // the layout of k ([B, H, T, 128] bf16), G counted from the chunk start:
-        //   Q<-_r = q_r exp(G_r),  K_tail_r = k_r exp(G_C - G_r)
+        // ---- chunk-relative operands of the state scan, G counted from the
+        // chunk start:
+        //   Q<-_r = q_r exp(G_r)       in the layout of k ([B, H, T, 128] bf16)
+        //   K_tail_r = k_r exp(G_C - G_r)   transposed per chunk ([chunks][128][64])
         // and gamma_C = exp(G_C) per key channel (fp32, [B H chunks][128]).
         // Formed in fp32 from the registers above, with the block decays bd_J.
         // (K<-_r = k_r exp(G_r) is only needed inside W = T' K<-, formed below.)
         {
             const size_t e0 = row0 * kDK + c;
+            uint2 kt[8];   // K_tail of this thread's 8 rows x 4 channels (zero past T)
             if (!SCALAR) {
                 float2 Fa = make_float2(1.f, 1.f), Fb = Fa, Ba = Fa, Bb = Fa;
 #pragma unroll
@@ -505,12 +499,10 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
                 pb = half ? Bb : fmul2(Bb, ob);
 #pragma unroll
                 for (int rr = 7; rr >= 0; --rr) {
-                    if (rbase + rr < nrows) {
-                        const size_t e = e0 + (size_t)(rbase + rr) * kDK;
-                        const float2 nk = make_float2(ik(rr), ik(rr));
-                        *reinterpret_cast<uint2 *>(Kto + e) =
-                            make_uint2(scale2p(kr[rr].x, PRO ? fmul2(pa, nk) : pa), scale2p(kr[rr].y, PRO ? fmul2(pb, nk) : pb));
-                    }
+                    const float2 nk = make_float2(ik(rr), ik(rr));
+                    kt[rr] = rbase + rr < nrows ? make_uint2(scale2p(kr[rr].x, PRO ? fmul2(pa, nk) : pa),
+                                                             scale2p(kr[rr].y, PRO ? fmul2(pb, nk) : pb))
+                                                : make_uint2(0u, 0u);
                     pa = fmul2(pa, make_float2(gv[rr].x, gv[rr].y));
                     pb = fmul2(pb, make_float2(gv[rr].z, gv[rr].w));
                 }
@@ -524,12 +516,33 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
                         const float2 fe = make_float2(ef * iq(rr), ef * iq(rr)), ft = make_float2(et * ik(rr), et * ik(rr));
                         const size_t e = e0 + (size_t)r * kDK;
                         *reinterpret_cast<uint2 *>(Qlo + e) = make_uint2(scale2p(qr[rr].x, fe), scale2p(qr[rr].y, fe));
-                        *reinterpret_cast<uint2 *>(Kto + e) = make_uint2(scale2p(kr[rr].x, ft), scale2p(kr[rr].y, ft));
+                        kt[rr] = make_uint2(scale2p(kr[rr].x, ft), scale2p(kr[rr].y, ft));
+                    } else {
+                        kt[rr] = make_uint2(0u, 0u);
                     }
                 }
                 if (R == 0 && half == 0) {
                     const float gl = __expf(Gl);
                     *reinterpret_cast<float4 *>(gamo + (size_t)ci * kDK + c) = make_float4(gl, gl, gl, gl);
+                }
+            }
+            // K_tail^T [128 channels][64 tokens] per chunk, the operand layout of
+            // the scan's state update: per channel, this thread's 8 consecutive
+            // tokens are one 16-byte store (the two halves of a warp fill whole
+            // 32-byte sectors); the tokens past T of a ragged chunk are zeros.
+            {
+                __nv_bfloat16 *kdst = Kto + ((size_t)ci * kDK + c) * kC + rbase;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint32_t sel = (j & 1) ? 0x7632u : 0x5410u;   // high or low bf16 of each pair
+                    uint32_t w[4];
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        const uint32_t a = (j < 2) ? kt[2 * m].x : kt[2 * m].y;
+                        const uint32_t b = (j < 2) ? kt[2 * m + 1].x : kt[2 * m + 1].y;
+                        w[m] = __byte_perm(a, b, sel);
+                    }
+                    *reinterpret_cast<uint4 *>(kdst + (size_t)j * kC) = make_uint4(w[0], w[1], w[2], w[3]);
                 }
             }
             if (GDR2) {
@@ -736,15 +749,19 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
         }
         __syncthreads();
 
-        // ---- W = T' K<- for the state scan, stored as W^T [128 channels][64 tokens].
+        // ---- W = T' K<- for the state scan, stored negated and token-major,
+        // -W [64 tokens][128 channels] (the layout of Q<-), so that the scan takes
+        // -S W^T and S Q<-^T in one product.
         // Per-channel gate: K<-_r = Khat_r * F_R with F_R = prod_{J<R} bd_J (row r
         // in block R), so W = sum_R (T'[:, block R] Khat_R) Diag(F_R): one fp32
         // accumulator per block, combined after the products.  Scalar gate: the
         // decay sits in T' (above) and Khat is k.  Warp w owns channels
         // 16w..16w+15 (two 8-channel tiles), all 64 tokens, in 4 token blocks.
+        // The fragments go to a staging tile (16-byte chunks XOR-swizzled by
+        // token, conflict free both ways), which is then stored in whole rows.
+        unsigned char *wstg = sm + OFF_KC;
         {
             const int c0 = 16 * warp;
-            unsigned char *stg = sm + OFF_KC + warp * 2048;   // 16 rows x 128 B, 16-byte chunks XOR-swizzled
             const uint32_t khat = smem_u32(sm + OFF_K);
 #pragma unroll
             for (int ct = 0; ct < 2; ++ct) {
@@ -780,26 +797,22 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
                         w4[2] = fmaf(accR[2], fr[R].x, w4[2]);
                         w4[3] = fmaf(accR[3], fr[R].y, w4[3]);
                     }
-                    // W^T[channel][token]: the fragment (tokens 16I + g (+8), channels
-                    // 2t, 2t + 1) is two 8x8 matrices; stored transposed, matrix h
-                    // lands in channel rows 8 ct .. 8 ct + 7, token chunk 2I + h.
-                    {
-                        const int row = 8 * ct + (lane & 7), chunk = (2 * I + ((lane >> 3) & 1)) ^ (row & 7);
-                        stsm_x2_trans(smem_u32(stg + row * 128 + chunk * 16), pack2(w4[0], w4[1]), pack2(w4[2], w4[3]));
-                    }
+                    // fragment: tokens 16I + g (+8), channels cs + 2t, + 1
+                    const int r0 = 16 * I + g, ck = cs >> 3;
+                    *reinterpret_cast<uint32_t *>(wstg + r0 * 256 + ((ck ^ (r0 & 7)) << 4) + 4 * t) = pack2(-w4[0], -w4[1]);
+                    *reinterpret_cast<uint32_t *>(wstg + (r0 + 8) * 256 + ((ck ^ (r0 & 7)) << 4) + 4 * t) =
+                        pack2(-w4[2], -w4[3]);
                 }
             }
-            __syncwarp();
-            // this warp's 16 rows (2 KB) of W^T to global: lane -> row lane/2, half a row
-            {
-                const int row = lane >> 1, h = lane & 1;
-                __nv_bfloat16 *dst = Wout + ((size_t)ci * kDK + c0 + row) * kC + 32 * h;
+        }
+        __syncthreads();
+        {
+            __nv_bfloat16 *wdst = Wout + (size_t)ci * kC * kDK;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int chunk = 4 * h + q;
-                    *reinterpret_cast<uint4 *>(dst + 8 * q) =
-                        *reinterpret_cast<const uint4 *>(stg + row * 128 + ((chunk ^ (row & 7)) << 4));
-                }
+            for (int q = tid; q < kC * 16; q += kThreads) {
+                const int r = q >> 4, ck = q & 15;
+                *reinterpret_cast<uint4 *>(wdst + r * kDK + 8 * ck) =
+                    *reinterpret_cast<const uint4 *>(wstg + r * 256 + ((ck ^ (r & 7)) << 4));
             }
         }
         // the next chunk overwrites Khat, T' and the staging area

@@ -183,10 +183,10 @@ def test_step_argument_validation(L):
 
 
 def _tc_workspace(B, H, T):
-    # per chunk: T' and Aqk (2 x 64 x 64 bf16), W^T (128 x 64 bf16) and gamma_C
-    # (128 fp32); per token: Q<-, K_tail (2 x 128 bf16)
+    # per chunk: T' and Aqk (2 x 64 x 64 bf16), -W and K_tail^T (2 x 64 x 128
+    # bf16, whole chunks) and gamma_C (128 fp32); per token: Q<- (128 bf16)
     nch = (T + 63) // 64
-    return B * H * (nch * (2 * 64 * 64 * 2 + 128 * 64 * 2 + 128 * 4) + T * 2 * 128 * 2)
+    return B * H * (nch * (2 * 64 * 64 * 2 + 2 * 128 * 64 * 2 + 128 * 4) + T * 128 * 2)
 
 
 def test_workspace_query(L):

@@ -73,12 +73,13 @@ constexpr int kLdA = 68;       // fp32 row stride: 16-byte rows, conflict-free f
 // shared memory (offsets from a 1024-byte aligned base)
 constexpr uint32_t OFF_K = 0;                      // Khat (or k), two swizzled panels   16 KB
 constexpr uint32_t OFF_Q = 16384;                  // Qhat (or q); then T' bf16 [64][72]   16 KB
-constexpr uint32_t OFF_KC = 32768;                 // Kchk; then -W staging [64][128] bf16  16 KB
+constexpr uint32_t OFF_KC = 32768;                 // Kchk                                 16 KB
 constexpr int kLdT = 72;                           // bf16 row stride of T' (ldmatrix conflict free)
 constexpr uint32_t OFF_BD = 49152;                 // bd[4][128], 1/bd[4][128] fp32         4 KB
 constexpr int kLdD = 24;       // row stride of the 16 x 16 blocks (conflict-free mma B fragments)
 constexpr uint32_t OFF_D = OFF_BD + 4096;          // D_i = N_ii^{-1}, [4][16][24]           6 KB
-constexpr uint32_t OFF_A = OFF_D + 4 * 16 * kLdD * 4;   // A
+constexpr uint32_t OFF_A = OFF_D + 4 * 16 * kLdD * 4;   // A; then the -W staging tile [64][128] bf16
+static_assert(kC * kLdA * 4 >= kC * kDK * 2, "the -W staging tile fits in the A tile");
 constexpr uint32_t OFF_AQ = OFF_A + kC * kLdA * 4; // Aqk, then Nt / X'
 constexpr uint32_t OFF_U = OFF_AQ + kC * kLdA * 4; // U_10, U_21, U_20 [3][16][24]
 constexpr uint32_t OFF_BETA = OFF_U + 3 * 16 * kLdD * 4;   // beta, two buffers by chunk parity
@@ -233,6 +234,20 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
     const int warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t = lane & 3;   // mma fragment coordinates
 
+    // -W of chunk cw leaves the staging tile in whole 256-byte token rows (16-byte
+    // chunks XOR-swizzled by token).  It runs during the next chunk's operand
+    // loads, so that their latency covers it; the A tile is next written by
+    // that chunk's block products.
+    const unsigned char *wstg = sm + OFF_A;
+    auto store_w = [&](int cw) {
+        __nv_bfloat16 *wdst = Wout + (size_t)cw * kC * kDK;
+#pragma unroll
+        for (int q = tid; q < kC * 16; q += kThreads) {
+            const int r = q >> 4, ck = q & 15;
+            *reinterpret_cast<uint4 *>(wdst + r * kDK + 8 * ck) =
+                *reinterpret_cast<const uint4 *>(wstg + r * 256 + ((ck ^ (r & 7)) << 4));
+        }
+    };
     int parity = 0;
     for (int ci = blockIdx.x; ci < total; ci += gridDim.x, parity ^= 1) {
         const int head = ci / nchunks;
@@ -272,6 +287,9 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
         const float *sinv = reinterpret_cast<const float *>(sm + OFF_INV) + (warp * 2 + half) * 16;
         auto iq = [&](int rr) { return PRO ? sinv[rr] : 1.f; };
         auto ik = [&](int rr) { return PRO ? sinv[8 + rr] : 1.f; };
+        // beta of row tid (warps 0-1), loaded with the operands so that its
+        // latency hides under theirs
+        const float beta_ld = (!GDR2 && tid < kC) ? __ldg(betag + row0 + min(tid, nrows - 1)) : 0.f;
         {
             // Unconditional loads from rows clamped into the chunk (a
             // conditional load makes the compiler wait for each one before the
@@ -292,6 +310,7 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
                     }
                 }
             }
+            if (ci != (int)blockIdx.x) store_w(ci - (int)gridDim.x);
 #pragma unroll
             for (int rr = 0; rr < 8; ++rr) {
                 if (rbase + rr >= nrows) {
@@ -359,8 +378,7 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
                 if (GDR2) {   // the gates sit in the operands; T' is (I + A)^{-1} itself
                     sBeta[tid] = tid < nrows ? 1.f : 0.f;
                 } else {
-                    const float bl = tid < nrows ? __ldg(betag + row0 + tid) : 0.f;
-                    sBeta[tid] = tid < nrows ? (PRO ? 1.f / (1.f + __expf(-bl)) : bl) : 0.f;
+                    sBeta[tid] = tid < nrows ? (PRO ? 1.f / (1.f + __expf(-beta_ld)) : beta_ld) : 0.f;
                 }
             }
             if (SCALAR && warp == 0) {
@@ -692,11 +710,15 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
                 *reinterpret_cast<float2 *>(&dst[g][8 * nt + 2 * t]) = make_float2(nt_[nt][0], nt_[nt][1]);
                 *reinterpret_cast<float2 *>(&dst[g + 8][8 * nt + 2 * t]) = make_float2(nt_[nt][2], nt_[nt][3]);
             }
-        } else {
-            // diagonal blocks D_i Diag(beta) and the zero blocks above them
-            for (int task = tid - 192; task < kC * 8; task += 64) {
-                const int r = task >> 3, g8 = task & 7, i = r >> 4, jb = g8 >> 1;
-                if (jb < i) continue;
+        }
+        // diagonal blocks D_i Diag(beta) and the zero blocks above them, 8
+        // columns of one row per task, two tasks per thread of every warp (the
+        // six warps above join after their product)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const int task = tid + kThreads * j;
+            const int r = task >> 3, g8 = task & 7, i = r >> 4, jb = g8 >> 1;
+            if (jb >= i) {
                 uint4 o = make_uint4(0u, 0u, 0u, 0u), os = o;
                 if (jb == i) {
                     const int ch = 8 * (g8 & 1), cl = 16 * jb + ch;
@@ -757,9 +779,8 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
         // accumulator per block, combined after the products.  Scalar gate: the
         // decay sits in T' (above) and Khat is k.  Warp w owns channels
         // 16w..16w+15 (two 8-channel tiles), all 64 tokens, in 4 token blocks.
-        // The fragments go to a staging tile (16-byte chunks XOR-swizzled by
-        // token, conflict free both ways), which is then stored in whole rows.
-        unsigned char *wstg = sm + OFF_KC;
+        // The fragments go to the staging tile (conflict free both ways), stored
+        // out during the next chunk's loads (or after the last chunk).
         {
             const int c0 = 16 * warp;
             const uint32_t khat = smem_u32(sm + OFF_K);
@@ -799,25 +820,19 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
                     }
                     // fragment: tokens 16I + g (+8), channels cs + 2t, + 1
                     const int r0 = 16 * I + g, ck = cs >> 3;
-                    *reinterpret_cast<uint32_t *>(wstg + r0 * 256 + ((ck ^ (r0 & 7)) << 4) + 4 * t) = pack2(-w4[0], -w4[1]);
-                    *reinterpret_cast<uint32_t *>(wstg + (r0 + 8) * 256 + ((ck ^ (r0 & 7)) << 4) + 4 * t) =
+                    unsigned char *ws = sm + OFF_A;
+                    *reinterpret_cast<uint32_t *>(ws + r0 * 256 + ((ck ^ (r0 & 7)) << 4) + 4 * t) = pack2(-w4[0], -w4[1]);
+                    *reinterpret_cast<uint32_t *>(ws + (r0 + 8) * 256 + ((ck ^ (r0 & 7)) << 4) + 4 * t) =
                         pack2(-w4[2], -w4[3]);
                 }
             }
         }
-        __syncthreads();
-        {
-            __nv_bfloat16 *wdst = Wout + (size_t)ci * kC * kDK;
-#pragma unroll
-            for (int q = tid; q < kC * 16; q += kThreads) {
-                const int r = q >> 4, ck = q & 15;
-                *reinterpret_cast<uint4 *>(wdst + r * kDK + 8 * ck) =
-                    *reinterpret_cast<const uint4 *>(wstg + r * 256 + ((ck ^ (r & 7)) << 4));
-            }
-        }
-        // the next chunk overwrites Khat, T' and the staging area
+        // the next chunk overwrites Khat and T', and stores the staged -W
         __syncthreads();
     }
+    // the -W of this CTA's last chunk (staged before the last barrier above)
+    if ((int)blockIdx.x < total)
+        store_w((int)blockIdx.x + ((total - 1 - (int)blockIdx.x) / (int)gridDim.x) * (int)gridDim.x);
 }
 
 int sm_count()

@@ -42,7 +42,8 @@
 //               [V_new^T | O^T] accumulator is double-buffered): O^T (TMEM) ->
 //               bf16 staging tile -> TMA store, then the O^T columns are
 //               zeroed for the chunk after next.  With OEPI the layer's gated output is
-//               fused in: y_t = Sigmoid(gate_t) * RMSNorm(o_t) per head
+//               fused in (and stored by these warps themselves):
+//               y_t = Sigmoid(gate_t) * RMSNorm(o_t) per head
 //               ("Token Mixer I", section "The Kimi Linear Model
 //               Architecture", the output equation before W_o), RMSNorm over
 //               the d_v channels in fp32 straight from the accumulator.
@@ -254,9 +255,9 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
     if (warp == 0) {
         // ================================================================ TMA producer, output stores
         if (lane == 1 && OEPI) {
-            // Gated output: the staging tile first receives the gate tile of chunk m
-            // (TMA), the epilogue overwrites it with y(m), the tile is stored, and as
-            // soon as the store has read it the gate tile of chunk m + 1 goes in.
+            // Gated output: the staging tile receives the gate tile of chunk m (TMA);
+            // the epilogue writes y(m) to global memory itself, and as soon as it has
+            // read the gate values the gate tile of chunk m + 1 goes in.
             auto load_gate = [&](int m) {
                 mbar_arrive_expect_tx(&bar[B_GATE_FULL], 16384);
                 tma_load_3d(sm + OFF_OST, &maps.og, &bar[B_GATE_FULL], 0, m * kC, head);
@@ -267,18 +268,11 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
                 load_gate(0);
                 loaded = 1;
             }
-            for (int m = 0; m < nchunks; ++m) {
-                if (!wait(B_EPI_FULL, (uint32_t)(m & 1))) break;
-                tma_store_3d(&maps.o, sm + OFF_OST, 0, m * kC, head);
-                tma_store_3d(&maps.o, sm + OFF_OST + 8192, 64, m * kC, head);
-                bulk_commit_group();
-                bulk_wait_read_all();
-                if (m + 1 < nchunks) {
-                    load_gate(m + 1);
-                    loaded = m + 2;
-                }
+            for (int m = 0; m + 1 < nchunks; ++m) {
+                if (!wait(B_EPI_FULL, (uint32_t)(m & 1))) break;   // the gate tile of m has been read
+                load_gate(m + 1);
+                loaded = m + 2;
             }
-            bulk_wait_all();   // the last store has completed before the CTA exits
             if (*abort_flag && loaded > 0)   // a gate tile still in flight lands before exit
                 mbar_wait(&bar[B_GATE_FULL], (uint32_t)((loaded - 1) & 1), kDrainBudget);
         }
@@ -541,11 +535,11 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
         // Plain: O^T -> bf16 staging tile -> TMA store (warp 0, lane 1).
         // OEPI: the gate tile of chunk m is TMA-loaded into the staging tile
         // (same layout as the output); per token the sum of squares over the 128
-        // channels (lanes, then the four warps), then
+        // channels (lanes, then the four warps); the gate values are read into
+        // registers, which frees the tile for the next gate load, and
         // y = o * rsqrt(mean o^2 + eps) * norm_w * Sigmoid(gate) is stored to
         // global memory straight from registers (32 consecutive channels per
-        // warp and token), which frees the tile for the next gate load as soon
-        // as it has been read.
+        // warp and token).
         const uint32_t lq = 32u * (warp & 3);
         const int i = (int)lq + lane;
         const uint32_t trow = tmem + (lq << 16);
@@ -632,9 +626,25 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
                     epi_sync();   // red is free again, rstd of these tokens written
                 }
                 if (!epi_all(waitw(B_GATE_FULL, (uint32_t)(m & 1)))) break;
-                // pass 2: 16 tokens per step; y replaces the gate element it was computed
-                // from, and the tile leaves by TMA store (rows past T are dropped)
-#pragma unroll 1
+                // the chunk's 64 gate values of this channel, packed in token pairs;
+                // then the tile goes back for the next chunk's gate
+                uint32_t zp[32];
+#pragma unroll
+                for (int jp = 0; jp < 32; ++jp) {
+                    const uint32_t t0 = 2u * jp, t1 = t0 + 1u;
+                    const uint32_t lo = *reinterpret_cast<const unsigned short *>(
+                        ost + (t0 >> 3) * 1024 + (t0 & 7) * 128 + ((c8 ^ (t0 & 7)) << 4));
+                    const uint32_t hi = *reinterpret_cast<const unsigned short *>(
+                        ost + (t1 >> 3) * 1024 + (t1 & 7) * 128 + ((c8 ^ (t1 & 7)) << 4));
+                    zp[jp] = lo | (hi << 16);
+                }
+                fence_async_smem();   // the next gate tile (TMA) overwrites what was read
+                warp_arrive(B_EPI_FULL);
+                // pass 2: 16 tokens per step; y goes to global memory from registers,
+                // 32 consecutive channels per warp and token (tokens past T dropped)
+                __nv_bfloat16 *yrow = O + ((size_t)head * T_len + (size_t)m * kC) * kD + i;
+                const int tvalid = T_len - m * kC;
+#pragma unroll
                 for (int cs = 0; cs < 4; ++cs) {
                     uint32_t r0[8], r1[8];
                     tmem_ld8(oc + 16 * cs, r0);
@@ -649,9 +659,10 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
                         f[4 * q4 + 3] = fv.w;
                     }
 #pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        z[j] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(
-                            ost + (2 * cs + (j >> 3)) * 1024 + (j & 7) * 128 + ((c8 ^ (uint32_t)(j & 7)) << 4)));
+                    for (int j = 0; j < 16; j += 2) {
+                        z[j] = __uint_as_float(zp[8 * cs + j / 2] << 16);
+                        z[j + 1] = __uint_as_float(zp[8 * cs + j / 2] & 0xffff0000u);
+                    }
                     tmem_ld_wait8(r0);
                     reg_touch8(r1);
                     // two tokens at a time: a = o * rstd / 2 * norm_w, y = a (1 + tanh(z / 2))
@@ -663,17 +674,15 @@ chunk_scan_kernel(const __grid_constant__ Maps maps, const float *__restrict__ g
                         const float2 hz = fmul2(make_float2(z[j], z[j + 1]), make_float2(0.5f, 0.5f));
                         const float2 y = ffma2(a, make_float2(tanh_approx(hz.x), tanh_approx(hz.y)), a);
                         const uint32_t yb = pack2_bf16(y.x, y.y);
-                        *reinterpret_cast<unsigned short *>(ost + (2 * cs + (j >> 3)) * 1024 + (j & 7) * 128 +
-                                                            ((c8 ^ (uint32_t)(j & 7)) << 4)) = (unsigned short)(yb & 0xffffu);
-                        *reinterpret_cast<unsigned short *>(ost + (2 * cs + (j >> 3)) * 1024 + ((j + 1) & 7) * 128 +
-                                                            ((c8 ^ (uint32_t)((j + 1) & 7)) << 4)) = (unsigned short)(yb >> 16);
+                        const int tt = 16 * cs + j;
+                        if (tt < tvalid) *reinterpret_cast<unsigned short *>(yrow + (size_t)tt * kD) = (unsigned short)(yb & 0xffffu);
+                        if (tt + 1 < tvalid)
+                            *reinterpret_cast<unsigned short *>(yrow + (size_t)(tt + 1) * kD) = (unsigned short)(yb >> 16);
                     }
                 }
                 zero_oacc();
                 tc_fence_before();
                 warp_arrive(B_OACC_EMPTY + bb);
-                fence_async_smem();   // the tile is read next by the TMA store
-                warp_arrive(B_EPI_FULL);
             }
         }
     }

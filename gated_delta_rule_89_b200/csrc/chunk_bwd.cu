@@ -656,65 +656,187 @@ bwd_grads(const T *__restrict__ qg, const T *__restrict__ kg, const T *__restric
         sP[r * 65 + pi] = -acc;   // dA (zero on and above the diagonal)
     }
     __syncthreads();
-    // decay-weighted contractions of dA (A_ri = beta_r sum_c k_rc k_ic E) and dAqk,
-    // four of the thread's rows at a time so the per-channel operands are read once
-    // for all four.  A row's terms past its own r are dropped (a select, so an
-    // exponential that overflows there never meets the zero it is multiplied by).
-    // row side: (r, c) collects over i <= r
+    // decay-weighted contractions of dA (A_ri = beta_r sum_c k_rc k_ic E) and dAqk:
+    // row side, (r, c) collects over i <= r; column side, (i, c) over r >= i.
     float xb[NR];
-#pragma unroll
-    for (int m0 = 0; m0 < NR; m0 += 4) {
-        float gr[4], sdk[4], sdq[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            gr[u] = sG[(h + RS * (m0 + u)) * LD + c];
-            sdk[u] = sdq[u] = 0.f;
-        }
-        const int rmax = h + RS * (m0 + 3);
-        for (int i = 0; i <= rmax; ++i) {
-            const float ki = sk[i * LD + c], gi = sG[i * LD + c];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int r = h + RS * (m0 + u);
-                const float kie = i <= r ? ki * __expf(gr[u] - gi) : 0.f;
-                sdk[u] = fmaf(sP[r * 65 + i], kie, sdk[u]);
-                sdq[u] = fmaf(sR[r * 65 + i], kie, sdq[u]);
+    if constexpr (!SCALAR) {
+        // Per-channel gate: in 16-token blocks, with base_R the log-decay just
+        // before block R (0 for R = 0), er_r = exp(G_r - base_R) <= 1,
+        // ep_i = exp(base_{I+1} - G_i) <= 1 and bd_R = exp(base_{R+1} - base_R),
+        //   exp(G_r - G_i) = er_r (prod_{I<J<R} bd_J) ep_i   (i in block I < R)
+        //                  = er_r ep_i / bd_R                 (both in block R)
+        // so no term needs an exponential of its own: the earlier blocks are
+        // combined by Horner steps with bd, the diagonal block by 1/bd_R, which
+        // the -5 bound keeps below e^80 (the decay-ratio scheme of the forward's
+        // prep, in fp32).  The A and Z tiles are free here: kc = k ep -> sX,
+        // er -> sY, bd and 1/bd -> sM.
+        float *skc = sX, *ser = sY, *sbd = sM, *sibd = sM + 4 * D;
+        for (int idx = tid; idx < kC * D; idx += kBT) {
+            const int r = idx / D, cc = idx - r * D, Rb = r >> 4;
+            const float base = Rb ? sG[(16 * Rb - 1) * LD + cc] : 0.f;
+            const float top = sG[(16 * Rb + 15) * LD + cc];
+            const float gr = sG[r * LD + cc];
+            const float er = __expf(gr - base);
+            ser[r * LD + cc] = er;
+            skc[r * LD + cc] = sk[r * LD + cc] * __expf(top - gr);
+            if ((r & 15) == 15) {   // the block's last row: er = bd_R
+                sbd[Rb * D + cc] = er;
+                sibd[Rb * D + cc] = 1.f / er;
             }
         }
+        __syncthreads();
+        // row side, four of the thread's rows at a time (they share a block)
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int m = m0 + u, r = h + RS * m;
-            const float sx = sdk[u] * sk[r * LD + c];    // sum_i dA_ri k_rc k_ic E
-            const float sxq = sdq[u] * sq[r * LD + c];   // sum_i dAqk_ri q_rc k_ic E
-            dk[m] = fmaf(sb[r], sdk[u], dk[m]);
-            dq[m] += sdq[u];
-            dG[m] += sb[r] * sx + sxq;
-            xb[m] = sx;
-        }
-    }
-    // column side: (i, c) collects over r >= i
+        for (int m0 = 0; m0 < NR; m0 += 4) {
+            const int rb = h + RS * m0, R = rb >> 4;
+            float ak[4] = {0.f, 0.f, 0.f, 0.f}, aq[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int I = 0; I < R; ++I) {
+                const float bdI = sbd[I * D + c];
+                float pk[4] = {0.f, 0.f, 0.f, 0.f}, pq[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+                for (int i = 16 * I; i < 16 * I + 16; ++i) {
+                    const float kc = skc[i * LD + c];
 #pragma unroll
-    for (int m0 = 0; m0 < NR; m0 += 4) {
-        float gi[4], sa[4];
+                    for (int u = 0; u < 4; ++u) {
+                        const int r = rb + RS * u;
+                        pk[u] = fmaf(sP[r * 65 + i], kc, pk[u]);
+                        pq[u] = fmaf(sR[r * 65 + i], kc, pq[u]);
+                    }
+                }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            gi[u] = sG[(h + RS * (m0 + u)) * LD + c];
-            sa[u] = 0.f;
-        }
-        for (int r = h + RS * m0; r < kC; ++r) {
-            const float gr = sG[r * LD + c], bk = sb[r] * sk[r * LD + c], qr = sq[r * LD + c];
+                for (int u = 0; u < 4; ++u) {
+                    ak[u] = fmaf(ak[u], bdI, pk[u]);
+                    aq[u] = fmaf(aq[u], bdI, pq[u]);
+                }
+            }
+            float pk[4] = {0.f, 0.f, 0.f, 0.f}, pq[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int i = 16 * R; i <= rb + RS * 3; ++i) {
+                const float kc = skc[i * LD + c];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int r = rb + RS * u;
+                    const float kk = i <= r ? kc : 0.f;
+                    pk[u] = fmaf(sP[r * 65 + i], kk, pk[u]);
+                    pq[u] = fmaf(sR[r * 65 + i], kk, pq[u]);
+                }
+            }
+            const float ibdR = sibd[R * D + c];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const int i = h + RS * (m0 + u);
-                const float e = r >= i ? __expf(gr - gi[u]) : 0.f;
-                sa[u] = fmaf(bk * sP[r * 65 + i] + sR[r * 65 + i] * qr, e, sa[u]);
+                const int m = m0 + u, r = rb + RS * u;
+                const float e = ser[r * LD + c];
+                const float sdk = e * fmaf(ibdR, pk[u], ak[u]);   // sum_i dA_ri k_ic E
+                const float sdq = e * fmaf(ibdR, pq[u], aq[u]);   // sum_i dAqk_ri k_ic E
+                const float sx = sdk * sk[r * LD + c];
+                const float sxq = sdq * sq[r * LD + c];
+                dk[m] = fmaf(sb[r], sdk, dk[m]);
+                dq[m] += sdq;
+                dG[m] += sb[r] * sx + sxq;
+                xb[m] = sx;
             }
         }
+        // column side, four of the thread's columns at a time
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int m = m0 + u;
-            dk[m] += sa[u];
-            dG[m] = fmaf(-sa[u], sk[(h + RS * m) * LD + c], dG[m]);
+        for (int m0 = 0; m0 < NR; m0 += 4) {
+            const int ib = h + RS * m0, I = ib >> 4;
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int R = kC / 16 - 1; R > I; --R) {
+                const float bdR = sbd[R * D + c];
+                float part[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+                for (int r = 16 * R; r < 16 * R + 16; ++r) {
+                    const float e = ser[r * LD + c];
+                    const float bk = sb[r] * sk[r * LD + c] * e, qe = sq[r * LD + c] * e;
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int i = ib + RS * u;
+                        part[u] = fmaf(bk, sP[r * 65 + i], fmaf(qe, sR[r * 65 + i], part[u]));
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) acc[u] = fmaf(acc[u], bdR, part[u]);
+            }
+            float pd[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int r = ib; r < 16 * I + 16; ++r) {
+                const float e = ser[r * LD + c];
+                const float bk = sb[r] * sk[r * LD + c] * e, qe = sq[r * LD + c] * e;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int i = ib + RS * u;
+                    const float t = fmaf(bk, sP[r * 65 + i], qe * sR[r * 65 + i]);
+                    pd[u] += r >= i ? t : 0.f;
+                }
+            }
+            const float ibdI = sibd[I * D + c], topI = sG[(16 * I + 15) * LD + c];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int m = m0 + u, i = ib + RS * u;
+                const float ep = __expf(topI - sG[i * LD + c]);
+                const float sa = ep * fmaf(ibdI, pd[u], acc[u]);   // sum_r (beta_r k_rc dA_ri + q_rc dAqk_ri) E
+                dk[m] += sa;
+                dG[m] = fmaf(-sa, sk[i * LD + c], dG[m]);
+            }
+        }
+    } else {
+        // Scalar gate (unbounded, so no block rescaling): one exponential per
+        // term.  Row side, four of the thread's rows at a time so the per-channel
+        // operands are read once for all four; a row's terms past its own r are
+        // dropped (a select, so an exponential that overflows there never meets
+        // the zero it is multiplied by).
+#pragma unroll
+        for (int m0 = 0; m0 < NR; m0 += 4) {
+            float gr[4], sdk[4], sdq[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                gr[u] = sG[(h + RS * (m0 + u)) * LD + c];
+                sdk[u] = sdq[u] = 0.f;
+            }
+            const int rmax = h + RS * (m0 + 3);
+            for (int i = 0; i <= rmax; ++i) {
+                const float ki = sk[i * LD + c], gi = sG[i * LD + c];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int r = h + RS * (m0 + u);
+                    const float kie = i <= r ? ki * __expf(gr[u] - gi) : 0.f;
+                    sdk[u] = fmaf(sP[r * 65 + i], kie, sdk[u]);
+                    sdq[u] = fmaf(sR[r * 65 + i], kie, sdq[u]);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int m = m0 + u, r = h + RS * m;
+                const float sx = sdk[u] * sk[r * LD + c];    // sum_i dA_ri k_rc k_ic E
+                const float sxq = sdq[u] * sq[r * LD + c];   // sum_i dAqk_ri q_rc k_ic E
+                dk[m] = fmaf(sb[r], sdk[u], dk[m]);
+                dq[m] += sdq[u];
+                dG[m] += sb[r] * sx + sxq;
+                xb[m] = sx;
+            }
+        }
+        // column side: (i, c) collects over r >= i
+#pragma unroll
+        for (int m0 = 0; m0 < NR; m0 += 4) {
+            float gi[4], sa[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                gi[u] = sG[(h + RS * (m0 + u)) * LD + c];
+                sa[u] = 0.f;
+            }
+            for (int r = h + RS * m0; r < kC; ++r) {
+                const float gr = sG[r * LD + c], bk = sb[r] * sk[r * LD + c], qr = sq[r * LD + c];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int i = h + RS * (m0 + u);
+                    const float e = r >= i ? __expf(gr - gi[u]) : 0.f;
+                    sa[u] = fmaf(bk * sP[r * 65 + i] + sR[r * 65 + i] * qr, e, sa[u]);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int m = m0 + u;
+                dk[m] += sa[u];
+                dG[m] = fmaf(-sa[u], sk[(h + RS * m) * LD + c], dG[m]);
+            }
         }
     }
     // dbeta_r += sum_c xb  (lanes, then the warps that share the rows)

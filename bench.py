@@ -53,14 +53,11 @@ DEFAULT_WORKLOAD = "kda_d128_t8192"
 # entry is ignored (traffic = null) as soon as any of the sources changes.
 TRAFFIC = {
     # B=1 capture doubled (4096 chunks; inputs and hand-off above L2 at both sizes):
-    # ut_prep 275.8 MB read + 224.1 MB written, chunk_scan 339.8 + 52.6 MB
-    "kda_d128_t8192": {"src_sha": "9f27d659ed1cb169", "bytes_per_launch": 1784652800},
-    # backward: bwd_prep 675.1 + 1553.3, bwd_fwd_scan 1126.1 + 771.1, bwd_rev_scan 1643.4 + 779.4,
-    # bwd_grads 2825.2 + 653.2 MB (chunk_bwd.cu unchanged since; the shared header changed
-    # only in the tensor-core workspace layout, which these kernels do not use)
-    "kda_d128_t8192_bwd": {"src_sha": "8d0a5075fc008e3b", "bytes_per_launch": 10026771200},
+    # ut_prep 276.7 MB read + 223.2 MB written, chunk_scan 339.9 + 53.0 MB
+    "kda_d128_t8192": {"src_sha": "0c12c160d8bf9a1b", "bytes_per_launch": 1785434112},
     # recurrent_step, one decode step: 547.4 MB read + 477.8 MB written (recurrent_step.cu
-    # unchanged since; same header note)
+    # unchanged since the capture; the shared header changed only in the tensor-core
+    # workspace layout, which this kernel does not use)
     "kda_decode_b256": {"src_sha": "83851ff3a738fcf9", "bytes_per_launch": 1025204480},
 }
 

@@ -73,8 +73,10 @@ inline BwdWs carve(void *ws, int B, int H, int T, int D)
 template <int D>
 struct PrepSmem {
     static constexpr int LD = D + 1;
-    static constexpr int K = 0, Q = K + kC * LD, G = Q + kC * LD, A = G + kC * LD, M = A + kC * 65, B = M + kC * 65;
-    static constexpr int TOTAL = B + kC;
+    static constexpr int LM = 68;   // M rows: 16-byte aligned for vector reads, columns conflict free
+    static constexpr int K = 0, Q = K + kC * LD, G = Q + kC * LD, A = G + kC * LD, M = A + kC * 65, B = M + kC * LM;
+    static constexpr int KR = B + kC, KC = KR + kC * LD, F = KC + kC * LD;   // per-channel gate only
+    static constexpr int TOTAL = F + 16 * D;
 };
 
 template <int D, typename T, bool SCALAR>
@@ -83,7 +85,7 @@ bwd_prep(const T *__restrict__ qg, const T *__restrict__ kg, const T *__restrict
          const float *__restrict__ betag, BwdWs w, int T_len, int nch)
 {
     using L = PrepSmem<D>;
-    constexpr int LD = L::LD, RS = kBT / D, NR = kC / RS;
+    constexpr int LD = L::LD, LM = L::LM, RS = kBT / D, NR = kC / RS;
     extern __shared__ float sm[];
     float *sk = sm + L::K, *sq = sm + L::Q, *sG = sm + L::G, *sA = sm + L::A, *sM = sm + L::M, *sb = sm + L::B;
     const int tid = threadIdx.x;
@@ -122,20 +124,72 @@ bwd_prep(const T *__restrict__ qg, const T *__restrict__ kg, const T *__restrict
     }
     // A (strictly lower, beta_r in) and Aqk (lower incl. the diagonal)
     float *Aqo = w.Aq + (size_t)ci * kC * kC;
-#pragma unroll 8
-    for (int idx = tid; idx < kC * kC; idx += kBT) {
-        const int r = idx >> 6, i = idx & 63;
-        float sa = 0.f, sq_ = 0.f;
-        if (i <= r) {
-            for (int c = 0; c < D; ++c) {
-                const float e = __expf(sG[r * LD + c] - sG[i * LD + c]);
-                const float ki = sk[i * LD + c] * e;
-                sa = fmaf(sk[r * LD + c], ki, sa);
-                sq_ = fmaf(sq[r * LD + c], ki, sq_);
+    if constexpr (!SCALAR) {
+        // In 16-token blocks (base_R the log-decay just before block R),
+        // exp(G_rc - G_ic) = er_r F ep_i with er_r = exp(G_r - base_R),
+        // ep_i = exp(base_{I+1} - G_i) and the per-channel block factor
+        // F = exp(base_R - base_{I+1}) (I < R; the product of the block decays
+        // between) or exp(base_R - base_{R+1}) (I = R; below e^80 under the -5
+        // bound).  So A and Aqk are sums of products of stored operands, four
+        // rows of one block per thread, with no exponential per term.
+        float *skr = sm + L::KR, *skc = sm + L::KC, *sF = sm + L::F;
+        __syncthreads();   // q has been read in its own form (Q<- above)
+        for (int idx = tid; idx < kC * D; idx += kBT) {
+            const int r = idx / D, cc = idx - r * D, Rb = r >> 4;
+            const float base = Rb ? sG[(16 * Rb - 1) * LD + cc] : 0.f;
+            const float top = sG[(16 * Rb + 15) * LD + cc];
+            const float gr = sG[r * LD + cc];
+            const float er = __expf(gr - base);
+            skr[r * LD + cc] = sk[r * LD + cc] * er;
+            sq[r * LD + cc] *= er;
+            skc[r * LD + cc] = sk[r * LD + cc] * __expf(top - gr);
+        }
+        for (int idx = tid; idx < 16 * D; idx += kBT) {
+            const int RI = idx / D, cc = idx - RI * D, R = RI >> 2, I = RI & 3;
+            const float baseR = R ? sG[(16 * R - 1) * LD + cc] : 0.f;
+            sF[RI * D + cc] = I <= R ? __expf(baseR - sG[(16 * I + 15) * LD + cc]) : 0.f;
+        }
+        __syncthreads();
+        const int i = tid & 63, r0 = tid >> 6, I = i >> 4;
+        for (int J = 0; J < kC / 16; ++J) {
+            float sa[4] = {0.f, 0.f, 0.f, 0.f}, sqv[4] = {0.f, 0.f, 0.f, 0.f};
+            if (I <= J) {
+                const float *f = sF + (4 * J + I) * D;
+#pragma unroll 4
+                for (int cc = 0; cc < D; ++cc) {
+                    const float kf = skc[i * LD + cc] * f[cc];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int r = r0 + 16 * J + 4 * u;
+                        sa[u] = fmaf(skr[r * LD + cc], kf, sa[u]);
+                        sqv[u] = fmaf(sq[r * LD + cc], kf, sqv[u]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {   // terms above the diagonal are dropped by a select
+                const int r = r0 + 16 * J + 4 * u;
+                sA[r * 65 + i] = i < r ? sb[r] * sa[u] : 0.f;
+                Aqo[r * kC + i] = i <= r ? sqv[u] : 0.f;
             }
         }
-        sA[r * 65 + i] = i < r ? sb[r] * sa : 0.f;
-        Aqo[r * kC + i] = sq_;
+    } else {
+        // scalar gate (unbounded): one exponential per term
+#pragma unroll 8
+        for (int idx = tid; idx < kC * kC; idx += kBT) {
+            const int r = idx >> 6, i = idx & 63;
+            float sa = 0.f, sq_ = 0.f;
+            if (i <= r) {
+                for (int c = 0; c < D; ++c) {
+                    const float e = __expf(sG[r * LD + c] - sG[i * LD + c]);
+                    const float ki = sk[i * LD + c] * e;
+                    sa = fmaf(sk[r * LD + c], ki, sa);
+                    sq_ = fmaf(sq[r * LD + c], ki, sq_);
+                }
+            }
+            sA[r * 65 + i] = i < r ? sb[r] * sa : 0.f;
+            Aqo[r * kC + i] = sq_;
+        }
     }
     __syncthreads();
     // M = (I + A)^{-1}: column j by forward substitution
@@ -147,16 +201,16 @@ bwd_prep(const T *__restrict__ qg, const T *__restrict__ kg, const T *__restrict
                 x = 1.f;
             } else if (r > j) {
                 float s = 0.f;
-                for (int m = j; m < r; ++m) s = fmaf(sA[r * 65 + m], sM[m * 65 + j], s);
+                for (int m = j; m < r; ++m) s = fmaf(sA[r * 65 + m], sM[m * LM + j], s);
                 x = -s;
             }
-            sM[r * 65 + j] = x;
+            sM[r * LM + j] = x;
         }
     }
     __syncthreads();
     float *Mo = w.M + (size_t)ci * kC * kC;
 #pragma unroll 8
-    for (int idx = tid; idx < kC * kC; idx += kBT) Mo[idx] = sM[(idx >> 6) * 65 + (idx & 63)];
+    for (int idx = tid; idx < kC * kC; idx += kBT) Mo[idx] = sM[(idx >> 6) * LM + (idx & 63)];
     // W = M Diag(beta) (K * gamma): the operand beta_i k_ic gamma_ic into sq
 #pragma unroll 8
     for (int idx = tid; idx < kC * D; idx += kBT) {
@@ -165,17 +219,22 @@ bwd_prep(const T *__restrict__ qg, const T *__restrict__ kg, const T *__restrict
     }
     __syncthreads();
     const int c = tid % D, h = tid / D;
-    {
-        float acc[NR];
+    // (16 of the thread's rows at a time; four columns of M per step, one
+    // 16-byte broadcast read per row)
+    for (int m0 = 0; m0 < NR; m0 += 16) {
+        float acc[16];
 #pragma unroll
-        for (int m = 0; m < NR; ++m) acc[m] = 0.f;
-        for (int i = 0; i < kC; ++i) {
-            const float b = sq[i * LD + c];
+        for (int m = 0; m < 16; ++m) acc[m] = 0.f;
+        for (int i = 0; i < kC; i += 4) {
+            const float b0 = sq[i * LD + c], b1 = sq[(i + 1) * LD + c], b2 = sq[(i + 2) * LD + c], b3 = sq[(i + 3) * LD + c];
 #pragma unroll
-            for (int m = 0; m < NR; ++m) acc[m] = fmaf(sM[(h + RS * m) * 65 + i], b, acc[m]);
+            for (int m = 0; m < 16; ++m) {
+                const float4 mv = *reinterpret_cast<const float4 *>(&sM[(h + RS * (m0 + m)) * LM + i]);
+                acc[m] = fmaf(mv.w, b3, fmaf(mv.z, b2, fmaf(mv.y, b1, fmaf(mv.x, b0, acc[m]))));
+            }
         }
 #pragma unroll
-        for (int m = 0; m < NR; ++m) w.W[(prow0 + h + RS * m) * D + c] = acc[m];
+        for (int m = 0; m < 16; ++m) w.W[(prow0 + h + RS * (m0 + m)) * D + c] = acc[m];
     }
     __syncthreads();
     // U = M Diag(beta) V (d_v = D)
@@ -185,17 +244,22 @@ bwd_prep(const T *__restrict__ qg, const T *__restrict__ kg, const T *__restrict
         sq[r * LD + j] = r < nrows ? sb[r] * to_f32<T>(vg[(row0 + r) * D + j]) : 0.f;
     }
     __syncthreads();
-    {
-        float acc[NR];
+    // (16 of the thread's rows at a time; four columns of M per step, one
+    // 16-byte broadcast read per row)
+    for (int m0 = 0; m0 < NR; m0 += 16) {
+        float acc[16];
 #pragma unroll
-        for (int m = 0; m < NR; ++m) acc[m] = 0.f;
-        for (int i = 0; i < kC; ++i) {
-            const float b = sq[i * LD + c];
+        for (int m = 0; m < 16; ++m) acc[m] = 0.f;
+        for (int i = 0; i < kC; i += 4) {
+            const float b0 = sq[i * LD + c], b1 = sq[(i + 1) * LD + c], b2 = sq[(i + 2) * LD + c], b3 = sq[(i + 3) * LD + c];
 #pragma unroll
-            for (int m = 0; m < NR; ++m) acc[m] = fmaf(sM[(h + RS * m) * 65 + i], b, acc[m]);
+            for (int m = 0; m < 16; ++m) {
+                const float4 mv = *reinterpret_cast<const float4 *>(&sM[(h + RS * (m0 + m)) * LM + i]);
+                acc[m] = fmaf(mv.w, b3, fmaf(mv.z, b2, fmaf(mv.y, b1, fmaf(mv.x, b0, acc[m]))));
+            }
         }
 #pragma unroll
-        for (int m = 0; m < NR; ++m) w.U[(prow0 + h + RS * m) * D + c] = acc[m];
+        for (int m = 0; m < 16; ++m) w.U[(prow0 + h + RS * (m0 + m)) * D + c] = acc[m];
     }
 }
 

@@ -311,13 +311,15 @@ ut_prep_kernel(const __nv_bfloat16 *__restrict__ kg, const __nv_bfloat16 *__rest
                 }
             }
             if (ci != (int)blockIdx.x) store_w(ci - (int)gridDim.x);
+            if (nrows < kC) {   // only the ragged last chunk of a head (a uniform branch)
 #pragma unroll
-            for (int rr = 0; rr < 8; ++rr) {
-                if (rbase + rr >= nrows) {
-                    kr[rr] = make_uint2(0u, 0u);
-                    qr[rr] = make_uint2(0u, 0u);
-                    if (GDR2) br[rr] = make_uint2(0u, 0u);
-                    if (!SCALAR) gv[rr] = make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int rr = 0; rr < 8; ++rr) {
+                    if (rbase + rr >= nrows) {
+                        kr[rr] = make_uint2(0u, 0u);
+                        qr[rr] = make_uint2(0u, 0u);
+                        if (GDR2) br[rr] = make_uint2(0u, 0u);
+                        if (!SCALAR) gv[rr] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
                 }
             }
             if (PRO) {

@@ -34,6 +34,8 @@
 //   4. bwd_grads    every chunk in parallel: dq, dk, dv, dg, dbeta
 // Decay ratios are only ever formed as exp of a difference that is <= 0.
 // Rows past the end of a partial last chunk act as identity tokens.
+#include <type_traits>
+
 #include "gdr_internal.cuh"
 
 namespace gdr {
@@ -496,6 +498,52 @@ bwd_rev_scan(const T *__restrict__ dOg, const float *__restrict__ dST, float *__
 }
 
 // ------------------------------------------------------------------ 4. per-chunk gradients
+// C[64][128] = sign * A[64][K] B[K][128] on the tensor cores (mma.sync
+// m16n8k8 with tf32 operands, rounded from fp32: about 2^-11 relative per
+// operand, fp32 accumulation), for the bf16 path's three 64 x 128 x 128
+// products.  A in shared memory (row stride lda), B in global or shared
+// memory (row stride ldb), C to shared memory (row stride ldc); warp w computes
+// rows 16 (w & 3) .. + 15 and columns 64 (w >> 2) .. + 63.  All 8 warps.
+__device__ __forceinline__ uint32_t tf32_rn(float x)
+{
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
+template <int K>
+__device__ __forceinline__ void mm_tf32_64x128(const float *A, int lda, const float *B, int ldb, float *C, int ldc,
+                                               float sign)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const int r0 = 16 * (warp & 3), n0 = 64 * (warp >> 2);
+    float acc[8][4];
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll 2
+    for (int k0 = 0; k0 < K; k0 += 8) {
+        const uint32_t a0 = tf32_rn(A[(r0 + g) * lda + k0 + t]), a1 = tf32_rn(A[(r0 + g + 8) * lda + k0 + t]);
+        const uint32_t a2 = tf32_rn(A[(r0 + g) * lda + k0 + t + 4]), a3 = tf32_rn(A[(r0 + g + 8) * lda + k0 + t + 4]);
+        const float *b = B + (size_t)(k0 + t) * ldb + n0 + g;
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+            const uint32_t b0 = tf32_rn(b[8 * nt]), b1 = tf32_rn(b[(size_t)4 * ldb + 8 * nt]);
+            asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+                         "{%8, %9}, {%0, %1, %2, %3};"
+                         : "+f"(acc[nt][0]), "+f"(acc[nt][1]), "+f"(acc[nt][2]), "+f"(acc[nt][3])
+                         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+        }
+    }
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+        const int col = n0 + 8 * nt + 2 * t;
+        C[(r0 + g) * ldc + col] = sign * acc[nt][0];
+        C[(r0 + g) * ldc + col + 1] = sign * acc[nt][1];
+        C[(r0 + g + 8) * ldc + col] = sign * acc[nt][2];
+        C[(r0 + g + 8) * ldc + col + 1] = sign * acc[nt][3];
+    }
+}
+
 template <int D>
 struct GradSmem {
     static constexpr int LD = D + 1;
@@ -551,8 +599,38 @@ bwd_grads(const T *__restrict__ qg, const T *__restrict__ kg, const T *__restric
     const float gcl = sG[(kC - 1) * LD + c];   // G at the chunk end
     float dgc = 0.f;                           // this thread's share of d G_C (channel c)
 
+    // The bf16 path at d = 128 takes its three 64 x 128 x 128 products on the
+    // tensor cores, through the P and R tiles (free until dAqk: 64 x 130 floats).
+    constexpr bool kTC = D == 128 && !std::is_same<T, float>::value;
+    float *sC = sP;
+    constexpr int LC = 130;
+    static_assert(L::R + kC * 65 - L::P >= kC * LC, "the product tile fits in the P and R tiles");
     // dQ<- = dO S  ->  dq += dQ<- gamma,  dG += dQ<- q gamma
-    {
+    if constexpr (kTC) {
+        mm_tf32_64x128<D>(sX, LD, Sn, D, sC, LC, 1.f);
+        __syncthreads();
+#pragma unroll
+        for (int m = 0; m < NR; ++m) {
+            const int r = h + RS * m;
+            const float ga = __expf(sG[r * LD + c]), a = sC[r * LC + c];
+            dq[m] = fmaf(a, ga, dq[m]);
+            dG[m] = fmaf(a * sq[r * LD + c], ga, dG[m]);
+        }
+        __syncthreads();
+        // dK_tail = V_new dS'  ->  dk += dK_tail gamma_C / gamma,  dG -= (same) k, dG_C += (same) k
+        mm_tf32_64x128<D>(sY, LD, dSn, D, sC, LC, 1.f);
+        __syncthreads();
+#pragma unroll
+        for (int m = 0; m < NR; ++m) {
+            const int r = h + RS * m;
+            const float t = sC[r * LC + c] * __expf(gcl - sG[r * LD + c]);
+            dk[m] += t;
+            const float tk = t * sk[r * LD + c];
+            dG[m] -= tk;
+            dgc += tk;
+        }
+        __syncthreads();   // the P and R tiles are free again
+    } else {
         float acc[NR];
 #pragma unroll
         for (int m = 0; m < NR; ++m) acc[m] = 0.f;
@@ -580,7 +658,8 @@ bwd_grads(const T *__restrict__ qg, const T *__restrict__ kg, const T *__restric
         sR[r * 65 + pi] = acc;
     }
     // dK_tail = V_new dS'  ->  dk += dK_tail gamma_C / gamma,  dG -= (same) k, dG_C += (same) k
-    {
+    // (on the tensor cores above for the bf16 path)
+    if constexpr (!kTC) {
         float acc[NR];
 #pragma unroll
         for (int m = 0; m < NR; ++m) acc[m] = 0.f;
@@ -644,7 +723,9 @@ bwd_grads(const T *__restrict__ qg, const T *__restrict__ kg, const T *__restric
     }
     __syncthreads();   // V read
     // dW = -dV_new S  -> sY
-    {
+    if constexpr (kTC) {
+        mm_tf32_64x128<D>(sX, LD, Sn, D, sY, LD, -1.f);
+    } else {
         float acc[NR];
 #pragma unroll
         for (int m = 0; m < NR; ++m) acc[m] = 0.f;

@@ -544,6 +544,46 @@ __device__ __forceinline__ void mm_tf32_64x128(const float *A, int lda, const fl
     }
 }
 
+// C[64][64] (=, or +=) A[64][K] Bm[64][K]^T on the tensor cores (as above),
+// both operands row-major in shared memory; with `lower` only the entries
+// with column <= row are stored (the others get 0).  Warp w computes rows
+// 16 (w & 3) .. + 15 and columns 32 (w >> 2) .. + 31.  All 8 warps.
+template <int K, bool ACC, bool LOWER>
+__device__ __forceinline__ void mm_tf32_64x64_nt(const float *A, int lda, const float *Bm, int ldb, float *C, int ldc)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const int r0 = 16 * (warp & 3), n0 = 32 * (warp >> 2);
+    float acc[4][4];
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll 2
+    for (int k0 = 0; k0 < K; k0 += 8) {
+        const uint32_t a0 = tf32_rn(A[(r0 + g) * lda + k0 + t]), a1 = tf32_rn(A[(r0 + g + 8) * lda + k0 + t]);
+        const uint32_t a2 = tf32_rn(A[(r0 + g) * lda + k0 + t + 4]), a3 = tf32_rn(A[(r0 + g + 8) * lda + k0 + t + 4]);
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) {
+            const float *b = Bm + (n0 + 8 * nt + g) * ldb + k0 + t;
+            const uint32_t b0 = tf32_rn(b[0]), b1 = tf32_rn(b[4]);
+            asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+                         "{%8, %9}, {%0, %1, %2, %3};"
+                         : "+f"(acc[nt][0]), "+f"(acc[nt][1]), "+f"(acc[nt][2]), "+f"(acc[nt][3])
+                         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+        }
+    }
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+        const int col = n0 + 8 * nt + 2 * t;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int row = r0 + g + 8 * (e >> 1), cc = col + (e & 1);
+            float v = acc[nt][e];
+            if (LOWER && cc > row) v = 0.f;
+            if (ACC) C[row * ldc + cc] += v;
+            else C[row * ldc + cc] = v;
+        }
+    }
+}
+
 template <int D>
 struct GradSmem {
     static constexpr int LD = D + 1;
@@ -649,13 +689,17 @@ bwd_grads(const T *__restrict__ qg, const T *__restrict__ kg, const T *__restric
         }
     }
     // dAqk = (dO V_new^T) on the lower triangle incl. the diagonal  -> sR
+    if constexpr (kTC) {
+        mm_tf32_64x64_nt<D, false, true>(sX, LD, sY, LD, sR, 65);
+    } else {
 #pragma unroll
-    for (int m = 0; m < kC / 4; ++m) {
-        const int r = pr + 4 * m;
-        float acc = 0.f;
-        if (pi <= r)
-            for (int j = 0; j < D; ++j) acc = fmaf(sX[r * LD + j], sY[pi * LD + j], acc);
-        sR[r * 65 + pi] = acc;
+        for (int m = 0; m < kC / 4; ++m) {
+            const int r = pr + 4 * m;
+            float acc = 0.f;
+            if (pi <= r)
+                for (int j = 0; j < D; ++j) acc = fmaf(sX[r * LD + j], sY[pi * LD + j], acc);
+            sR[r * 65 + pi] = acc;
+        }
     }
     // dK_tail = V_new dS'  ->  dk += dK_tail gamma_C / gamma,  dG -= (same) k, dG_C += (same) k
     // (on the tensor cores above for the bf16 path)
@@ -714,12 +758,16 @@ bwd_grads(const T *__restrict__ qg, const T *__restrict__ kg, const T *__restric
         }
     }
     // dT' = dV_new V^T  -> sP
+    if constexpr (kTC) {
+        mm_tf32_64x64_nt<D, false, false>(sX, LD, sY, LD, sP, 65);
+    } else {
 #pragma unroll
-    for (int m = 0; m < kC / 4; ++m) {
-        const int r = pr + 4 * m;
-        float acc = 0.f;
-        for (int j = 0; j < D; ++j) acc = fmaf(sX[r * LD + j], sY[pi * LD + j], acc);
-        sP[r * 65 + pi] = acc;
+        for (int m = 0; m < kC / 4; ++m) {
+            const int r = pr + 4 * m;
+            float acc = 0.f;
+            for (int j = 0; j < D; ++j) acc = fmaf(sX[r * LD + j], sY[pi * LD + j], acc);
+            sP[r * 65 + pi] = acc;
+        }
     }
     __syncthreads();   // V read
     // dW = -dV_new S  -> sY
@@ -746,12 +794,16 @@ bwd_grads(const T *__restrict__ qg, const T *__restrict__ kg, const T *__restric
     }
     __syncthreads();
     // dT' += dW K<-^T
+    if constexpr (kTC) {
+        mm_tf32_64x64_nt<D, true, false>(sY, LD, sX, LD, sP, 65);
+    } else {
 #pragma unroll
-    for (int m = 0; m < kC / 4; ++m) {
-        const int r = pr + 4 * m;
-        float acc = 0.f;
-        for (int cc = 0; cc < D; ++cc) acc = fmaf(sY[r * LD + cc], sX[pi * LD + cc], acc);
-        sP[r * 65 + pi] += acc;
+        for (int m = 0; m < kC / 4; ++m) {
+            const int r = pr + 4 * m;
+            float acc = 0.f;
+            for (int cc = 0; cc < D; ++cc) acc = fmaf(sY[r * LD + cc], sX[pi * LD + cc], acc);
+            sP[r * 65 + pi] += acc;
+        }
     }
     // dK<- = T'^T dW = Diag(beta) M^T dW  ->  dk += dK<- gamma,  dG += dK<- k gamma
     {

@@ -584,6 +584,42 @@ __device__ __forceinline__ void mm_tf32_64x64_nt(const float *A, int lda, const 
     }
 }
 
+// General form: out(row, col, v) receives every element of the 64 x N product
+// A B (fp32 accumulation of tf32 operands), where A(row, k) is A[row * lda + k]
+// (or A[k * lda + row] with TA) and B(k, col) is B[k * ldb + col] (or
+// B[col * ldb + k] with TB).  N = 64 or 128; warp w computes rows 16 (w & 3)
+// .. + 15 and columns N / 2 (w >> 2) .. + N / 2 - 1.  All 8 warps.
+template <int N, int K, bool TA, bool TB, typename Out>
+__device__ __forceinline__ void mm_tf32_any(const float *A, int lda, const float *B, int ldb, Out out)
+{
+    constexpr int NT = N / 16;   // n-tiles of 8 columns per warp
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const int r0 = 16 * (warp & 3), n0 = (N / 2) * (warp >> 2);
+    auto a_at = [&](int row, int k) { return TA ? A[k * lda + row] : A[row * lda + k]; };
+    auto b_at = [&](int k, int col) { return TB ? B[col * ldb + k] : B[(size_t)k * ldb + col]; };
+    float acc[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll 2
+    for (int k0 = 0; k0 < K; k0 += 8) {
+        const uint32_t a0 = tf32_rn(a_at(r0 + g, k0 + t)), a1 = tf32_rn(a_at(r0 + g + 8, k0 + t));
+        const uint32_t a2 = tf32_rn(a_at(r0 + g, k0 + t + 4)), a3 = tf32_rn(a_at(r0 + g + 8, k0 + t + 4));
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int col = n0 + 8 * nt + g;
+            const uint32_t b0 = tf32_rn(b_at(k0 + t, col)), b1 = tf32_rn(b_at(k0 + t + 4, col));
+            asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+                         "{%8, %9}, {%0, %1, %2, %3};"
+                         : "+f"(acc[nt][0]), "+f"(acc[nt][1]), "+f"(acc[nt][2]), "+f"(acc[nt][3])
+                         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+        }
+    }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) out(r0 + g + 8 * (e >> 1), n0 + 8 * nt + 2 * t + (e & 1), acc[nt][e]);
+}
+
 template <int D>
 struct GradSmem {
     static constexpr int LD = D + 1;
@@ -742,7 +778,11 @@ bwd_grads(const T *__restrict__ qg, const T *__restrict__ kg, const T *__restric
         sY[r * LD + j] = r < nrows ? to_f32<T>(vg[(row0 + r) * D + j]) : 0.f;   // V
     }
     __syncthreads();
-    {
+    if constexpr (kTC) {
+        mm_tf32_any<D, kC, true, false>(sM, 65, sX, LD, [&](int r, int cc, float v) {
+            if (r < nrows) dvg[(row0 + r) * D + cc] = from_f32<T>(sb[r] * v);
+        });
+    } else {
         float acc[NR];
 #pragma unroll
         for (int m = 0; m < NR; ++m) acc[m] = 0.f;
@@ -806,7 +846,18 @@ bwd_grads(const T *__restrict__ qg, const T *__restrict__ kg, const T *__restric
         }
     }
     // dK<- = T'^T dW = Diag(beta) M^T dW  ->  dk += dK<- gamma,  dG += dK<- k gamma
-    {
+    if constexpr (kTC) {
+        __syncthreads();   // K<- (sX) has been read: the product goes there
+        mm_tf32_any<D, kC, true, false>(sM, 65, sY, LD, [&](int r, int cc, float v) { sX[r * LD + cc] = v; });
+        __syncthreads();
+#pragma unroll
+        for (int m = 0; m < NR; ++m) {
+            const int r = h + RS * m;
+            const float t = sb[r] * sX[r * LD + c] * __expf(sG[r * LD + c]);
+            dk[m] += t;
+            dG[m] = fmaf(t, sk[r * LD + c], dG[m]);
+        }
+    } else {
         float acc[NR];
 #pragma unroll
         for (int m = 0; m < NR; ++m) acc[m] = 0.f;
@@ -836,21 +887,28 @@ bwd_grads(const T *__restrict__ qg, const T *__restrict__ kg, const T *__restric
     __syncthreads();
     // dA = -M^T dM M^T on the strict lower triangle: first Z = dM M^T -> sY (as 64 x 65)
     float *sZ = sY;
+    if constexpr (kTC) {
+        mm_tf32_any<kC, kC, false, true>(sP, 65, sM, 65, [&](int r, int cc, float v) { sZ[r * 65 + cc] = v; });
+        __syncthreads();
+        mm_tf32_any<kC, kC, true, false>(sM, 65, sZ, 65,
+                                         [&](int r, int cc, float v) { sP[r * 65 + cc] = cc < r ? -v : 0.f; });
+    } else {
 #pragma unroll
-    for (int m = 0; m < kC / 4; ++m) {
-        const int r = pr + 4 * m;
-        float acc = 0.f;
-        for (int kk = 0; kk < kC; ++kk) acc = fmaf(sP[r * 65 + kk], sM[pi * 65 + kk], acc);
-        sZ[r * 65 + pi] = acc;
-    }
-    __syncthreads();
+        for (int m = 0; m < kC / 4; ++m) {
+            const int r = pr + 4 * m;
+            float acc = 0.f;
+            for (int kk = 0; kk < kC; ++kk) acc = fmaf(sP[r * 65 + kk], sM[pi * 65 + kk], acc);
+            sZ[r * 65 + pi] = acc;
+        }
+        __syncthreads();
 #pragma unroll
-    for (int m = 0; m < kC / 4; ++m) {
-        const int r = pr + 4 * m;
-        float acc = 0.f;
-        if (pi < r)
-            for (int kk = 0; kk < kC; ++kk) acc = fmaf(sM[kk * 65 + r], sZ[kk * 65 + pi], acc);
-        sP[r * 65 + pi] = -acc;   // dA (zero on and above the diagonal)
+        for (int m = 0; m < kC / 4; ++m) {
+            const int r = pr + 4 * m;
+            float acc = 0.f;
+            if (pi < r)
+                for (int kk = 0; kk < kC; ++kk) acc = fmaf(sM[kk * 65 + r], sZ[kk * 65 + pi], acc);
+            sP[r * 65 + pi] = -acc;   // dA (zero on and above the diagonal)
+        }
     }
     __syncthreads();
     // decay-weighted contractions of dA (A_ri = beta_r sum_c k_rc k_ic E) and dAqk:

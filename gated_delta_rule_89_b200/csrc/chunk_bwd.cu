@@ -71,6 +71,132 @@ inline BwdWs carve(void *ws, int B, int H, int T, int D)
     return w;
 }
 
+// ------------------------------------------------------------------ tensor-core products
+// The bf16 path at d = 128 runs its larger products on the tensor cores
+// (mma.sync m16n8k8 with tf32 operands, rounded from fp32: about 2^-11
+// relative per operand, fp32 accumulation); the fp32 path, whose bar is 1e-4,
+// keeps them on CUDA cores.
+//
+__device__ __forceinline__ uint32_t tf32_rn(float x)
+{
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
+// C[64][128] = sign * A[64][K] B[K][128]: A in shared memory (row stride lda),
+// B in global or shared memory (row stride ldb), C to shared memory (row
+// stride ldc); warp w computes rows 16 (w & 3) .. + 15 and columns 64 (w >> 2)
+// .. + 63.  All 8 warps.
+template <int K>
+__device__ __forceinline__ void mm_tf32_64x128(const float *A, int lda, const float *B, int ldb, float *C, int ldc,
+                                               float sign)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const int r0 = 16 * (warp & 3), n0 = 64 * (warp >> 2);
+    float acc[8][4];
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll 2
+    for (int k0 = 0; k0 < K; k0 += 8) {
+        const uint32_t a0 = tf32_rn(A[(r0 + g) * lda + k0 + t]), a1 = tf32_rn(A[(r0 + g + 8) * lda + k0 + t]);
+        const uint32_t a2 = tf32_rn(A[(r0 + g) * lda + k0 + t + 4]), a3 = tf32_rn(A[(r0 + g + 8) * lda + k0 + t + 4]);
+        const float *b = B + (size_t)(k0 + t) * ldb + n0 + g;
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+            const uint32_t b0 = tf32_rn(b[8 * nt]), b1 = tf32_rn(b[(size_t)4 * ldb + 8 * nt]);
+            asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+                         "{%8, %9}, {%0, %1, %2, %3};"
+                         : "+f"(acc[nt][0]), "+f"(acc[nt][1]), "+f"(acc[nt][2]), "+f"(acc[nt][3])
+                         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+        }
+    }
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+        const int col = n0 + 8 * nt + 2 * t;
+        C[(r0 + g) * ldc + col] = sign * acc[nt][0];
+        C[(r0 + g) * ldc + col + 1] = sign * acc[nt][1];
+        C[(r0 + g + 8) * ldc + col] = sign * acc[nt][2];
+        C[(r0 + g + 8) * ldc + col + 1] = sign * acc[nt][3];
+    }
+}
+
+// C[64][64] (=, or +=) A[64][K] Bm[64][K]^T on the tensor cores (as above),
+// both operands row-major in shared memory; with `lower` only the entries
+// with column <= row are stored (the others get 0).  Warp w computes rows
+// 16 (w & 3) .. + 15 and columns 32 (w >> 2) .. + 31.  All 8 warps.
+template <int K, bool ACC, bool LOWER>
+__device__ __forceinline__ void mm_tf32_64x64_nt(const float *A, int lda, const float *Bm, int ldb, float *C, int ldc)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const int r0 = 16 * (warp & 3), n0 = 32 * (warp >> 2);
+    float acc[4][4];
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll 2
+    for (int k0 = 0; k0 < K; k0 += 8) {
+        const uint32_t a0 = tf32_rn(A[(r0 + g) * lda + k0 + t]), a1 = tf32_rn(A[(r0 + g + 8) * lda + k0 + t]);
+        const uint32_t a2 = tf32_rn(A[(r0 + g) * lda + k0 + t + 4]), a3 = tf32_rn(A[(r0 + g + 8) * lda + k0 + t + 4]);
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) {
+            const float *b = Bm + (n0 + 8 * nt + g) * ldb + k0 + t;
+            const uint32_t b0 = tf32_rn(b[0]), b1 = tf32_rn(b[4]);
+            asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+                         "{%8, %9}, {%0, %1, %2, %3};"
+                         : "+f"(acc[nt][0]), "+f"(acc[nt][1]), "+f"(acc[nt][2]), "+f"(acc[nt][3])
+                         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+        }
+    }
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+        const int col = n0 + 8 * nt + 2 * t;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int row = r0 + g + 8 * (e >> 1), cc = col + (e & 1);
+            float v = acc[nt][e];
+            if (LOWER && cc > row) v = 0.f;
+            if (ACC) C[row * ldc + cc] += v;
+            else C[row * ldc + cc] = v;
+        }
+    }
+}
+
+// General form: out(row, col, v) receives every element of the 64 x N product
+// A B (fp32 accumulation of tf32 operands), where A(row, k) is A[row * lda + k]
+// (or A[k * lda + row] with TA) and B(k, col) is B[k * ldb + col] (or
+// B[col * ldb + k] with TB).  N = 64 or 128; warp w computes rows 16 (w & 3)
+// .. + 15 and columns N / 2 (w >> 2) .. + N / 2 - 1.  All 8 warps.
+template <int N, int K, bool TA, bool TB, typename Out>
+__device__ __forceinline__ void mm_tf32_any(const float *A, int lda, const float *B, int ldb, Out out)
+{
+    constexpr int NT = N / 16;   // n-tiles of 8 columns per warp
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const int r0 = 16 * (warp & 3), n0 = (N / 2) * (warp >> 2);
+    auto a_at = [&](int row, int k) { return TA ? A[k * lda + row] : A[row * lda + k]; };
+    auto b_at = [&](int k, int col) { return TB ? B[col * ldb + k] : B[(size_t)k * ldb + col]; };
+    float acc[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll 2
+    for (int k0 = 0; k0 < K; k0 += 8) {
+        const uint32_t a0 = tf32_rn(a_at(r0 + g, k0 + t)), a1 = tf32_rn(a_at(r0 + g + 8, k0 + t));
+        const uint32_t a2 = tf32_rn(a_at(r0 + g, k0 + t + 4)), a3 = tf32_rn(a_at(r0 + g + 8, k0 + t + 4));
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int col = n0 + 8 * nt + g;
+            const uint32_t b0 = tf32_rn(b_at(k0 + t, col)), b1 = tf32_rn(b_at(k0 + t + 4, col));
+            asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+                         "{%8, %9}, {%0, %1, %2, %3};"
+                         : "+f"(acc[nt][0]), "+f"(acc[nt][1]), "+f"(acc[nt][2]), "+f"(acc[nt][3])
+                         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+        }
+    }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) out(r0 + g + 8 * (e >> 1), n0 + 8 * nt + 2 * t + (e & 1), acc[nt][e]);
+}
+
 // ------------------------------------------------------------------ 1. prep
 template <int D>
 struct PrepSmem {
@@ -88,6 +214,7 @@ bwd_prep(const T *__restrict__ qg, const T *__restrict__ kg, const T *__restrict
 {
     using L = PrepSmem<D>;
     constexpr int LD = L::LD, LM = L::LM, RS = kBT / D, NR = kC / RS;
+    constexpr bool kTC = D == 128 && !std::is_same<T, float>::value;   // tensor-core products (bf16 path)
     extern __shared__ float sm[];
     float *sk = sm + L::K, *sq = sm + L::Q, *sG = sm + L::G, *sA = sm + L::A, *sM = sm + L::M, *sb = sm + L::B;
     const int tid = threadIdx.x;
@@ -221,22 +348,27 @@ bwd_prep(const T *__restrict__ qg, const T *__restrict__ kg, const T *__restrict
     }
     __syncthreads();
     const int c = tid % D, h = tid / D;
-    // (16 of the thread's rows at a time; four columns of M per step, one
-    // 16-byte broadcast read per row)
-    for (int m0 = 0; m0 < NR; m0 += 16) {
-        float acc[16];
+    if constexpr (kTC) {
+        mm_tf32_any<D, kC, false, false>(sM, LM, sq, LD,
+                                         [&](int r, int cc, float v) { w.W[(prow0 + r) * D + cc] = v; });
+    } else {
+        // (16 of the thread's rows at a time; four columns of M per step, one
+        // 16-byte broadcast read per row)
+        for (int m0 = 0; m0 < NR; m0 += 16) {
+            float acc[16];
 #pragma unroll
-        for (int m = 0; m < 16; ++m) acc[m] = 0.f;
-        for (int i = 0; i < kC; i += 4) {
-            const float b0 = sq[i * LD + c], b1 = sq[(i + 1) * LD + c], b2 = sq[(i + 2) * LD + c], b3 = sq[(i + 3) * LD + c];
+            for (int m = 0; m < 16; ++m) acc[m] = 0.f;
+            for (int i = 0; i < kC; i += 4) {
+                const float b0 = sq[i * LD + c], b1 = sq[(i + 1) * LD + c], b2 = sq[(i + 2) * LD + c], b3 = sq[(i + 3) * LD + c];
 #pragma unroll
-            for (int m = 0; m < 16; ++m) {
-                const float4 mv = *reinterpret_cast<const float4 *>(&sM[(h + RS * (m0 + m)) * LM + i]);
-                acc[m] = fmaf(mv.w, b3, fmaf(mv.z, b2, fmaf(mv.y, b1, fmaf(mv.x, b0, acc[m]))));
+                for (int m = 0; m < 16; ++m) {
+                    const float4 mv = *reinterpret_cast<const float4 *>(&sM[(h + RS * (m0 + m)) * LM + i]);
+                    acc[m] = fmaf(mv.w, b3, fmaf(mv.z, b2, fmaf(mv.y, b1, fmaf(mv.x, b0, acc[m]))));
+                }
             }
-        }
 #pragma unroll
-        for (int m = 0; m < 16; ++m) w.W[(prow0 + h + RS * (m0 + m)) * D + c] = acc[m];
+            for (int m = 0; m < 16; ++m) w.W[(prow0 + h + RS * (m0 + m)) * D + c] = acc[m];
+        }
     }
     __syncthreads();
     // U = M Diag(beta) V (d_v = D)
@@ -246,22 +378,27 @@ bwd_prep(const T *__restrict__ qg, const T *__restrict__ kg, const T *__restrict
         sq[r * LD + j] = r < nrows ? sb[r] * to_f32<T>(vg[(row0 + r) * D + j]) : 0.f;
     }
     __syncthreads();
-    // (16 of the thread's rows at a time; four columns of M per step, one
-    // 16-byte broadcast read per row)
-    for (int m0 = 0; m0 < NR; m0 += 16) {
-        float acc[16];
+    if constexpr (kTC) {
+        mm_tf32_any<D, kC, false, false>(sM, LM, sq, LD,
+                                         [&](int r, int cc, float v) { w.U[(prow0 + r) * D + cc] = v; });
+    } else {
+        // (16 of the thread's rows at a time; four columns of M per step, one
+        // 16-byte broadcast read per row)
+        for (int m0 = 0; m0 < NR; m0 += 16) {
+            float acc[16];
 #pragma unroll
-        for (int m = 0; m < 16; ++m) acc[m] = 0.f;
-        for (int i = 0; i < kC; i += 4) {
-            const float b0 = sq[i * LD + c], b1 = sq[(i + 1) * LD + c], b2 = sq[(i + 2) * LD + c], b3 = sq[(i + 3) * LD + c];
+            for (int m = 0; m < 16; ++m) acc[m] = 0.f;
+            for (int i = 0; i < kC; i += 4) {
+                const float b0 = sq[i * LD + c], b1 = sq[(i + 1) * LD + c], b2 = sq[(i + 2) * LD + c], b3 = sq[(i + 3) * LD + c];
 #pragma unroll
-            for (int m = 0; m < 16; ++m) {
-                const float4 mv = *reinterpret_cast<const float4 *>(&sM[(h + RS * (m0 + m)) * LM + i]);
-                acc[m] = fmaf(mv.w, b3, fmaf(mv.z, b2, fmaf(mv.y, b1, fmaf(mv.x, b0, acc[m]))));
+                for (int m = 0; m < 16; ++m) {
+                    const float4 mv = *reinterpret_cast<const float4 *>(&sM[(h + RS * (m0 + m)) * LM + i]);
+                    acc[m] = fmaf(mv.w, b3, fmaf(mv.z, b2, fmaf(mv.y, b1, fmaf(mv.x, b0, acc[m]))));
+                }
             }
-        }
 #pragma unroll
-        for (int m = 0; m < 16; ++m) w.U[(prow0 + h + RS * (m0 + m)) * D + c] = acc[m];
+            for (int m = 0; m < 16; ++m) w.U[(prow0 + h + RS * (m0 + m)) * D + c] = acc[m];
+        }
     }
 }
 
@@ -498,128 +635,6 @@ bwd_rev_scan(const T *__restrict__ dOg, const float *__restrict__ dST, float *__
 }
 
 // ------------------------------------------------------------------ 4. per-chunk gradients
-// C[64][128] = sign * A[64][K] B[K][128] on the tensor cores (mma.sync
-// m16n8k8 with tf32 operands, rounded from fp32: about 2^-11 relative per
-// operand, fp32 accumulation), for the bf16 path's three 64 x 128 x 128
-// products.  A in shared memory (row stride lda), B in global or shared
-// memory (row stride ldb), C to shared memory (row stride ldc); warp w computes
-// rows 16 (w & 3) .. + 15 and columns 64 (w >> 2) .. + 63.  All 8 warps.
-__device__ __forceinline__ uint32_t tf32_rn(float x)
-{
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return r;
-}
-
-template <int K>
-__device__ __forceinline__ void mm_tf32_64x128(const float *A, int lda, const float *B, int ldb, float *C, int ldc,
-                                               float sign)
-{
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-    const int r0 = 16 * (warp & 3), n0 = 64 * (warp >> 2);
-    float acc[8][4];
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-#pragma unroll 2
-    for (int k0 = 0; k0 < K; k0 += 8) {
-        const uint32_t a0 = tf32_rn(A[(r0 + g) * lda + k0 + t]), a1 = tf32_rn(A[(r0 + g + 8) * lda + k0 + t]);
-        const uint32_t a2 = tf32_rn(A[(r0 + g) * lda + k0 + t + 4]), a3 = tf32_rn(A[(r0 + g + 8) * lda + k0 + t + 4]);
-        const float *b = B + (size_t)(k0 + t) * ldb + n0 + g;
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-            const uint32_t b0 = tf32_rn(b[8 * nt]), b1 = tf32_rn(b[(size_t)4 * ldb + 8 * nt]);
-            asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-                         "{%8, %9}, {%0, %1, %2, %3};"
-                         : "+f"(acc[nt][0]), "+f"(acc[nt][1]), "+f"(acc[nt][2]), "+f"(acc[nt][3])
-                         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-        }
-    }
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-        const int col = n0 + 8 * nt + 2 * t;
-        C[(r0 + g) * ldc + col] = sign * acc[nt][0];
-        C[(r0 + g) * ldc + col + 1] = sign * acc[nt][1];
-        C[(r0 + g + 8) * ldc + col] = sign * acc[nt][2];
-        C[(r0 + g + 8) * ldc + col + 1] = sign * acc[nt][3];
-    }
-}
-
-// C[64][64] (=, or +=) A[64][K] Bm[64][K]^T on the tensor cores (as above),
-// both operands row-major in shared memory; with `lower` only the entries
-// with column <= row are stored (the others get 0).  Warp w computes rows
-// 16 (w & 3) .. + 15 and columns 32 (w >> 2) .. + 31.  All 8 warps.
-template <int K, bool ACC, bool LOWER>
-__device__ __forceinline__ void mm_tf32_64x64_nt(const float *A, int lda, const float *Bm, int ldb, float *C, int ldc)
-{
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-    const int r0 = 16 * (warp & 3), n0 = 32 * (warp >> 2);
-    float acc[4][4];
-#pragma unroll
-    for (int nt = 0; nt < 4; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-#pragma unroll 2
-    for (int k0 = 0; k0 < K; k0 += 8) {
-        const uint32_t a0 = tf32_rn(A[(r0 + g) * lda + k0 + t]), a1 = tf32_rn(A[(r0 + g + 8) * lda + k0 + t]);
-        const uint32_t a2 = tf32_rn(A[(r0 + g) * lda + k0 + t + 4]), a3 = tf32_rn(A[(r0 + g + 8) * lda + k0 + t + 4]);
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt) {
-            const float *b = Bm + (n0 + 8 * nt + g) * ldb + k0 + t;
-            const uint32_t b0 = tf32_rn(b[0]), b1 = tf32_rn(b[4]);
-            asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-                         "{%8, %9}, {%0, %1, %2, %3};"
-                         : "+f"(acc[nt][0]), "+f"(acc[nt][1]), "+f"(acc[nt][2]), "+f"(acc[nt][3])
-                         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-        }
-    }
-#pragma unroll
-    for (int nt = 0; nt < 4; ++nt) {
-        const int col = n0 + 8 * nt + 2 * t;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int row = r0 + g + 8 * (e >> 1), cc = col + (e & 1);
-            float v = acc[nt][e];
-            if (LOWER && cc > row) v = 0.f;
-            if (ACC) C[row * ldc + cc] += v;
-            else C[row * ldc + cc] = v;
-        }
-    }
-}
-
-// General form: out(row, col, v) receives every element of the 64 x N product
-// A B (fp32 accumulation of tf32 operands), where A(row, k) is A[row * lda + k]
-// (or A[k * lda + row] with TA) and B(k, col) is B[k * ldb + col] (or
-// B[col * ldb + k] with TB).  N = 64 or 128; warp w computes rows 16 (w & 3)
-// .. + 15 and columns N / 2 (w >> 2) .. + N / 2 - 1.  All 8 warps.
-template <int N, int K, bool TA, bool TB, typename Out>
-__device__ __forceinline__ void mm_tf32_any(const float *A, int lda, const float *B, int ldb, Out out)
-{
-    constexpr int NT = N / 16;   // n-tiles of 8 columns per warp
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-    const int r0 = 16 * (warp & 3), n0 = (N / 2) * (warp >> 2);
-    auto a_at = [&](int row, int k) { return TA ? A[k * lda + row] : A[row * lda + k]; };
-    auto b_at = [&](int k, int col) { return TB ? B[col * ldb + k] : B[(size_t)k * ldb + col]; };
-    float acc[NT][4];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-#pragma unroll 2
-    for (int k0 = 0; k0 < K; k0 += 8) {
-        const uint32_t a0 = tf32_rn(a_at(r0 + g, k0 + t)), a1 = tf32_rn(a_at(r0 + g + 8, k0 + t));
-        const uint32_t a2 = tf32_rn(a_at(r0 + g, k0 + t + 4)), a3 = tf32_rn(a_at(r0 + g + 8, k0 + t + 4));
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            const int col = n0 + 8 * nt + g;
-            const uint32_t b0 = tf32_rn(b_at(k0 + t, col)), b1 = tf32_rn(b_at(k0 + t + 4, col));
-            asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-                         "{%8, %9}, {%0, %1, %2, %3};"
-                         : "+f"(acc[nt][0]), "+f"(acc[nt][1]), "+f"(acc[nt][2]), "+f"(acc[nt][3])
-                         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-        }
-    }
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) out(r0 + g + 8 * (e >> 1), n0 + 8 * nt + 2 * t + (e & 1), acc[nt][e]);
-}
-
 template <int D>
 struct GradSmem {
     static constexpr int LD = D + 1;

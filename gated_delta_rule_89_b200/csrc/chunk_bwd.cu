@@ -161,17 +161,20 @@ __device__ __forceinline__ void mm_tf32_64x64_nt(const float *A, int lda, const 
     }
 }
 
-// General form: out(row, col, v) receives every element of the 64 x N product
+// General form: out(row, col, v) receives every element of the M x N product
 // A B (fp32 accumulation of tf32 operands), where A(row, k) is A[row * lda + k]
 // (or A[k * lda + row] with TA) and B(k, col) is B[k * ldb + col] (or
-// B[col * ldb + k] with TB).  N = 64 or 128; warp w computes rows 16 (w & 3)
-// .. + 15 and columns N / 2 (w >> 2) .. + N / 2 - 1.  All 8 warps.
-template <int N, int K, bool TA, bool TB, typename Out>
+// B[col * ldb + k] with TB).  M = 64 (warp w: rows 16 (w & 3) .. + 15, columns
+// N / 2 (w >> 2) .. + N / 2 - 1) or M = 32 (rows 16 (w & 1) .. + 15, columns
+// N / 4 (w >> 1) .. + N / 4 - 1); N a multiple of 32.  All 8 warps.
+template <int N, int K, bool TA, bool TB, int M = 64, typename Out>
 __device__ __forceinline__ void mm_tf32_any(const float *A, int lda, const float *B, int ldb, Out out)
 {
-    constexpr int NT = N / 16;   // n-tiles of 8 columns per warp
+    static_assert(M == 64 || M == 32, "64 or 32 rows");
+    constexpr int MW = M / 16, NW = 8 / MW;   // warps along the rows, along the columns
+    constexpr int NT = N / NW / 8;            // n-tiles of 8 columns per warp
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-    const int r0 = 16 * (warp & 3), n0 = (N / 2) * (warp >> 2);
+    const int r0 = 16 * (warp % MW), n0 = (N / NW) * (warp / MW);
     auto a_at = [&](int row, int k) { return TA ? A[k * lda + row] : A[row * lda + k]; };
     auto b_at = [&](int k, int col) { return TB ? B[col * ldb + k] : B[(size_t)k * ldb + col]; };
     float acc[NT][4];
@@ -409,22 +412,33 @@ bwd_prep(const T *__restrict__ qg, const T *__restrict__ kg, const T *__restrict
 // dV_new) and 2 state rows x 8 channels of the state update, reading 16-byte
 // operand vectors (rows padded to D + 4 floats).
 template <int D>
-struct FwdSmem {
+struct FwdSmem {   // W, K_tail and G_C in two buffers, by chunk parity
     static constexpr int L4 = D + 4;
-    static constexpr int S = 0, W = S + kTile * L4, KT = W + kC * L4, VN = KT + kC * L4, GC = VN + kC * (kTile + 1);
-    static constexpr int TOTAL = GC + D;
+    static constexpr int S = 0, W = S + kTile * L4, KT = W + 2 * kC * L4, VN = KT + 2 * kC * L4,
+                         GC = VN + kC * (kTile + 1);
+    static constexpr int TOTAL = GC + 2 * D;
 };
 
-// K_tail rows of chunk n into kt, G_C into gc
+// 16-byte asynchronous global -> shared copies (cp.async), committed in groups
+__device__ __forceinline__ void cp16(float *smem, const float *gmem)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(smem))),
+                 "l"(gmem)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// rows [0, kC) x D floats of a per-token workspace part into a shared tile of row stride D + 4
 template <int D>
-__device__ __forceinline__ void load_ktail(float *kt, float *gc, const BwdWs &w, size_t prow0, int tid)
+__device__ __forceinline__ void cp_rows(float *dst, const float *src, int tid)
 {
     constexpr int L4 = D + 4;
-    for (int c = tid; c < D; c += kBT) gc[c] = w.G[(prow0 + kC - 1) * D + c];
 #pragma unroll 4
     for (int idx = tid; idx < kC * D / 4; idx += kBT) {
         const int r = idx / (D / 4), c4 = idx - r * (D / 4);
-        *reinterpret_cast<float4 *>(kt + r * L4 + 4 * c4) = *reinterpret_cast<const float4 *>(w.Kt + (prow0 + r) * D + 4 * c4);
+        cp16(dst + r * L4 + 4 * c4, src + (size_t)r * D + 4 * c4);
     }
 }
 
@@ -471,7 +485,7 @@ __device__ __forceinline__ void outer_rows(float (&acc)[JPT][8], const float *X,
     }
 }
 
-template <int D>
+template <int D, bool TC>
 __global__ void __launch_bounds__(kBT)
 bwd_fwd_scan(const float *__restrict__ S0, BwdWs w, int nch)
 {
@@ -488,28 +502,55 @@ bwd_fwd_scan(const float *__restrict__ S0, BwdWs w, int nch)
     }
     const int vj = tid & 15, vr = 4 * (tid >> 4);               // V_new: rows vr..vr+3, state rows vj, vj+16
     const int cg = tid % NCG, jb0 = JPT * (tid / NCG), c0 = 8 * cg;   // update: channels c0..c0+7
+    // the W, K_tail and G_C of chunk n + 1 load (cp.async) while chunk n is computed
+    auto issue = [&](int n) {
+        const size_t prow = (size_t)head * nch * kC + (size_t)n * kC;
+        const int b = n & 1;
+        cp_rows<D>(sW + b * kC * L4, w.W + prow * D, tid);
+        cp_rows<D>(sKt + b * kC * L4, w.Kt + prow * D, tid);
+        for (int c4 = tid; c4 < D / 4; c4 += kBT) cp16(gc + b * D + 4 * c4, w.G + (prow + kC - 1) * D + 4 * c4);
+        cp_commit();
+    };
+    if (nch > 0) issue(0);
     for (int n = 0; n < nch; ++n) {
         const size_t prow0 = (size_t)head * nch * kC + (size_t)n * kC;
-        __syncthreads();
+        const float *cW = sW + (n & 1) * kC * L4, *cKt = sKt + (n & 1) * kC * L4, *cgc = gc + (n & 1) * D;
+        __syncthreads();   // chunk n - 1 is done with the other buffers and with sS
         float *ck = w.Sck + ((size_t)(head * nch + n) * D + i0) * D;
         for (int idx = tid; idx < kTile * D; idx += kBT) ck[idx] = sS[(idx / D) * L4 + idx % D];
-#pragma unroll 4
-        for (int idx = tid; idx < kC * D / 4; idx += kBT) {
-            const int r = idx / (D / 4), c4 = idx - r * (D / 4);
-            *reinterpret_cast<float4 *>(sW + r * L4 + 4 * c4) = *reinterpret_cast<const float4 *>(w.W + (prow0 + r) * D + 4 * c4);
-        }
-        load_ktail<D>(sKt, gc, w, prow0, tid);
+        if (n + 1 < nch) issue(n + 1);
+        else cp_commit();   // (an empty group keeps the count)
+        float u[4][2];
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < 2; ++b) u[a][b] = w.U[(prow0 + vr + a) * D + i0 + vj + 16 * b];
+        cp_wait<1>();      // chunk n's copies have landed
         __syncthreads();
+        if constexpr (TC) {
+            // V_new = U - W S^T: 64 tokens x this tile's 32 state rows, over 128 channels
+            mm_tf32_any<kTile, D, false, true>(cW, L4, sS, L4, [&](int r, int j, float v) {
+                const float x = w.U[(prow0 + r) * D + i0 + j] - v;
+                sVn[r * TL + j] = x;
+                w.Vn[(prow0 + r) * D + i0 + j] = x;
+            });
+            __syncthreads();
+            // S <- S Diag(gamma_C) + V_new^T K_tail: 32 state rows x 128 channels, over 64 tokens
+            mm_tf32_any<D, kC, true, false, kTile>(sVn, TL, cKt, L4, [&](int j, int cc, float v) {
+                sS[j * L4 + cc] = fmaf(sS[j * L4 + cc], __expf(cgc[cc]), v);
+            });
+            continue;
+        }
         // V_new = U - W S^T (this tile's d_v columns)
         {
             float acc[4][2] = {};
-            dot_4x2<D>(acc, sW, vr, sS, vj, vj + 16);
+            dot_4x2<D>(acc, cW, vr, sS, vj, vj + 16);
 #pragma unroll
             for (int a = 0; a < 4; ++a)
 #pragma unroll
                 for (int b = 0; b < 2; ++b) {
                     const int r = vr + a, j = vj + 16 * b;
-                    const float x = w.U[(prow0 + r) * D + i0 + j] - acc[a][b];
+                    const float x = u[a][b] - acc[a][b];
                     sVn[r * TL + j] = x;
                     w.Vn[(prow0 + r) * D + i0 + j] = x;
                 }
@@ -520,22 +561,23 @@ bwd_fwd_scan(const float *__restrict__ S0, BwdWs w, int nch)
 #pragma unroll
         for (int b = 0; b < JPT; ++b)
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc[b][e] = sS[(jb0 + b) * L4 + c0 + e] * __expf(gc[c0 + e]);
-        outer_rows<D, JPT>(acc, sVn, TL, sKt, jb0, c0, 1.f);
+            for (int e = 0; e < 8; ++e) acc[b][e] = sS[(jb0 + b) * L4 + c0 + e] * __expf(cgc[c0 + e]);
+        outer_rows<D, JPT>(acc, sVn, TL, cKt, jb0, c0, 1.f);
         __syncthreads();
 #pragma unroll
         for (int b = 0; b < JPT; ++b)
 #pragma unroll
             for (int e = 0; e < 8; ++e) sS[(jb0 + b) * L4 + c0 + e] = acc[b][e];
     }
+    cp_wait<0>();
 }
 
 // ------------------------------------------------------------------ 3. reverse state scan
 template <int D>
-struct RevSmem {
+struct RevSmem {   // Aqk, K_tail, Q<- and W of a chunk each in a buffer of its own
     static constexpr int L4 = D + 4;
     static constexpr int DS = 0, AQ = DS + kTile * L4, DO = AQ + kC * 68, DVN = DO + kC * (kTile + 1),
-                         KT = DVN + kC * (kTile + 1), GC = KT + kC * L4;
+                         KT = DVN + kC * (kTile + 1), QL = KT + kC * L4, W = QL + kC * L4, GC = W + kC * L4;
     static constexpr int TOTAL = GC + D;
 };
 
@@ -549,7 +591,7 @@ bwd_rev_scan(const T *__restrict__ dOg, const float *__restrict__ dST, float *__
     constexpr int NCG = D / 8, JPT = kTile * NCG / kBT;
     extern __shared__ float sm[];
     float *sdS = sm + L::DS, *sAq = sm + L::AQ, *sdO = sm + L::DO, *sdVn = sm + L::DVN, *sKt = sm + L::KT,
-          *gc = sm + L::GC;
+          *sQl = sm + L::QL, *sWt = sm + L::W, *gc = sm + L::GC;
     const int tid = threadIdx.x;
     const int head = blockIdx.x, i0 = blockIdx.y * kTile;
     for (int idx = tid; idx < kTile * D; idx += kBT) {
@@ -562,19 +604,43 @@ bwd_rev_scan(const T *__restrict__ dOg, const float *__restrict__ dST, float *__
         const int t0 = n * kC, nrows = min(kC, T_len - t0);
         const size_t row0 = (size_t)head * T_len + t0, prow0 = (size_t)head * nch * kC + t0;
         __syncthreads();
-        float *ck = w.dSck + ((size_t)(head * nch + n) * D + i0) * D;
-        for (int idx = tid; idx < kTile * D; idx += kBT) ck[idx] = sdS[(idx / D) * L4 + idx % D];
+        // every operand of the chunk in one batch of asynchronous copies (Aqk,
+        // K_tail, Q<-, W, G_C), then dO through registers, so that the latencies
+        // overlap
         const float *aq = w.Aq + (size_t)(head * nch + n) * kC * kC;
 #pragma unroll 4
-        for (int idx = tid; idx < kC * kC / 4; idx += kBT)
-            *reinterpret_cast<float4 *>(sAq + (idx >> 4) * 68 + 4 * (idx & 15)) = *reinterpret_cast<const float4 *>(aq + 4 * idx);
+        for (int idx = tid; idx < kC * kC / 4; idx += kBT) cp16(sAq + (idx >> 4) * 68 + 4 * (idx & 15), aq + 4 * idx);
+        cp_rows<D>(sKt, w.Kt + prow0 * D, tid);
+        cp_rows<D>(sQl, w.Ql + prow0 * D, tid);
+        cp_rows<D>(sWt, w.W + prow0 * D, tid);
+        for (int c4 = tid; c4 < D / 4; c4 += kBT) cp16(gc + 4 * c4, w.G + (prow0 + kC - 1) * D + 4 * c4);
+        cp_commit();
+        float *ck = w.dSck + ((size_t)(head * nch + n) * D + i0) * D;
+        for (int idx = tid; idx < kTile * D; idx += kBT) ck[idx] = sdS[(idx / D) * L4 + idx % D];
 #pragma unroll 8
         for (int idx = tid; idx < kC * kTile; idx += kBT) {
             const int r = idx / kTile, j = idx - r * kTile;
             sdO[r * TL + j] = r < nrows ? to_f32<T>(dOg[(row0 + r) * D + i0 + j]) : 0.f;
         }
-        load_ktail<D>(sKt, gc, w, prow0, tid);
+        cp_wait<0>();
         __syncthreads();
+        if constexpr (D == 128 && !std::is_same<T, float>::value) {   // tensor cores (bf16 path)
+            // dV_new = K_tail dS^T + Aqk^T dO: 64 tokens x 32 state rows
+            mm_tf32_any<kTile, D, false, true>(sKt, L4, sdS, L4, [&](int r, int j, float v) { sdVn[r * TL + j] = v; });
+            mm_tf32_any<kTile, kC, true, false>(sAq, 68, sdO, TL, [&](int r, int j, float v) {
+                const float x = sdVn[r * TL + j] + v;
+                sdVn[r * TL + j] = x;
+                w.dVn[(prow0 + r) * D + i0 + j] = x;
+            });
+            __syncthreads();
+            // dS <- dS Diag(gamma_C) + dO^T Q<- - dV_new^T W: 32 state rows x 128 channels
+            mm_tf32_any<D, kC, true, false, kTile>(sdO, TL, sQl, L4, [&](int j, int cc, float v) {
+                sdS[j * L4 + cc] = fmaf(sdS[j * L4 + cc], __expf(gc[cc]), v);
+            });
+            mm_tf32_any<D, kC, true, false, kTile>(sdVn, TL, sWt, L4,
+                                                  [&](int j, int cc, float v) { sdS[j * L4 + cc] -= v; });
+            continue;
+        }
         // dV_new = Aqk^T dO + K_tail dS^T  (Aqk is zero above the diagonal)
         {
             float acc[4][2] = {};
@@ -601,27 +667,14 @@ bwd_rev_scan(const T *__restrict__ dOg, const float *__restrict__ dST, float *__
                 }
         }
         __syncthreads();
-        // dS <- dS Diag(gamma_C) + dO^T Q<- - dV_new^T W  (Q<-, then W, staged in the K_tail buffer)
+        // dS <- dS Diag(gamma_C) + dO^T Q<- - dV_new^T W
         float acc[JPT][8];
 #pragma unroll
         for (int b = 0; b < JPT; ++b)
 #pragma unroll
             for (int e = 0; e < 8; ++e) acc[b][e] = sdS[(jb0 + b) * L4 + c0 + e] * __expf(gc[c0 + e]);
-#pragma unroll 4
-        for (int idx = tid; idx < kC * D / 4; idx += kBT) {
-            const int r = idx / (D / 4), c4 = idx - r * (D / 4);
-            *reinterpret_cast<float4 *>(sKt + r * L4 + 4 * c4) = *reinterpret_cast<const float4 *>(w.Ql + (prow0 + r) * D + 4 * c4);
-        }
-        __syncthreads();
-        outer_rows<D, JPT>(acc, sdO, TL, sKt, jb0, c0, 1.f);
-        __syncthreads();
-#pragma unroll 4
-        for (int idx = tid; idx < kC * D / 4; idx += kBT) {
-            const int r = idx / (D / 4), c4 = idx - r * (D / 4);
-            *reinterpret_cast<float4 *>(sKt + r * L4 + 4 * c4) = *reinterpret_cast<const float4 *>(w.W + (prow0 + r) * D + 4 * c4);
-        }
-        __syncthreads();
-        outer_rows<D, JPT>(acc, sdVn, TL, sKt, jb0, c0, -1.f);
+        outer_rows<D, JPT>(acc, sdO, TL, sQl, jb0, c0, 1.f);
+        outer_rows<D, JPT>(acc, sdVn, TL, sWt, jb0, c0, -1.f);
         __syncthreads();
 #pragma unroll
         for (int b = 0; b < JPT; ++b)
@@ -1183,7 +1236,7 @@ cudaError_t launch_typed(const BwdArgs &a, cudaStream_t st, int *launches)
         ++*launches;
     }
     {
-        auto kern = bwd_fwd_scan<D>;
+        auto kern = bwd_fwd_scan<D, D == 128 && !std::is_same<T, float>::value>;
         const size_t bytes = sizeof(float) * FwdSmem<D>::TOTAL;
         if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes))) return e;
         kern<<<dim3(BH, D / kTile), kBT, bytes, st>>>(a.S0, w, nch);

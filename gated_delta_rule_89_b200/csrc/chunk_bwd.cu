@@ -412,11 +412,10 @@ bwd_prep(const T *__restrict__ qg, const T *__restrict__ kg, const T *__restrict
 // dV_new) and 2 state rows x 8 channels of the state update, reading 16-byte
 // operand vectors (rows padded to D + 4 floats).
 template <int D>
-struct FwdSmem {   // W, K_tail and G_C in two buffers, by chunk parity
+struct FwdSmem {   // one buffer each for W, K_tail and G_C: two CTAs fit on an SM
     static constexpr int L4 = D + 4;
-    static constexpr int S = 0, W = S + kTile * L4, KT = W + 2 * kC * L4, VN = KT + 2 * kC * L4,
-                         GC = VN + kC * (kTile + 1);
-    static constexpr int TOTAL = GC + 2 * D;
+    static constexpr int S = 0, W = S + kTile * L4, KT = W + kC * L4, VN = KT + kC * L4, GC = VN + kC * (kTile + 1);
+    static constexpr int TOTAL = GC + D;
 };
 
 // 16-byte asynchronous global -> shared copies (cp.async), committed in groups
@@ -502,30 +501,24 @@ bwd_fwd_scan(const float *__restrict__ S0, BwdWs w, int nch)
     }
     const int vj = tid & 15, vr = 4 * (tid >> 4);               // V_new: rows vr..vr+3, state rows vj, vj+16
     const int cg = tid % NCG, jb0 = JPT * (tid / NCG), c0 = 8 * cg;   // update: channels c0..c0+7
-    // the W, K_tail and G_C of chunk n + 1 load (cp.async) while chunk n is computed
-    auto issue = [&](int n) {
-        const size_t prow = (size_t)head * nch * kC + (size_t)n * kC;
-        const int b = n & 1;
-        cp_rows<D>(sW + b * kC * L4, w.W + prow * D, tid);
-        cp_rows<D>(sKt + b * kC * L4, w.Kt + prow * D, tid);
-        for (int c4 = tid; c4 < D / 4; c4 += kBT) cp16(gc + b * D + 4 * c4, w.G + (prow + kC - 1) * D + 4 * c4);
-        cp_commit();
-    };
-    if (nch > 0) issue(0);
+    // W, K_tail and G_C of the chunk in one batch of asynchronous copies; the
+    // other CTA on the SM computes while they land
+    const float *cW = sW, *cKt = sKt, *cgc = gc;
     for (int n = 0; n < nch; ++n) {
         const size_t prow0 = (size_t)head * nch * kC + (size_t)n * kC;
-        const float *cW = sW + (n & 1) * kC * L4, *cKt = sKt + (n & 1) * kC * L4, *cgc = gc + (n & 1) * D;
-        __syncthreads();   // chunk n - 1 is done with the other buffers and with sS
+        __syncthreads();   // chunk n - 1 is done with the buffers and with sS
+        cp_rows<D>(sW, w.W + prow0 * D, tid);
+        cp_rows<D>(sKt, w.Kt + prow0 * D, tid);
+        for (int c4 = tid; c4 < D / 4; c4 += kBT) cp16(gc + 4 * c4, w.G + (prow0 + kC - 1) * D + 4 * c4);
+        cp_commit();
         float *ck = w.Sck + ((size_t)(head * nch + n) * D + i0) * D;
         for (int idx = tid; idx < kTile * D; idx += kBT) ck[idx] = sS[(idx / D) * L4 + idx % D];
-        if (n + 1 < nch) issue(n + 1);
-        else cp_commit();   // (an empty group keeps the count)
         float u[4][2];
 #pragma unroll
         for (int a = 0; a < 4; ++a)
 #pragma unroll
             for (int b = 0; b < 2; ++b) u[a][b] = w.U[(prow0 + vr + a) * D + i0 + vj + 16 * b];
-        cp_wait<1>();      // chunk n's copies have landed
+        cp_wait<0>();
         __syncthreads();
         if constexpr (TC) {
             // V_new = U - W S^T: 64 tokens x this tile's 32 state rows, over 128 channels

@@ -27,8 +27,8 @@
 // Warp roles (448 threads):
 //   warp 0      TMA producer (lane 0): all tiles of a chunk land in one of
 //               two stages and complete one barrier; gamma_C in two slots.
-//               Lane 1 issues the TMA stores of the output tiles (and, for
-//               the gated output, the loads of the gate tiles).
+//               Lane 1 issues the TMA stores of the output tiles (for the
+//               gated output instead the loads of the gate tiles).
 //   warp 1      TMEM allocation and the MMA issuer (one lane), in the order
 //               XO(n) = S_n [Q<-; -W]^T (in two halves, each issued once its
 //               half of the bf16 S_n is in smem), SO(n) = V_new^T(n)
@@ -37,11 +37,11 @@
 //   warps 2-9   the state conversions, split by columns between warps 2-5
 //               and 6-9: on the sequential path S (TMEM) -> bf16 smem and
 //               V_new^T (TMEM) -> bf16 smem; off it, in the gaps while the
-//               tensor core runs, S *= gamma_C in TMEM.
+//               tensor core runs, gamma_C S into the other TMEM region.
 //   warps 10-13 the output epilogue, one chunk behind the MMAs (the
-//               [V_new^T | O^T] accumulator is double-buffered): O^T (TMEM) ->
-//               bf16 staging tile -> TMA store, then the O^T columns are
-//               zeroed for the chunk after next.  With OEPI the layer's gated output is
+//               TMEM regions alternate by chunk): O^T (TMEM) -> bf16 staging
+//               tile -> TMA store, then the O^T columns are zeroed for the
+//               chunk after next.  With OEPI the layer's gated output is
 //               fused in (and stored by these warps themselves):
 //               y_t = Sigmoid(gate_t) * RMSNorm(o_t) per head
 //               ("Token Mixer I", section "The Kimi Linear Model

@@ -55,6 +55,7 @@ CASES = [
     (1, 1, 1, 128, "per_channel", torch.bfloat16, "softplus_n02_clamp5"),
     (2, 1, 300, 128, "per_channel", torch.bfloat16, "long_context_mix"),
     (1, 2, 150, 64, "per_channel", torch.float32, "softplus_n01_plus1_clamp5"),
+    (1, 1, 130, 128, "per_channel", torch.float32, "softplus_n02_clamp5"),   # d = 128 fp32: CUDA-core products
     (1, 1, 97, 64, "scalar", torch.float32, "scalar_softplus_n01_plus2"),
 ]
 

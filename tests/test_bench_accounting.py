@@ -47,3 +47,21 @@ def test_traffic_is_keyed_to_sources():
     for name, ent in bench.TRAFFIC.items():
         assert name in W.WORKLOADS
         assert len(ent["src_sha"]) == 16 and ent["bytes_per_launch"] > 0
+
+
+def test_traffic_only_for_the_sources_it_was_measured_on(tmp_path):
+    # the stored DRAM figure is reported only while the path's sources hash to the
+    # value recorded with it; other sources, or a batch-overridden workload (used
+    # for small profiler captures), report none
+    import dataclasses
+    w = W.WORKLOADS["kda_d128_t8192"]
+    peaks = {"hbm_gbs": 6453.4, "bf16_tflops": 1679.3, "source": "test"}
+    other = tmp_path / "other.cu"
+    other.write_text("// not a source of the path\n")
+    assert bench.roofline(w, 1e-3, peaks, [str(other)])["traffic"] is None
+    wb = dataclasses.replace(w, B=1, name=f"{w.name}_b1")
+    assert bench.roofline(wb, 1e-3, peaks, bench.kernel_sources(w))["traffic"] is None
+    # the fractions: against the measured copy peak and against the datasheet figure
+    r = bench.roofline(w, 1e-3, peaks, [str(other)])
+    assert abs(r["frac"] - bench.algorithmic_bytes(w) / 1e-3 / 1e9 / 6453.4) < 1e-4
+    assert abs(r["frac_vs_spec"] - bench.algorithmic_bytes(w) / 1e-3 / 1e9 / bench.SPEC_HBM_GBS) < 1e-4

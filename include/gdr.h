@@ -192,8 +192,10 @@ int gdr_chunk_fwd_gated(const void *q, const void *k, const void *v, const float
  * Gating"; the training path of the section "Gated Delta Networks"): the
  * states at chunk boundaries are recomputed, the state gradient runs through
  * the chunks in reverse, and the rest is parallel over chunks.  fp32
- * arithmetic throughout.  The -5 bound on a per-channel g passes the gradient
- * where g >= -5 and blocks it below.
+ * arithmetic; for bf16 inputs at d = 128 the matrix products take tf32
+ * operands (rounded from fp32) on the tensor cores, accumulating in fp32.
+ * The -5 bound on a per-channel g passes the gradient where g >= -5 and
+ * blocks it below.
  *
  *   q, k, v, g, beta, S0   as gdr_chunk_fwd (S0 NULL -> zeros)
  *   dO     [B,H,T,d_v]   dtype                  gradient of O
